@@ -1,0 +1,377 @@
+"""Pins for the fp64 oracle: facts the pages and the mathematics fix, checked
+without trusting the oracle itself.
+
+Each ``pin_*`` takes a loaded oracle library handle (so the same pins can be run
+against deliberately broken copies of the oracle, see test_oracle_mutants.py)
+and raises AssertionError when the oracle disagrees with the fact.
+
+Sources: the RWKV transformer-math page (aicassindra.com, tm_rwkv_math) --
+sections "The WKV operator: attention with a fixed decay", "Why it collapses
+into a recurrence", "Numerical stability: carry the exponent", "A worked
+example, one channel", "Token shift: a two-tap causal convolution"; the aiwiki
+"RWKV" page (eq. 1 and its one-token decode step); the vanos001 "RWKV
+(Attention-RNN Hybrid)" page (decode step written with a negative stored decay).
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "worked_example.txt")
+
+
+def read_golden(path=GOLDEN):
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            key, val = (x.strip() for x in line.split("=", 1))
+            nums = [float(x) for x in val.split()]
+            vals[key] = nums if len(nums) > 1 else nums[0]
+    return vals
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _rand_case(seed, B=2, T=17, C=5, k_std=1.0, w_lo=-3.0, w_hi=1.0):
+    r = _rng(seed)
+    w = np.exp(r.uniform(w_lo, w_hi, C))
+    u = r.normal(0.0, 0.5, C)
+    k = r.normal(0.0, k_std, (B, T, C))
+    v = r.normal(0.0, 1.0, (B, T, C))
+    return w, u, k, v
+
+
+def _accum(st):
+    """True accumulators (A, B) = (a e^p, b e^p) of a [3, ...] state."""
+    return st[0] * np.exp(st[2]), st[1] * np.exp(st[2])
+
+
+# ----------------------------------------------------------------------------
+# The page's worked example
+# ----------------------------------------------------------------------------
+
+def pin_worked_example(L):
+    g = read_golden()
+    w = np.array([g["w"]])
+    u = np.array([g["u"]])
+    k = np.array(g["k"]).reshape(1, 3, 1)
+    v = np.array(g["v"]).reshape(1, 3, 1)
+    tol = 5e-5  # the page prints 4 decimals
+    yd, _ = oracle.wkv_direct(w, u, k, v, L=L)
+    yr, _, _, _ = oracle.wkv_recurrent(w, u, k, v, L=L)
+    yn = oracle.wkv_naive(w, u, k, v, L=L)
+    for y in (yd, yr, yn):
+        assert abs(y[0, 2, 0] - g["wkv_last"]) <= tol, (y[0, 2, 0], g["wkv_last"])
+    # the page's intermediate accumulators, through the stored state
+    _, _, st1, _ = oracle.wkv_recurrent(w, u, k[:, :1], v[:, :1], L=L)
+    A0, B0 = _accum(st1)
+    assert abs(A0[0, 0] - g["A_0"]) <= tol and abs(B0[0, 0] - g["B_0"]) <= tol, (A0, B0)
+    _, _, st2, _ = oracle.wkv_recurrent(w, u, k[:, :2], v[:, :2], L=L)
+    A1, B1 = _accum(st2)
+    assert abs(A1[0, 0] - g["A_1"]) <= tol and abs(B1[0, 0] - g["B_1"]) <= tol, (A1, B1)
+    # the page's numerator and denominator are sums of three terms each printed to
+    # 4 decimals, so each carries up to 2e-4 of rounding; their ratio then agrees
+    # with y to 3.9 * (2e-4/19.6 + 2e-4/5.07) < 2e-4
+    assert abs(g["numerator"] / g["denominator"] - yd[0, 2, 0]) <= 2e-4
+    assert abs(math.exp(-g["w"]) - g["decay"]) <= tol
+
+
+# ----------------------------------------------------------------------------
+# Three routes to the same number
+# ----------------------------------------------------------------------------
+
+def pin_routes_agree(L):
+    for seed, (B, T, C) in enumerate([(1, 1, 1), (2, 17, 5), (1, 64, 64), (3, 33, 7)]):
+        w, u, k, v = _rand_case(100 + seed, B, T, C)
+        yd, sd = oracle.wkv_direct(w, u, k, v, L=L)
+        yr, sr, _, _ = oracle.wkv_recurrent(w, u, k, v, L=L)
+        yn = oracle.wkv_naive(w, u, k, v, L=L)
+        assert np.all(np.isfinite(yd)) and np.all(np.isfinite(yr))
+        scale = np.maximum(sd, 1e-300)
+        assert np.max(np.abs(yd - yr) / scale) <= 1e-12
+        assert np.max(np.abs(yd - yn) / scale) <= 1e-12
+        assert np.max(np.abs(sd - sr) / scale) <= 1e-12
+
+
+def pin_brute_force_high_precision(L):
+    """eq. 1 in 40-digit arithmetic (mpmath) on tiny inputs; the fp64 routes must sit
+    within a few hundred ulps of the exact value."""
+    import mpmath
+    mpmath.mp.dps = 40
+    w, u, k, v = _rand_case(7, B=1, T=9, C=3, k_std=2.0)
+    yd, sd = oracle.wkv_direct(w, u, k, v, L=L)
+    yr, _, _, _ = oracle.wkv_recurrent(w, u, k, v, L=L)
+    for c in range(3):
+        for t in range(9):
+            num = mpmath.mpf(0)
+            den = mpmath.mpf(0)
+            for i in range(t):
+                e = mpmath.exp(-(t - 1 - i) * mpmath.mpf(w[c]) + mpmath.mpf(k[0, i, c]))
+                num += e * mpmath.mpf(v[0, i, c])
+                den += e
+            e = mpmath.exp(mpmath.mpf(u[c]) + mpmath.mpf(k[0, t, c]))
+            num += e * mpmath.mpf(v[0, t, c])
+            den += e
+            exact = float(num / den)
+            assert abs(yd[0, t, c] - exact) <= 1e-13 * sd[0, t, c], (t, c)
+            assert abs(yr[0, t, c] - exact) <= 1e-13 * sd[0, t, c], (t, c)
+
+
+# ----------------------------------------------------------------------------
+# Special cases and closed forms
+# ----------------------------------------------------------------------------
+
+def pin_first_position_is_v(L):
+    """The sum over the past is empty at the first position, so y = v (any k, u, w)."""
+    w, u, k, v = _rand_case(11, B=2, T=5, C=9, k_std=5.0)
+    yr, _, _, _ = oracle.wkv_recurrent(w, u, k, v, L=L)
+    assert np.array_equal(yr[:, 0, :], v[:, 0, :])
+    yd, _ = oracle.wkv_direct(w, u, k, v, L=L)
+    assert np.max(np.abs(yd[:, 0, :] - v[:, 0, :]) / np.maximum(np.abs(v[:, 0, :]), 1e-300)) <= 4e-16
+    yr1, _, _, _ = oracle.wkv_recurrent(w, u, k[:, :1], v[:, :1], L=L)
+    assert np.array_equal(yr1[:, 0, :], v[:, 0, :])
+
+
+def pin_convex_bound(L):
+    """Numerator and denominator share their weights: y_t lies within [min v, max v] of i <= t."""
+    w, u, k, v = _rand_case(12, B=2, T=50, C=8, k_std=3.0)
+    for y in (oracle.wkv_direct(w, u, k, v, L=L)[0], oracle.wkv_recurrent(w, u, k, v, L=L)[0]):
+        lo = np.minimum.accumulate(v, axis=1)
+        hi = np.maximum.accumulate(v, axis=1)
+        assert np.all(y >= lo - 1e-12) and np.all(y <= hi + 1e-12)
+
+
+def pin_running_mean(L):
+    """w = 0, u = 0, constant k: every weight is equal, so y_t is the mean of v_0..v_t."""
+    B, T, C = 2, 40, 6
+    r = _rng(13)
+    v = r.normal(0, 1, (B, T, C))
+    k = np.full((B, T, C), 0.3)
+    w = np.zeros(C)
+    u = np.zeros(C)
+    mean = np.cumsum(v, axis=1) / np.arange(1, T + 1)[None, :, None]
+    for y in (oracle.wkv_direct(w, u, k, v, L=L)[0], oracle.wkv_recurrent(w, u, k, v, L=L)[0],
+              oracle.wkv_naive(w, u, k, v, L=L)):
+        assert np.max(np.abs(y - mean)) <= 1e-13
+
+
+def pin_two_tap_softmax(L):
+    """Huge decay (w = 1e4): only the most recent past token (undecayed, i = t-1) and the
+    current token survive, so y_t is a two-way softmax of (k_{t-1}, u + k_t) over
+    (v_{t-1}, v_t).  Pins the off-by-one in the decay exponent."""
+    B, T, C = 1, 12, 4
+    r = _rng(14)
+    k = r.normal(0, 1.5, (B, T, C))
+    v = r.normal(0, 1, (B, T, C))
+    u = r.normal(0, 0.5, C)
+    w = np.full(C, 1e4)
+    ep = np.exp(k[:, :-1])
+    ec = np.exp(u[None, None, :] + k[:, 1:])
+    want = (ep * v[:, :-1] + ec * v[:, 1:]) / (ep + ec)
+    for y in (oracle.wkv_direct(w, u, k, v, L=L)[0], oracle.wkv_recurrent(w, u, k, v, L=L)[0]):
+        assert np.max(np.abs(y[:, 1:] - want)) <= 1e-13
+        assert np.array_equal(y[:, 0], v[:, 0]) or np.max(np.abs(y[:, 0] - v[:, 0])) <= 1e-15
+
+
+def pin_bonus_to_minus_infinity(L):
+    """u -> -inf removes the current token: with w = 1e4 the output is then v_{t-1} for
+    t >= 1; the first position keeps its limit y_0 = v_0."""
+    B, T, C = 1, 10, 3
+    r = _rng(15)
+    k = r.normal(0, 1, (B, T, C))
+    v = r.normal(0, 1, (B, T, C))
+    w = np.full(C, 1e4)
+    yr = oracle.wkv_recurrent(w, np.full(C, -1e4), k, v, L=L)[0]
+    assert np.array_equal(yr[:, 0], v[:, 0])
+    assert np.max(np.abs(yr[:, 1:] - v[:, :-1])) <= 1e-15
+    yd = oracle.wkv_direct(w, np.full(C, -600.0), k, v, L=L)[0]  # e^-600 is tiny but not 0
+    assert np.max(np.abs(yd[:, 1:] - v[:, :-1])) <= 1e-15
+    # with an ordinary decay, u = -1e4 gives the past-only average: check against
+    # the same case with the current token's key pushed to -inf by hand
+    w2 = np.exp(r.uniform(-3, 1, C))
+    y_cut = oracle.wkv_recurrent(w2, np.full(C, -1e4), k, v, L=L)[0]
+    for t in range(1, T):
+        kk = k.copy()
+        kk[:, t] = -1e4  # current key removed; past unchanged
+        y_ref = oracle.wkv_recurrent(w2, np.zeros(C), kk[:, : t + 1], v[:, : t + 1], L=L)[0]
+        assert np.max(np.abs(y_cut[:, t] - y_ref[:, t])) <= 1e-13
+
+
+def pin_key_shift_invariance(L):
+    """k -> k + c scales every weight by e^c: y is unchanged and the running maximum
+    shifts by exactly c (keys up to 40 plus a shift of 100: no inf/NaN)."""
+    w, u, k, v = _rand_case(16, B=2, T=60, C=5, k_std=3.0, w_lo=-5)
+    k = k.copy()
+    k[:, ::7, ::2] = 40.0
+    y0, _, st0, _ = oracle.wkv_recurrent(w, u, k, v, L=L)
+    y1, _, st1, _ = oracle.wkv_recurrent(w, u, k + 100.0, v, L=L)
+    assert np.all(np.isfinite(y1)) and np.all(np.isfinite(st1))
+    assert np.max(np.abs(y1 - y0)) <= 1e-12
+    assert np.max(np.abs(st1[2] - st0[2] - 100.0)) <= 1e-11
+    assert np.max(np.abs(st1[:2] - st0[:2]) / np.maximum(np.abs(st0[:2]), 1e-300)) <= 1e-11
+    yd0, _ = oracle.wkv_direct(w, u, k, v, L=L)
+    yd1, _ = oracle.wkv_direct(w, u, k + 100.0, v, L=L)
+    assert np.all(np.isfinite(yd1)) and np.max(np.abs(yd1 - yd0)) <= 1e-12
+
+
+def pin_value_affine(L):
+    """Weights sum to one after normalising: y(alpha v + beta) = alpha y(v) + beta."""
+    w, u, k, v = _rand_case(17, B=1, T=30, C=4)
+    y0 = oracle.wkv_recurrent(w, u, k, v, L=L)[0]
+    y1 = oracle.wkv_recurrent(w, u, k, -2.5 * v + 3.0, L=L)[0]
+    assert np.max(np.abs(y1 - (-2.5 * y0 + 3.0))) <= 1e-12
+    yd0 = oracle.wkv_direct(w, u, k, v, L=L)[0]
+    yd1 = oracle.wkv_direct(w, u, k, -2.5 * v + 3.0, L=L)[0]
+    assert np.max(np.abs(yd1 - (-2.5 * yd0 + 3.0))) <= 1e-12
+
+
+def pin_running_max_closed_form(L):
+    """The stored exponent after t tokens is max_{i<=t} (k_i - (t - i) w), and b >= 1
+    (the maximising token contributes e^0)."""
+    w, u, k, v = _rand_case(18, B=2, T=25, C=6, k_std=2.0)
+    for T in (1, 2, 7, 25):
+        _, _, st, _ = oracle.wkv_recurrent(w, u, k[:, :T], v[:, :T], L=L)
+        i = np.arange(T)[None, :, None]
+        want = np.max(k[:, :T] - (T - 1 - i) * w[None, None, :], axis=1)
+        assert np.max(np.abs(st[2] - want)) <= 1e-12
+        assert np.all(st[1] >= 1.0 - 1e-15)
+
+
+def pin_naive_accumulators(L):
+    """The stored state's true accumulators equal the plain two-accumulator sums
+    a_t = sum_i e^{-(t-i) w + k_i} v_i, b_t = sum_i e^{-(t-i) w + k_i}."""
+    w, u, k, v = _rand_case(19, B=1, T=15, C=4)
+    _, _, st, _ = oracle.wkv_recurrent(w, u, k, v, L=L)
+    A, Bs = _accum(st)
+    i = np.arange(15)[None, :, None]
+    wt = np.exp(-(14 - i) * w[None, None, :] + k)
+    assert np.max(np.abs(A - np.sum(wt * v, axis=1)) / np.sum(wt * np.abs(v), axis=1)) <= 1e-13
+    assert np.max(np.abs(Bs - np.sum(wt, axis=1)) / np.sum(wt, axis=1)) <= 1e-13
+
+
+def pin_prefill_then_decode(L):
+    """Prefill produces the state, decode steps continue from it: the sequence cut at any
+    point and resumed from the stored state gives the uncut result, bit for bit."""
+    w, u, k, v = _rand_case(20, B=2, T=21, C=3, k_std=3.0)
+    y, s, st, sa = oracle.wkv_recurrent(w, u, k, v, L=L)
+    for cut in (0, 1, 8, 20):
+        y1, _, st1, sa1 = oracle.wkv_recurrent(w, u, k[:, :cut], v[:, :cut], L=L)
+        y2, _, st2, sa2 = oracle.wkv_recurrent(w, u, k[:, cut:], v[:, cut:], state_in=st1, sacc_in=sa1, L=L)
+        assert np.array_equal(np.concatenate([y1, y2], axis=1), y)
+        assert np.array_equal(st2, st) and np.array_equal(sa2, sa)
+    # token by token, as a decode loop does
+    stt, sat = None, None
+    for t in range(21):
+        yt, _, stt, sat = oracle.wkv_recurrent(w, u, k[:, t:t + 1], v[:, t:t + 1], state_in=stt,
+                                               sacc_in=sat, L=L)
+        assert np.array_equal(yt[:, 0], y[:, t])
+    assert np.array_equal(stt, st)
+
+
+def pin_decode_layer_indexing(L):
+    """Decode rows are [N, L, C] with parameters [L, C]: row (n, l) uses layer l's w, u."""
+    N, Ly, C = 3, 4, 5
+    r = _rng(21)
+    w = np.exp(r.uniform(-3, 1, (Ly, C)))
+    u = r.normal(0, 0.5, (Ly, C))
+    k = r.normal(0, 1, (N, Ly, C))
+    v = r.normal(0, 1, (N, Ly, C))
+    st = np.stack([r.normal(0, 1, (N, Ly, C)), 1 + np.abs(r.normal(0, 1, (N, Ly, C))),
+                   r.normal(0, 1, (N, Ly, C))])
+    y, _, st2, _ = oracle.decode_step(w, u, k, v, st, L=L)
+    for l in range(Ly):
+        yl, _, stl, _ = oracle.wkv_recurrent(w[l], u[l], k[:, l:l + 1], v[:, l:l + 1], state_in=st[:, :, l],
+                                             L=L)
+        assert np.array_equal(yl[:, 0], y[:, l])
+        assert np.array_equal(stl, st2[:, :, l])
+
+
+def pin_negative_decay_convention(L):
+    """One page writes the step with a stored decay that is negative and added
+    (p + w_stored).  With w_stored = -w it is the same step; read as +w it no longer
+    reproduces the worked example's 3.8619."""
+    g = read_golden()
+
+    def step_added_decay(state, kk, vv, w_stored, uu):
+        a, b, p = state
+        m = max(p, uu + kk)
+        y = (a * math.exp(p - m) + math.exp(uu + kk - m) * vv) / (b * math.exp(p - m) + math.exp(uu + kk - m))
+        m2 = max(p + w_stored, kk)
+        a = a * math.exp(p + w_stored - m2) + vv * math.exp(kk - m2)
+        b = b * math.exp(p + w_stored - m2) + math.exp(kk - m2)
+        return y, (a, b, m2)
+
+    def run(w_stored):
+        st = (0.0, 0.0, oracle.P_EMPTY)
+        ys = []
+        for kk, vv in zip(g["k"], g["v"]):
+            y, st = step_added_decay(st, kk, vv, w_stored, g["u"])
+            ys.append(y)
+        return ys, st
+
+    w = np.array([g["w"]])
+    u = np.array([g["u"]])
+    k = np.array(g["k"]).reshape(1, 3, 1)
+    v = np.array(g["v"]).reshape(1, 3, 1)
+    yr, _, st, _ = oracle.wkv_recurrent(w, u, k, v, L=L)
+    ys, stp = run(-g["w"])
+    assert ys == list(yr[0, :, 0]) and stp == (st[0, 0, 0], st[1, 0, 0], st[2, 0, 0])
+    ys_wrong, _ = run(+g["w"])
+    assert abs(ys_wrong[2] - g["wkv_last"]) > 1e-2
+
+
+def pin_token_shift(L):
+    """xbar_t = mu x_t + (1 - mu) x_{t-1}: mu = 1 passes x_t, mu = 0 passes the previous token,
+    mu = 1/2 is the exact midpoint; the token before t = 0 is x_last, else zero."""
+    B, T, C = 2, 7, 5
+    r = _rng(22)
+    x = r.normal(0, 1, (B, T, C))
+    xl = r.normal(0, 1, (B, C))
+    prev = np.concatenate([xl[:, None], x[:, :-1]], axis=1)
+    prev0 = np.concatenate([np.zeros((B, 1, C)), x[:, :-1]], axis=1)
+    assert np.array_equal(oracle.token_shift(np.ones(C), x, xl, L=L), x)
+    assert np.array_equal(oracle.token_shift(np.zeros(C), x, xl, L=L), prev)
+    assert np.array_equal(oracle.token_shift(np.full(C, 0.5), x, xl, L=L), (x + prev) / 2)
+    assert np.array_equal(oracle.token_shift(np.full(C, 0.5), x, None, L=L), (x + prev0) / 2)
+    mu = r.uniform(0, 1, C)
+    xb = oracle.token_shift(mu, x, xl, L=L)
+    # per channel the result lies between the two taps
+    assert np.all(xb >= np.minimum(x, prev) - 1e-15) and np.all(xb <= np.maximum(x, prev) + 1e-15)
+    # decode form: one token from the previous one, [N, L, C] rows with [L, C] mu
+    mu2 = r.uniform(0, 1, (3, C))
+    xt = r.normal(0, 1, (B, 3, C))
+    xp = r.normal(0, 1, (B, 3, C))
+    xb2 = oracle.decode_token_shift(mu2, xt, xp, L=L)
+    for l in range(3):
+        want = oracle.token_shift(mu2[l], xt[:, l:l + 1], xp[:, l], L=L)[:, 0]
+        assert np.array_equal(xb2[:, l], want)
+    assert np.array_equal(oracle.decode_token_shift(np.ones((3, C)), xt, xp, L=L), xt)
+
+
+ALL_PINS = [
+    pin_worked_example,
+    pin_routes_agree,
+    pin_brute_force_high_precision,
+    pin_first_position_is_v,
+    pin_convex_bound,
+    pin_running_mean,
+    pin_two_tap_softmax,
+    pin_bonus_to_minus_infinity,
+    pin_key_shift_invariance,
+    pin_value_affine,
+    pin_running_max_closed_form,
+    pin_naive_accumulators,
+    pin_prefill_then_decode,
+    pin_decode_layer_indexing,
+    pin_negative_decay_convention,
+    pin_token_shift,
+]

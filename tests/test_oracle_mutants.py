@@ -1,0 +1,62 @@
+"""The pins are strong enough: every plausible slip planted in a copy of the oracle
+(a dropped term, a wrong sign or index, a transposed operand) fails at least one pin.
+
+Each mutant is the oracle's C source with one textual substitution, compiled with
+gcc into a temporary library; the oracle itself is never modified.
+"""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+import oracle
+from oracle_pins import ALL_PINS
+
+MUTANTS = {
+    "decay_exponent_off_by_one": ("exp(-(double)(t - 1 - i) * w[c]", "exp(-(double)(t - i) * w[c]"),
+    "direct_drops_bonus": ("double e = exp(u[c] + k[at3(b, t, c, T, C)]);",
+                           "double e = exp(k[at3(b, t, c, T, C)]);"),
+    "direct_includes_current_in_past": ("for (int64_t i = 0; i < t; ++i)", "for (int64_t i = 0; i <= t; ++i)"),
+    "direct_drops_current_value": ("num += e * v[at3(b, t, c, T, C)];", "num += e;"),
+    "output_max_ignores_bonus": ("double q = fmax(p, u[c] + kt);", "double q = fmax(p, kt);"),
+    "update_decay_sign": ("double p_new = fmax(p - w[c], kt);", "double p_new = fmax(p + w[c], kt);"),
+    "update_drops_decay": ("double keep = exp(p - w[c] - p_new);", "double keep = exp(p - p_new);"),
+    "update_drops_value": ("a = keep * a + add * vt;", "a = keep * a + add;"),
+    "denominator_gets_value": ("bb = keep * bb + add;", "bb = keep * bb + add * vt;"),
+    "output_transposed_operand": ("(w_past * a + w_now * vt) / den", "(w_past * bb + w_now * vt) / den"),
+    "output_bonus_on_past": ("double w_now = exp(u[c] + kt - q);", "double w_now = exp(kt - q);"),
+    "naive_decay_sign": ("double decay = exp(-w[c]);", "double decay = exp(w[c]);"),
+    "naive_update_before_output": ("a = decay * a + exp(kt) * vt;", "a = a + exp(kt) * vt;"),
+    "state_in_swaps_b_p": ("bb = state_in[BC + bc];", "bb = state_in[2 * BC + bc];"),
+    "state_out_drops_p": ("state_out[2 * BC + bc] = p;", "state_out[2 * BC + bc] = 0.0;"),
+    "lerp_weight_swapped": ("(1.0 - mu[c]) * prev", "mu[c] * prev"),
+    "lerp_previous_token_index": ("prev = x[at3(b, t - 1, c, T, C)];", "prev = x[at3(b, t, c, T, C)];"),
+    "layout_transposed": ("return ((size_t)b * (size_t)T + (size_t)t) * (size_t)C + (size_t)c;",
+                          "return ((size_t)b * (size_t)C + (size_t)c) * (size_t)T + (size_t)t;"),
+    "magnitude_scale_signed": ("sa = keep * sa + add * fabs(vt);", "sa = keep * sa + add * vt;"),
+}
+
+
+def _failing_pins(lib):
+    failed = []
+    for pin in ALL_PINS:
+        try:
+            pin(lib)
+        except AssertionError:
+            failed.append(pin.__name__)
+    return failed
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="gcc needed to build mutants")
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(oracle._SRC).read()
+    assert src.count(old) >= 1, f"mutation site for {name} not found"
+    mutant_src = tmp_path / "mutant.c"
+    mutant_src.write_text(src.replace(old, new))
+    so = tmp_path / "libmutant.so"
+    oracle.build(force=True, src=str(mutant_src), out=str(so))
+    lib = oracle.load(str(so))
+    assert _failing_pins(lib), f"mutant {name} passed every pin"
