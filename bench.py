@@ -1,0 +1,496 @@
+#!/usr/bin/env python
+"""Benchmark of the RWKV-4 WKV operator on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (one step = one pass of the whole hot path over one batch): prefill of
+B=8 sequences x T=1024 tokens x C=768 channels in fp32 (keys N(0,3) with 1% set to
++40, values N(0,1), w = exp(U(-5,1)), u ~ N(0,0.5)) through wkv_forward, which also
+returns the final state, then one fused decode step (token shift + WKV update) that
+continues all 8 sequences from that state.  Metric: WKV forward B*T*C elements/s.
+The same JSON line also carries the decode throughput of 256 sessions x 32 layers x
+4096 channels (tokens/s, a token being one session's step through all 32 layers).
+
+Timing: W untimed warm-up steps, then exactly K steps replayed from CUDA graphs,
+bracketed by a barrier and a device synchronise, timed with CUDA events; the max over
+ranks is taken.  Six input sets (453 MB, over three times the 126 MB L2) rotate
+between steps so no step finds its inputs in L2.  The forward kernel's own launch
+time comes from CUDA events recorded around each forward launch inside the graph.
+
+--impl reference times the fp64 CPU oracle (plain C, OpenMP) on this workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "fwd_8x1024x768"
+METRIC = "WKV forward B*T*C elements/s"
+N_SETS = 6
+GRAPH_STEPS = 60
+ALG_BYTES_PER_ELEM = {"f32": 12, "bf16": 6}     # k + v read, y written, per element
+DECODE_ALG_BYTES_PER_ELEM = 48                    # x_t, x_prev, k, v, a, b, p in; a, b, p, y, xbar out
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=6000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------
+# clocks
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms in the background."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0, t1):
+        rows = [s for (t, s) in self.samples if t0 <= t <= t1]
+        window = "timed"
+        if len(rows) < 3:
+            rows = [s for (t, s) in self.samples if t0 - 1.5 <= t <= t1 + 0.2]
+            window = "timed+preroll"
+        if not rows:
+            return None
+        mhz, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            p = [x.strip() for x in r.split(",")]
+            try:
+                mhz.append(float(p[1]))
+                mx.append(float(p[2]))
+            except (ValueError, IndexError):
+                continue
+            for name, val in zip(names, p[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(mhz), "window": window}
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+def kernel_source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_attention_rnn_wkv_b200", "csrc")
+    for name in ("wkv_device.cuh", "wkv_forward_chunked.cu"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch of the forward kernel from the committed ncu summary, if it
+    was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"wkv_fwd_chunked_{workload}.md")
+    try:
+        txt = open(path).read()
+    except OSError:
+        return None
+    m_src = re.search(r"kernel_source_digest:\s*([0-9a-f]+)", txt)
+    m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not m_src or not m_tr or m_src.group(1) != kernel_source_digest():
+        return None
+    return float(m_tr.group(1))
+
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline leg and --impl reference)
+# ----------------------------------------------------------------------------
+
+def time_oracle(spec, inputs, min_seconds, min_passes):
+    import oracle
+    w, u, k, v = inputs
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        oracle.wkv_recurrent(w, u, k, v)
+        passes += 1
+        el = time.perf_counter() - t0
+        if passes >= min_passes and el >= min_seconds:
+            break
+    n = spec.B * spec.T * spec.C
+    return n * passes / el, passes, el, oracle.num_threads()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import synth
+    spec = synth.FORWARD[WORKLOAD]
+    inputs = synth.forward_inputs(spec)
+    import oracle
+    for _ in range(max(args.warmup, 0)):
+        oracle.wkv_recurrent(*inputs)
+    n = spec.B * spec.T * spec.C
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.wkv_recurrent(*inputs)
+    el = time.perf_counter() - t0
+    value = n * args.steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": spec.B, "T": spec.T, "C": spec.C, "io": "f32"},
+        "cpu_baseline": {"value": value, "unit": "elements/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"each step: the whole {spec.B}x{spec.T}x{spec.C} prefill through the fp64 "
+                                   f"stabilised recurrence (no decode step)"},
+        "e2e": {"value": value, "unit": "elements/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+
+class ForwardSet:
+    """One rotating input set: the prefill batch plus the decode token that follows it."""
+
+    def __init__(self, spec, seed, dev):
+        import numpy as np
+        import torch
+        import synth
+        s = synth.ForwardSpec(spec.name, spec.B, spec.T, spec.C, spec.dtype, spec.k_std, spec.w_lo, spec.w_hi,
+                              spec.spike_prob, spec.spike_value, seed)
+        w, u, k, v = synth.forward_inputs(s)
+        self.host = (k, v)
+        self.w = torch.from_numpy(w).to(dev)
+        self.u = torch.from_numpy(u).to(dev)
+        self.k = torch.from_numpy(k).to(dev)
+        self.v = torch.from_numpy(v).to(dev)
+        self.y = torch.empty_like(self.k)
+        self.state = torch.empty((3, spec.B, spec.C), dtype=torch.float32, device=dev)
+        B, C = spec.B, spec.C
+        r = np.random.default_rng(seed)
+        self.mu = torch.from_numpy(r.uniform(0, 1, (1, C)).astype(np.float32)).to(dev)
+        self.w1 = self.w.reshape(1, C)
+        self.u1 = self.u.reshape(1, C)
+        self.x_t = torch.from_numpy(r.normal(0, 1, (B, 1, C)).astype(np.float32)).to(dev)
+        self.x_prev = torch.from_numpy(r.normal(0, 1, (B, 1, C)).astype(np.float32)).to(dev)
+        self.k1 = torch.from_numpy(r.normal(0, 1, (B, 1, C)).astype(np.float32)).to(dev)
+        self.v1 = torch.from_numpy(r.normal(0, 1, (B, 1, C)).astype(np.float32)).to(dev)
+        self.xbar1 = torch.empty_like(self.x_t)
+        self.y1 = torch.empty_like(self.x_t)
+        self.state4 = self.state.view(3, B, 1, C)
+
+
+def step(wkv, s, ws, ev=None):
+    """One pass of the hot path: prefill forward (with state_out) then the fused decode step."""
+    if ev is not None:
+        ev[0].record()
+    wkv.wkv_forward(s.w, s.u, s.k, s.v, workspace=ws, y=s.y, state_out=s.state)
+    if ev is not None:
+        ev[1].record()
+    wkv.wkv_decode_step_fused(s.mu, s.w1, s.u1, s.x_t, s.x_prev, s.k1, s.v1, s.state4, xbar=s.xbar1, y=s.y1)
+
+
+def capture(torch, wkv, sets, ws, nsteps, with_events):
+    g = torch.cuda.CUDAGraph()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nsteps)] \
+        if with_events else [None] * nsteps
+    with torch.cuda.graph(g):
+        for i in range(nsteps):
+            step(wkv, sets[i % len(sets)], ws, evs[i])
+    return g, evs
+
+
+def decode_bench(torch, wkv, dev, steps):
+    """256 sessions x 32 layers x 4096 channels, fused decode, 4 input sets in rotation."""
+    import numpy as np
+    N, L, C = 256, 32, 4096
+    g = torch.Generator(device=dev)
+    g.manual_seed(1005)
+    mu = torch.rand((L, C), generator=g, device=dev)
+    w = torch.exp(torch.rand((L, C), generator=g, device=dev) * 6 - 5)
+    u = torch.randn((L, C), generator=g, device=dev) * 0.5
+    st = torch.empty((3, N, L, C), device=dev)
+    st[2].normal_(1.0, 1.0, generator=g)
+    st[1].normal_(0.0, 1.0, generator=g).abs_().add_(1.0)
+    st[0].normal_(0.0, 1.0, generator=g).mul_(st[1])
+    sets = [tuple(torch.randn((N, L, C), generator=g, device=dev) for _ in range(3)) for _ in range(4)]
+    xbar = torch.empty((N, L, C), device=dev)
+    y = torch.empty((N, L, C), device=dev)
+
+    def one(i):
+        x_t, k, v = sets[i % 4]
+        x_prev = sets[(i - 1) % 4][0]
+        wkv.wkv_decode_step_fused(mu, w, u, x_t, x_prev, k, v, st, xbar=xbar, y=y)
+
+    for i in range(4):
+        one(i)
+    nper = 8
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        for i in range(nper):
+            one(i)
+    gr.replay()
+    torch.cuda.synchronize()
+    reps = max(1, steps // nper)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        gr.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (reps * nper)
+    del gr
+    return {"workload": f"decode_{N}x{L}x{C}", "metric": "decode tokens/s (session steps through all 32 layers)",
+            "value": N / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": reps * nper,
+            "hbm_gbs": DECODE_ALG_BYTES_PER_ELEM * N * L * C / (ms * 1e-3) / 1e9}
+
+
+def e2e_bench(torch, wkv, sets, ws, steps, dev):
+    """Through the public API with host buffers: per step, copy k and v from pinned host
+    memory, run the step, read y back to pinned host memory.  Copies ride a second
+    stream so the next step's upload overlaps this step's kernels and download."""
+    pinned_in = [(torch.from_numpy(s.host[0]).pin_memory(), torch.from_numpy(s.host[1]).pin_memory()) for s in sets]
+    pinned_out = [torch.empty(s.y.shape, dtype=s.y.dtype).pin_memory() for s in sets]
+    h2d = sum(a.numel() * a.element_size() for a in pinned_in[0])
+    d2h = pinned_out[0].numel() * pinned_out[0].element_size()
+    comp = torch.cuda.current_stream()
+    copy = torch.cuda.Stream()
+    uploaded = [torch.cuda.Event() for _ in sets]
+    consumed = [torch.cuda.Event() for _ in sets]
+    for e in consumed:
+        e.record(comp)
+
+    def run(n):
+        for i in range(n):
+            j = i % len(sets)
+            s = sets[j]
+            with torch.cuda.stream(copy):
+                copy.wait_event(consumed[j])
+                s.k.copy_(pinned_in[j][0], non_blocking=True)
+                s.v.copy_(pinned_in[j][1], non_blocking=True)
+                uploaded[j].record(copy)
+            comp.wait_event(uploaded[j])
+            step(wkv, s, ws)
+            pinned_out[j].copy_(s.y, non_blocking=True)
+            consumed[j].record(comp)
+
+    run(len(sets))
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    run(steps)
+    e1.record(comp)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return ms, h2d, d2h
+
+
+def run_ours(args):
+    import torch
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    import linear_attention_rnn_wkv_b200 as wkv
+    import synth
+
+    spec = synth.FORWARD[WORKLOAD]
+    n_elem = spec.B * spec.T * spec.C
+    sets = [ForwardSet(spec, spec.seed + 100 * rank + i, dev) for i in range(N_SETS)]
+    ws = wkv.Workspace(dev, wkv.workspace_size(spec.B, spec.T, spec.C))
+    path = wkv.auto_path(spec.B, spec.T, spec.C)
+
+    # eager warm-up (sets kernel attributes, first-touch), then W untimed graph steps
+    for s in sets:
+        step(wkv, s, ws)
+    torch.cuda.synchronize()
+    wkv.forward_status(ws.buf)
+
+    K = args.steps
+    per = min(GRAPH_STEPS, K)
+    main_g, main_ev = capture(torch, wkv, sets, ws, per, with_events=True)
+    rem = K % per
+    rem_g = capture(torch, wkv, sets, ws, rem, with_events=False)[0] if rem else None
+    reps = K // per
+    warm_g, _ = capture(torch, wkv, sets, ws, min(max(args.warmup, 1), GRAPH_STEPS), with_events=False)
+    for _ in range(max(1, (args.warmup + GRAPH_STEPS - 1) // GRAPH_STEPS)):
+        warm_g.replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    if rank == 0:
+        clocks.start()
+    # pre-roll the same graph for ~1 s so the clock record covers sustained load
+    t_pre = time.time()
+    while time.time() - t_pre < 1.0:
+        main_g.replay()
+        torch.cuda.synchronize()
+
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    e0.record()
+    for _ in range(reps):
+        main_g.replay()
+    if rem_g is not None:
+        rem_g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(world)
+    clocks.stop()
+    wkv.forward_status(ws.buf)
+
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world)
+    ms_per_step = ms_total / K
+    value = world * n_elem / (ms_per_step * 1e-3)
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in main_ev)
+    fwd_ms = max_over_ranks(fwd_ms, world)
+
+    peaks, peak_kind = measured_peaks()
+    alg = ALG_BYTES_PER_ELEM[spec.dtype] * n_elem
+    achieved = alg / (fwd_ms * 1e-3) / 1e9
+    traffic = profiled_traffic(WORKLOAD)
+
+    del main_g, rem_g, warm_g
+    dec = None if args.no_decode else decode_bench(torch, wkv, dev, 400)
+    e2e = None
+    if not args.no_e2e:
+        ms_e2e, h2d, d2h = e2e_bench(torch, wkv, sets, ws, min(K, 240), dev)
+        ms_e2e = max_over_ranks(ms_e2e, world)
+        e2e = {"value": world * n_elem / (ms_e2e * 1e-3), "unit": "elements/s", "ms_per_step": ms_e2e,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        rate, passes, el, cores = time_oracle(spec, synth.forward_inputs(spec), 5.0, 3)
+        cpu = {"value": rate, "unit": "elements/s", "cores": cores, "kind": "oracle",
+               "sample": f"{passes} passes of the whole {spec.B}x{spec.T}x{spec.C} prefill through the fp64 "
+                         f"stabilised recurrence ({el:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": spec.B, "T": spec.T, "C": spec.C, "io": spec.dtype,
+                       "step": "prefill forward (with final state) + one fused decode step of the same batch",
+                       "forward_path": path, "l2": f"{N_SETS} rotating input sets "
+                                                    f"({N_SETS * 3 * n_elem * 4 / 1e6:.0f} MB > 3x L2)",
+                       "graph": f"CUDA graphs of {per} steps"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                         "kernel": f"wkv_forward ({path})", "launch_ms": fwd_ms,
+                         "alg_bytes_per_launch": alg, "peak_kind": f"{peak_kind} hbm_gbs"},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 2 * K,
+            "decode": dec,
+            "clocks": clocks.summary(t_wall0, t_wall1) if rank == 0 else None,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+/*
+ * wkv.h -- C ABI of the B200 (sm_100a) RWKV-4 WKV library (libwkv_b200.so).
+ *
+ * The operator ("RWKV" transformer-math page, aicassindra.com, section "The WKV
+ * operator: attention with a fixed decay"; aiwiki "RWKV", eq. 1), per channel c,
+ * 0-based position t:
+ *
+ *   wkv_t = ( sum_{i<t} e^{-(t-1-i) w + k_i} v_i + e^{u + k_t} v_t )
+ *         / ( sum_{i<t} e^{-(t-1-i) w + k_i}     + e^{u + k_t} )
+ *
+ * w >= 0 is the per-channel decay rate (the decay per step is e^{-w}; the pages
+ * take w = exp(omega) > 0), u the per-channel bonus of the current token.
+ *
+ * The state of one channel is the triple (a, b, p) with true accumulators
+ *   A = a e^p = sum_i e^{-(t-i) w + k_i} v_i,   B = b e^p = sum_i e^{-(t-i) w + k_i}
+ * over the tokens i <= t consumed so far (same page, section "Numerical stability:
+ * carry the exponent").  p is a free exponent offset: (a e^d, b e^d, p - d) is the
+ * same state.  The empty state is a = b = 0, p = -1e38.  A state buffer holds three
+ * planes: [3][rows][C] = (a plane, b plane, p plane), fp32.
+ *
+ * Conventions for every call below
+ *  - Pointers are DEVICE pointers owned by the caller (e.g. torch tensors).  The
+ *    library allocates nothing and keeps no per-call state.
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream): they validate
+ *    their arguments on the host, enqueue the kernel(s) and return.
+ *  - Argument errors are reported synchronously by the return value and nothing is
+ *    enqueued: sizes < 0 or whose products overflow int64 -> WKV_ERR_INVALID_ARG;
+ *    a required pointer that is NULL -> WKV_ERR_INVALID_ARG; a device pointer not
+ *    16-byte aligned -> WKV_ERR_MISALIGNED; an unknown dtype/path ->
+ *    WKV_ERR_UNSUPPORTED.  A launch failure returns WKV_ERR_CUDA
+ *    (wkv_last_cuda_error() gives the cudaError_t).  Faults inside a kernel show
+ *    up, as for any CUDA kernel, at the caller's next synchronisation.
+ *  - A size of 0 in any dimension is a valid empty call (nothing is written,
+ *    except that wkv_forward with T = 0 still writes state_out).
+ *  - Tensors are dense row-major with the innermost (channel) dimension
+ *    contiguous.  Any C is accepted; C a multiple of 4 (fp32) or 8 (bf16) takes the
+ *    vectorised bulk-copy path.
+ *  - There is no CPU fallback: every entry point runs CUDA kernels for sm_100a.
+ */
+#ifndef WKV_B200_H
+#define WKV_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum wkv_status {
+    WKV_OK = 0,
+    WKV_ERR_INVALID_ARG = 1,  /* bad size, NULL pointer, workspace too small */
+    WKV_ERR_MISALIGNED = 2,   /* a device pointer is not 16-byte aligned */
+    WKV_ERR_UNSUPPORTED = 3,  /* unknown dtype, path or chunk length */
+    WKV_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+    WKV_ERR_TIMEOUT = 5       /* a device-side wait gave up (see wkv_forward_status) */
+} wkv_status;
+
+typedef enum wkv_dtype {
+    WKV_F32 = 0,   /* k, v, y in fp32 */
+    WKV_BF16 = 1   /* k, v, y in bf16 (y rounded to nearest even); state and w, u stay fp32 */
+} wkv_dtype;
+
+typedef enum wkv_path {
+    WKV_PATH_AUTO = 0,     /* pick from the measured table for (B*C, T, dtype) */
+    WKV_PATH_SERIAL = 1,   /* one thread per (b, c) scanning all of T */
+    WKV_PATH_CHUNKED = 2   /* time-parallel: chunk summaries, carry scan, fix-up */
+} wkv_path;
+
+/*
+ * Forward (prefill) over [B, T, C].
+ *
+ * Computes wkv_t for every (b, t, c) (the equation above) and, if state_out is not
+ * NULL, the state after the last token, which wkv_decode_step continues exactly
+ * ("RWKV and Recurrent Models With Transformer Quality", multigrid.ai, section
+ * "Prefill, decode, and where each form is used": prefill produces the state after
+ * the last prompt token; decode steps from it).
+ *
+ *   w, u       [C] fp32 (w >= 0)
+ *   k, v       [B, T, C] in dtype io
+ *   y          [B, T, C] in dtype io (written)
+ *   state_out  [3][B][C] fp32 (a, b, p) or NULL
+ *   workspace  caller-owned device scratch of ws_bytes >= wkv_forward_workspace_size();
+ *              it must be zero-filled once before its first use (wkv_workspace_init)
+ *              and must not be used by two calls that can overlap on the GPU.
+ *              It may be NULL when the size query returns 0.
+ * Returns WKV_ERR_INVALID_ARG when ws_bytes is too small for the chosen path.
+ */
+wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, wkv_dtype io, const float* w, const float* u,
+                       const void* k, const void* v, void* y, float* state_out, void* workspace,
+                       size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * As wkv_forward, plus:
+ *   state_in  [3][B][C] fp32 (a, b, p) to continue from, or NULL for the empty state
+ *             (resumable / piecewise prefill; state_out may alias state_in);
+ *   path      WKV_PATH_AUTO, WKV_PATH_SERIAL or WKV_PATH_CHUNKED;
+ *   chunk     time steps per chunk for the chunked path (0 = default; else 4, 8 or 16
+ *             steps per warp).
+ */
+wkv_status wkv_forward_ex(int64_t B, int64_t T, int64_t C, wkv_dtype io, const float* w, const float* u,
+                          const void* k, const void* v, const float* state_in, void* y, float* state_out,
+                          void* workspace, size_t ws_bytes, wkv_path path, int chunk, cudaStream_t stream);
+
+/* Workspace bytes wkv_forward needs for this shape (the largest over all paths). */
+size_t wkv_forward_workspace_size(int64_t B, int64_t T, int64_t C, wkv_dtype io);
+
+/* Zero-fill a workspace (once, before its first use). */
+wkv_status wkv_workspace_init(void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Synchronises `stream`, then reports and clears the device-side error word of a
+ * workspace: WKV_ERR_TIMEOUT if a chunked forward launched with it gave up waiting
+ * for a predecessor's carry (its outputs are then invalid), else WKV_OK.
+ */
+wkv_status wkv_forward_status(void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * One decode step for N sessions x L layers x C channels: for every row (n, l) and
+ * channel c, emit wkv for the token (k, v) from the stored state and fold the token
+ * into the state (aiwiki "RWKV": the one-token decode step; transformer-math page,
+ * section "Numerical stability: carry the exponent").
+ *   w, u         [L][C] fp32 (layer l's parameters)
+ *   k, v, y      [N][L][C] fp32
+ *   state_inout  [3][N][L][C] fp32 (a, b, p), updated in place
+ * With L = 1 and N = B, state_out of wkv_forward continues the same sequences.
+ */
+wkv_status wkv_decode_step(int64_t N, int64_t L, int64_t C, const float* w, const float* u, const float* k,
+                           const float* v, float* state_inout, float* y, cudaStream_t stream);
+
+/*
+ * Token shift (transformer-math page, section "Token shift: a two-tap causal
+ * convolution"): xbar_t = mu * x_t + (1 - mu) * x_{t-1}, per channel.
+ *   mu      [C] fp32
+ *   x, xbar [B, T, C] fp32 (xbar must not alias x)
+ *   x_last  [B][C] fp32, the token before t = 0, or NULL for zeros (causal padding)
+ */
+wkv_status token_shift_mix(int64_t B, int64_t T, int64_t C, const float* mu, const float* x, const float* x_last,
+                           float* xbar, cudaStream_t stream);
+
+/*
+ * Fused decode step: the token-shift lerp and the WKV decode step in one kernel.
+ *   mu, w, u      [L][C] fp32
+ *   x_t, x_prev   [N][L][C] fp32: this token's input and the previous token's
+ *   xbar          [N][L][C] fp32: mu * x_t + (1 - mu) * x_prev (written)
+ *   k, v, y       [N][L][C] fp32: the token's key and value; y = its wkv (written)
+ *   state_inout   [3][N][L][C] fp32, updated in place
+ * The caller makes x_t the next call's x_prev (pointer swap, no copy).
+ */
+wkv_status wkv_decode_step_fused(int64_t N, int64_t L, int64_t C, const float* mu, const float* w,
+                                 const float* u, const float* x_t, const float* x_prev, float* xbar,
+                                 const float* k, const float* v, float* state_inout, float* y,
+                                 cudaStream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char* wkv_status_string(wkv_status status);
+
+/* The cudaError_t of the last WKV_ERR_CUDA returned on this host thread (0 if none). */
+int wkv_last_cuda_error(void);
+
+/* The path WKV_PATH_AUTO picks for this shape (WKV_PATH_SERIAL or WKV_PATH_CHUNKED). */
+wkv_path wkv_forward_auto_path(int64_t B, int64_t T, int64_t C, wkv_dtype io);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int wkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WKV_B200_H */

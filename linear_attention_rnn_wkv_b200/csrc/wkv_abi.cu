@@ -1,0 +1,248 @@
+// C ABI of the WKV library: argument validation, path choice, launches.
+// Declarations and the contract of every entry point are in include/wkv.h.
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include "wkv.h"
+#include "wkv_device.cuh"
+#include "wkv_internal.h"
+
+namespace {
+
+using namespace wkvb;
+
+thread_local int g_last_cuda_error = 0;
+
+// Library-owned status block for launches that run without a workspace (the
+// serial path): word 0 is the device error code, word 1 the failing unit.
+__device__ uint32_t g_status_block[4];
+
+wkv_status cuda_fail(cudaError_t e) {
+    g_last_cuda_error = (int)e;
+    return WKV_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool mul_ok(int64_t a, int64_t b, int64_t* out) {
+    if (a < 0 || b < 0) return false;
+    if (a != 0 && b > INT64_MAX / a) return false;
+    *out = a * b;
+    return true;
+}
+
+bool sizes_ok(int64_t A, int64_t B, int64_t C, int64_t* total) {
+    int64_t ab;
+    return mul_ok(A, B, &ab) && mul_ok(ab, C, total);
+}
+
+uint32_t* status_word() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    static uint32_t* cache[64] = {nullptr};
+    if (dev < 0 || dev >= 64) return nullptr;
+    if (!cache[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_block) != cudaSuccess) return nullptr;
+        cache[dev] = static_cast<uint32_t*>(p);
+    }
+    return cache[dev];
+}
+
+// Default path table: the chunked scan exposes T-parallelism and wins unless there
+// are enough independent channels to fill every SM with serial scans.
+wkv_path auto_path(int64_t B, int64_t T, int64_t C, wkv_dtype io) {
+    (void)io;
+    const int64_t BC = B * C;
+    if (T <= 64 && BC >= 148 * 1024) return WKV_PATH_SERIAL;
+    return WKV_PATH_CHUNKED;
+}
+
+wkv_status forward_impl(int64_t B, int64_t T, int64_t C, wkv_dtype io, const float* w, const float* u,
+                        const void* k, const void* v, const float* state_in, void* y, float* state_out,
+                        void* workspace, size_t ws_bytes, wkv_path path, int chunk, uint32_t spin_limit,
+                        int64_t drop_unit, cudaStream_t stream) {
+    int64_t n = 0, BC = 0;
+    if (!sizes_ok(B, T, C, &n) || !mul_ok(B, C, &BC) || BC > INT64_MAX / 3) return WKV_ERR_INVALID_ARG;
+    if (io != WKV_F32 && io != WKV_BF16) return WKV_ERR_UNSUPPORTED;
+    if (path != WKV_PATH_AUTO && path != WKV_PATH_SERIAL && path != WKV_PATH_CHUNKED) return WKV_ERR_UNSUPPORTED;
+    if (chunk != 0 && chunk != 4 && chunk != 8 && chunk != 16) return WKV_ERR_UNSUPPORTED;
+    if (BC == 0) return WKV_OK;
+    if (!w || !u) return WKV_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(u) || !aligned16(state_in) || !aligned16(state_out) || !aligned16(workspace))
+        return WKV_ERR_MISALIGNED;
+    if (T == 0) {
+        if (!state_out) return WKV_OK;
+        cudaError_t e = launch_state_passthrough(BC, state_in, state_out, stream);
+        return e == cudaSuccess ? WKV_OK : cuda_fail(e);
+    }
+    if (!k || !v || !y) return WKV_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(y)) return WKV_ERR_MISALIGNED;
+
+    ForwardArgs a;
+    a.B = B;
+    a.T = T;
+    a.C = C;
+    a.io = (int)io;
+    a.w = w;
+    a.u = u;
+    a.k = k;
+    a.v = v;
+    a.state_in = state_in;
+    a.y = y;
+    a.state_out = state_out;
+    a.spin_limit = spin_limit;
+
+    if (path == WKV_PATH_AUTO) path = auto_path(B, T, C, io);
+    if (path == WKV_PATH_SERIAL) {
+        a.err = workspace && ws_bytes >= kWsHeaderBytes ? &static_cast<WsHeader*>(workspace)->error : status_word();
+        if (!a.err) return cuda_fail(cudaGetLastError());
+        const int64_t grid = B * ((C + 127) / 128);
+        if (grid > INT32_MAX) return WKV_ERR_UNSUPPORTED;
+        cudaError_t e = launch_forward_serial(a, stream);
+        return e == cudaSuccess ? WKV_OK : cuda_fail(e);
+    }
+    ChunkGeom g;
+    if (!chunk_geometry(B, T, C, (int)io, chunk, &g)) return WKV_ERR_UNSUPPORTED;
+    if (g.U > INT32_MAX) return WKV_ERR_UNSUPPORTED;
+    if (!workspace || ws_bytes < g.ws_bytes) return WKV_ERR_INVALID_ARG;
+    a.err = &static_cast<WsHeader*>(workspace)->error;
+    cudaError_t e = launch_forward_chunked(a, g, workspace, drop_unit, stream);
+    return e == cudaSuccess ? WKV_OK : cuda_fail(e);
+}
+
+bool f32_args_ok(std::initializer_list<const void*> ps) {
+    for (const void* p : ps)
+        if (!aligned16(p)) return false;
+    return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t wkv_forward_workspace_size(int64_t B, int64_t T, int64_t C, wkv_dtype io) {
+    int64_t n = 0;
+    if (!sizes_ok(B, T, C, &n) || n == 0) return kWsHeaderBytes;
+    size_t best = kWsHeaderBytes;
+    for (int chunk : {4, 8, 16}) {
+        ChunkGeom g;
+        if (chunk_geometry(B, T, C, (int)io, chunk, &g) && g.ws_bytes > best) best = g.ws_bytes;
+    }
+    return best;
+}
+
+wkv_status wkv_workspace_init(void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (!workspace) return ws_bytes == 0 ? WKV_OK : WKV_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return WKV_ERR_MISALIGNED;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, ws_bytes, stream);
+    return e == cudaSuccess ? WKV_OK : cuda_fail(e);
+}
+
+wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, wkv_dtype io, const float* w, const float* u, const void* k,
+                       const void* v, void* y, float* state_out, void* workspace, size_t ws_bytes,
+                       cudaStream_t stream) {
+    return forward_impl(B, T, C, io, w, u, k, v, nullptr, y, state_out, workspace, ws_bytes, WKV_PATH_AUTO, 0,
+                        kSpinLimitDefault, -1, stream);
+}
+
+wkv_status wkv_forward_ex(int64_t B, int64_t T, int64_t C, wkv_dtype io, const float* w, const float* u,
+                          const void* k, const void* v, const float* state_in, void* y, float* state_out,
+                          void* workspace, size_t ws_bytes, wkv_path path, int chunk, cudaStream_t stream) {
+    return forward_impl(B, T, C, io, w, u, k, v, state_in, y, state_out, workspace, ws_bytes, path, chunk,
+                        kSpinLimitDefault, -1, stream);
+}
+
+wkv_status wkv_forward_status(void* workspace, size_t ws_bytes, cudaStream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    uint32_t* word = nullptr;
+    if (workspace) {
+        if (ws_bytes < kWsHeaderBytes) return WKV_ERR_INVALID_ARG;
+        word = &static_cast<WsHeader*>(workspace)->error;
+    } else {
+        word = status_word();
+        if (!word) return cuda_fail(cudaGetLastError());
+    }
+    uint32_t code = 0;
+    e = cudaMemcpy(&code, word, sizeof(code), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (code == kDevOk) return WKV_OK;
+    // clear the error; a workspace is zero-filled whole (counters, epoch and flags restart
+    // together, so no flag of an earlier launch can match a later epoch)
+    if (workspace) {
+        e = cudaMemset(workspace, 0, ws_bytes);
+    } else {
+        const uint32_t zero[2] = {0, 0};
+        e = cudaMemcpy(word, zero, sizeof(zero), cudaMemcpyHostToDevice);
+    }
+    if (e != cudaSuccess) return cuda_fail(e);
+    return WKV_ERR_TIMEOUT;
+}
+
+wkv_status wkv_decode_step(int64_t N, int64_t L, int64_t C, const float* w, const float* u, const float* k,
+                           const float* v, float* state_inout, float* y, cudaStream_t stream) {
+    int64_t n = 0;
+    if (!sizes_ok(N, L, C, &n) || n > INT64_MAX / 3) return WKV_ERR_INVALID_ARG;
+    if (n == 0) return WKV_OK;
+    if (!w || !u || !k || !v || !state_inout || !y) return WKV_ERR_INVALID_ARG;
+    if (!f32_args_ok({w, u, k, v, state_inout, y})) return WKV_ERR_MISALIGNED;
+    cudaError_t e = launch_decode_step(N, L, C, nullptr, w, u, nullptr, nullptr, nullptr, k, v, state_inout, y,
+                                       stream);
+    return e == cudaSuccess ? WKV_OK : cuda_fail(e);
+}
+
+wkv_status wkv_decode_step_fused(int64_t N, int64_t L, int64_t C, const float* mu, const float* w, const float* u,
+                                 const float* x_t, const float* x_prev, float* xbar, const float* k, const float* v,
+                                 float* state_inout, float* y, cudaStream_t stream) {
+    int64_t n = 0;
+    if (!sizes_ok(N, L, C, &n) || n > INT64_MAX / 3) return WKV_ERR_INVALID_ARG;
+    if (n == 0) return WKV_OK;
+    if (!mu || !w || !u || !x_t || !x_prev || !xbar || !k || !v || !state_inout || !y) return WKV_ERR_INVALID_ARG;
+    if (!f32_args_ok({mu, w, u, x_t, x_prev, xbar, k, v, state_inout, y})) return WKV_ERR_MISALIGNED;
+    cudaError_t e = launch_decode_step(N, L, C, mu, w, u, x_t, x_prev, xbar, k, v, state_inout, y, stream);
+    return e == cudaSuccess ? WKV_OK : cuda_fail(e);
+}
+
+wkv_status token_shift_mix(int64_t B, int64_t T, int64_t C, const float* mu, const float* x, const float* x_last,
+                           float* xbar, cudaStream_t stream) {
+    int64_t n = 0;
+    if (!sizes_ok(B, T, C, &n)) return WKV_ERR_INVALID_ARG;
+    if (n == 0) return WKV_OK;
+    if (!mu || !x || !xbar) return WKV_ERR_INVALID_ARG;
+    if (!f32_args_ok({mu, x, x_last, xbar})) return WKV_ERR_MISALIGNED;
+    cudaError_t e = launch_token_shift(B, T, C, mu, x, x_last, xbar, stream);
+    return e == cudaSuccess ? WKV_OK : cuda_fail(e);
+}
+
+const char* wkv_status_string(wkv_status status) {
+    switch (status) {
+        case WKV_OK: return "WKV_OK";
+        case WKV_ERR_INVALID_ARG: return "WKV_ERR_INVALID_ARG";
+        case WKV_ERR_MISALIGNED: return "WKV_ERR_MISALIGNED";
+        case WKV_ERR_UNSUPPORTED: return "WKV_ERR_UNSUPPORTED";
+        case WKV_ERR_CUDA: return "WKV_ERR_CUDA";
+        case WKV_ERR_TIMEOUT: return "WKV_ERR_TIMEOUT";
+    }
+    return "WKV_ERR_UNKNOWN";
+}
+
+int wkv_last_cuda_error(void) { return g_last_cuda_error; }
+
+wkv_path wkv_forward_auto_path(int64_t B, int64_t T, int64_t C, wkv_dtype io) { return auto_path(B, T, C, io); }
+
+int wkv_version(void) { return 100; }
+
+// Test hook (not in wkv.h): a chunked forward in which `drop_unit` never publishes its
+// carry and every bounded wait gives up after `spin_limit` polls.  The successor of the
+// dropped unit then runs out its wait, records WKV_ERR_TIMEOUT in the workspace, and the
+// launch still completes.  Used to check that the error path returns control.
+wkv_status wkv_testhook_forward_drop(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
+                                     const float* v, float* y, void* workspace, size_t ws_bytes,
+                                     int64_t drop_unit, uint32_t spin_limit, cudaStream_t stream) {
+    return forward_impl(B, T, C, WKV_F32, w, u, k, v, nullptr, y, nullptr, workspace, ws_bytes, WKV_PATH_CHUNKED,
+                        0, spin_limit, drop_unit, stream);
+}
+
+}  // extern "C"

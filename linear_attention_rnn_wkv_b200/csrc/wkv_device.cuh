@@ -1,0 +1,241 @@
+// Device-side numerics shared by the WKV kernels (sm_100a).
+//
+// Notation follows the RWKV transformer-math page (aicassindra.com, tm_rwkv_math),
+// section "Numerical stability: carry the exponent": a channel's state is (a, b, p)
+// with true accumulators A = a e^p, B = b e^p, and every exponent handed to exp is
+// <= 0 (up to rounding).
+//
+// Two exponent domains are used:
+//  * natural (the ABI's): exp(x) is evaluated as 2^(x * log2 e);
+//  * base 2 (inside the forward kernels): k, w, u and p are pre-multiplied by
+//    log2 e once, so exp is a single ex2.  States cross the ABI in natural units.
+//
+// Rounding: the page's update p' = max(p - w, k), a' = e^{p-w-p'} a + e^{k-p'} v
+// rounds p - w every step.  In fp32 that rounding error is the same every step (w
+// is constant and p stays in one binade), so A = a e^p drifts linearly.  Two
+// evaluation choices, both exactly the page's arithmetic in real numbers, remove
+// the drift:
+//  (1) the history factor's exponent is evaluated as (p - p') - w.  When p' = p - w
+//      (no new maximum) this is the tiny rounding residual of p', recovered exactly
+//      (Sterbenz), and the factor e^x is applied as a + x' a with x' = e^x - 1 from
+//      a short Taylor polynomial -- forming 1 + x' would round it away;
+//  (2) in long scans the exponent is kept anchored, p = anc - n w (one fused
+//      multiply-add from the token that set the maximum), so p itself carries a
+//      single rounding instead of one per step.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace wkvb {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.69314718055994531f;
+// Exponent of the empty state (a = b = 0): finite so p - w never forms inf - inf.
+constexpr float kPEmpty = -1e38f;
+
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+// ---------------------------------------------------------------------------
+// Hardware approximations (MUFU): 2^x and 1/x, flush-to-zero.
+// ex2.approx of a large negative argument returns +0, which is the intended
+// weight of the empty state.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float rcp(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// exp in the chosen domain
+template <bool NAT>
+__device__ __forceinline__ float expd(float x) {
+    return NAT ? ex2(x * kLog2e) : ex2(x);
+}
+
+// e^y - 1 (NAT) or 2^y - 1 (base 2) for |y| well below 1: fourth-order Taylor
+// polynomial of e^z - 1 in z = y (or y ln 2); relative error < 1e-8 for |z| < 2^-4.
+// The argument is clamped to [-1, 1] so degenerate (empty-state) inputs stay finite.
+template <bool NAT>
+__device__ __forceinline__ float expm1d_small(float y) {
+    float z = fminf(fmaxf(NAT ? y : y * kLn2, -1.f), 1.f);
+    return z * fmaf(z, fmaf(z, fmaf(z, 1.f / 24.f, 1.f / 6.f), 0.5f), 1.f);
+}
+
+// ---------------------------------------------------------------------------
+// Output of the current token from a state:  q = max(p, u + k),
+//   y = (e^{p-q} a + e^{u+k-q} v) / (e^{p-q} b + e^{u+k-q}).
+// One of the two weights is exactly 1, so a single exp is needed.
+// uk = u + k in the domain's units.
+// ---------------------------------------------------------------------------
+template <bool NAT>
+__device__ __forceinline__ float wkv_output(float a, float b, float p, float uk, float v) {
+    float d = p - uk;
+    float e = expd<NAT>(-fabsf(d));
+    bool hist = d >= 0.f;
+    float sa = hist ? 1.f : e;
+    float sv = hist ? e : 1.f;
+    return fmaf(sv, v, sa * a) * rcp(fmaf(sa, b, sv));
+}
+
+// ---------------------------------------------------------------------------
+// Fold token (k, v) into the state:  p' = max(p - w, k),
+//   a' = e^{p-w-p'} a + e^{k-p'} v,  b' = e^{p-w-p'} b + e^{k-p'}.
+// pd is the candidate p - w (the caller may compute it from an anchor).
+// ---------------------------------------------------------------------------
+template <bool NAT>
+__device__ __forceinline__ void wkv_fold(float& a, float& b, float& p, float pd, float k, float v, float w) {
+    bool keep = pd >= k;                   // history still holds the maximum
+    float pn = keep ? pd : k;
+    float x = (p - pn) - w;                // keep: rounding residual of pd; else p - k - w
+    float f = expd<NAT>(keep ? (k - pn) : x);
+    float m = keep ? expm1d_small<NAT>(x) : f;
+    float nf = keep ? f : 1.f;
+    a = fmaf(nf, v, fmaf(m, a, keep ? a : 0.f));
+    b = nf + fmaf(m, b, keep ? b : 0.f);
+    p = pn;
+}
+
+// ---------------------------------------------------------------------------
+// Anchored segment record (base-2 units): accumulators (a, b) relative to the
+// exponent p = anc - n w, where anc is the key (or carried exponent) that set
+// the maximum and n the number of steps it has decayed since.
+// The identity (empty segment) is (0, 0, kPEmpty, 0).
+// ---------------------------------------------------------------------------
+struct Rec {
+    float a, b, anc, n;
+};
+
+__device__ __forceinline__ Rec rec_identity() { return Rec{0.f, 0.f, kPEmpty, 0.f}; }
+
+__device__ __forceinline__ float rec_p(const Rec& r, float w2) { return fmaf(-r.n, w2, r.anc); }
+
+// left (earlier) then right (later, spanning len steps): the left decays over len
+// steps (the telescoping of the decay factor, transformer-math page, section "Why
+// it collapses into a recurrence"), then the larger exponent becomes the reference.
+__device__ __forceinline__ Rec rec_combine(const Rec& L, const Rec& R, float len, float w2) {
+    float nl = L.n + len;
+    float pl_old = fmaf(-L.n, w2, L.anc);
+    float pl = fmaf(-nl, w2, L.anc);
+    float pr = fmaf(-R.n, w2, R.anc);
+    bool keep = pl >= pr;
+    Rec o;
+    if (keep) {
+        // left keeps the maximum: its factor is 2^{(pl_old - pl) - len w2}, a rounding residual
+        float x = fmaf(-len, w2, pl_old - pl);
+        float m = expm1d_small<false>(x);
+        float f = ex2(pr - pl);
+        o.a = fmaf(f, R.a, fmaf(m, L.a, L.a));
+        o.b = fmaf(f, R.b, fmaf(m, L.b, L.b));
+        o.anc = L.anc;
+        o.n = nl;
+    } else {
+        float f = ex2(pl - pr);
+        o.a = fmaf(f, L.a, R.a);
+        o.b = fmaf(f, L.b, R.b);
+        o.anc = R.anc;
+        o.n = R.n;
+    }
+    return o;
+}
+
+// ---------------------------------------------------------------------------
+// I/O element conversions
+// ---------------------------------------------------------------------------
+template <typename T>
+struct io;
+
+template <>
+struct io<float> {
+    static __device__ __forceinline__ float load(const float* p) { return *p; }
+    static __device__ __forceinline__ void store(float* p, float x) { *p = x; }
+    static __device__ __forceinline__ float to_f(float x) { return x; }
+    static __device__ __forceinline__ float from_f(float x) { return x; }
+};
+
+template <>
+struct io<__nv_bfloat16> {
+    static __device__ __forceinline__ float load(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+    static __device__ __forceinline__ void store(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
+    static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+    static __device__ __forceinline__ __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+
+// ---------------------------------------------------------------------------
+// Async bulk copies (TMA engine, non-tensor form) and mbarriers.  No cluster
+// multicast is used anywhere.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// Returns true once the phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Global -> shared bulk copy of `bytes` (multiple of 16, both addresses 16-B aligned),
+// completion signalled on `bar` as transaction bytes.
+__device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// GPU-scope acquire/release on 32-bit flags (decoupled look-back).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ float4 ld_relaxed_f4(const float4* p) {
+    float4 r;
+    asm volatile("ld.relaxed.gpu.global.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+                 : "l"(p)
+                 : "memory");
+    return r;
+}
+
+}  // namespace wkvb

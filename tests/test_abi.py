@@ -1,0 +1,91 @@
+"""The C ABI library loads and exports every declared entry point; host-side argument
+validation works without a GPU (no kernel is launched by these calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_rnn_wkv_b200 as wkv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wkv.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+\*?([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "while")))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("wkv_forward", "wkv_decode_step", "token_shift_mix", "wkv_decode_step_fused",
+                 "wkv_forward_workspace_size", "wkv_forward_status", "wkv_status_string"):
+        assert must in names, names
+
+
+def test_library_exports_every_declared_symbol():
+    L = wkv.lib()
+    missing = [n for n in declared_functions() if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_status_strings():
+    L = wkv.lib()
+    for code, name in wkv.STATUS.items():
+        assert L.wkv_status_string(code).decode() == name
+    assert L.wkv_version() == 100
+
+
+I64 = ctypes.c_int64
+FAKE = 0x10000  # a 16-byte aligned, never dereferenced address
+
+
+def _fwd(B, T, C, io=0, w=FAKE, u=FAKE, k=FAKE, v=FAKE, y=FAKE, st=None, ws=FAKE, nbytes=1 << 30, path=0, chunk=0):
+    return wkv.lib().wkv_forward_ex(B, T, C, io, w, u, k, v, None, y, st, ws, nbytes, path, chunk, None)
+
+
+def test_forward_validation_without_launch():
+    assert _fwd(-1, 4, 4) == 1                   # negative size
+    assert _fwd(1 << 40, 1 << 40, 4) == 1        # product overflows int64
+    assert _fwd(1, 4, 4, io=7) == 3              # unknown dtype
+    assert _fwd(1, 4, 4, path=9) == 3            # unknown path
+    assert _fwd(1, 4, 4, chunk=5) == 3           # unsupported chunk
+    assert _fwd(1, 4, 4, w=None) == 1            # null parameter
+    assert _fwd(1, 4, 4, k=None) == 1            # null input
+    assert _fwd(1, 4, 4, y=FAKE + 4) == 2        # misaligned output
+    assert _fwd(1, 4, 4, k=FAKE + 8) == 2        # misaligned input
+    assert _fwd(1, 4, 4, path=2, nbytes=16) == 1  # workspace too small for the chunked path
+    assert _fwd(0, 4, 4) == 0 and _fwd(3, 4, 0) == 0  # empty calls are no-ops
+
+
+def test_decode_and_shift_validation_without_launch():
+    L = wkv.lib()
+    assert L.wkv_decode_step(-2, 1, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert L.wkv_decode_step(2, 1, 4, FAKE, FAKE, None, FAKE, FAKE, FAKE, None) == 1
+    assert L.wkv_decode_step(2, 1, 4, FAKE, FAKE, FAKE + 4, FAKE, FAKE, FAKE, None) == 2
+    assert L.wkv_decode_step(0, 1, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 0
+    assert L.wkv_decode_step_fused(2, 1, 4, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert L.token_shift_mix(1, 4, 4, FAKE, FAKE, FAKE + 4, FAKE, None) == 2
+    assert L.token_shift_mix(1, 4, 4, None, FAKE, None, FAKE, None) == 1
+    assert L.token_shift_mix(1, 0, 4, FAKE, FAKE, None, FAKE, None) == 0
+
+
+def test_workspace_size_query():
+    for (B, T, C) in [(1, 64, 64), (8, 1024, 768), (1, 16384, 4096), (3, 5, 7)]:
+        n = wkv.lib().wkv_forward_workspace_size(B, T, C, 0)
+        # header + one flag and two 16-byte records per channel-tile of the smallest chunk
+        assert n >= 64 + 2 * 16 * B * C * ((T + 15) // 16)
+    assert wkv.lib().wkv_forward_workspace_size(0, 10, 10, 0) == 64
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    k = torch.zeros(1, 4, 4)
+    with pytest.raises(TypeError):
+        wkv.wkv_forward(torch.ones(4), torch.zeros(4), k, k)
+    with pytest.raises(TypeError):
+        wkv.token_shift_mix(torch.ones(4), k)
