@@ -11,7 +11,7 @@ namespace wkvb {
 enum : uint32_t { kDevOk = 0, kDevTimeoutCarry = 1, kDevTimeoutCopy = 2, kDevBadWorkspace = 3 };
 
 // Bounded-wait limits (iterations of a poll loop that sleeps ~64 ns per miss).
-constexpr uint32_t kSpinLimitDefault = 1u << 24;  // ~1 s
+constexpr uint32_t kSpinLimitDefault = 1u << 18;  // a few hundred ms of polling
 
 struct ForwardArgs {
     int64_t B, T, C;
