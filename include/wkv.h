@@ -154,6 +154,32 @@ wkv_status wkv_decode_step_fused(int64_t N, int64_t L, int64_t C, const float* m
                                  const float* k, const float* v, float* state_inout, float* y,
                                  cudaStream_t stream);
 
+/*
+ * wkv_forward_ex on the chunked path for callers that cannot allocate device memory
+ * (for instance code running inside another framework's memory pool, or under a
+ * budget that forbids cudaMalloc after start-up).  The pages have no counterpart: this
+ * is a packaging of the same chunked kernel, not a different computation.
+ *
+ * Same arguments, layouts and results as wkv_forward_ex with path = WKV_PATH_CHUNKED,
+ * minus the workspace: the scratch lives in a fixed 32 MiB device array inside the
+ * library, which every GPU that loads the library keeps until the process exits.  The
+ * call allocates nothing (no cudaMalloc, no allocating library routine).
+ *  - Shapes whose scratch would exceed 32 MiB are rejected with WKV_ERR_INVALID_ARG
+ *    before anything is enqueued (e.g. 8 x 1024 x 768 fp32 needs ~6.3 MB; 1 x 16384 x
+ *    4096 fp32 needs more and is rejected).  T must be >= 1; B = 0 or C = 0 is a no-op.
+ *  - All calls on a device share the array and it keeps the last call's contents; each
+ *    call clears the counters that must start at zero.  Calls that can overlap on the
+ *    GPU race on the array: order them (same stream, or events).
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current and zero-fills the array once;
+ *    make that first call before any stream capture.
+ *  - A device-side wait that runs out (only possible when calls overlap) is recorded
+ *    in the array and cleared by the next call; it is not reported to the caller.
+ */
+wkv_status wkv_forward_chunked_noalloc(int64_t B, int64_t T, int64_t C, wkv_dtype io, const float* w,
+                                       const float* u, const void* k, const void* v, const float* state_in,
+                                       void* y, float* state_out, cudaStream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char* wkv_status_string(wkv_status status);
 
