@@ -10,18 +10,19 @@
 //  * base 2 (inside the forward kernels): k, w, u and p are pre-multiplied by
 //    log2 e once, so exp is a single ex2.  States cross the ABI in natural units.
 //
-// Rounding: the page's update p' = max(p - w, k), a' = e^{p-w-p'} a + e^{k-p'} v
-// rounds p - w every step.  In fp32 that rounding error is the same every step (w
-// is constant and p stays in one binade), so A = a e^p drifts linearly.  Two
-// evaluation choices, both exactly the page's arithmetic in real numbers, remove
-// the drift:
-//  (1) the history factor's exponent is evaluated as (p - p') - w.  When p' = p - w
-//      (no new maximum) this is the tiny rounding residual of p', recovered exactly
-//      (Sterbenz), and the factor e^x is applied as a + x' a with x' = e^x - 1 from
-//      a short Taylor polynomial -- forming 1 + x' would round it away;
-//  (2) in long scans the exponent is kept anchored, p = anc - n w (one fused
-//      multiply-add from the token that set the maximum), so p itself carries a
-//      single rounding instead of one per step.
+// Rounding.  The page's update p' = max(p - w, k), a' = e^{p-w-p'} a + e^{k-p'} v
+// rounds p - w at every step, and in fp32 that rounding error repeats (w is constant
+// and p stays in one binade), so the true accumulators A = a e^p drift linearly.  Two
+// ways of evaluating the same real-number arithmetic avoid it:
+//  (1) scans keep (a, b) relative to the exact exponent anc - n w, where anc is the key
+//      (or carried exponent) that set the maximum and n counts the steps since: the
+//      history then decays by incrementing n, without touching a or b, and rounding
+//      enters only through the argument of each exp (once per term).  Used by the
+//      forward kernels and the segment records (Rec);
+//  (2) the decode step, whose state crosses the ABI as an explicit p, evaluates the
+//      history factor's exponent as (p - p') - w -- the exact rounding residual of p'
+//      when p' = p - w -- and applies it as a + (e^x - 1) a with a Taylor polynomial
+//      for e^x - 1 (wkv_fold).  Over 128 steps that keeps the state within a few 1e-6.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -104,10 +105,10 @@ __device__ __forceinline__ void wkv_fold(float& a, float& b, float& p, float pd,
 }
 
 // ---------------------------------------------------------------------------
-// Anchored segment record (base-2 units): accumulators (a, b) relative to the
-// exponent p = anc - n w, where anc is the key (or carried exponent) that set
-// the maximum and n the number of steps it has decayed since.
-// The identity (empty segment) is (0, 0, kPEmpty, 0).
+// Anchored segment record (base-2 units): accumulators (a, b) relative to the exact
+// exponent anc - n w (a real number; rec_p gives its fp32 value with one rounding).
+// Decaying a record by `len` steps only adds len to n.  The identity (empty segment)
+// is (0, 0, kPEmpty, 0).
 // ---------------------------------------------------------------------------
 struct Rec {
     float a, b, anc, n;
@@ -119,31 +120,46 @@ __device__ __forceinline__ float rec_p(const Rec& r, float w2) { return fmaf(-r.
 
 // left (earlier) then right (later, spanning len steps): the left decays over len
 // steps (the telescoping of the decay factor, transformer-math page, section "Why
-// it collapses into a recurrence"), then the larger exponent becomes the reference.
+// it collapses into a recurrence"); the larger exponent stays the reference and the
+// other record is scaled onto it with one exp.
 __device__ __forceinline__ Rec rec_combine(const Rec& L, const Rec& R, float len, float w2) {
-    float nl = L.n + len;
-    float pl_old = fmaf(-L.n, w2, L.anc);
-    float pl = fmaf(-nl, w2, L.anc);
-    float pr = fmaf(-R.n, w2, R.anc);
-    bool keep = pl >= pr;
+    const float nl = L.n + len;
+    const float pl = fmaf(-nl, w2, L.anc);
+    const float pr = fmaf(-R.n, w2, R.anc);
+    const bool keep = pl >= pr;
+    const float f = ex2(-fabsf(pl - pr));
     Rec o;
     if (keep) {
-        // left keeps the maximum: its factor is 2^{(pl_old - pl) - len w2}, a rounding residual
-        float x = fmaf(-len, w2, pl_old - pl);
-        float m = expm1d_small<false>(x);
-        float f = ex2(pr - pl);
-        o.a = fmaf(f, R.a, fmaf(m, L.a, L.a));
-        o.b = fmaf(f, R.b, fmaf(m, L.b, L.b));
+        o.a = fmaf(f, R.a, L.a);
+        o.b = fmaf(f, R.b, L.b);
         o.anc = L.anc;
         o.n = nl;
     } else {
-        float f = ex2(pl - pr);
         o.a = fmaf(f, L.a, R.a);
         o.b = fmaf(f, L.b, R.b);
         o.anc = R.anc;
         o.n = R.n;
     }
     return o;
+}
+
+// One token of a long scan in the anchored form (base-2 units): output from the
+// state before the token, then fold the token in.  (a, b) are relative to anc - n w.
+__device__ __forceinline__ float scan_step(float& a, float& b, float& anc, float& n, float k2, float v, float u2,
+                                           float w2) {
+    const float p = fmaf(-n, w2, anc);
+    const float y = wkv_output<false>(a, b, p, u2 + k2, v);
+    const float n1 = n + 1.f;
+    const float pd = fmaf(-n1, w2, anc);   // the history's exponent after decaying one step
+    const bool keep = pd >= k2;            // history still holds the maximum
+    const float e = ex2(-fabsf(k2 - pd));  // the smaller of the two weights
+    const float sa = keep ? 1.f : e;
+    const float sv = keep ? e : 1.f;
+    a = fmaf(sv, v, sa * a);
+    b = fmaf(sa, b, sv);
+    anc = keep ? anc : k2;
+    n = keep ? n1 : 0.f;
+    return y;
 }
 
 // ---------------------------------------------------------------------------

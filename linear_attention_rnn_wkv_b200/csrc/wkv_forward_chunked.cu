@@ -4,9 +4,7 @@
 // "Why it collapses into a recurrence"), so the state after a span of tokens is an
 // associative fold: a segment is summarised by (a, b, p) relative to its own running
 // maximum, and two adjacent segments combine by decaying the earlier one over the
-// later one's length and re-referencing to the larger exponent.  The summaries use
-// the anchored record of wkv_device.cuh (p = anc - n w) so that exponents carry one
-// rounding, not one per step.
+// later one's length and re-referencing to the larger exponent (rec_combine).
 //
 // Work decomposition.  A unit is a tile of Ts = NW * LC time steps by Cg = 32 * V
 // channels of one sequence.  Units are handed out by an atomic ticket in
@@ -20,27 +18,64 @@
 //      completion on an mbarrier; per-element loads when rows are not 16-byte
 //      multiples);
 //   2. each warp summarises its chunk from the empty state: the exact maximum
-//      exponent max_i (k_i - (LC-1-i) w) first, then one exp per element;
+//      exponent M = max_i (k_i - (LC-1-i) w) first (kept as the record's exponent, a
+//      single rounding), then one exp per element;
 //   3. one thread per channel scans the NW chunk summaries (exclusive prefixes stay
 //      in shared memory; the inclusive one is the tile aggregate);
-//   4. warp 0 publishes the aggregate, then looks back over the predecessor tiles of
-//      the same channel group (decoupled look-back, Merrill & Garland 2016): it
-//      combines aggregates until it meets an inclusive prefix, and publishes its own
-//      inclusive prefix.  Every wait is bounded; on expiry the error word is set and
-//      the missing carry is taken as empty, so no successor can hang;
+//   4. warp 0 publishes the aggregate and looks back over the predecessor tiles of
+//      the same channel group (decoupled look-back, Merrill & Garland 2016).  The 32
+//      lanes poll the flags of 32 predecessors at once and stop at the nearest one
+//      holding an inclusive prefix; the records in between are then loaded together
+//      and folded, so a look-back costs a few L2 round trips whatever its depth.
+//      Every wait is bounded; on expiry the error word is set and the missing carry
+//      is taken as empty, so no successor can hang;
 //   5. every warp combines the tile carry with its chunk's exclusive prefix and
-//      re-scans its chunk from shared memory, writing y.
+//      re-scans its chunk from shared memory, writing y.  Within a chunk the output
+//      and the state update share one exp: the state is kept relative to a reference
+//      exponent r that decays with the history, so the new token's weight relative to
+//      it is the output's weight times the per-channel constant 2^(w - u); r moves to
+//      the current token only when that token dominates (see lazy_step).  Channels
+//      with |u| or w too large for that constant fall back to the page's form.
 // The last time segment's inclusive prefix is the final state (state_out).
 #include "wkv_device.cuh"
 #include "wkv_internal.h"
 
+// Tile shape per I/O type: V channels per lane (32 V per tile) and NW warps (chunks).
+#ifndef WKV_F32_V
+#define WKV_F32_V 2
+#endif
+#ifndef WKV_F32_NW
+#define WKV_F32_NW 8
+#endif
+#ifndef WKV_BF16_V
+#define WKV_BF16_V 4
+#endif
+#ifndef WKV_BF16_NW
+#define WKV_BF16_NW 4
+#endif
+
 namespace wkvb {
 namespace {
 
-// ---- vector I/O of V adjacent channels ----
+// ---- vector I/O of V adjacent channels (shared or global memory) ----
 template <typename TIO, int V>
 struct Vec;
 
+template <>
+struct Vec<float, 1> {
+    static __device__ __forceinline__ void load(const float* p, float (&o)[1]) { o[0] = *p; }
+    static __device__ __forceinline__ void store(float* p, const float (&o)[1]) { *p = o[0]; }
+};
+template <>
+struct Vec<float, 2> {
+    static __device__ __forceinline__ void load(const float* p, float (&o)[2]) {
+        float2 t = *reinterpret_cast<const float2*>(p);
+        o[0] = t.x; o[1] = t.y;
+    }
+    static __device__ __forceinline__ void store(float* p, const float (&o)[2]) {
+        *reinterpret_cast<float2*>(p) = make_float2(o[0], o[1]);
+    }
+};
 template <>
 struct Vec<float, 4> {
     static __device__ __forceinline__ void load(const float* p, float (&o)[4]) {
@@ -52,38 +87,48 @@ struct Vec<float, 4> {
     }
 };
 
-template <>
-struct Vec<float, 1> {
-    static __device__ __forceinline__ void load(const float* p, float (&o)[1]) { o[0] = *p; }
-    static __device__ __forceinline__ void store(float* p, const float (&o)[1]) { *p = o[0]; }
-};
+__device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
+__device__ __forceinline__ uint32_t bf_pack(float lo, float hi) {
+    __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&t);
+}
 
+template <>
+struct Vec<__nv_bfloat16, 1> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&o)[1]) { o[0] = __bfloat162float(*p); }
+    static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&o)[1]) { *p = __float2bfloat16_rn(o[0]); }
+};
+template <>
+struct Vec<__nv_bfloat16, 2> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&o)[2]) {
+        uint32_t t = *reinterpret_cast<const uint32_t*>(p);
+        o[0] = bf_lo(t); o[1] = bf_hi(t);
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&o)[2]) {
+        *reinterpret_cast<uint32_t*>(p) = bf_pack(o[0], o[1]);
+    }
+};
 template <>
 struct Vec<__nv_bfloat16, 4> {
     static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&o)[4]) {
         uint2 t = *reinterpret_cast<const uint2*>(p);
-        o[0] = __uint_as_float(t.x << 16);
-        o[1] = __uint_as_float(t.x & 0xFFFF0000u);
-        o[2] = __uint_as_float(t.y << 16);
-        o[3] = __uint_as_float(t.y & 0xFFFF0000u);
+        o[0] = bf_lo(t.x); o[1] = bf_hi(t.x); o[2] = bf_lo(t.y); o[3] = bf_hi(t.y);
     }
     static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&o)[4]) {
-        __nv_bfloat162 lo = __floats2bfloat162_rn(o[0], o[1]);
-        __nv_bfloat162 hi = __floats2bfloat162_rn(o[2], o[3]);
-        uint2 t;
-        t.x = *reinterpret_cast<uint32_t*>(&lo);
-        t.y = *reinterpret_cast<uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(p) = t;
+        *reinterpret_cast<uint2*>(p) = make_uint2(bf_pack(o[0], o[1]), bf_pack(o[2], o[3]));
     }
 };
-
 template <>
-struct Vec<__nv_bfloat16, 1> {
-    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&o)[1]) {
-        o[0] = __bfloat162float(*p);
+struct Vec<__nv_bfloat16, 8> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&o)[8]) {
+        uint4 t = *reinterpret_cast<const uint4*>(p);
+        o[0] = bf_lo(t.x); o[1] = bf_hi(t.x); o[2] = bf_lo(t.y); o[3] = bf_hi(t.y);
+        o[4] = bf_lo(t.z); o[5] = bf_hi(t.z); o[6] = bf_lo(t.w); o[7] = bf_hi(t.w);
     }
-    static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&o)[1]) {
-        *p = __float2bfloat16_rn(o[0]);
+    static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&o)[8]) {
+        *reinterpret_cast<uint4*>(p) = make_uint4(bf_pack(o[0], o[1]), bf_pack(o[2], o[3]), bf_pack(o[4], o[5]),
+                                                  bf_pack(o[6], o[7]));
     }
 };
 
@@ -103,6 +148,36 @@ __device__ __forceinline__ Rec rec_unpack(const float4& f) { return Rec{f.x, f.y
 __device__ __forceinline__ Rec rec_from_state(const float* st, int64_t bc, int64_t BC) {
     return Rec{st[bc], st[BC + bc], st[2 * BC + bc] * kLog2e, 0.f};
 }
+
+// One token within a chunk, one exp for both the output and the update.
+// State (a, b) is relative to the reference exponent r = R - n w (base 2, exact real;
+// the history decays by counting n), i.e. A = a 2^r.  With D = (u + k) - r, E = 2^-|D|:
+//   D <= 0 (history dominates): y = (a + E v)/(b + E); the new token's weight relative to
+//          the decayed reference r - w is 2^(k - r + w) = E * c with c = 2^(w - u), so
+//          a += E c v, b += E c, n += 1;
+//   D > 0  (token dominates):   y = (E a + v)/(E b + 1); re-reference to u + k:
+//          a = E a + c v, b = E b + c, R = u + k, n = 1.
+// Exact in real arithmetic; valid while c and its reciprocal stay far from the fp32
+// range limits (callers check |u|, w <= kLazyLimit).
+__device__ __forceinline__ float lazy_step(float& a, float& b, float& R, float& n, float k2, float v, float u2,
+                                           float w2, float c) {
+    const float r = fmaf(-n, w2, R);
+    const float uk = u2 + k2;
+    const float d = uk - r;
+    const float e = ex2(-fabsf(d));
+    const bool cur = d > 0.f;
+    const float sa = cur ? e : 1.f;
+    const float sv = cur ? 1.f : e;
+    const float t = sa * a;
+    const float y = fmaf(sv, v, t) * rcp(fmaf(sa, b, sv));
+    const float nw = sv * c;
+    a = fmaf(nw, v, t);
+    b = fmaf(sa, b, nw);
+    R = cur ? uk : R;
+    n = cur ? 1.f : n + 1.f;
+    return y;
+}
+constexpr float kLazyLimit = 40.f;  // base-2 units: c = 2^(w - u) within 2^(+-80)
 
 template <typename TIO, int V, int NW, int LC, bool BULK>
 __global__ void __launch_bounds__(NW * 32) chunked_kernel(ForwardArgs args, ChunkParams cp) {
@@ -168,6 +243,20 @@ __global__ void __launch_bounds__(NW * 32) chunked_kernel(ForwardArgs args, Chun
                 bulk_g2s(vs + r * Cg, vg + (int64_t)r * C, row_bytes, bar);
             }
         }
+    }
+
+    // per-thread channels and parameters (base-2 units), while the copies fly
+    const int cl = lane * V;  // first channel of this lane within the tile
+    const bool lane_active = cl < nch;
+    float w2[V], u2[V];
+#pragma unroll
+    for (int q = 0; q < V; ++q) {
+        const bool ok = lane_active && (cl + q < nch);
+        w2[q] = ok ? args.w[c0 + cl + q] * kLog2e : 0.f;
+        u2[q] = ok ? args.u[c0 + cl + q] * kLog2e : 0.f;
+    }
+
+    if (BULK) {
         bool timed_out = false;
         for (uint32_t it = 0; !mbar_try_wait(bar, 0); ++it) {
             if (it >= args.spin_limit) {
@@ -192,61 +281,45 @@ __global__ void __launch_bounds__(NW * 32) chunked_kernel(ForwardArgs args, Chun
         __syncthreads();
     }
 
-    // per-thread channels and parameters (base-2 units)
-    const int cl = lane * V;  // first channel of this lane within the tile
-    const bool lane_active = cl < nch;
-    float w2[V], u2[V];
-#pragma unroll
-    for (int q = 0; q < V; ++q) {
-        const int64_t c = c0 + cl + q;
-        const bool ok = lane_active && (cl + q < nch);
-        w2[q] = ok ? args.w[c] * kLog2e : 0.f;
-        u2[q] = ok ? args.u[c] * kLog2e : 0.f;
-    }
-
     // ---- 2. chunk summaries from the empty state ----
     const int r_begin = warp * LC;
     const int r_cnt = max(0, min(LC, len - r_begin));
     if (lane_active) {
-        float M[V], anc[V], nn[V];
+        float gx[LC][V], M[V];
 #pragma unroll
-        for (int q = 0; q < V; ++q) {
-            M[q] = kPEmpty;
-            anc[q] = kPEmpty;
-            nn[q] = 0.f;
-        }
-        for (int i = 0; i < r_cnt; ++i) {
-            float kk[V];
-            Vec<TIO, V>::load(ks + (r_begin + i) * Cg + cl, kk);
-            const float back = (float)(r_cnt - 1 - i);
+        for (int q = 0; q < V; ++q) M[q] = kPEmpty;
 #pragma unroll
-            for (int q = 0; q < V; ++q) {
-                const float k2 = kk[q] * kLog2e;
-                const float gq = fmaf(-back, w2[q], k2);
-                if (gq > M[q]) {
-                    M[q] = gq;
-                    anc[q] = k2;
-                    nn[q] = back;
+        for (int i = 0; i < LC; ++i) {
+            if (i < r_cnt) {
+                float kk[V];
+                Vec<TIO, V>::load(ks + (r_begin + i) * Cg + cl, kk);
+                const float back = (float)(r_cnt - 1 - i);
+#pragma unroll
+                for (int q = 0; q < V; ++q) {
+                    gx[i][q] = fmaf(-back, w2[q], kk[q] * kLog2e);
+                    M[q] = fmaxf(M[q], gx[i][q]);
                 }
             }
         }
         float sa[V], sb[V];
 #pragma unroll
         for (int q = 0; q < V; ++q) sa[q] = sb[q] = 0.f;
-        for (int i = 0; i < r_cnt; ++i) {
-            float kk[V], vv[V];
-            Vec<TIO, V>::load(ks + (r_begin + i) * Cg + cl, kk);
-            Vec<TIO, V>::load(vs + (r_begin + i) * Cg + cl, vv);
-            const float back = (float)(r_cnt - 1 - i);
 #pragma unroll
-            for (int q = 0; q < V; ++q) {
-                const float e = ex2(fmaf(-back, w2[q], kk[q] * kLog2e) - M[q]);
-                sa[q] = fmaf(e, vv[q], sa[q]);
-                sb[q] += e;
+        for (int i = 0; i < LC; ++i) {
+            if (i < r_cnt) {
+                float vv[V];
+                Vec<TIO, V>::load(vs + (r_begin + i) * Cg + cl, vv);
+#pragma unroll
+                for (int q = 0; q < V; ++q) {
+                    const float e = ex2(gx[i][q] - M[q]);
+                    sa[q] = fmaf(e, vv[q], sa[q]);
+                    sb[q] += e;
+                }
             }
         }
+        // the record's exponent is M itself (anchor M, zero steps since)
 #pragma unroll
-        for (int q = 0; q < V; ++q) recs[warp * Cg + cl + q] = Rec{sa[q], sb[q], anc[q], nn[q]};
+        for (int q = 0; q < V; ++q) recs[warp * Cg + cl + q] = Rec{sa[q], sb[q], M[q], 0.f};
     }
     __syncthreads();
 
@@ -254,6 +327,7 @@ __global__ void __launch_bounds__(NW * 32) chunked_kernel(ForwardArgs args, Chun
     for (int cc = tid; cc < nch; cc += NT) {
         const float w2c = args.w[c0 + cc] * kLog2e;
         Rec run = rec_identity();
+#pragma unroll
         for (int w = 0; w < NW; ++w) {
             const int lw = max(0, min(LC, len - w * LC));
             Rec r = recs[w * Cg + cc];
@@ -266,9 +340,8 @@ __global__ void __launch_bounds__(NW * 32) chunked_kernel(ForwardArgs args, Chun
 
     // ---- 4. decoupled look-back across time segments (warp 0) ----
     if (warp == 0) {
-        const int64_t uidx = unit;
-        const bool publish = uidx != cp.drop_unit;
-        Rec carry[V], inc[V];
+        const bool publish = unit != cp.drop_unit;
+        Rec carry[V];
         if (j == 0) {
 #pragma unroll
             for (int q = 0; q < V; ++q) {
@@ -281,80 +354,100 @@ __global__ void __launch_bounds__(NW * 32) chunked_kernel(ForwardArgs args, Chun
             if (lane_active) {
 #pragma unroll
                 for (int q = 0; q < V; ++q)
-                    if (cl + q < nch) cp.agg[uidx * Cg + cl + q] = rec_pack(aggs[cl + q]);
+                    if (cl + q < nch) cp.agg[unit * Cg + cl + q] = rec_pack(aggs[cl + q]);
             }
             __threadfence();
             __syncwarp();
-            if (lane == 0 && publish) st_release_u32(&cp.flags[uidx], (epoch30 << 2) | 1u);
-            // look back
+            if (lane == 0 && publish) st_release_u32(&cp.flags[unit], (epoch30 << 2) | 1u);
+
             Rec run[V];
 #pragma unroll
             for (int q = 0; q < V; ++q) run[q] = rec_identity();
             float span = 0.f;
-            int64_t pred = j - 1;
+            int64_t hi = j - 1;  // newest predecessor not folded yet
             while (true) {
-                const int64_t pu = pred * cp.G + g;
-                // lane 0 polls; then every lane acquires the flag itself (at least the state lane 0
-                // saw: flags only move AGG -> INCL within a launch) before reading the record
-                uint32_t f = 0;
-                bool ready = false;
-                if (lane == 0) {
-                    for (uint32_t it = 0; it <= args.spin_limit; ++it) {
-                        f = ld_acquire_u32(&cp.flags[pu]);
-                        if ((f >> 2) == epoch30 && (f & 3u) != 0u) {
-                            ready = true;
-                            break;
-                        }
-                        __nanosleep(64);
+                // lane i watches predecessor hi - i
+                const int64_t mine = hi - lane;
+                const bool valid = mine >= 0;
+                const uint32_t* myflag = &cp.flags[(valid ? mine : 0) * cp.G + g];
+                uint32_t st = valid ? 0u : 3u;  // invalid lanes never block
+                int m = -1;                     // lanes 0..m get folded
+                bool found_incl = false;
+                for (uint32_t it = 0; it <= args.spin_limit; ++it) {
+                    if (st == 0u) {
+                        const uint32_t f = ld_acquire_u32(myflag);
+                        if ((f >> 2) == epoch30 && (f & 3u) != 0u) st = f & 3u;
                     }
+                    const unsigned incl = __ballot_sync(0xffffffffu, valid && st == 2u);
+                    const unsigned ready = __ballot_sync(0xffffffffu, st != 0u);
+                    const int last = (int)min64(31, hi);  // last valid lane
+                    const int stop = incl ? (__ffs(incl) - 1) : last;
+                    const unsigned need = stop >= 31 ? 0xffffffffu : ((2u << stop) - 1u);
+                    if ((ready & need) == need) {
+                        m = stop;
+                        found_incl = incl != 0;
+                        break;
+                    }
+                    __nanosleep(64);
                 }
-                ready = __shfl_sync(0xffffffffu, ready, 0);
-                if (!ready) {
-                    // the predecessor never published: record it, take its carry as empty
+                if (m < 0) {
+                    // a predecessor never published: record it, take the rest of the carry as empty
                     if (lane == 0) {
                         atomicCAS(&cp.hdr->error, kDevOk, kDevTimeoutCarry);
-                        cp.hdr->error_unit = (uint32_t)uidx;
+                        cp.hdr->error_unit = (uint32_t)unit;
                     }
                     break;
                 }
-                f = __shfl_sync(0xffffffffu, f, 0);
-                if (lane != 0) {
-                    for (uint32_t it = 0; it <= args.spin_limit; ++it) {
-                        const uint32_t mine = ld_acquire_u32(&cp.flags[pu]);
-                        if ((mine >> 2) == epoch30 && (mine & 3u) >= (f & 3u)) break;
-                        __nanosleep(64);
-                    }
-                }
-                const bool inclusive = (f & 3u) == 2u;
-                const float4* src = inclusive ? cp.incl : cp.agg;
-                if (lane_active) {
+                // Lane i acquired predecessor hi - i's flag; after the warp barrier every
+                // lane reads the records behind the flags with L1-bypassing loads (the
+                // producer wrote them before its fence and release).  Fold predecessors
+                // hi .. hi - m, newest first, loading four at a time.
+                __syncwarp();
+                for (int i0 = 0; i0 <= m; i0 += 4) {
+                    float4 buf[4][V];
+                    uint32_t sts[4];
 #pragma unroll
-                    for (int q = 0; q < V; ++q) {
-                        if (cl + q < nch) {
-                            Rec r = rec_unpack(ld_relaxed_f4(src + pu * Cg + cl + q));
-                            run[q] = rec_combine(r, run[q], span, w2[q]);
+                    for (int ii = 0; ii < 4; ++ii) {
+                        const int i = i0 + ii;
+                        sts[ii] = __shfl_sync(0xffffffffu, st, i & 31);
+                        if (i <= m && lane_active) {
+                            const float4* src = (sts[ii] == 2u) ? cp.incl : cp.agg;
+                            const int64_t pu = (hi - i) * cp.G + g;
+#pragma unroll
+                            for (int q = 0; q < V; ++q)
+                                if (cl + q < nch) buf[ii][q] = ld_relaxed_f4(src + pu * Cg + cl + q);
                         }
                     }
+#pragma unroll
+                    for (int ii = 0; ii < 4; ++ii) {
+                        if (i0 + ii <= m && lane_active) {
+#pragma unroll
+                            for (int q = 0; q < V; ++q)
+                                if (cl + q < nch) run[q] = rec_combine(rec_unpack(buf[ii][q]), run[q], span, w2[q]);
+                        }
+                        if (i0 + ii <= m) span += (float)Ts;
+                    }
                 }
-                if (inclusive || pred == 0) break;
-                span += (float)Ts;
-                --pred;
+                if (found_incl) break;
+                hi -= (int64_t)(m + 1);
+                if (hi < 0) break;
             }
 #pragma unroll
             for (int q = 0; q < V; ++q) carry[q] = run[q];
         }
         // inclusive prefix of this unit
+        Rec inc[V];
 #pragma unroll
         for (int q = 0; q < V; ++q)
             inc[q] = (cl + q < nch) ? rec_combine(carry[q], aggs[cl + q], (float)len, w2[q]) : rec_identity();
         if (lane_active) {
 #pragma unroll
             for (int q = 0; q < V; ++q)
-                if (cl + q < nch) cp.incl[uidx * Cg + cl + q] = rec_pack(inc[q]);
+                if (cl + q < nch) cp.incl[unit * Cg + cl + q] = rec_pack(inc[q]);
         }
         __threadfence();
         __syncwarp();
-        if (lane == 0 && publish) st_release_u32(&cp.flags[uidx], (epoch30 << 2) | 2u);
+        if (lane == 0 && publish) st_release_u32(&cp.flags[unit], (epoch30 << 2) | 2u);
         if (lane_active) {
 #pragma unroll
             for (int q = 0; q < V; ++q) carry_s[cl + q] = carry[q];
@@ -375,31 +468,63 @@ __global__ void __launch_bounds__(NW * 32) chunked_kernel(ForwardArgs args, Chun
 
     // ---- 5. re-scan each chunk from its carry, emitting y ----
     if (lane_active && r_cnt > 0) {
-        float a[V], bb[V], p[V];
+        float a[V], bb[V], R[V], nn[V];
 #pragma unroll
         for (int q = 0; q < V; ++q) {
             const Rec cr = rec_combine(carry_s[cl + q], recs[warp * Cg + cl + q], (float)r_begin, w2[q]);
             a[q] = cr.a;
             bb[q] = cr.b;
-            p[q] = rec_p(cr, w2[q]);
+            R[q] = cr.anc;
+            nn[q] = cr.n;
         }
-        for (int i = 0; i < r_cnt; ++i) {
-            const int r = r_begin + i;
-            float kk[V], vv[V], yy[V];
-            Vec<TIO, V>::load(ks + r * Cg + cl, kk);
-            Vec<TIO, V>::load(vs + r * Cg + cl, vv);
+        bool lazy_ok = true;
 #pragma unroll
-            for (int q = 0; q < V; ++q) {
-                const float k2 = kk[q] * kLog2e;
-                yy[q] = wkv_output<false>(a[q], bb[q], p[q], u2[q] + k2, vv[q]);
-                wkv_fold<false>(a[q], bb[q], p[q], p[q] - w2[q], k2, vv[q], w2[q]);
+        for (int q = 0; q < V; ++q) lazy_ok = lazy_ok && fabsf(u2[q]) <= kLazyLimit && w2[q] <= kLazyLimit;
+        if (lazy_ok) {
+            float c[V];
+#pragma unroll
+            for (int q = 0; q < V; ++q) c[q] = ex2(w2[q] - u2[q]);
+#pragma unroll
+            for (int i = 0; i < LC; ++i) {
+                if (i < r_cnt) {
+                    const int r = r_begin + i;
+                    float kk[V], vv[V], yy[V];
+                    Vec<TIO, V>::load(ks + r * Cg + cl, kk);
+                    Vec<TIO, V>::load(vs + r * Cg + cl, vv);
+#pragma unroll
+                    for (int q = 0; q < V; ++q)
+                        yy[q] = lazy_step(a[q], bb[q], R[q], nn[q], kk[q] * kLog2e, vv[q], u2[q], w2[q], c[q]);
+                    if (V == 1 || cl + V <= nch) {
+                        Vec<TIO, V>::store(yg + (int64_t)r * C + cl, yy);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < V; ++q)
+                            if (cl + q < nch) io<TIO>::store(yg + (int64_t)r * C + cl + q, yy[q]);
+                    }
+                }
             }
-            if (V == 1 || cl + V <= nch) {
-                Vec<TIO, V>::store(yg + (int64_t)r * C + cl, yy);
-            } else {
+        } else {
+            float p[V];
 #pragma unroll
-                for (int q = 0; q < V; ++q)
-                    if (cl + q < nch) io<TIO>::store(yg + (int64_t)r * C + cl + q, yy[q]);
+            for (int q = 0; q < V; ++q) p[q] = fmaf(-nn[q], w2[q], R[q]);
+            for (int i = 0; i < r_cnt; ++i) {
+                const int r = r_begin + i;
+                float kk[V], vv[V], yy[V];
+                Vec<TIO, V>::load(ks + r * Cg + cl, kk);
+                Vec<TIO, V>::load(vs + r * Cg + cl, vv);
+#pragma unroll
+                for (int q = 0; q < V; ++q) {
+                    const float k2 = kk[q] * kLog2e;
+                    yy[q] = wkv_output<false>(a[q], bb[q], p[q], u2[q] + k2, vv[q]);
+                    wkv_fold<false>(a[q], bb[q], p[q], p[q] - w2[q], k2, vv[q], w2[q]);
+                }
+                if (V == 1 || cl + V <= nch) {
+                    Vec<TIO, V>::store(yg + (int64_t)r * C + cl, yy);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < V; ++q)
+                        if (cl + q < nch) io<TIO>::store(yg + (int64_t)r * C + cl + q, yy[q]);
+                }
             }
         }
     }
@@ -438,9 +563,8 @@ cudaError_t launch_t(const ForwardArgs& a, const ChunkGeom& g, const ChunkParams
     return cudaGetLastError();
 }
 
-template <typename TIO, int V, bool BULK>
+template <typename TIO, int V, int NW, bool BULK>
 cudaError_t launch_lc(const ForwardArgs& a, const ChunkGeom& g, const ChunkParams& cp, cudaStream_t s) {
-    constexpr int NW = 4;
     switch (g.LC) {
         case 4: return launch_t<TIO, V, NW, 4, BULK>(a, g, cp, s);
         case 8: return launch_t<TIO, V, NW, 8, BULK>(a, g, cp, s);
@@ -454,10 +578,10 @@ cudaError_t launch_lc(const ForwardArgs& a, const ChunkGeom& g, const ChunkParam
 bool chunk_geometry(int64_t B, int64_t T, int64_t C, int io, int chunk, ChunkGeom* g) {
     const int esize = io == 1 ? 2 : 4;
     const bool bulk = ((C * esize) % 16) == 0;
-    const int LC = chunk == 0 ? 8 : chunk;
+    const int LC = chunk == 0 ? 16 : chunk;
     if (LC != 4 && LC != 8 && LC != 16) return false;
-    g->V = bulk ? 4 : 1;
-    g->NW = 4;
+    g->V = bulk ? (io == 1 ? WKV_BF16_V : WKV_F32_V) : 1;
+    g->NW = bulk ? (io == 1 ? WKV_BF16_NW : WKV_F32_NW) : 4;
     g->LC = LC;
     g->bulk = bulk;
     g->Cg = 32 * g->V;
@@ -485,9 +609,11 @@ cudaError_t launch_forward_chunked(const ForwardArgs& a, const ChunkGeom& g, voi
     cp.incl = cp.agg + (size_t)g.U * (size_t)g.Cg;
     cp.drop_unit = drop_unit;
     if (a.io == 1) {
-        return g.bulk ? launch_lc<__nv_bfloat16, 4, true>(a, g, cp, s) : launch_lc<__nv_bfloat16, 1, false>(a, g, cp, s);
+        return g.bulk ? launch_lc<__nv_bfloat16, WKV_BF16_V, WKV_BF16_NW, true>(a, g, cp, s)
+                      : launch_lc<__nv_bfloat16, 1, 4, false>(a, g, cp, s);
     }
-    return g.bulk ? launch_lc<float, 4, true>(a, g, cp, s) : launch_lc<float, 1, false>(a, g, cp, s);
+    return g.bulk ? launch_lc<float, WKV_F32_V, WKV_F32_NW, true>(a, g, cp, s)
+                  : launch_lc<float, 1, 4, false>(a, g, cp, s);
 }
 
 }  // namespace wkvb

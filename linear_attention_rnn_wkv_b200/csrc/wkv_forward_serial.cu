@@ -2,8 +2,8 @@
 //
 // The recurrence is the running-maximum form of the RWKV transformer-math page
 // (aicassindra.com, tm_rwkv_math), section "Numerical stability: carry the
-// exponent", evaluated token after token with the exponent anchored (p = anc - n w,
-// one rounding) so long scans do not drift.
+// exponent", evaluated token after token in the anchored form of scan_step: the
+// history decays by counting steps, so long scans do not drift.
 //
 // Data movement (bulk path, C a multiple of 16 bytes): a CTA owns NT consecutive
 // channels of one sequence.  Tiles of TS time steps x NT channels of k and v are
@@ -19,7 +19,7 @@ namespace {
 
 template <typename TIO>
 struct SerialChannel {
-    float a, b, p, anc, n;
+    float a, b, anc, n;
     float w2, u2;
 
     __device__ __forceinline__ void init(const float* w, const float* u, const float* state_in, int64_t bc,
@@ -29,32 +29,21 @@ struct SerialChannel {
         if (state_in) {
             a = state_in[bc];
             b = state_in[BC + bc];
-            p = state_in[2 * BC + bc] * kLog2e;
+            anc = state_in[2 * BC + bc] * kLog2e;
         } else {
             a = 0.f;
             b = 0.f;
-            p = kPEmpty;
+            anc = kPEmpty;
         }
-        anc = p;
         n = 0.f;
     }
 
-    __device__ __forceinline__ float step(float kk, float vv) {
-        float k2 = kk * kLog2e;
-        float y = wkv_output<false>(a, b, p, u2 + k2, vv);
-        float n1 = n + 1.f;
-        float pd = fmaf(-n1, w2, anc);
-        bool keep = pd >= k2;
-        wkv_fold<false>(a, b, p, pd, k2, vv, w2);
-        anc = keep ? anc : k2;
-        n = keep ? n1 : 0.f;
-        return y;
-    }
+    __device__ __forceinline__ float step(float kk, float vv) { return scan_step(a, b, anc, n, kk * kLog2e, vv, u2, w2); }
 
     __device__ __forceinline__ void store_state(float* state_out, int64_t bc, int64_t BC) {
         state_out[bc] = a;
         state_out[BC + bc] = b;
-        state_out[2 * BC + bc] = p * kLn2;
+        state_out[2 * BC + bc] = fmaf(-n, w2, anc) * kLn2;
     }
 };
 
