@@ -76,8 +76,12 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     import torch
     import linear_attention_rnn_wkv_b200 as wkv
     noalloc = _noalloc(wkv.lib())
-    # 1 x 16384 x 4096 fp32 needs more than the 32 MiB scratch: refused before any launch
-    rc = noalloc(1, 16384, 4096, 0, 16, 16, 16, 16, None, 16, None, torch.cuda.current_stream().cuda_stream)
+    # a shape whose scratch exceeds 32 MiB on every tile the library may pick
+    # (65536 x 8192 channel-steps: at least 2 x 16 B x 8192 x 512 = 128 MiB of records):
+    # refused before any launch
+    need = wkv.workspace_size(1, 65536, 8192)
+    assert need > 32 << 20
+    rc = noalloc(1, 65536, 8192, 0, 16, 16, 16, 16, None, 16, None, torch.cuda.current_stream().cuda_stream)
     assert rc == 1  # WKV_ERR_INVALID_ARG
     assert noalloc(2, 0, 8, 0, 16, 16, 16, 16, None, 16, None, None) == 1
     assert noalloc(0, 5, 8, 0, 16, 16, 16, 16, None, 16, None, None) == 0
