@@ -126,7 +126,7 @@ size_t wkv_forward_workspace_size(int64_t B, int64_t T, int64_t C, wkv_dtype io)
     int64_t n = 0;
     if (!sizes_ok(B, T, C, &n) || n == 0) return kWsHeaderBytes;
     size_t best = kWsHeaderBytes;
-    for (int chunk : {4, 8, 16}) {
+    for (int chunk : {0, 4, 8, 16}) {
         ChunkGeom g;
         if (chunk_geometry(B, T, C, (int)io, chunk, &g) && g.ws_bytes > best) best = g.ws_bytes;
     }

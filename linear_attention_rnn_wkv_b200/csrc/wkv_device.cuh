@@ -163,6 +163,47 @@ __device__ __forceinline__ float scan_step(float& a, float& b, float& anc, float
 }
 
 // ---------------------------------------------------------------------------
+// Record packing and the one-exp chunk step used by the chunked forward kernels
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float4 rec_pack(const Rec& r) { return make_float4(r.a, r.b, r.anc, r.n); }
+__device__ __forceinline__ Rec rec_unpack(const float4& f) { return Rec{f.x, f.y, f.z, f.w}; }
+
+// Natural-units state (a, b, p) -> anchored base-2 record.
+__device__ __forceinline__ Rec rec_from_state(const float* st, int64_t bc, int64_t BC) {
+    return Rec{st[bc], st[BC + bc], st[2 * BC + bc] * kLog2e, 0.f};
+}
+
+// One token within a chunk, one exp for both the output and the update.
+// State (a, b) is relative to the reference exponent r = R - n w (base 2, exact real;
+// the history decays by counting n), i.e. A = a 2^r.  With D = (u + k) - r, E = 2^-|D|:
+//   D <= 0 (history dominates): y = (a + E v)/(b + E); the new token's weight relative to
+//          the decayed reference r - w is 2^(k - r + w) = E * c with c = 2^(w - u), so
+//          a += E c v, b += E c, n += 1;
+//   D > 0  (token dominates):   y = (E a + v)/(E b + 1); re-reference to u + k:
+//          a = E a + c v, b = E b + c, R = u + k, n = 1.
+// Exact in real arithmetic; valid while c and its reciprocal stay far from the fp32
+// range limits (callers check |u|, w <= kLazyLimit).
+__device__ __forceinline__ float lazy_step(float& a, float& b, float& R, float& n, float k2, float v, float u2,
+                                           float w2, float c) {
+    const float r = fmaf(-n, w2, R);
+    const float uk = u2 + k2;
+    const float d = uk - r;
+    const float e = ex2(-fabsf(d));
+    const bool cur = d > 0.f;
+    const float sa = cur ? e : 1.f;
+    const float sv = cur ? 1.f : e;
+    const float t = sa * a;
+    const float y = fmaf(sv, v, t) * rcp(fmaf(sa, b, sv));
+    const float nw = sv * c;
+    a = fmaf(nw, v, t);
+    b = fmaf(sa, b, nw);
+    R = cur ? uk : R;
+    n = cur ? 1.f : n + 1.f;
+    return y;
+}
+constexpr float kLazyLimit = 40.f;  // base-2 units: c = 2^(w - u) within 2^(+-80)
+
+// ---------------------------------------------------------------------------
 // I/O element conversions
 // ---------------------------------------------------------------------------
 template <typename T>
@@ -240,6 +281,25 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Makes earlier relaxed loads acquire: later accesses see what their writers released.
+__device__ __forceinline__ void fence_acquire_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");

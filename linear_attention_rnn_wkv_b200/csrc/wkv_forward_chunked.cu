@@ -39,6 +39,7 @@
 // The last time segment's inclusive prefix is the final state (state_out).
 #include "wkv_device.cuh"
 #include "wkv_internal.h"
+#include "wkv_vec.cuh"
 
 // Tile shape per I/O type: V channels per lane (32 V per tile) and NW warps (chunks).
 #ifndef WKV_F32_V
@@ -57,81 +58,6 @@
 namespace wkvb {
 namespace {
 
-// ---- vector I/O of V adjacent channels (shared or global memory) ----
-template <typename TIO, int V>
-struct Vec;
-
-template <>
-struct Vec<float, 1> {
-    static __device__ __forceinline__ void load(const float* p, float (&o)[1]) { o[0] = *p; }
-    static __device__ __forceinline__ void store(float* p, const float (&o)[1]) { *p = o[0]; }
-};
-template <>
-struct Vec<float, 2> {
-    static __device__ __forceinline__ void load(const float* p, float (&o)[2]) {
-        float2 t = *reinterpret_cast<const float2*>(p);
-        o[0] = t.x; o[1] = t.y;
-    }
-    static __device__ __forceinline__ void store(float* p, const float (&o)[2]) {
-        *reinterpret_cast<float2*>(p) = make_float2(o[0], o[1]);
-    }
-};
-template <>
-struct Vec<float, 4> {
-    static __device__ __forceinline__ void load(const float* p, float (&o)[4]) {
-        float4 t = *reinterpret_cast<const float4*>(p);
-        o[0] = t.x; o[1] = t.y; o[2] = t.z; o[3] = t.w;
-    }
-    static __device__ __forceinline__ void store(float* p, const float (&o)[4]) {
-        *reinterpret_cast<float4*>(p) = make_float4(o[0], o[1], o[2], o[3]);
-    }
-};
-
-__device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
-__device__ __forceinline__ uint32_t bf_pack(float lo, float hi) {
-    __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&t);
-}
-
-template <>
-struct Vec<__nv_bfloat16, 1> {
-    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&o)[1]) { o[0] = __bfloat162float(*p); }
-    static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&o)[1]) { *p = __float2bfloat16_rn(o[0]); }
-};
-template <>
-struct Vec<__nv_bfloat16, 2> {
-    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&o)[2]) {
-        uint32_t t = *reinterpret_cast<const uint32_t*>(p);
-        o[0] = bf_lo(t); o[1] = bf_hi(t);
-    }
-    static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&o)[2]) {
-        *reinterpret_cast<uint32_t*>(p) = bf_pack(o[0], o[1]);
-    }
-};
-template <>
-struct Vec<__nv_bfloat16, 4> {
-    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&o)[4]) {
-        uint2 t = *reinterpret_cast<const uint2*>(p);
-        o[0] = bf_lo(t.x); o[1] = bf_hi(t.x); o[2] = bf_lo(t.y); o[3] = bf_hi(t.y);
-    }
-    static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&o)[4]) {
-        *reinterpret_cast<uint2*>(p) = make_uint2(bf_pack(o[0], o[1]), bf_pack(o[2], o[3]));
-    }
-};
-template <>
-struct Vec<__nv_bfloat16, 8> {
-    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&o)[8]) {
-        uint4 t = *reinterpret_cast<const uint4*>(p);
-        o[0] = bf_lo(t.x); o[1] = bf_hi(t.x); o[2] = bf_lo(t.y); o[3] = bf_hi(t.y);
-        o[4] = bf_lo(t.z); o[5] = bf_hi(t.z); o[6] = bf_lo(t.w); o[7] = bf_hi(t.w);
-    }
-    static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&o)[8]) {
-        *reinterpret_cast<uint4*>(p) = make_uint4(bf_pack(o[0], o[1]), bf_pack(o[2], o[3]), bf_pack(o[4], o[5]),
-                                                  bf_pack(o[6], o[7]));
-    }
-};
-
 struct ChunkParams {
     int64_t groups_per_b, G, S;
     uint32_t* flags;  // [U]
@@ -140,44 +66,6 @@ struct ChunkParams {
     WsHeader* hdr;
     int64_t drop_unit;
 };
-
-__device__ __forceinline__ float4 rec_pack(const Rec& r) { return make_float4(r.a, r.b, r.anc, r.n); }
-__device__ __forceinline__ Rec rec_unpack(const float4& f) { return Rec{f.x, f.y, f.z, f.w}; }
-
-// Natural-units state (a, b, p) -> anchored base-2 record.
-__device__ __forceinline__ Rec rec_from_state(const float* st, int64_t bc, int64_t BC) {
-    return Rec{st[bc], st[BC + bc], st[2 * BC + bc] * kLog2e, 0.f};
-}
-
-// One token within a chunk, one exp for both the output and the update.
-// State (a, b) is relative to the reference exponent r = R - n w (base 2, exact real;
-// the history decays by counting n), i.e. A = a 2^r.  With D = (u + k) - r, E = 2^-|D|:
-//   D <= 0 (history dominates): y = (a + E v)/(b + E); the new token's weight relative to
-//          the decayed reference r - w is 2^(k - r + w) = E * c with c = 2^(w - u), so
-//          a += E c v, b += E c, n += 1;
-//   D > 0  (token dominates):   y = (E a + v)/(E b + 1); re-reference to u + k:
-//          a = E a + c v, b = E b + c, R = u + k, n = 1.
-// Exact in real arithmetic; valid while c and its reciprocal stay far from the fp32
-// range limits (callers check |u|, w <= kLazyLimit).
-__device__ __forceinline__ float lazy_step(float& a, float& b, float& R, float& n, float k2, float v, float u2,
-                                           float w2, float c) {
-    const float r = fmaf(-n, w2, R);
-    const float uk = u2 + k2;
-    const float d = uk - r;
-    const float e = ex2(-fabsf(d));
-    const bool cur = d > 0.f;
-    const float sa = cur ? e : 1.f;
-    const float sv = cur ? 1.f : e;
-    const float t = sa * a;
-    const float y = fmaf(sv, v, t) * rcp(fmaf(sa, b, sv));
-    const float nw = sv * c;
-    a = fmaf(nw, v, t);
-    b = fmaf(sa, b, nw);
-    R = cur ? uk : R;
-    n = cur ? 1.f : n + 1.f;
-    return y;
-}
-constexpr float kLazyLimit = 40.f;  // base-2 units: c = 2^(w - u) within 2^(+-80)
 
 template <typename TIO, int V, int NW, int LC, bool BULK>
 __global__ void __launch_bounds__(NW * 32) chunked_kernel(ForwardArgs args, ChunkParams cp) {
@@ -578,10 +466,18 @@ cudaError_t launch_lc(const ForwardArgs& a, const ChunkGeom& g, const ChunkParam
 bool chunk_geometry(int64_t B, int64_t T, int64_t C, int io, int chunk, ChunkGeom* g) {
     const int esize = io == 1 ? 2 : 4;
     const bool bulk = ((C * esize) % 16) == 0;
-    const int LC = chunk == 0 ? 16 : chunk;
-    if (LC != 4 && LC != 8 && LC != 16) return false;
-    g->V = bulk ? (io == 1 ? WKV_BF16_V : WKV_F32_V) : 1;
-    g->NW = bulk ? (io == 1 ? WKV_BF16_NW : WKV_F32_NW) : 4;
+    if (chunk != 0 && chunk != 4 && chunk != 8 && chunk != 16) return false;
+    // bulk rows run the pipelined kernel (default 16 steps per chunk); chunk 4 and ragged
+    // rows run the one-unit-per-CTA kernel above
+    g->pipe = bulk && chunk != 4;
+    const int LC = chunk != 0 ? chunk : 16;
+    if (g->pipe) {
+        g->V = io == 1 ? 4 : 2;
+        g->NW = 8;
+    } else {
+        g->V = bulk ? (io == 1 ? WKV_BF16_V : WKV_F32_V) : 1;
+        g->NW = bulk ? (io == 1 ? WKV_BF16_NW : WKV_F32_NW) : 4;
+    }
     g->LC = LC;
     g->bulk = bulk;
     g->Cg = 32 * g->V;
@@ -590,13 +486,20 @@ bool chunk_geometry(int64_t B, int64_t T, int64_t C, int io, int chunk, ChunkGeo
     g->G = B * g->groups_per_b;
     g->S = (T + g->Ts - 1) / g->Ts;
     g->U = g->G * g->S;
-    const size_t flags = ((size_t)g->U * 4 + 15) / 16 * 16;
-    g->ws_bytes = kWsHeaderBytes + flags + 2 * (size_t)g->U * (size_t)g->Cg * 16;
+    if (g->pipe) {
+        // tagged four-word records, aggregate and inclusive prefix per tile-channel
+        g->ws_bytes = kWsHeaderBytes + 2 * (size_t)g->U * (size_t)g->Cg * 32;
+    } else {
+        // flag per tile, 16-byte aggregate and inclusive records per tile-channel
+        const size_t flags = ((size_t)g->U * 4 + 15) / 16 * 16;
+        g->ws_bytes = kWsHeaderBytes + flags + 2 * (size_t)g->U * (size_t)g->Cg * 16;
+    }
     return true;
 }
 
 cudaError_t launch_forward_chunked(const ForwardArgs& a, const ChunkGeom& g, void* ws, int64_t drop_unit,
                                    cudaStream_t s) {
+    if (g.pipe) return launch_forward_pipe(a, g, ws, drop_unit, s);
     unsigned char* base = static_cast<unsigned char*>(ws);
     const size_t flags_bytes = ((size_t)g.U * 4 + 15) / 16 * 16;
     ChunkParams cp;

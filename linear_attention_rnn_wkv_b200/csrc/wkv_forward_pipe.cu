@@ -1,0 +1,585 @@
+// Persistent, warp-specialised chunked WKV forward (the default chunked path when
+// rows are 16-byte multiples).
+//
+// Same arithmetic and the same inter-CTA protocol as chunked_kernel (wkv_forward_
+// chunked.cu): a unit is a tile of Ts = NWS * LC time steps by Cg = 32 * V channels;
+// units are taken by an atomic ticket in time-segment-major order; each unit's chunk
+// summaries fold into a tile aggregate, a decoupled look-back over earlier segments of
+// the same channel group yields the carry, and the chunks are re-scanned from the
+// carry to write y (the decay telescopes: RWKV transformer-math page, aicassindra.com,
+// section "Why it collapses into a recurrence").
+//
+// What changes is the schedule.  One CTA per SM runs for the whole launch and keeps
+// NS units in flight in a shared-memory ring; each role is a set of warps that moves
+// from unit to unit on its own, handing over through mbarriers:
+//   producer  (1 warp)   takes the next ticket, announces the unit (`tick`), and
+//                        issues the TMA bulk copies of its k and v rows (`full`);
+//   summarise (NWS warps) chunk summaries, the in-tile scan, the aggregate record
+//                        published for other CTAs (`summ`);
+//   look-back (1 warp)   starts as soon as the unit is announced, while its rows are
+//                        still loading: folds the predecessors' records into the carry,
+//                        then combines it with the aggregate and publishes the
+//                        inclusive prefix (`carry`);
+//   emit      (NWS warps) re-scan each chunk from its carry and write y, then free the
+//                        stage (`empty`) for the producer.
+// So a unit's load, its look-back and the arithmetic of neighbouring units overlap,
+// and no warp waits at a CTA-wide barrier.  All waits are bounded (error word on
+// expiry, then the pipeline keeps moving).  Deadlock freedom: roles handle a CTA's units
+// in ticket order and every cross-CTA wait is on a smaller ticket, so the oldest
+// unfinished unit in the whole grid can always complete.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "wkv_device.cuh"
+#include "wkv_internal.h"
+#include "wkv_vec.cuh"
+
+// Rows per TMA box (a tile of Ts rows is fetched as Ts / kBoxRows boxes per array).
+#ifndef WKV_PIPE_BOXR
+#define WKV_PIPE_BOXR 32
+#endif
+
+namespace wkvb {
+namespace {
+
+constexpr int kBoxRows = WKV_PIPE_BOXR;
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Bounded wait on an mbarrier phase; returns false if it ran out.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
+    for (uint32_t it = 0; !mbar_try_wait(bar, parity); ++it) {
+        if (it >= limit) return false;
+        __nanosleep(32);
+    }
+    return true;
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* tm, int x, int y, int z, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+            smem_u32(dst)),
+        "l"(tm), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+struct PipeParams {
+    int64_t groups_per_b, G, S, U;
+    uint64_t* agg;      // [U][Cg][4] tagged words: a tile's aggregate
+    uint64_t* incl;     // [U][Cg][4] tagged words: its inclusive prefix
+    WsHeader* hdr;
+    int64_t drop_unit;  // test hook: this unit never publishes its records (-1: none)
+};
+
+// A published record is four 64-bit words, (a | tag), (b | tag), (anc | tag), (n | tag):
+// the value's bits in the low half, the launch epoch and the record kind in the high
+// half.  Aligned 64-bit accesses are single-copy atomic, so a reader that finds the
+// expected tag in all four words holds one consistent record; nothing else has to be
+// ordered, so neither side needs a fence or a separate flag.  The anchored exponent
+// (anc, n) travels unrounded.
+__device__ __forceinline__ void publish_rec(uint64_t* dst, const Rec& r, uint32_t tag) {
+    const uint64_t t = (uint64_t)tag << 32;
+    st_relaxed_u64(dst + 0, t | __float_as_uint(r.a));
+    st_relaxed_u64(dst + 1, t | __float_as_uint(r.b));
+    st_relaxed_u64(dst + 2, t | __float_as_uint(r.anc));
+    st_relaxed_u64(dst + 3, t | __float_as_uint(r.n));
+}
+
+__device__ __forceinline__ bool read_rec(const uint64_t* src, uint32_t tag, Rec& out) {
+    const uint64_t w0 = ld_relaxed_u64(src + 0);
+    const uint64_t w1 = ld_relaxed_u64(src + 1);
+    const uint64_t w2 = ld_relaxed_u64(src + 2);
+    const uint64_t w3 = ld_relaxed_u64(src + 3);
+    if ((uint32_t)(w0 >> 32) != tag || (uint32_t)(w1 >> 32) != tag || (uint32_t)(w2 >> 32) != tag ||
+        (uint32_t)(w3 >> 32) != tag)
+        return false;
+    out = Rec{__uint_as_float((uint32_t)w0), __uint_as_float((uint32_t)w1), __uint_as_float((uint32_t)w2),
+              __uint_as_float((uint32_t)w3)};
+    return true;
+}
+
+constexpr size_t align128(size_t x) { return (x + 127) / 128 * 128; }
+
+template <typename TIO, int V, int NWS, int LC, int NS>
+struct PipeLayout {
+    static constexpr int Cg = 32 * V;
+    static constexpr int Ts = NWS * LC;
+    static constexpr size_t tile = sizeof(TIO) * Ts * Cg;  // one array (k or v)
+    static constexpr size_t recs_off = 2 * tile;           // Rec [NWS][Cg]
+    static constexpr size_t carry_off = recs_off + sizeof(Rec) * NWS * Cg;
+    static constexpr size_t stage = align128(carry_off + sizeof(Rec) * Cg);
+    static constexpr size_t bars_off = NS * stage;           // 5 mbarriers per stage
+    static constexpr size_t misc_off = bars_off + NS * 5 * 8;  // stage unit ids, epoch, end index
+    static constexpr size_t total = misc_off + NS * 8 + 24;
+};
+
+enum { kFull = 0, kTick = 1, kChunks = 2, kCarry = 3, kEmpty = 4 };
+
+template <typename TIO, int V, int NWS, int LC, int NS>
+__global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
+    pipe_kernel(ForwardArgs args, PipeParams pp, const __grid_constant__ CUtensorMap tmk,
+                const __grid_constant__ CUtensorMap tmv) {
+    using Lay = PipeLayout<TIO, V, NWS, LC, NS>;
+    constexpr int Cg = Lay::Cg;
+    constexpr int Ts = Lay::Ts;
+    constexpr int W_S0 = 1, W_L0 = 1 + NWS, W_E0 = 1 + NWS + NS;
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bars_off);
+    int64_t* stage_unit = reinterpret_cast<int64_t*>(smem + Lay::misc_off);
+    uint32_t* s_epoch = reinterpret_cast<uint32_t*>(stage_unit + NS);
+    volatile int64_t* s_iend = reinterpret_cast<volatile int64_t*>(stage_unit + NS + 1);
+    auto bar = [&](int s, int kind) { return &bars[s * 5 + kind]; };
+    auto ktile = [&](int s) { return reinterpret_cast<TIO*>(smem + s * Lay::stage); };
+    auto vtile = [&](int s) { return reinterpret_cast<TIO*>(smem + s * Lay::stage + Lay::tile); };
+    auto recs = [&](int s) { return reinterpret_cast<Rec*>(smem + s * Lay::stage + Lay::recs_off); };
+    auto carries = [&](int s) { return reinterpret_cast<Rec*>(smem + s * Lay::stage + Lay::carry_off); };
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int64_t T = args.T, C = args.C, BC = args.B * args.C;
+    const uint32_t lim = args.spin_limit;
+
+    if (tid == 0) {
+        *s_epoch = (*reinterpret_cast<volatile uint32_t*>(&pp.hdr->epoch) + 1u) & 0x3FFFFFFFu;
+        *s_iend = INT64_MAX;
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(bar(s, kFull), 1);
+            mbar_init(bar(s, kTick), 1);
+            mbar_init(bar(s, kChunks), NWS);
+            mbar_init(bar(s, kCarry), 1);
+            mbar_init(bar(s, kEmpty), NWS);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const uint32_t epoch30 = *s_epoch;
+    const uint32_t tag_agg = (epoch30 << 2) | 1u, tag_incl = (epoch30 << 2) | 2u;
+    auto report = [&](uint32_t code) { atomicCAS(&pp.hdr->error, kDevOk, code); };
+
+    struct Geo {
+        int64_t j, g, b, c0, t0;
+        int len, nch;
+    };
+    auto geo = [&](int64_t unit) {
+        Geo q;
+        q.j = unit / pp.G;
+        q.g = unit % pp.G;
+        q.b = q.g / pp.groups_per_b;
+        q.c0 = (q.g % pp.groups_per_b) * Cg;
+        q.t0 = q.j * Ts;
+        q.len = (int)min64(Ts, T - q.t0);
+        q.nch = (int)min64(Cg, C - q.c0);
+        return q;
+    };
+
+    if (warp == 0) {
+        // ------------------------------- producer -------------------------------
+        if (lane == 0) {
+            for (int64_t i = 0;; ++i) {
+                const int s = (int)(i % NS);
+                if (i >= NS && !mbar_wait(bar(s, kEmpty), (uint32_t)((i / NS - 1) & 1), lim)) report(kDevTimeoutCopy);
+                const uint32_t t = atomicAdd(&pp.hdr->ticket, 1u);
+                if (t >= (uint32_t)pp.U + gridDim.x) report(kDevBadWorkspace);
+                if (t >= (uint32_t)pp.U) {
+                    *s_iend = i;
+                    stage_unit[s] = -1;
+                    mbar_arrive(bar(s, kTick));
+                    mbar_arrive(bar(s, kFull));
+                    break;
+                }
+                const int64_t unit = t;
+                stage_unit[s] = unit;
+                mbar_arrive(bar(s, kTick));
+                const Geo q = geo(unit);
+                constexpr int BR = kBoxRows < Ts ? kBoxRows : Ts;
+                mbar_arrive_expect_tx(bar(s, kFull), 2u * (uint32_t)(Ts * Cg * sizeof(TIO)));
+#pragma unroll
+                for (int r0 = 0; r0 < Ts; r0 += BR) {
+                    tma_load_3d(ktile(s) + r0 * Cg, &tmk, (int)q.c0, (int)(q.t0 + r0), (int)q.b, bar(s, kFull));
+                    tma_load_3d(vtile(s) + r0 * Cg, &tmv, (int)q.c0, (int)(q.t0 + r0), (int)q.b, bar(s, kFull));
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp < W_L0) {
+        // ------------------------------- summarise ------------------------------
+        // Every warp summarises its own chunk of the tile and signals the stage.
+        const int sw = warp - W_S0;
+        for (int64_t i = 0;; ++i) {
+            const int s = (int)(i % NS);
+            const uint32_t ph = (uint32_t)((i / NS) & 1);
+            if (!mbar_wait(bar(s, kFull), ph, lim) && lane == 0) report(kDevTimeoutCopy);
+            const int64_t unit = stage_unit[s];
+            if (unit < 0) break;
+            const Geo q = geo(unit);
+            const int cl = lane * V;
+            const bool lane_active = cl < q.nch;
+            const int r_begin = sw * LC;
+            const int r_cnt = max(0, min(LC, q.len - r_begin));
+            float w2[V];
+#pragma unroll
+            for (int c = 0; c < V; ++c) w2[c] = (lane_active && cl + c < q.nch) ? args.w[q.c0 + cl + c] * kLog2e : 0.f;
+            if (lane_active) {
+                float gx[LC][V], M[V], sa[V], sb[V];
+#pragma unroll
+                for (int c = 0; c < V; ++c) {
+                    M[c] = kPEmpty;
+                    sa[c] = sb[c] = 0.f;
+                }
+                const TIO* kt = ktile(s);
+                const TIO* vt = vtile(s);
+#pragma unroll
+                for (int r = 0; r < LC; ++r) {
+                    if (r < r_cnt) {
+                        float kk[V];
+                        Vec<TIO, V>::load(kt + (r_begin + r) * Cg + cl, kk);
+                        const float back = (float)(r_cnt - 1 - r);
+#pragma unroll
+                        for (int c = 0; c < V; ++c) {
+                            gx[r][c] = fmaf(-back, w2[c], kk[c] * kLog2e);
+                            M[c] = fmaxf(M[c], gx[r][c]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < LC; ++r) {
+                    if (r < r_cnt) {
+                        float vv[V];
+                        Vec<TIO, V>::load(vt + (r_begin + r) * Cg + cl, vv);
+#pragma unroll
+                        for (int c = 0; c < V; ++c) {
+                            const float e = ex2(gx[r][c] - M[c]);
+                            sa[c] = fmaf(e, vv[c], sa[c]);
+                            sb[c] += e;
+                        }
+                    }
+                }
+                Rec* rc = recs(s);
+#pragma unroll
+                for (int c = 0; c < V; ++c) rc[sw * Cg + cl + c] = Rec{sa[c], sb[c], M[c], 0.f};
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(s, kChunks));
+        }
+    } else if (warp < W_E0) {
+        // ------------------------------- look-back ------------------------------
+        // Look-back warp l owns ring stage l: units i = l, l + NS, ...
+        const int s = warp - W_L0;
+        for (int64_t i = s;; i += NS) {
+            const uint32_t ph = (uint32_t)((i / NS) & 1);
+            bool got = false, gone = false;
+            for (uint32_t it = 0; it <= lim; ++it) {
+                if (mbar_try_wait(bar(s, kTick), ph)) {
+                    got = true;
+                    break;
+                }
+                if (*s_iend < i) {  // past the end (the sentinel unit itself still arrives)
+                    gone = true;
+                    break;
+                }
+                __nanosleep(32);
+            }
+            if (gone) break;
+            if (!got && lane == 0) report(kDevTimeoutCopy);
+            const int64_t unit = stage_unit[s];
+            if (unit < 0) {
+                if (lane == 0) mbar_arrive(bar(s, kCarry));
+                break;
+            }
+            const Geo q = geo(unit);
+            const int cl = lane * V;
+            const bool lane_active = cl < q.nch;
+            float w2[V];
+#pragma unroll
+            for (int c = 0; c < V; ++c) w2[c] = (lane_active && cl + c < q.nch) ? args.w[q.c0 + cl + c] * kLog2e : 0.f;
+            // scan the chunk summaries (exclusive prefixes for the emitters) and publish the
+            // tile aggregate for later segments before looking back
+            if (!mbar_wait(bar(s, kChunks), ph, lim) && lane == 0) report(kDevTimeoutCarry);
+            Rec agg[V];
+            if (lane_active) {
+                Rec* rc = recs(s);
+#pragma unroll
+                for (int c = 0; c < V; ++c) agg[c] = rec_identity();
+#pragma unroll
+                for (int w = 0; w < NWS; ++w) {
+                    const int lw = max(0, min(LC, q.len - w * LC));
+#pragma unroll
+                    for (int c = 0; c < V; ++c) {
+                        const Rec r = rc[w * Cg + cl + c];
+                        rc[w * Cg + cl + c] = agg[c];  // exclusive prefix of chunk w
+                        if (lw > 0) agg[c] = rec_combine(agg[c], r, (float)lw, w2[c]);
+                    }
+                }
+                if (q.j > 0 && unit != pp.drop_unit) {
+#pragma unroll
+                    for (int c = 0; c < V; ++c)
+                        if (cl + c < q.nch) publish_rec(pp.agg + (unit * Cg + cl + c) * 4, agg[c], tag_agg);
+                }
+            }
+            Rec run[V];
+            if (q.j == 0) {
+#pragma unroll
+                for (int c = 0; c < V; ++c) {
+                    const int cc = cl + c;
+                    run[c] = (args.state_in && cc < q.nch) ? rec_from_state(args.state_in, q.b * C + q.c0 + cc, BC)
+                                                           : rec_identity();
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < V; ++c) run[c] = rec_identity();
+                // Each lane looks back for its own channels: fold the newest predecessor's
+                // inclusive prefix if it is there, else its aggregate and step further back;
+                // back off while neither has been published.
+                float span[V];
+                int64_t hi[V];
+                bool done[V];
+#pragma unroll
+                for (int c = 0; c < V; ++c) {
+                    span[c] = 0.f;
+                    hi[c] = q.j - 1;
+                    done[c] = !(lane_active && cl + c < q.nch);
+                }
+                uint32_t nap = 64;
+                bool all_done = false;
+                for (uint32_t it = 0; it <= lim && !all_done; ++it) {
+                    bool progressed = false;
+                    all_done = true;
+#pragma unroll
+                    for (int c = 0; c < V; ++c) {
+                        if (done[c]) continue;
+                        const int64_t off = ((hi[c] * pp.G + q.g) * Cg + cl + c) * 4;
+                        Rec r;
+                        if (read_rec(pp.incl + off, tag_incl, r)) {
+                            run[c] = rec_combine(r, run[c], span[c], w2[c]);
+                            done[c] = true;
+                            progressed = true;
+                        } else if (read_rec(pp.agg + off, tag_agg, r)) {
+                            run[c] = rec_combine(r, run[c], span[c], w2[c]);
+                            span[c] += (float)Ts;
+                            progressed = true;
+                            if (--hi[c] < 0) done[c] = true;
+                        }
+                        all_done = all_done && done[c];
+                    }
+                    if (!all_done && !progressed) {
+                        __nanosleep(nap);
+                        nap = nap < 1024 ? nap * 2 : 1024;
+                    } else if (progressed) {
+                        nap = 64;
+                    }
+                }
+                if (!all_done) {
+                    report(kDevTimeoutCarry);
+                    pp.hdr->error_unit = (uint32_t)unit;
+                }
+            }
+            // hand the carry to the emitters first, then publish the inclusive prefix
+            Rec inc[V];
+            if (lane_active) {
+                Rec* cs = carries(s);
+#pragma unroll
+                for (int c = 0; c < V; ++c) {
+                    inc[c] = rec_combine(run[c], agg[c], (float)q.len, w2[c]);
+                    cs[cl + c] = run[c];
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(s, kCarry));
+            if (lane_active) {
+#pragma unroll
+                for (int c = 0; c < V; ++c) {
+                    if (cl + c < q.nch) {
+                        if (unit != pp.drop_unit) publish_rec(pp.incl + (unit * Cg + cl + c) * 4, inc[c], tag_incl);
+                        if (q.j == pp.S - 1 && args.state_out) {
+                            const int64_t bc = q.b * C + q.c0 + cl + c;
+                            args.state_out[bc] = inc[c].a;
+                            args.state_out[BC + bc] = inc[c].b;
+                            args.state_out[2 * BC + bc] = rec_p(inc[c], w2[c]) * kLn2;
+                        }
+                    }
+                }
+            }
+        }
+    } else {
+        // --------------------------------- emit ---------------------------------
+        const int ew = warp - W_E0;  // chunk index
+        for (int64_t i = 0;; ++i) {
+            const int s = (int)(i % NS);
+            const uint32_t ph = (uint32_t)((i / NS) & 1);
+            if (!mbar_wait(bar(s, kCarry), ph, lim) && lane == 0) report(kDevTimeoutCarry);
+            (void)mbar_wait(bar(s, kFull), ph, lim);  // already complete; orders the tile reads
+            const int64_t unit = stage_unit[s];
+            if (unit < 0) break;
+            const Geo q = geo(unit);
+            const int cl = lane * V;
+            const int r_begin = ew * LC;
+            const int r_cnt = max(0, min(LC, q.len - r_begin));
+            if (cl < q.nch && r_cnt > 0) {
+                float w2[V], u2[V], a[V], bb[V], R[V], nn[V];
+                bool lazy_ok = true;
+#pragma unroll
+                for (int c = 0; c < V; ++c) {
+                    const bool ok = cl + c < q.nch;
+                    w2[c] = ok ? args.w[q.c0 + cl + c] * kLog2e : 0.f;
+                    u2[c] = ok ? args.u[q.c0 + cl + c] * kLog2e : 0.f;
+                    const Rec cr = rec_combine(carries(s)[cl + c], recs(s)[ew * Cg + cl + c], (float)r_begin, w2[c]);
+                    a[c] = cr.a;
+                    bb[c] = cr.b;
+                    R[c] = cr.anc;
+                    nn[c] = cr.n;
+                    lazy_ok = lazy_ok && fabsf(u2[c]) <= kLazyLimit && w2[c] <= kLazyLimit;
+                }
+                const TIO* kt = ktile(s);
+                const TIO* vt = vtile(s);
+                TIO* yg = static_cast<TIO*>(args.y) + (q.b * T + q.t0) * C + q.c0;
+                if (lazy_ok) {
+                    float cw[V];
+#pragma unroll
+                    for (int c = 0; c < V; ++c) cw[c] = ex2(w2[c] - u2[c]);
+#pragma unroll
+                    for (int r = 0; r < LC; ++r) {
+                        if (r < r_cnt) {
+                            const int row = r_begin + r;
+                            float kk[V], vv[V], yy[V];
+                            Vec<TIO, V>::load(kt + row * Cg + cl, kk);
+                            Vec<TIO, V>::load(vt + row * Cg + cl, vv);
+#pragma unroll
+                            for (int c = 0; c < V; ++c)
+                                yy[c] = lazy_step(a[c], bb[c], R[c], nn[c], kk[c] * kLog2e, vv[c], u2[c], w2[c], cw[c]);
+                            Vec<TIO, V>::store(yg + (int64_t)row * C + cl, yy);
+                        }
+                    }
+                } else {
+                    float p[V];
+#pragma unroll
+                    for (int c = 0; c < V; ++c) p[c] = fmaf(-nn[c], w2[c], R[c]);
+                    for (int r = 0; r < r_cnt; ++r) {
+                        const int row = r_begin + r;
+                        float kk[V], vv[V], yy[V];
+                        Vec<TIO, V>::load(kt + row * Cg + cl, kk);
+                        Vec<TIO, V>::load(vt + row * Cg + cl, vv);
+#pragma unroll
+                        for (int c = 0; c < V; ++c) {
+                            const float k2 = kk[c] * kLog2e;
+                            yy[c] = wkv_output<false>(a[c], bb[c], p[c], u2[c] + k2, vv[c]);
+                            wkv_fold<false>(a[c], bb[c], p[c], p[c] - w2[c], k2, vv[c], w2[c]);
+                        }
+                        Vec<TIO, V>::store(yg + (int64_t)row * C + cl, yy);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(s, kEmpty));
+        }
+    }
+
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const uint32_t finished = atomicAdd(&pp.hdr->done, 1u) + 1u;
+        if (finished == gridDim.x) {
+            atomicExch(&pp.hdr->ticket, 0u);
+            atomicExch(&pp.hdr->done, 0u);
+            atomicExch(&pp.hdr->epoch, epoch30);
+        }
+    }
+}
+
+// Tensor maps for k and v viewed as [B][T][C] (3-D, channels innermost), box = one tile.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+bool make_tile_map(CUtensorMap* tm, const void* base, int64_t B, int64_t T, int64_t C, int io, int Cg, int Ts) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t es = io == 1 ? 2 : 4;
+    cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[2] = {(cuuint64_t)C * es, (cuuint64_t)T * (cuuint64_t)C * es};
+    cuuint32_t box[3] = {(cuuint32_t)Cg, (cuuint32_t)Ts, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(tm, io == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+                          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <typename TIO, int V, int NWS, int LC>
+cudaError_t launch_pipe_t(const ForwardArgs& a, const ChunkGeom& g, const PipeParams& pp, cudaStream_t s) {
+    // as many stages as fit in the 227 KB a CTA may use (at most 5)
+    constexpr size_t stage = PipeLayout<TIO, V, NWS, LC, 1>::stage;
+    constexpr size_t budget = 232448 - 512;
+    constexpr int NS = (int)(budget / (stage + 64) > 5 ? 5 : budget / (stage + 64));
+    static_assert(NS >= 2, "tile too large for a two-stage ring");
+    using Lay = PipeLayout<TIO, V, NWS, LC, NS>;
+    auto kern = pipe_kernel<TIO, V, NWS, LC, NS>;
+    CUtensorMap tmk, tmv;
+    constexpr int BR = kBoxRows < Lay::Ts ? kBoxRows : Lay::Ts;
+    static_assert(Lay::Ts % BR == 0, "tile rows must be a multiple of the box rows");
+    if (!make_tile_map(&tmk, a.k, a.B, a.T, a.C, a.io, Lay::Cg, BR) ||
+        !make_tile_map(&tmv, a.v, a.B, a.T, a.C, a.io, Lay::Cg, BR))
+        return cudaErrorInvalidValue;
+    static uint64_t attr_done = 0;  // per device; set once so captured launches issue no attribute call
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static int sms[64] = {0};
+    if (dev >= 64 || !(attr_done & (1ull << dev))) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::total);
+        if (e != cudaSuccess) return e;
+        int n = 0;
+        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) {
+            sms[dev] = n;
+            attr_done |= 1ull << dev;
+        }
+    }
+    const int64_t nsm = dev < 64 ? sms[dev] : 148;
+    const int64_t grid = g.U < nsm ? g.U : nsm;
+    kern<<<(unsigned)grid, (1 + 2 * NWS + NS) * 32, Lay::total, s>>>(a, pp, tmk, tmv);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_forward_pipe(const ForwardArgs& a, const ChunkGeom& g, void* ws, int64_t drop_unit,
+                                cudaStream_t s) {
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    PipeParams pp;
+    pp.groups_per_b = g.groups_per_b;
+    pp.G = g.G;
+    pp.S = g.S;
+    pp.U = g.U;
+    pp.hdr = reinterpret_cast<WsHeader*>(base);
+    pp.agg = reinterpret_cast<uint64_t*>(base + kWsHeaderBytes);
+    pp.incl = pp.agg + (size_t)g.U * (size_t)g.Cg * 4;
+    pp.drop_unit = drop_unit;
+    if (a.io == 1) {
+        if (g.V == 4 && g.NW == 8 && g.LC == 8) return launch_pipe_t<__nv_bfloat16, 4, 8, 8>(a, g, pp, s);
+        if (g.V == 4 && g.NW == 8 && g.LC == 16) return launch_pipe_t<__nv_bfloat16, 4, 8, 16>(a, g, pp, s);
+        return cudaErrorInvalidValue;
+    }
+    if (g.V == 2 && g.NW == 8 && g.LC == 8) return launch_pipe_t<float, 2, 8, 8>(a, g, pp, s);
+    if (g.V == 2 && g.NW == 8 && g.LC == 16) return launch_pipe_t<float, 2, 8, 16>(a, g, pp, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace wkvb

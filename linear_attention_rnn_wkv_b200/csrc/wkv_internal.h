@@ -36,6 +36,7 @@ struct ChunkGeom {
     int NW;       // warps per CTA (= chunks per tile)
     int LC;       // time steps per chunk
     bool bulk;    // rows copied with cp.async.bulk
+    bool pipe;    // persistent warp-specialised kernel (wkv_forward_pipe.cu)
     int64_t Cg;   // channels per tile (32 * V)
     int64_t Ts;   // time steps per tile (NW * LC)
     int64_t groups_per_b;
@@ -65,6 +66,10 @@ struct WsHeader {
 // so a launch captured in a CUDA graph stays correct on every replay).
 cudaError_t launch_forward_chunked(const ForwardArgs& a, const ChunkGeom& g, void* ws, int64_t drop_unit,
                                    cudaStream_t s);
+
+// Persistent warp-specialised variant (bulk rows, chunk 8 or 16); same workspace layout.
+cudaError_t launch_forward_pipe(const ForwardArgs& a, const ChunkGeom& g, void* ws, int64_t drop_unit,
+                                cudaStream_t s);
 
 // ----- T == 0: state_out = state_in (or the empty state) -----
 cudaError_t launch_state_passthrough(int64_t BC, const float* state_in, float* state_out, cudaStream_t s);

@@ -80,7 +80,7 @@ def test_workspace_size_query():
         # header + a flag per tile + two 16-byte records per channel per tile; tiles span
         # 16 to 128 time steps and up to 128 channels (rounded up), so the size lies between
         lo = 64 + 2 * 16 * B * C * ((T + 127) // 128)
-        hi = 64 + 16 + (4 + 2 * 16 * 128) * B * (C + 31) // 32 * ((T + 15) // 16)
+        hi = 64 + 16 + (4 + 2 * 32 * 128) * B * (C + 31) // 32 * ((T + 15) // 16)
         assert lo <= n <= hi, (n, lo, hi)
     assert wkv.lib().wkv_forward_workspace_size(0, 10, 10, 0) == 64
 
