@@ -298,6 +298,16 @@ __device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
     asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
+// Two adjacent 64-bit words in one 16-byte access (p 16-byte aligned); each word is its
+// own single-copy-atomic element, the pair is not.
+__device__ __forceinline__ void ld_relaxed_v2u64(const uint64_t* p, uint64_t& x, uint64_t& y) {
+    asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(x), "=l"(y) : "l"(p) : "memory");
+}
+
+__device__ __forceinline__ void st_relaxed_v2u64(uint64_t* p, uint64_t x, uint64_t y) {
+    asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(x), "l"(y) : "memory");
+}
+
 // Makes earlier relaxed loads acquire: later accesses see what their writers released.
 __device__ __forceinline__ void fence_acquire_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 

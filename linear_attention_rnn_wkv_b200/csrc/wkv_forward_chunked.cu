@@ -472,7 +472,7 @@ bool chunk_geometry(int64_t B, int64_t T, int64_t C, int io, int chunk, ChunkGeo
     g->pipe = bulk && chunk != 4;
     const int LC = chunk != 0 ? chunk : 16;
     if (g->pipe) {
-        g->V = io == 1 ? 4 : 2;
+        g->V = 2;  // a lane owns a channel pair: 64 channels per tile (256-byte fp32 / 128-byte bf16 rows)
         g->NW = 8;
     } else {
         g->V = bulk ? (io == 1 ? WKV_BF16_V : WKV_F32_V) : 1;
@@ -487,8 +487,8 @@ bool chunk_geometry(int64_t B, int64_t T, int64_t C, int io, int chunk, ChunkGeo
     g->S = (T + g->Ts - 1) / g->Ts;
     g->U = g->G * g->S;
     if (g->pipe) {
-        // tagged four-word records, aggregate and inclusive prefix per tile-channel
-        g->ws_bytes = kWsHeaderBytes + 2 * (size_t)g->U * (size_t)g->Cg * 32;
+        // one slot of four tagged words per tile-channel (aggregate, then inclusive prefix)
+        g->ws_bytes = kWsHeaderBytes + (size_t)g->U * (size_t)g->Cg * 32;
     } else {
         // flag per tile, 16-byte aggregate and inclusive records per tile-channel
         const size_t flags = ((size_t)g->U * 4 + 15) / 16 * 16;

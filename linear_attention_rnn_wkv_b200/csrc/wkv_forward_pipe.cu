@@ -12,14 +12,15 @@
 // What changes is the schedule.  One CTA per SM runs for the whole launch and keeps
 // NS units in flight in a shared-memory ring; each role is a set of warps that moves
 // from unit to unit on its own, handing over through mbarriers:
-//   producer  (1 warp)   takes the next ticket, announces the unit (`tick`), and
-//                        issues the TMA bulk copies of its k and v rows (`full`);
-//   summarise (NWS warps) chunk summaries, the in-tile scan, the aggregate record
-//                        published for other CTAs (`summ`);
-//   look-back (1 warp)   starts as soon as the unit is announced, while its rows are
-//                        still loading: folds the predecessors' records into the carry,
-//                        then combines it with the aggregate and publishes the
-//                        inclusive prefix (`carry`);
+//   producer  (1 warp)   announces the unit of its (prefetched) ticket (`tick`), and
+//                        issues the TMA copies of its k and v rows and of its channels'
+//                        w and u (`full`);
+//   summarise (NWS warps) one chunk summary each (`chunks`);
+//   look-back (NS warps, one per ring stage) starts as soon as the unit is announced,
+//                        while its rows are still loading: folds the predecessors'
+//                        records into the carry; once the summaries are in, scans them
+//                        and publishes the tile aggregate (or, if the carry is already
+//                        known, the inclusive prefix); hands the carry over (`carry`);
 //   emit      (NWS warps) re-scan each chunk from its carry and write y, then free the
 //                        stage (`empty`) for the producer.
 // So a unit's load, its look-back and the arithmetic of neighbouring units overlap,
@@ -33,6 +34,31 @@
 #include "wkv_device.cuh"
 #include "wkv_internal.h"
 #include "wkv_vec.cuh"
+
+// Per-unit event trace (profiling builds only): compiled with -DWKV_TRACE, the kernel
+// stamps %globaltimer at each hand-over of every unit into the buffer registered with
+// wkv_trace_set_buffer ([units][11] u64: events 0..9 below, slot 10 the SM id).  Normal
+// builds define the hooks away.
+#ifdef WKV_TRACE
+__device__ unsigned long long* g_wkv_trace = nullptr;
+extern "C" cudaError_t wkv_trace_set_buffer(void* p) { return cudaMemcpyToSymbol(g_wkv_trace, &p, sizeof(p)); }
+__device__ __forceinline__ void wkv_trace(int64_t unit, int ev) {
+    if (!g_wkv_trace) return;
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    g_wkv_trace[unit * 11 + ev] = t;
+    if (ev == 0) {
+        unsigned sm;
+        asm volatile("mov.u32 %0, %smid;" : "=r"(sm));
+        g_wkv_trace[unit * 11 + 10] = sm;
+    }
+}
+#define WKV_TRACE_EVENT(unit, ev) wkv_trace(unit, ev)
+#else
+#define WKV_TRACE_EVENT(unit, ev) ((void)0)
+#endif
+// events: 0 ticket, 1 tile loaded, 2 chunks summarised, 3 look-back start, 4 summaries
+// scanned, 5 carry known, 6 carry handed over, 7 records published, 8 emit start, 9 emit end
 
 // Rows per TMA box (a tile of Ts rows is fetched as Ts / kBoxRows boxes per array).
 #ifndef WKV_PIPE_BOXR
@@ -71,38 +97,72 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* tm, in
 
 struct PipeParams {
     int64_t groups_per_b, G, S, U;
-    uint64_t* agg;      // [U][Cg][4] tagged words: a tile's aggregate
-    uint64_t* incl;     // [U][Cg][4] tagged words: its inclusive prefix
+    uint64_t* slot;     // [U][Cg][4] tagged words: a tile's aggregate, later its inclusive prefix
     WsHeader* hdr;
     int64_t drop_unit;  // test hook: this unit never publishes its records (-1: none)
 };
 
 // A published record is four 64-bit words, (a | tag), (b | tag), (anc | tag), (n | tag):
 // the value's bits in the low half, the launch epoch and the record kind in the high
-// half.  Aligned 64-bit accesses are single-copy atomic, so a reader that finds the
-// expected tag in all four words holds one consistent record; nothing else has to be
-// ordered, so neither side needs a fence or a separate flag.  The anchored exponent
-// (anc, n) travels unrounded.
-__device__ __forceinline__ void publish_rec(uint64_t* dst, const Rec& r, uint32_t tag) {
-    const uint64_t t = (uint64_t)tag << 32;
-    st_relaxed_u64(dst + 0, t | __float_as_uint(r.a));
-    st_relaxed_u64(dst + 1, t | __float_as_uint(r.b));
-    st_relaxed_u64(dst + 2, t | __float_as_uint(r.anc));
-    st_relaxed_u64(dst + 3, t | __float_as_uint(r.n));
+// half.  Aligned 64-bit accesses are single-copy atomic, so a reader that finds one tag
+// in all four words holds one consistent record; nothing else has to be ordered, so
+// neither side needs a fence or a separate flag.  The anchored exponent (anc, n) travels
+// unrounded.  Each tile has one slot per channel: the tile's aggregate is published there
+// first and later overwritten by its inclusive prefix (same thread, so every word takes
+// the second value after the first); a reader that catches the overwrite half done sees
+// mixed tags and reads again.  A tile's slots are stored word-major, [4][Cg] words, so a
+// lane moves the same word of its two channels with one 16-byte access and a warp's
+// access is contiguous.
+__device__ __forceinline__ uint64_t tagged(uint32_t tag, float x) { return ((uint64_t)tag << 32) | __float_as_uint(x); }
+
+template <int Cg>
+__device__ __forceinline__ void publish_pair(uint64_t* tile_slots, int cl, const Rec& r0, const Rec& r1, uint32_t tag) {
+    st_relaxed_v2u64(tile_slots + 0 * Cg + cl, tagged(tag, r0.a), tagged(tag, r1.a));
+    st_relaxed_v2u64(tile_slots + 1 * Cg + cl, tagged(tag, r0.b), tagged(tag, r1.b));
+    st_relaxed_v2u64(tile_slots + 2 * Cg + cl, tagged(tag, r0.anc), tagged(tag, r1.anc));
+    st_relaxed_v2u64(tile_slots + 3 * Cg + cl, tagged(tag, r0.n), tagged(tag, r1.n));
 }
 
-__device__ __forceinline__ bool read_rec(const uint64_t* src, uint32_t tag, Rec& out) {
-    const uint64_t w0 = ld_relaxed_u64(src + 0);
-    const uint64_t w1 = ld_relaxed_u64(src + 1);
-    const uint64_t w2 = ld_relaxed_u64(src + 2);
-    const uint64_t w3 = ld_relaxed_u64(src + 3);
-    if ((uint32_t)(w0 >> 32) != tag || (uint32_t)(w1 >> 32) != tag || (uint32_t)(w2 >> 32) != tag ||
-        (uint32_t)(w3 >> 32) != tag)
-        return false;
-    out = Rec{__uint_as_float((uint32_t)w0), __uint_as_float((uint32_t)w1), __uint_as_float((uint32_t)w2),
-              __uint_as_float((uint32_t)w3)};
-    return true;
+struct RawPair {
+    uint64_t w[4][2];  // word i of channel cl + c
+};
+
+template <int Cg>
+__device__ __forceinline__ RawPair load_pair(const uint64_t* tile_slots, int cl) {
+    RawPair r;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ld_relaxed_v2u64(tile_slots + i * Cg + cl, r.w[i][0], r.w[i][1]);
+    return r;
 }
+
+// 2: both channels hold an inclusive prefix, 1: both an aggregate, 0: nothing usable yet
+// (stale, half written, or the two channels caught at different kinds).
+__device__ __forceinline__ int pair_kind(const RawPair& r, uint32_t tag_agg, uint32_t tag_incl, Rec& o0, Rec& o1) {
+    const uint32_t t0 = (uint32_t)(r.w[0][0] >> 32);
+    bool same = true;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) same = same && (uint32_t)(r.w[i][c] >> 32) == t0;
+    if (!same || (t0 != tag_agg && t0 != tag_incl)) return 0;
+    o0 = Rec{__uint_as_float((uint32_t)r.w[0][0]), __uint_as_float((uint32_t)r.w[1][0]),
+             __uint_as_float((uint32_t)r.w[2][0]), __uint_as_float((uint32_t)r.w[3][0])};
+    o1 = Rec{__uint_as_float((uint32_t)r.w[0][1]), __uint_as_float((uint32_t)r.w[1][1]),
+             __uint_as_float((uint32_t)r.w[2][1]), __uint_as_float((uint32_t)r.w[3][1])};
+    return t0 == tag_incl ? 2 : 1;
+}
+
+// w and u of a tile's channels copied into its stage with the rows (1), or read from
+// global memory by each warp (0).
+#ifndef WKV_PIPE_WU_SMEM
+#define WKV_PIPE_WU_SMEM 0
+#endif
+
+// Predecessor slots read per look-back round trip.
+#ifndef WKV_PIPE_LOOKAHEAD
+#define WKV_PIPE_LOOKAHEAD 1
+#endif
+constexpr int kLook = WKV_PIPE_LOOKAHEAD;
 
 constexpr size_t align128(size_t x) { return (x + 127) / 128 * 128; }
 
@@ -113,7 +173,8 @@ struct PipeLayout {
     static constexpr size_t tile = sizeof(TIO) * Ts * Cg;  // one array (k or v)
     static constexpr size_t recs_off = 2 * tile;           // Rec [NWS][Cg]
     static constexpr size_t carry_off = recs_off + sizeof(Rec) * NWS * Cg;
-    static constexpr size_t stage = align128(carry_off + sizeof(Rec) * Cg);
+    static constexpr size_t wu_off = carry_off + sizeof(Rec) * Cg;  // float w[Cg], u[Cg] of the tile's channels
+    static constexpr size_t stage = align128(wu_off + 2 * sizeof(float) * Cg);
     static constexpr size_t bars_off = NS * stage;           // 5 mbarriers per stage
     static constexpr size_t misc_off = bars_off + NS * 5 * 8;  // stage unit ids, epoch, end index
     static constexpr size_t total = misc_off + NS * 8 + 24;
@@ -126,6 +187,7 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
     pipe_kernel(ForwardArgs args, PipeParams pp, const __grid_constant__ CUtensorMap tmk,
                 const __grid_constant__ CUtensorMap tmv) {
     using Lay = PipeLayout<TIO, V, NWS, LC, NS>;
+    static_assert(V == 2, "a lane owns one channel pair (records move as pairs)");
     constexpr int Cg = Lay::Cg;
     constexpr int Ts = Lay::Ts;
     constexpr int W_S0 = 1, W_L0 = 1 + NWS, W_E0 = 1 + NWS + NS;
@@ -139,6 +201,8 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
     auto vtile = [&](int s) { return reinterpret_cast<TIO*>(smem + s * Lay::stage + Lay::tile); };
     auto recs = [&](int s) { return reinterpret_cast<Rec*>(smem + s * Lay::stage + Lay::recs_off); };
     auto carries = [&](int s) { return reinterpret_cast<Rec*>(smem + s * Lay::stage + Lay::carry_off); };
+    auto wtile = [&](int s) { return reinterpret_cast<float*>(smem + s * Lay::stage + Lay::wu_off); };
+    auto utile = [&](int s) { return wtile(s) + Cg; };
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -182,6 +246,8 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
     if (warp == 0) {
         // ------------------------------- producer -------------------------------
         if (lane == 0) {
+            // A ticket is taken only once a stage is free: a unit that holds a ticket starts
+            // at once, so no later unit ever waits on one that sits idle.
             for (int64_t i = 0;; ++i) {
                 const int s = (int)(i % NS);
                 if (i >= NS && !mbar_wait(bar(s, kEmpty), (uint32_t)((i / NS - 1) & 1), lim)) report(kDevTimeoutCopy);
@@ -195,11 +261,19 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
                     break;
                 }
                 const int64_t unit = t;
+                WKV_TRACE_EVENT(unit, 0);
                 stage_unit[s] = unit;
                 mbar_arrive(bar(s, kTick));
                 const Geo q = geo(unit);
                 constexpr int BR = kBoxRows < Ts ? kBoxRows : Ts;
-                mbar_arrive_expect_tx(bar(s, kFull), 2u * (uint32_t)(Ts * Cg * sizeof(TIO)));
+                // w and u of the tile's channels ride along: nch * 4 bytes is a multiple of 16
+                // because bulk rows need C * sizeof(TIO) % 16 == 0 and c0 is a multiple of 64
+                const uint32_t wu_bytes = WKV_PIPE_WU_SMEM ? (uint32_t)q.nch * 4u : 0u;
+                mbar_arrive_expect_tx(bar(s, kFull), 2u * (uint32_t)(Ts * Cg * sizeof(TIO)) + 2u * wu_bytes);
+                if (WKV_PIPE_WU_SMEM) {
+                    bulk_g2s(wtile(s), args.w + q.c0, wu_bytes, bar(s, kFull));
+                    bulk_g2s(utile(s), args.u + q.c0, wu_bytes, bar(s, kFull));
+                }
 #pragma unroll
                 for (int r0 = 0; r0 < Ts; r0 += BR) {
                     tma_load_3d(ktile(s) + r0 * Cg, &tmk, (int)q.c0, (int)(q.t0 + r0), (int)q.b, bar(s, kFull));
@@ -218,6 +292,7 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
             if (!mbar_wait(bar(s, kFull), ph, lim) && lane == 0) report(kDevTimeoutCopy);
             const int64_t unit = stage_unit[s];
             if (unit < 0) break;
+            if (sw == 0 && lane == 0) WKV_TRACE_EVENT(unit, 1);
             const Geo q = geo(unit);
             const int cl = lane * V;
             const bool lane_active = cl < q.nch;
@@ -225,7 +300,10 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
             const int r_cnt = max(0, min(LC, q.len - r_begin));
             float w2[V];
 #pragma unroll
-            for (int c = 0; c < V; ++c) w2[c] = (lane_active && cl + c < q.nch) ? args.w[q.c0 + cl + c] * kLog2e : 0.f;
+            for (int c = 0; c < V; ++c)
+                w2[c] = (lane_active && cl + c < q.nch)
+                            ? (WKV_PIPE_WU_SMEM ? wtile(s)[cl + c] : args.w[q.c0 + cl + c]) * kLog2e
+                            : 0.f;
             if (lane_active) {
                 float gx[LC][V], M[V], sa[V], sb[V];
 #pragma unroll
@@ -267,6 +345,7 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(s, kChunks));
+            if (sw == 0 && lane == 0) WKV_TRACE_EVENT(unit, 2);
         }
     } else if (warp < W_E0) {
         // ------------------------------- look-back ------------------------------
@@ -302,6 +381,7 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
             // scan the chunk summaries (exclusive prefixes for the emitters) and publish the
             // tile aggregate for later segments before looking back
             if (!mbar_wait(bar(s, kChunks), ph, lim) && lane == 0) report(kDevTimeoutCarry);
+            if (lane == 0) WKV_TRACE_EVENT(unit, 3);
             Rec agg[V];
             if (lane_active) {
                 Rec* rc = recs(s);
@@ -317,12 +397,10 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
                         if (lw > 0) agg[c] = rec_combine(agg[c], r, (float)lw, w2[c]);
                     }
                 }
-                if (q.j > 0 && unit != pp.drop_unit) {
-#pragma unroll
-                    for (int c = 0; c < V; ++c)
-                        if (cl + c < q.nch) publish_rec(pp.agg + (unit * Cg + cl + c) * 4, agg[c], tag_agg);
-                }
+                // (nch is even, so a lane's two channels are both in range or both out)
+                if (q.j > 0 && unit != pp.drop_unit) publish_pair<Cg>(pp.slot + unit * 4 * Cg, cl, agg[0], agg[1], tag_agg);
             }
+            if (lane == 0) WKV_TRACE_EVENT(unit, 4);
             Rec run[V];
             if (q.j == 0) {
 #pragma unroll
@@ -334,76 +412,80 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
             } else {
 #pragma unroll
                 for (int c = 0; c < V; ++c) run[c] = rec_identity();
-                // Each lane looks back for its own channels: fold the newest predecessor's
-                // inclusive prefix if it is there, else its aggregate and step further back;
-                // back off while neither has been published.
-                float span[V];
-                int64_t hi[V];
-                bool done[V];
-#pragma unroll
-                for (int c = 0; c < V; ++c) {
-                    span[c] = 0.f;
-                    hi[c] = q.j - 1;
-                    done[c] = !(lane_active && cl + c < q.nch);
-                }
+                // Each lane looks back for its channel pair, reading the slots of the kLook
+                // newest unfolded predecessors in one round trip: it folds aggregates from the
+                // newest backwards and stops at the first inclusive prefix (the carry is then
+                // known) or at the first slot that is not yet published.
+                float span = 0.f;
+                int64_t hi = q.j - 1;
+                bool done = !lane_active;
                 uint32_t nap = 64;
                 bool all_done = false;
                 for (uint32_t it = 0; it <= lim && !all_done; ++it) {
-                    bool progressed = false;
-                    all_done = true;
+                    if (!done) {
+                        RawPair raw[kLook];
 #pragma unroll
-                    for (int c = 0; c < V; ++c) {
-                        if (done[c]) continue;
-                        const int64_t off = ((hi[c] * pp.G + q.g) * Cg + cl + c) * 4;
-                        Rec r;
-                        if (read_rec(pp.incl + off, tag_incl, r)) {
-                            run[c] = rec_combine(r, run[c], span[c], w2[c]);
-                            done[c] = true;
+                        for (int d = 0; d < kLook; ++d)
+                            if (hi - d >= 0) raw[d] = load_pair<Cg>(pp.slot + ((hi - d) * pp.G + q.g) * 4 * Cg, cl);
+                        bool progressed = false;
+#pragma unroll
+                        for (int d = 0; d < kLook; ++d) {
+                            if (done) break;
+                            Rec r0, r1;
+                            const int kind = pair_kind(raw[d], tag_agg, tag_incl, r0, r1);
+                            if (kind == 0) break;
+                            run[0] = rec_combine(r0, run[0], span, w2[0]);
+                            run[1] = rec_combine(r1, run[1], span, w2[1]);
                             progressed = true;
-                        } else if (read_rec(pp.agg + off, tag_agg, r)) {
-                            run[c] = rec_combine(r, run[c], span[c], w2[c]);
-                            span[c] += (float)Ts;
-                            progressed = true;
-                            if (--hi[c] < 0) done[c] = true;
+                            if (kind == 2) {
+                                done = true;
+                            } else {
+                                span += (float)Ts;
+                                if (--hi < 0) done = true;
+                            }
                         }
-                        all_done = all_done && done[c];
+                        if (!done && !progressed) {
+                            __nanosleep(nap);
+                            nap = nap < 1024 ? nap * 2 : 1024;
+                        } else if (progressed) {
+                            nap = 64;
+                        }
                     }
-                    if (!all_done && !progressed) {
-                        __nanosleep(nap);
-                        nap = nap < 1024 ? nap * 2 : 1024;
-                    } else if (progressed) {
-                        nap = 64;
-                    }
+                    all_done = __all_sync(0xffffffffu, done);
                 }
                 if (!all_done) {
                     report(kDevTimeoutCarry);
                     pp.hdr->error_unit = (uint32_t)unit;
                 }
             }
-            // hand the carry to the emitters first, then publish the inclusive prefix
+            if (lane == 0) WKV_TRACE_EVENT(unit, 5);
+            // publish the inclusive prefix (it overwrites the aggregate), then hand the carry
+            // to the emitters
             Rec inc[V];
+            if (lane_active) {
+#pragma unroll
+                for (int c = 0; c < V; ++c) inc[c] = rec_combine(run[c], agg[c], (float)q.len, w2[c]);
+                if (unit != pp.drop_unit) publish_pair<Cg>(pp.slot + unit * 4 * Cg, cl, inc[0], inc[1], tag_incl);
+            }
+            if (lane == 0) WKV_TRACE_EVENT(unit, 7);
             if (lane_active) {
                 Rec* cs = carries(s);
 #pragma unroll
-                for (int c = 0; c < V; ++c) {
-                    inc[c] = rec_combine(run[c], agg[c], (float)q.len, w2[c]);
-                    cs[cl + c] = run[c];
-                }
+                for (int c = 0; c < V; ++c) cs[cl + c] = run[c];
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(s, kCarry));
-            if (lane_active) {
+            if (lane == 0) {
+                WKV_TRACE_EVENT(unit, 6);
+                mbar_arrive(bar(s, kCarry));
+            }
+            if (lane_active && q.j == pp.S - 1 && args.state_out) {
 #pragma unroll
                 for (int c = 0; c < V; ++c) {
-                    if (cl + c < q.nch) {
-                        if (unit != pp.drop_unit) publish_rec(pp.incl + (unit * Cg + cl + c) * 4, inc[c], tag_incl);
-                        if (q.j == pp.S - 1 && args.state_out) {
-                            const int64_t bc = q.b * C + q.c0 + cl + c;
-                            args.state_out[bc] = inc[c].a;
-                            args.state_out[BC + bc] = inc[c].b;
-                            args.state_out[2 * BC + bc] = rec_p(inc[c], w2[c]) * kLn2;
-                        }
-                    }
+                    if (cl + c >= q.nch) continue;
+                    const int64_t bc = q.b * C + q.c0 + cl + c;
+                    args.state_out[bc] = inc[c].a;
+                    args.state_out[BC + bc] = inc[c].b;
+                    args.state_out[2 * BC + bc] = rec_p(inc[c], w2[c]) * kLn2;
                 }
             }
         }
@@ -417,6 +499,7 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
             (void)mbar_wait(bar(s, kFull), ph, lim);  // already complete; orders the tile reads
             const int64_t unit = stage_unit[s];
             if (unit < 0) break;
+            if (ew == 0 && lane == 0) WKV_TRACE_EVENT(unit, 8);
             const Geo q = geo(unit);
             const int cl = lane * V;
             const int r_begin = ew * LC;
@@ -427,8 +510,8 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
 #pragma unroll
                 for (int c = 0; c < V; ++c) {
                     const bool ok = cl + c < q.nch;
-                    w2[c] = ok ? args.w[q.c0 + cl + c] * kLog2e : 0.f;
-                    u2[c] = ok ? args.u[q.c0 + cl + c] * kLog2e : 0.f;
+                    w2[c] = ok ? (WKV_PIPE_WU_SMEM ? wtile(s)[cl + c] : args.w[q.c0 + cl + c]) * kLog2e : 0.f;
+                    u2[c] = ok ? (WKV_PIPE_WU_SMEM ? utile(s)[cl + c] : args.u[q.c0 + cl + c]) * kLog2e : 0.f;
                     const Rec cr = rec_combine(carries(s)[cl + c], recs(s)[ew * Cg + cl + c], (float)r_begin, w2[c]);
                     a[c] = cr.a;
                     bb[c] = cr.b;
@@ -476,6 +559,7 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
                 }
             }
             __syncwarp();
+            if (ew == 0 && lane == 0) WKV_TRACE_EVENT(unit, 9);
             if (lane == 0) mbar_arrive(bar(s, kEmpty));
         }
     }
@@ -569,12 +653,11 @@ cudaError_t launch_forward_pipe(const ForwardArgs& a, const ChunkGeom& g, void* 
     pp.S = g.S;
     pp.U = g.U;
     pp.hdr = reinterpret_cast<WsHeader*>(base);
-    pp.agg = reinterpret_cast<uint64_t*>(base + kWsHeaderBytes);
-    pp.incl = pp.agg + (size_t)g.U * (size_t)g.Cg * 4;
+    pp.slot = reinterpret_cast<uint64_t*>(base + kWsHeaderBytes);
     pp.drop_unit = drop_unit;
     if (a.io == 1) {
-        if (g.V == 4 && g.NW == 8 && g.LC == 8) return launch_pipe_t<__nv_bfloat16, 4, 8, 8>(a, g, pp, s);
-        if (g.V == 4 && g.NW == 8 && g.LC == 16) return launch_pipe_t<__nv_bfloat16, 4, 8, 16>(a, g, pp, s);
+        if (g.V == 2 && g.NW == 8 && g.LC == 8) return launch_pipe_t<__nv_bfloat16, 2, 8, 8>(a, g, pp, s);
+        if (g.V == 2 && g.NW == 8 && g.LC == 16) return launch_pipe_t<__nv_bfloat16, 2, 8, 16>(a, g, pp, s);
         return cudaErrorInvalidValue;
     }
     if (g.V == 2 && g.NW == 8 && g.LC == 8) return launch_pipe_t<float, 2, 8, 8>(a, g, pp, s);
