@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--profile-forward", metavar="WORKLOAD", default=None,
+                    help="only run 2 + 3 eager forward launches of a forward workload (e.g. fwd_1x16384x4096) "
+                         "and exit: a short, self-contained command to capture under a profiler")
     return ap.parse_args()
 
 
@@ -507,8 +510,34 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def profile_forward(name):
+    """Two warm-up and three profiled eager forward launches (with the final state) of one
+    forward workload on one input set; checks the workspace status afterwards."""
+    import torch
+    import linear_attention_rnn_wkv_b200 as wkv
+    import synth
+    spec = synth.FORWARD[name]
+    dev = torch.device("cuda", 0)
+    w, u, k, v = synth.forward_inputs(spec)
+    td = torch.bfloat16 if spec.dtype == "bf16" else torch.float32
+    w, u = torch.from_numpy(w).to(dev), torch.from_numpy(u).to(dev)
+    k, v = torch.from_numpy(k).to(dev).to(td), torch.from_numpy(v).to(dev).to(td)
+    y = torch.empty_like(k)
+    st = torch.empty((3, spec.B, spec.C), dtype=torch.float32, device=dev)
+    ws = wkv.Workspace(dev, wkv.workspace_size(spec.B, spec.T, spec.C, td))
+    for _ in range(5):
+        wkv.wkv_forward(w, u, k, v, want_state=True, workspace=ws, y=y, state_out=st)
+    torch.cuda.synchronize()
+    wkv.forward_status(ws.buf)
+    print(json.dumps({"profile_forward": name, "launches": 5, "B": spec.B, "T": spec.T, "C": spec.C,
+                      "io": spec.dtype}))
+
+
 def main():
     args = parse()
+    if args.profile_forward:
+        profile_forward(args.profile_forward)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

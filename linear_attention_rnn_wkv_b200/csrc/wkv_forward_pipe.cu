@@ -78,13 +78,20 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Bounded wait on an mbarrier phase; returns false if it ran out.
+// Suspend-time hint of the mbarrier waits, in nanoseconds (0: poll with a short sleep).
+#ifndef WKV_WAIT_HINT
+#define WKV_WAIT_HINT 1000
+#endif
+
+// Bounded wait on an mbarrier phase; returns false if it ran out.  With a hint, a waiting
+// warp is parked by the hardware instead of spinning, so it takes no issue slots from the
+// warps that do the work.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
-    for (uint32_t it = 0; !mbar_try_wait(bar, parity); ++it) {
+    for (uint32_t it = 0;; ++it) {
+        if (WKV_WAIT_HINT ? mbar_try_wait_hint(bar, parity, WKV_WAIT_HINT) : mbar_try_wait(bar, parity)) return true;
         if (it >= limit) return false;
-        __nanosleep(32);
+        if (!WKV_WAIT_HINT) __nanosleep(32);
     }
-    return true;
 }
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* tm, int x, int y, int z, uint64_t* bar) {
@@ -156,6 +163,11 @@ __device__ __forceinline__ int pair_kind(const RawPair& r, uint32_t tag_agg, uin
 // global memory by each warp (0).
 #ifndef WKV_PIPE_WU_SMEM
 #define WKV_PIPE_WU_SMEM 0
+#endif
+
+// Summaries and the emitters' per-token step on f32x2 pairs (1) or per channel (0).
+#ifndef WKV_PIPE_PACKED
+#define WKV_PIPE_PACKED 1
 #endif
 
 // Predecessor slots read per look-back round trip.
@@ -304,7 +316,42 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
                 w2[c] = (lane_active && cl + c < q.nch)
                             ? (WKV_PIPE_WU_SMEM ? wtile(s)[cl + c] : args.w[q.c0 + cl + c]) * kLog2e
                             : 0.f;
-            if (lane_active) {
+            if (lane_active && WKV_PIPE_PACKED) {
+                // the same arithmetic as below on the lane's channel pair with f32x2 ops
+                const TIO* kt = ktile(s);
+                const TIO* vt = vtile(s);
+                const float2 w2p = make_float2(w2[0], w2[1]);
+                const float2 L2 = make_float2(kLog2e, kLog2e);
+                float2 gx[LC];
+                float M0 = kPEmpty, M1 = kPEmpty;
+#pragma unroll
+                for (int r = 0; r < LC; ++r) {
+                    if (r < r_cnt) {
+                        float kk[V];
+                        Vec<TIO, V>::load(kt + (r_begin + r) * Cg + cl, kk);
+                        const float back = -(float)(r_cnt - 1 - r);
+                        gx[r] = __ffma2_rn(make_float2(back, back), w2p, __fmul2_rn(make_float2(kk[0], kk[1]), L2));
+                        M0 = fmaxf(M0, gx[r].x);
+                        M1 = fmaxf(M1, gx[r].y);
+                    }
+                }
+                const float2 nM = make_float2(-M0, -M1);
+                float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int r = 0; r < LC; ++r) {
+                    if (r < r_cnt) {
+                        float vv[V];
+                        Vec<TIO, V>::load(vt + (r_begin + r) * Cg + cl, vv);
+                        const float2 x = __fadd2_rn(gx[r], nM);
+                        const float2 e = make_float2(ex2(x.x), ex2(x.y));
+                        sa = __ffma2_rn(e, make_float2(vv[0], vv[1]), sa);
+                        sb = __fadd2_rn(sb, e);
+                    }
+                }
+                Rec* rc = recs(s);
+                rc[sw * Cg + cl] = Rec{sa.x, sb.x, M0, 0.f};
+                rc[sw * Cg + cl + 1] = Rec{sa.y, sb.y, M1, 0.f};
+            } else if (lane_active) {
                 float gx[LC][V], M[V], sa[V], sb[V];
 #pragma unroll
                 for (int c = 0; c < V; ++c) {
@@ -355,7 +402,7 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
             const uint32_t ph = (uint32_t)((i / NS) & 1);
             bool got = false, gone = false;
             for (uint32_t it = 0; it <= lim; ++it) {
-                if (mbar_try_wait(bar(s, kTick), ph)) {
+                if (WKV_WAIT_HINT ? mbar_try_wait_hint(bar(s, kTick), ph, WKV_WAIT_HINT) : mbar_try_wait(bar(s, kTick), ph)) {
                     got = true;
                     break;
                 }
@@ -363,7 +410,7 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
                     gone = true;
                     break;
                 }
-                __nanosleep(32);
+                if (!WKV_WAIT_HINT) __nanosleep(32);
             }
             if (gone) break;
             if (!got && lane == 0) report(kDevTimeoutCopy);
@@ -522,7 +569,48 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
                 const TIO* kt = ktile(s);
                 const TIO* vt = vtile(s);
                 TIO* yg = static_cast<TIO*>(args.y) + (q.b * T + q.t0) * C + q.c0;
-                if (lazy_ok) {
+                if (lazy_ok && WKV_PIPE_PACKED) {
+                    // lazy_step on the lane's channel pair with f32x2 ops; the reference is
+                    // kept negated (nR = -R) and u + k formed with one FMA, so no negation
+                    // is needed inside the loop
+                    const float2 L2 = make_float2(kLog2e, kLog2e), nL2 = make_float2(-kLog2e, -kLog2e);
+                    const float2 u2p = make_float2(u2[0], u2[1]), nu2p = make_float2(-u2[0], -u2[1]);
+                    const float2 w2p = make_float2(w2[0], w2[1]);
+                    const float2 cwp = make_float2(ex2(w2[0] - u2[0]), ex2(w2[1] - u2[1]));
+                    const float2 one = make_float2(1.f, 1.f);
+                    float2 ap = make_float2(a[0], a[1]), bp = make_float2(bb[0], bb[1]);
+                    float2 nRp = make_float2(-R[0], -R[1]), np = make_float2(nn[0], nn[1]);
+#pragma unroll
+                    for (int r = 0; r < LC; ++r) {
+                        if (r < r_cnt) {
+                            const int row = r_begin + r;
+                            float kk[V], vv[V], yy[V];
+                            Vec<TIO, V>::load(kt + row * Cg + cl, kk);
+                            Vec<TIO, V>::load(vt + row * Cg + cl, vv);
+                            const float2 kp = make_float2(kk[0], kk[1]), vp = make_float2(vv[0], vv[1]);
+                            const float2 uk = __ffma2_rn(kp, L2, u2p);
+                            const float2 nuk = __ffma2_rn(kp, nL2, nu2p);
+                            const float2 d = __ffma2_rn(np, w2p, __fadd2_rn(nRp, uk));  // (u + k) - (R - n w)
+                            const bool c0 = d.x > 0.f, c1 = d.y > 0.f;
+                            const float e0 = ex2(-fabsf(d.x)), e1 = ex2(-fabsf(d.y));
+                            const float2 sa = make_float2(c0 ? e0 : 1.f, c1 ? e1 : 1.f);
+                            const float2 sv = make_float2(c0 ? 1.f : e0, c1 ? 1.f : e1);
+                            const float2 t = __fmul2_rn(sa, ap);
+                            const float2 num = __ffma2_rn(sv, vp, t);
+                            const float2 den = __ffma2_rn(sa, bp, sv);
+                            const float2 yv = __fmul2_rn(num, make_float2(rcp(den.x), rcp(den.y)));
+                            const float2 nw = __fmul2_rn(sv, cwp);
+                            ap = __ffma2_rn(nw, vp, t);
+                            bp = __ffma2_rn(sa, bp, nw);
+                            nRp = make_float2(c0 ? nuk.x : nRp.x, c1 ? nuk.y : nRp.y);
+                            const float2 n1 = __fadd2_rn(np, one);
+                            np = make_float2(c0 ? 1.f : n1.x, c1 ? 1.f : n1.y);
+                            yy[0] = yv.x;
+                            yy[1] = yv.y;
+                            Vec<TIO, V>::store(yg + (int64_t)row * C + cl, yy);
+                        }
+                    }
+                } else if (lazy_ok) {
                     float cw[V];
 #pragma unroll
                     for (int c = 0; c < V; ++c) cw[c] = ex2(w2[c] - u2[c]);
