@@ -165,6 +165,12 @@ __device__ __forceinline__ int pair_kind(const RawPair& r, uint32_t tag_agg, uin
 #define WKV_PIPE_WU_SMEM 0
 #endif
 
+// Emitters re-scan a chunk in the fixed frame of its largest exponent (1), or carry a
+// moving reference token by token (0; always used where the frame's range check fails).
+#ifndef WKV_PIPE_FRAME
+#define WKV_PIPE_FRAME 1
+#endif
+
 // Summaries and the emitters' per-token step on f32x2 pairs (1) or per channel (0).
 #ifndef WKV_PIPE_PACKED
 #define WKV_PIPE_PACKED 1
@@ -186,7 +192,8 @@ struct PipeLayout {
     static constexpr size_t recs_off = 2 * tile;           // Rec [NWS][Cg]
     static constexpr size_t carry_off = recs_off + sizeof(Rec) * NWS * Cg;
     static constexpr size_t wu_off = carry_off + sizeof(Rec) * Cg;  // float w[Cg], u[Cg] of the tile's channels
-    static constexpr size_t stage = align128(wu_off + 2 * sizeof(float) * Cg);
+    static constexpr size_t mx_off = wu_off + (WKV_PIPE_WU_SMEM ? 2 * sizeof(float) * Cg : 0);  // float [NWS][Cg]: each chunk's max exponent
+    static constexpr size_t stage = align128(mx_off + sizeof(float) * NWS * Cg);
     static constexpr size_t bars_off = NS * stage;           // 5 mbarriers per stage
     static constexpr size_t misc_off = bars_off + NS * 5 * 8;  // stage unit ids, epoch, end index
     static constexpr size_t total = misc_off + NS * 8 + 24;
@@ -215,6 +222,7 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
     auto carries = [&](int s) { return reinterpret_cast<Rec*>(smem + s * Lay::stage + Lay::carry_off); };
     auto wtile = [&](int s) { return reinterpret_cast<float*>(smem + s * Lay::stage + Lay::wu_off); };
     auto utile = [&](int s) { return wtile(s) + Cg; };
+    auto chunk_max = [&](int s) { return reinterpret_cast<float*>(smem + s * Lay::stage + Lay::mx_off); };
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -351,6 +359,7 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
                 Rec* rc = recs(s);
                 rc[sw * Cg + cl] = Rec{sa.x, sb.x, M0, 0.f};
                 rc[sw * Cg + cl + 1] = Rec{sa.y, sb.y, M1, 0.f};
+                *reinterpret_cast<float2*>(chunk_max(s) + sw * Cg + cl) = make_float2(M0, M1);
             } else if (lane_active) {
                 float gx[LC][V], M[V], sa[V], sb[V];
 #pragma unroll
@@ -388,7 +397,10 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
                 }
                 Rec* rc = recs(s);
 #pragma unroll
-                for (int c = 0; c < V; ++c) rc[sw * Cg + cl + c] = Rec{sa[c], sb[c], M[c], 0.f};
+                for (int c = 0; c < V; ++c) {
+                    rc[sw * Cg + cl + c] = Rec{sa[c], sb[c], M[c], 0.f};
+                    chunk_max(s)[sw * Cg + cl + c] = M[c];
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(s, kChunks));
@@ -569,7 +581,81 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
                 const TIO* kt = ktile(s);
                 const TIO* vt = vtile(s);
                 TIO* yg = static_cast<TIO*>(args.y) + (q.b * T + q.t0) * C + q.c0;
-                if (lazy_ok && WKV_PIPE_PACKED) {
+                // Fixed-frame re-scan.  Seen from the chunk's last row, each token's weight
+                // e_i = 2^(k_i - (L-1-i) w - G) and the carried-in history K do not change from
+                // row to row (everything decays at the same rate), so with running sums S of
+                // K + e_i v_i and K + e_i over earlier rows and c = 2^(w - u)
+                //   y_r = (S^a + e_r v_r / c) / (S^b + e_r / c):
+                // no re-referencing and no selects, and only S is carried from row to row (the
+                // first row of a sequence without history returns v itself, as the
+                // recurrence does; the rearranged form v + (S^a - S^b v) / (...) would do that
+                // by itself but cancels badly when the history dominates).  The frame G lies
+                // at most 100 above the larger of the history and the first token (so no term
+                // that matters can be flushed), at most 64 below the history (so K stays finite)
+                // and high enough that no later token's term can overflow; a chunk whose range
+                // leaves no such G takes the token-by-token path below.
+                bool frame_ok = false;
+                float2 fSa, fSb, fnG, fic;
+                if (WKV_PIPE_FRAME && lazy_ok) {
+                    float k0[V];
+                    Vec<TIO, V>::load(kt + r_begin * Cg + cl, k0);
+                    float fa[V], fb[V], fg[V], fi[V];
+                    bool ok = true;
+                    const float fc = (float)r_cnt;
+#pragma unroll
+                    for (int c = 0; c < V; ++c) {
+                        const float M = chunk_max(s)[ew * Cg + cl + c];
+                        const float hK = fmaf(-fc, w2[c], fmaf(-nn[c], w2[c], R[c]));  // history, at the last row
+                        const float h0 = fmaf(-(fc - 1.f), w2[c], k0[c] * kLog2e);        // first token, same
+                        const float bonus = u2[c] - w2[c];
+                        const float dom = fminf(fmaxf(hK, h0), fmaxf(hK, h0 + bonus));
+                        const float G = fmaxf(fminf(M, dom + 100.f), hK - 64.f);
+                        ok = ok && (M - G + fmaxf(bonus, 0.f) <= 100.f);
+                        const float sc = ex2(hK - G);
+                        fa[c] = a[c] * sc;
+                        fb[c] = bb[c] * sc;
+                        fg[c] = -G;
+                        fi[c] = ex2(bonus);
+                    }
+                    frame_ok = ok;
+                    fSa = make_float2(fa[0], fa[1]);
+                    fSb = make_float2(fb[0], fb[1]);
+                    fnG = make_float2(fg[0], fg[1]);
+                    fic = make_float2(fi[0], fi[1]);
+                }
+                if (frame_ok) {
+                    const float2 L2 = make_float2(kLog2e, kLog2e);
+                    const float2 w2p = make_float2(w2[0], w2[1]);
+                    const float back0 = 1.f - (float)r_cnt;  // -(steps from row 0 to the last row)
+#pragma unroll
+                    for (int r = 0; r < LC; ++r) {
+                        if (r < r_cnt) {
+                            const int row = r_begin + r;
+                            float kk[V], vv[V], yy[V];
+                            Vec<TIO, V>::load(kt + row * Cg + cl, kk);
+                            Vec<TIO, V>::load(vt + row * Cg + cl, vv);
+                            const float2 vp = make_float2(vv[0], vv[1]);
+                            // k - G first: the large cancellation happens inside one rounding
+                            const float back = back0 + (float)r;
+                            const float2 x = __ffma2_rn(make_float2(back, back), w2p,
+                                                        __ffma2_rn(make_float2(kk[0], kk[1]), L2, fnG));
+                            const float2 e = make_float2(ex2(x.x), ex2(x.y));
+                            const float2 ec = __fmul2_rn(e, fic);
+                            const float2 num = __ffma2_rn(ec, vp, fSa);
+                            const float2 den = __fadd2_rn(fSb, ec);
+                            const float2 yv = __fmul2_rn(num, make_float2(rcp(den.x), rcp(den.y)));
+                            yy[0] = yv.x;
+                            yy[1] = yv.y;
+                            if (r == 0) {
+                                if (fSb.x == 0.f) yy[0] = vv[0];
+                                if (fSb.y == 0.f) yy[1] = vv[1];
+                            }
+                            fSa = __ffma2_rn(e, vp, fSa);
+                            fSb = __fadd2_rn(fSb, e);
+                            Vec<TIO, V>::store(yg + (int64_t)row * C + cl, yy);
+                        }
+                    }
+                } else if (lazy_ok && WKV_PIPE_PACKED) {
                     // lazy_step on the lane's channel pair with f32x2 ops; the reference is
                     // kept negated (nR = -R) and u + k formed with one FMA, so no negation
                     // is needed inside the loop
@@ -699,7 +785,7 @@ cudaError_t launch_pipe_t(const ForwardArgs& a, const ChunkGeom& g, const PipePa
     constexpr size_t stage = PipeLayout<TIO, V, NWS, LC, 1>::stage;
     constexpr size_t budget = 232448 - 512;
     constexpr int NS = (int)(budget / (stage + 64) > 5 ? 5 : budget / (stage + 64));
-    static_assert(NS >= 2, "tile too large for a two-stage ring");
+    static_assert(NS >= 3, "tile too large for a three-stage ring");
     using Lay = PipeLayout<TIO, V, NWS, LC, NS>;
     auto kern = pipe_kernel<TIO, V, NWS, LC, NS>;
     CUtensorMap tmk, tmv;
