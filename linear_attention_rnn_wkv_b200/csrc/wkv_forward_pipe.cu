@@ -28,161 +28,13 @@
 // expiry, then the pipeline keeps moving).  Deadlock freedom: roles handle a CTA's units
 // in ticket order and every cross-CTA wait is on a smaller ticket, so the oldest
 // unfinished unit in the whole grid can always complete.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include "wkv_device.cuh"
 #include "wkv_internal.h"
 #include "wkv_vec.cuh"
-
-// Per-unit event trace (profiling builds only): compiled with -DWKV_TRACE, the kernel
-// stamps %globaltimer at each hand-over of every unit into the buffer registered with
-// wkv_trace_set_buffer ([units][11] u64: events 0..9 below, slot 10 the SM id).  Normal
-// builds define the hooks away.
-#ifdef WKV_TRACE
-__device__ unsigned long long* g_wkv_trace = nullptr;
-extern "C" cudaError_t wkv_trace_set_buffer(void* p) { return cudaMemcpyToSymbol(g_wkv_trace, &p, sizeof(p)); }
-__device__ __forceinline__ void wkv_trace(int64_t unit, int ev) {
-    if (!g_wkv_trace) return;
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    g_wkv_trace[unit * 11 + ev] = t;
-    if (ev == 0) {
-        unsigned sm;
-        asm volatile("mov.u32 %0, %smid;" : "=r"(sm));
-        g_wkv_trace[unit * 11 + 10] = sm;
-    }
-}
-#define WKV_TRACE_EVENT(unit, ev) wkv_trace(unit, ev)
-#else
-#define WKV_TRACE_EVENT(unit, ev) ((void)0)
-#endif
-// events: 0 ticket, 1 tile loaded, 2 chunks summarised, 3 look-back start, 4 summaries
-// scanned, 5 carry known, 6 carry handed over, 7 records published, 8 emit start, 9 emit end
-
-// Rows per TMA box (a tile of Ts rows is fetched as Ts / kBoxRows boxes per array).
-#ifndef WKV_PIPE_BOXR
-#define WKV_PIPE_BOXR 32
-#endif
+#include "wkv_pipe_common.cuh"
 
 namespace wkvb {
 namespace {
-
-constexpr int kBoxRows = WKV_PIPE_BOXR;
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ void named_sync(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// Suspend-time hint of the mbarrier waits, in nanoseconds (0: poll with a short sleep).
-#ifndef WKV_WAIT_HINT
-#define WKV_WAIT_HINT 1000
-#endif
-
-// Bounded wait on an mbarrier phase; returns false if it ran out.  With a hint, a waiting
-// warp is parked by the hardware instead of spinning, so it takes no issue slots from the
-// warps that do the work.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
-    for (uint32_t it = 0;; ++it) {
-        if (WKV_WAIT_HINT ? mbar_try_wait_hint(bar, parity, WKV_WAIT_HINT) : mbar_try_wait(bar, parity)) return true;
-        if (it >= limit) return false;
-        if (!WKV_WAIT_HINT) __nanosleep(32);
-    }
-}
-
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* tm, int x, int y, int z, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
-            smem_u32(dst)),
-        "l"(tm), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
-        : "memory");
-}
-
-struct PipeParams {
-    int64_t groups_per_b, G, S, U;
-    uint64_t* slot;     // [U][Cg][4] tagged words: a tile's aggregate, later its inclusive prefix
-    WsHeader* hdr;
-    int64_t drop_unit;  // test hook: this unit never publishes its records (-1: none)
-};
-
-// A published record is four 64-bit words, (a | tag), (b | tag), (anc | tag), (n | tag):
-// the value's bits in the low half, the launch epoch and the record kind in the high
-// half.  Aligned 64-bit accesses are single-copy atomic, so a reader that finds one tag
-// in all four words holds one consistent record; nothing else has to be ordered, so
-// neither side needs a fence or a separate flag.  The anchored exponent (anc, n) travels
-// unrounded.  Each tile has one slot per channel: the tile's aggregate is published there
-// first and later overwritten by its inclusive prefix (same thread, so every word takes
-// the second value after the first); a reader that catches the overwrite half done sees
-// mixed tags and reads again.  A tile's slots are stored word-major, [4][Cg] words, so a
-// lane moves the same word of its two channels with one 16-byte access and a warp's
-// access is contiguous.
-__device__ __forceinline__ uint64_t tagged(uint32_t tag, float x) { return ((uint64_t)tag << 32) | __float_as_uint(x); }
-
-template <int Cg>
-__device__ __forceinline__ void publish_pair(uint64_t* tile_slots, int cl, const Rec& r0, const Rec& r1, uint32_t tag) {
-    st_relaxed_v2u64(tile_slots + 0 * Cg + cl, tagged(tag, r0.a), tagged(tag, r1.a));
-    st_relaxed_v2u64(tile_slots + 1 * Cg + cl, tagged(tag, r0.b), tagged(tag, r1.b));
-    st_relaxed_v2u64(tile_slots + 2 * Cg + cl, tagged(tag, r0.anc), tagged(tag, r1.anc));
-    st_relaxed_v2u64(tile_slots + 3 * Cg + cl, tagged(tag, r0.n), tagged(tag, r1.n));
-}
-
-struct RawPair {
-    uint64_t w[4][2];  // word i of channel cl + c
-};
-
-template <int Cg>
-__device__ __forceinline__ RawPair load_pair(const uint64_t* tile_slots, int cl) {
-    RawPair r;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) ld_relaxed_v2u64(tile_slots + i * Cg + cl, r.w[i][0], r.w[i][1]);
-    return r;
-}
-
-// 2: both channels hold an inclusive prefix, 1: both an aggregate, 0: nothing usable yet
-// (stale, half written, or the two channels caught at different kinds).
-__device__ __forceinline__ int pair_kind(const RawPair& r, uint32_t tag_agg, uint32_t tag_incl, Rec& o0, Rec& o1) {
-    const uint32_t t0 = (uint32_t)(r.w[0][0] >> 32);
-    bool same = true;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int c = 0; c < 2; ++c) same = same && (uint32_t)(r.w[i][c] >> 32) == t0;
-    if (!same || (t0 != tag_agg && t0 != tag_incl)) return 0;
-    o0 = Rec{__uint_as_float((uint32_t)r.w[0][0]), __uint_as_float((uint32_t)r.w[1][0]),
-             __uint_as_float((uint32_t)r.w[2][0]), __uint_as_float((uint32_t)r.w[3][0])};
-    o1 = Rec{__uint_as_float((uint32_t)r.w[0][1]), __uint_as_float((uint32_t)r.w[1][1]),
-             __uint_as_float((uint32_t)r.w[2][1]), __uint_as_float((uint32_t)r.w[3][1])};
-    return t0 == tag_incl ? 2 : 1;
-}
-
-// w and u of a tile's channels copied into its stage with the rows (1), or read from
-// global memory by each warp (0).
-#ifndef WKV_PIPE_WU_SMEM
-#define WKV_PIPE_WU_SMEM 0
-#endif
-
-// Emitters re-scan a chunk in the fixed frame of its largest exponent (1), or carry a
-// moving reference token by token (0; always used where the frame's range check fails).
-#ifndef WKV_PIPE_FRAME
-#define WKV_PIPE_FRAME 1
-#endif
-
-// Summaries and the emitters' per-token step on f32x2 pairs (1) or per channel (0).
-#ifndef WKV_PIPE_PACKED
-#define WKV_PIPE_PACKED 1
-#endif
-
-// Predecessor slots read per look-back round trip.
-#ifndef WKV_PIPE_LOOKAHEAD
-#define WKV_PIPE_LOOKAHEAD 1
-#endif
-constexpr int kLook = WKV_PIPE_LOOKAHEAD;
-
-constexpr size_t align128(size_t x) { return (x + 127) / 128 * 128; }
 
 template <typename TIO, int V, int NWS, int LC, int NS>
 struct PipeLayout {
@@ -191,15 +43,19 @@ struct PipeLayout {
     static constexpr size_t tile = sizeof(TIO) * Ts * Cg;  // one array (k or v)
     static constexpr size_t recs_off = 2 * tile;           // Rec [NWS][Cg]
     static constexpr size_t carry_off = recs_off + sizeof(Rec) * NWS * Cg;
-    static constexpr size_t wu_off = carry_off + sizeof(Rec) * Cg;  // float w[Cg], u[Cg] of the tile's channels
-    static constexpr size_t mx_off = wu_off + (WKV_PIPE_WU_SMEM ? 2 * sizeof(float) * Cg : 0);  // float [NWS][Cg]: each chunk's max exponent
+    static constexpr size_t mx_off = carry_off + sizeof(Rec) * Cg;  // float [NWS][Cg]: each chunk's max exponent
     static constexpr size_t stage = align128(mx_off + sizeof(float) * NWS * Cg);
-    static constexpr size_t bars_off = NS * stage;           // 5 mbarriers per stage
-    static constexpr size_t misc_off = bars_off + NS * 5 * 8;  // stage unit ids, epoch, end index
+    static constexpr int BR = kBoxRows < Ts ? kBoxRows : Ts;  // rows per TMA box
+    static constexpr int NB = Ts / BR;                           // boxes per array
+    static constexpr int NBAR = 4 + NB;                          // mbarriers per stage
+    static constexpr size_t bars_off = NS * stage;
+    static constexpr size_t misc_off = bars_off + NS * NBAR * 8;  // stage unit ids, epoch, end index
     static constexpr size_t total = misc_off + NS * 8 + 24;
+    static constexpr size_t per_stage = stage + NBAR * 8 + 8;  // what one more stage costs
 };
 
-enum { kFull = 0, kTick = 1, kChunks = 2, kCarry = 3, kEmpty = 4 };
+// per stage: kTick, kChunks, kCarry, kEmpty, then one `full` barrier per TMA box of rows
+enum { kTick = 0, kChunks = 1, kCarry = 2, kEmpty = 3, kFull0 = 4 };
 
 template <typename TIO, int V, int NWS, int LC, int NS>
 __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
@@ -215,13 +71,12 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
     int64_t* stage_unit = reinterpret_cast<int64_t*>(smem + Lay::misc_off);
     uint32_t* s_epoch = reinterpret_cast<uint32_t*>(stage_unit + NS);
     volatile int64_t* s_iend = reinterpret_cast<volatile int64_t*>(stage_unit + NS + 1);
-    auto bar = [&](int s, int kind) { return &bars[s * 5 + kind]; };
+    constexpr int NB = Lay::NB, BR = Lay::BR;
+    auto bar = [&](int s, int kind) { return &bars[s * Lay::NBAR + kind]; };
     auto ktile = [&](int s) { return reinterpret_cast<TIO*>(smem + s * Lay::stage); };
     auto vtile = [&](int s) { return reinterpret_cast<TIO*>(smem + s * Lay::stage + Lay::tile); };
     auto recs = [&](int s) { return reinterpret_cast<Rec*>(smem + s * Lay::stage + Lay::recs_off); };
     auto carries = [&](int s) { return reinterpret_cast<Rec*>(smem + s * Lay::stage + Lay::carry_off); };
-    auto wtile = [&](int s) { return reinterpret_cast<float*>(smem + s * Lay::stage + Lay::wu_off); };
-    auto utile = [&](int s) { return wtile(s) + Cg; };
     auto chunk_max = [&](int s) { return reinterpret_cast<float*>(smem + s * Lay::stage + Lay::mx_off); };
 
     const int tid = threadIdx.x;
@@ -234,7 +89,7 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
         *s_epoch = (*reinterpret_cast<volatile uint32_t*>(&pp.hdr->epoch) + 1u) & 0x3FFFFFFFu;
         *s_iend = INT64_MAX;
         for (int s = 0; s < NS; ++s) {
-            mbar_init(bar(s, kFull), 1);
+            for (int b = 0; b < NB; ++b) mbar_init(bar(s, kFull0 + b), 1);
             mbar_init(bar(s, kTick), 1);
             mbar_init(bar(s, kChunks), NWS);
             mbar_init(bar(s, kCarry), 1);
@@ -277,7 +132,7 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
                     *s_iend = i;
                     stage_unit[s] = -1;
                     mbar_arrive(bar(s, kTick));
-                    mbar_arrive(bar(s, kFull));
+                    for (int b = 0; b < NB; ++b) mbar_arrive(bar(s, kFull0 + b));
                     break;
                 }
                 const int64_t unit = t;
@@ -285,19 +140,14 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
                 stage_unit[s] = unit;
                 mbar_arrive(bar(s, kTick));
                 const Geo q = geo(unit);
-                constexpr int BR = kBoxRows < Ts ? kBoxRows : Ts;
-                // w and u of the tile's channels ride along: nch * 4 bytes is a multiple of 16
-                // because bulk rows need C * sizeof(TIO) % 16 == 0 and c0 is a multiple of 64
-                const uint32_t wu_bytes = WKV_PIPE_WU_SMEM ? (uint32_t)q.nch * 4u : 0u;
-                mbar_arrive_expect_tx(bar(s, kFull), 2u * (uint32_t)(Ts * Cg * sizeof(TIO)) + 2u * wu_bytes);
-                if (WKV_PIPE_WU_SMEM) {
-                    bulk_g2s(wtile(s), args.w + q.c0, wu_bytes, bar(s, kFull));
-                    bulk_g2s(utile(s), args.u + q.c0, wu_bytes, bar(s, kFull));
-                }
+                // each box of BR rows (k and v) completes its own barrier, so the summarisers
+                // of the first chunks start while later rows are still in flight
 #pragma unroll
-                for (int r0 = 0; r0 < Ts; r0 += BR) {
-                    tma_load_3d(ktile(s) + r0 * Cg, &tmk, (int)q.c0, (int)(q.t0 + r0), (int)q.b, bar(s, kFull));
-                    tma_load_3d(vtile(s) + r0 * Cg, &tmv, (int)q.c0, (int)(q.t0 + r0), (int)q.b, bar(s, kFull));
+                for (int b = 0; b < NB; ++b) {
+                    uint64_t* fb = bar(s, kFull0 + b);
+                    mbar_arrive_expect_tx(fb, 2u * (uint32_t)(BR * Cg * sizeof(TIO)));
+                    tma_load_3d(ktile(s) + b * BR * Cg, &tmk, (int)q.c0, (int)(q.t0 + b * BR), (int)q.b, fb);
+                    tma_load_3d(vtile(s) + b * BR * Cg, &tmv, (int)q.c0, (int)(q.t0 + b * BR), (int)q.b, fb);
                 }
             }
         }
@@ -309,7 +159,7 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
         for (int64_t i = 0;; ++i) {
             const int s = (int)(i % NS);
             const uint32_t ph = (uint32_t)((i / NS) & 1);
-            if (!mbar_wait(bar(s, kFull), ph, lim) && lane == 0) report(kDevTimeoutCopy);
+            if (!mbar_wait(bar(s, kFull0 + sw * LC / BR), ph, lim) && lane == 0) report(kDevTimeoutCopy);
             const int64_t unit = stage_unit[s];
             if (unit < 0) break;
             if (sw == 0 && lane == 0) WKV_TRACE_EVENT(unit, 1);
@@ -322,7 +172,7 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
 #pragma unroll
             for (int c = 0; c < V; ++c)
                 w2[c] = (lane_active && cl + c < q.nch)
-                            ? (WKV_PIPE_WU_SMEM ? wtile(s)[cl + c] : args.w[q.c0 + cl + c]) * kLog2e
+                            ? args.w[q.c0 + cl + c] * kLog2e
                             : 0.f;
             if (lane_active && WKV_PIPE_PACKED) {
                 // the same arithmetic as below on the lane's channel pair with f32x2 ops
@@ -438,9 +288,12 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
 #pragma unroll
             for (int c = 0; c < V; ++c) w2[c] = (lane_active && cl + c < q.nch) ? args.w[q.c0 + cl + c] * kLog2e : 0.f;
             // scan the chunk summaries (exclusive prefixes for the emitters) and publish the
-            // tile aggregate for later segments before looking back
+            // tile aggregate for later segments before looking back; the first read of the
+            // newest predecessor's slot is issued first, so its round trip overlaps the scan
             if (!mbar_wait(bar(s, kChunks), ph, lim) && lane == 0) report(kDevTimeoutCarry);
             if (lane == 0) WKV_TRACE_EVENT(unit, 3);
+            RawPair first;
+            if (q.j > 0 && lane_active) first = load_pair<Cg>(pp.slot + ((q.j - 1) * pp.G + q.g) * 4 * Cg, cl);
             Rec agg[V];
             if (lane_active) {
                 Rec* rc = recs(s);
@@ -485,7 +338,10 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
                         RawPair raw[kLook];
 #pragma unroll
                         for (int d = 0; d < kLook; ++d)
-                            if (hi - d >= 0) raw[d] = load_pair<Cg>(pp.slot + ((hi - d) * pp.G + q.g) * 4 * Cg, cl);
+                            if (hi - d >= 0)
+                                raw[d] = (it == 0 && d == 0)
+                                             ? first
+                                             : load_pair<Cg>(pp.slot + ((hi - d) * pp.G + q.g) * 4 * Cg, cl);
                         bool progressed = false;
 #pragma unroll
                         for (int d = 0; d < kLook; ++d) {
@@ -555,7 +411,7 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
             const int s = (int)(i % NS);
             const uint32_t ph = (uint32_t)((i / NS) & 1);
             if (!mbar_wait(bar(s, kCarry), ph, lim) && lane == 0) report(kDevTimeoutCarry);
-            (void)mbar_wait(bar(s, kFull), ph, lim);  // already complete; orders the tile reads
+            (void)mbar_wait(bar(s, kFull0 + ew * LC / BR), ph, lim);  // already complete; orders the tile reads
             const int64_t unit = stage_unit[s];
             if (unit < 0) break;
             if (ew == 0 && lane == 0) WKV_TRACE_EVENT(unit, 8);
@@ -569,8 +425,8 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
 #pragma unroll
                 for (int c = 0; c < V; ++c) {
                     const bool ok = cl + c < q.nch;
-                    w2[c] = ok ? (WKV_PIPE_WU_SMEM ? wtile(s)[cl + c] : args.w[q.c0 + cl + c]) * kLog2e : 0.f;
-                    u2[c] = ok ? (WKV_PIPE_WU_SMEM ? utile(s)[cl + c] : args.u[q.c0 + cl + c]) * kLog2e : 0.f;
+                    w2[c] = ok ? args.w[q.c0 + cl + c] * kLog2e : 0.f;
+                    u2[c] = ok ? args.u[q.c0 + cl + c] * kLog2e : 0.f;
                     const Rec cr = rec_combine(carries(s)[cl + c], recs(s)[ew * Cg + cl + c], (float)r_begin, w2[c]);
                     a[c] = cr.a;
                     bb[c] = cr.b;
@@ -750,49 +606,21 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
     }
 }
 
-// Tensor maps for k and v viewed as [B][T][C] (3-D, channels innermost), box = one tile.
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
-bool make_tile_map(CUtensorMap* tm, const void* base, int64_t B, int64_t T, int64_t C, int io, int Cg, int Ts) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t es = io == 1 ? 2 : 4;
-    cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
-    cuuint64_t strides[2] = {(cuuint64_t)C * es, (cuuint64_t)T * (cuuint64_t)C * es};
-    cuuint32_t box[3] = {(cuuint32_t)Cg, (cuuint32_t)Ts, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    const CUresult r = fn(tm, io == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
-                          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 template <typename TIO, int V, int NWS, int LC>
 cudaError_t launch_pipe_t(const ForwardArgs& a, const ChunkGeom& g, const PipeParams& pp, cudaStream_t s) {
     // as many stages as fit in the 227 KB a CTA may use (at most 5)
-    constexpr size_t stage = PipeLayout<TIO, V, NWS, LC, 1>::stage;
-    constexpr size_t budget = 232448 - 512;
-    constexpr int NS = (int)(budget / (stage + 64) > 5 ? 5 : budget / (stage + 64));
+    constexpr size_t per_stage = PipeLayout<TIO, V, NWS, LC, 1>::per_stage;
+    constexpr size_t budget = 232448 - 24;  // the most dynamic shared memory a CTA may use, minus the misc words
+    constexpr int NS = (int)(budget / per_stage > 5 ? 5 : budget / per_stage);
     static_assert(NS >= 3, "tile too large for a three-stage ring");
     using Lay = PipeLayout<TIO, V, NWS, LC, NS>;
+    static_assert(Lay::total <= 232448, "shared memory layout over the per-CTA limit");
     auto kern = pipe_kernel<TIO, V, NWS, LC, NS>;
     CUtensorMap tmk, tmv;
-    constexpr int BR = kBoxRows < Lay::Ts ? kBoxRows : Lay::Ts;
-    static_assert(Lay::Ts % BR == 0, "tile rows must be a multiple of the box rows");
-    if (!make_tile_map(&tmk, a.k, a.B, a.T, a.C, a.io, Lay::Cg, BR) ||
-        !make_tile_map(&tmv, a.v, a.B, a.T, a.C, a.io, Lay::Cg, BR))
+    static_assert(Lay::Ts % Lay::BR == 0, "tile rows must be a multiple of the box rows");
+    static_assert(LC <= Lay::BR && Lay::BR % LC == 0, "a chunk must lie inside one box");
+    if (!make_tile_map(&tmk, a.k, a.B, a.T, a.C, a.io, Lay::Cg, Lay::BR) ||
+        !make_tile_map(&tmv, a.v, a.B, a.T, a.C, a.io, Lay::Cg, Lay::BR))
         return cudaErrorInvalidValue;
     static uint64_t attr_done = 0;  // per device; set once so captured launches issue no attribute call
     int dev = 0;

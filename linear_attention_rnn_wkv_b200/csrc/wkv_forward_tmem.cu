@@ -1,0 +1,828 @@
+// Persistent, warp-specialised chunked WKV forward that parks each tile in tensor memory
+// (the default chunked path when rows are 16-byte multiples).
+//
+// The arithmetic and the inter-CTA protocol are those of the shared-memory pipeline
+// (wkv_forward_pipe.cu): a unit is a tile of Ts = 8 * LC time steps by 64 channels; units
+// are taken by an atomic ticket in time-segment-major order; each unit's chunk summaries
+// fold into a tile aggregate, a decoupled look-back over earlier segments of the same
+// channel group yields the carry, and each chunk is re-scanned from its carry to write y
+// (the decay telescopes: RWKV transformer-math page, aicassindra.com, section "Why it
+// collapses into a recurrence").
+//
+// What changes is where a tile waits for its carry.  A unit's k and v rows are needed
+// twice, by the summaries and, after the look-back, by the re-scan; in between the tile
+// sits idle for several microseconds.  Here the TMA lands a tile in a shared-memory stage,
+// each summarising warp copies its chunk into its quadrant of the SM's tensor memory
+// (tcgen05.st, 512 columns x 128 lanes x 32 bits) while it reads it, and the stage is
+// free again as soon as the summaries are done.  The emitting warp of the same quadrant
+// reads the chunk back (tcgen05.ld) once the carry is known.  Tensor memory holds 4
+// (fp32) or 8 (bf16) units, so that many units per SM wait for carries at once while
+// only 2-4 shared-memory stages are needed for the loads.
+//
+// Roles (20 warps):
+//   warp 0          producer: a ticket once a stage and a unit slot are free, the unit's
+//                   TMA box copies (`full`, one barrier per box of rows); also allocates
+//                   and frees the tensor memory;
+//   warps 1-3       look-back, round robin over units: scan the chunk summaries, publish
+//                   the aggregate, fold predecessors' records into the carry, publish
+//                   the inclusive prefix, hand the carry over (`carry`);
+//   warps 4-11      summarise chunk c = warp - 4: summary record, rows into tensor memory
+//                   (`chunks`; the stage is released, `dempty`);
+//   warps 12-19     emit chunk c = warp - 12 (same quadrant as its summariser): rows back
+//                   from tensor memory, re-scan in a fixed frame, y to HBM (`uempty`).
+// All waits are bounded (error word on expiry, then the pipeline keeps moving), and the
+// tensor memory is freed on every path before the CTA exits.  Deadlock freedom: a ticket
+// is taken only when its stage and slot are free, roles handle a CTA's units in ticket
+// order, and every cross-CTA wait is on a smaller ticket.
+#include <type_traits>
+
+#include "wkv_device.cuh"
+#include "wkv_internal.h"
+#include "wkv_vec.cuh"
+#include "wkv_pipe_common.cuh"
+
+#ifdef WKV_TRACE
+extern "C" cudaError_t wkv_trace_set_buffer(void* p) { return cudaMemcpyToSymbol(g_wkv_trace, &p, sizeof(p)); }
+#endif
+
+namespace wkvb {
+namespace {
+
+// ---------------------------------------------------------------------------
+// Tensor memory (tcgen05) helpers.  A warp reaches the 32 lanes of its quadrant
+// (warp index mod 4); the 32x32b shape gives thread i lane (quadrant * 32 + i) and N
+// consecutive 32-bit columns.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+template <int N>
+struct TmemIO;
+
+template <>
+struct TmemIO<8> {
+    static __device__ __forceinline__ void st(uint32_t taddr, const uint32_t (&r)[8]) {
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                     : "memory");
+    }
+    static __device__ __forceinline__ void ld(uint32_t taddr, uint32_t (&r)[8]) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];" : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]) : "r"(taddr)
+                     : "memory");
+    }
+    // completes this thread's earlier loads; the operands tie r's later uses to it
+    static __device__ __forceinline__ void wait_ld(uint32_t (&r)[8]) {
+        asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7])::"memory");
+    }
+    // completes this thread's earlier stores before r's registers are reused
+    static __device__ __forceinline__ void wait_st(uint32_t (&r)[8]) {
+        asm volatile("tcgen05.wait::st.sync.aligned;" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7])::"memory");
+    }
+};
+
+template <>
+struct TmemIO<16> {
+    static __device__ __forceinline__ void st(uint32_t taddr, const uint32_t (&r)[16]) {
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+                     : "memory");
+    }
+    static __device__ __forceinline__ void ld(uint32_t taddr, uint32_t (&r)[16]) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];" : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]) : "r"(taddr)
+                     : "memory");
+    }
+    // completes this thread's earlier loads; the operands tie r's later uses to it
+    static __device__ __forceinline__ void wait_ld(uint32_t (&r)[16]) {
+        asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])::"memory");
+    }
+    // completes this thread's earlier stores before r's registers are reused
+    static __device__ __forceinline__ void wait_st(uint32_t (&r)[16]) {
+        asm volatile("tcgen05.wait::st.sync.aligned;" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])::"memory");
+    }
+};
+
+
+// A lane's two channels of one row as 32-bit words: two fp32 words, or one bf16 pair.
+template <typename TIO>
+struct Pk;
+template <>
+struct Pk<float> {
+    static constexpr int W = 2;
+    static __device__ __forceinline__ void load(const float* p, uint32_t* w) {
+        const float2 f = *reinterpret_cast<const float2*>(p);
+        w[0] = __float_as_uint(f.x);
+        w[1] = __float_as_uint(f.y);
+    }
+    static __device__ __forceinline__ float2 unpack(const uint32_t* w) {
+        return make_float2(__uint_as_float(w[0]), __uint_as_float(w[1]));
+    }
+};
+template <>
+struct Pk<__nv_bfloat16> {
+    static constexpr int W = 1;
+    static __device__ __forceinline__ void load(const __nv_bfloat16* p, uint32_t* w) {
+        w[0] = *reinterpret_cast<const uint32_t*>(p);
+    }
+    static __device__ __forceinline__ float2 unpack(const uint32_t* w) { return make_float2(bf_lo(w[0]), bf_hi(w[0])); }
+};
+
+constexpr int kNWS = 8;   // chunks per tile (summarising warps, emitting warps)
+constexpr int kNL = 3;    // look-back warps
+constexpr int kCg = 64;   // channels per tile (a lane owns a pair)
+constexpr int kThreads = (1 + kNL + 2 * kNWS) * 32;
+
+template <typename TIO, int LC, int NS, int NT>
+struct TmLayout {
+    static constexpr int Cg = kCg;
+    static constexpr int Ts = kNWS * LC;
+    static constexpr size_t tile = sizeof(TIO) * Ts * Cg;  // one array (k or v)
+    static constexpr size_t stage = align128(2 * tile);     // shared-memory stage: k tile, v tile
+    // unit slot: chunk records [NWS][Cg], carries [Cg], chunk maxima [NWS][Cg]
+    static constexpr size_t recs_off = 0;
+    static constexpr size_t carry_off = recs_off + sizeof(Rec) * kNWS * Cg;
+    static constexpr size_t mx_off = carry_off + sizeof(Rec) * Cg;
+    static constexpr size_t slot = align128(mx_off + sizeof(float) * kNWS * Cg);
+    static constexpr int BR = kBoxRows < Ts ? kBoxRows : Ts;  // rows per TMA box
+    static constexpr int NB = Ts / BR;
+    static constexpr size_t slots_off = NS * stage;
+    static constexpr size_t bars_off = slots_off + NT * slot;
+    static constexpr int NBARS = NS * (NB + 1) + NT * 3;  // per stage: NB full + 1 empty; per slot: chunks, carry, empty
+    static constexpr size_t misc_off = bars_off + NBARS * 8;  // slot unit ids [NT], end index, epoch, tensor memory base
+    static constexpr size_t total = misc_off + NT * 8 + 8 + 8;
+    // tensor memory: words per row per lane, columns per chunk array, per chunk, per unit and quadrant
+    static constexpr int W = Pk<TIO>::W;
+    static constexpr int CPA = LC * W;
+    static constexpr int CPC = 2 * CPA;
+    static constexpr int CPU = (kNWS / 4) * CPC;
+    static constexpr int SR = 8 / W;   // rows per tensor-memory slice (8 words: two slices of k and v
+    static constexpr int SW = SR * W;  // stay in registers while the next pair is read)
+    static_assert(NT * CPU <= 512, "unit slots exceed the tensor memory");
+    static_assert(LC % SR == 0, "slices must tile a chunk");
+};
+
+template <typename TIO, int LC, int NS, int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+    tmem_kernel(ForwardArgs args, PipeParams pp, const __grid_constant__ CUtensorMap tmk,
+                const __grid_constant__ CUtensorMap tmv) {
+    using Lay = TmLayout<TIO, LC, NS, NT>;
+    constexpr int V = 2;
+    constexpr int Cg = Lay::Cg, Ts = Lay::Ts, NB = Lay::NB, BR = Lay::BR, W = Lay::W, SR = Lay::SR, SW = Lay::SW;
+    constexpr int W_L0 = 1, W_S0 = 1 + kNL, W_E0 = 1 + kNL + kNWS;
+    static_assert(W_S0 % 4 == 0 && W_E0 % 4 == 0, "a chunk's summariser and emitter must share a quadrant");
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bars_off);
+    int64_t* slot_unit = reinterpret_cast<int64_t*>(smem + Lay::misc_off);
+    volatile int64_t* s_iend = reinterpret_cast<volatile int64_t*>(slot_unit + NT);
+    uint32_t* s_epoch = reinterpret_cast<uint32_t*>(slot_unit + NT + 1);
+    uint32_t* s_tmem = s_epoch + 1;
+    auto dfull = [&](int s, int b) { return &bars[s * (NB + 1) + b]; };
+    auto dempty = [&](int s) { return &bars[s * (NB + 1) + NB]; };
+    auto chunks_bar = [&](int t) { return &bars[NS * (NB + 1) + t * 3 + 0]; };
+    auto carry_bar = [&](int t) { return &bars[NS * (NB + 1) + t * 3 + 1]; };
+    auto uempty = [&](int t) { return &bars[NS * (NB + 1) + t * 3 + 2]; };
+    auto ktile = [&](int s) { return reinterpret_cast<TIO*>(smem + s * Lay::stage); };
+    auto vtile = [&](int s) { return reinterpret_cast<TIO*>(smem + s * Lay::stage + Lay::tile); };
+    auto slotp = [&](int t) { return smem + Lay::slots_off + t * Lay::slot; };
+    auto recs = [&](int t) { return reinterpret_cast<Rec*>(slotp(t) + Lay::recs_off); };
+    auto carries = [&](int t) { return reinterpret_cast<Rec*>(slotp(t) + Lay::carry_off); };
+    auto chunk_max = [&](int t) { return reinterpret_cast<float*>(slotp(t) + Lay::mx_off); };
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int64_t T = args.T, C = args.C, BC = args.B * args.C;
+    const uint32_t lim = args.spin_limit;
+
+    if (warp == 0) {
+        tmem_alloc(s_tmem, 512);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        *s_epoch = (*reinterpret_cast<volatile uint32_t*>(&pp.hdr->epoch) + 1u) & 0x3FFFFFFFu;
+        *s_iend = INT64_MAX;
+        for (int s = 0; s < NS; ++s) {
+            for (int b = 0; b < NB; ++b) mbar_init(dfull(s, b), 1);
+            mbar_init(dempty(s), kNWS);
+        }
+        for (int t = 0; t < NT; ++t) {
+            mbar_init(chunks_bar(t), kNWS);
+            mbar_init(carry_bar(t), 1);
+            mbar_init(uempty(t), kNWS);
+        }
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t epoch30 = *s_epoch;
+    const uint32_t tag_agg = (epoch30 << 2) | 1u, tag_incl = (epoch30 << 2) | 2u;
+    auto report = [&](uint32_t code) { atomicCAS(&pp.hdr->error, kDevOk, code); };
+    // this warp's quadrant; the columns of chunk c's array a (0 k, 1 v) in unit slot t
+    const uint32_t tq = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    auto tcol = [&](int t, int c, int a) { return (uint32_t)(t * Lay::CPU + (c >> 2) * Lay::CPC + a * Lay::CPA); };
+
+    struct Geo {
+        int64_t j, g, b, c0, t0;
+        int len, nch;
+    };
+    auto geo = [&](int64_t unit) {
+        Geo q;
+        q.j = unit / pp.G;
+        q.g = unit % pp.G;
+        q.b = q.g / pp.groups_per_b;
+        q.c0 = (q.g % pp.groups_per_b) * Cg;
+        q.t0 = q.j * Ts;
+        q.len = (int)min64(Ts, T - q.t0);
+        q.nch = (int)min64(Cg, C - q.c0);
+        return q;
+    };
+
+    if (warp == 0) {
+        // ------------------------------- producer -------------------------------
+        if (lane == 0) {
+            for (int64_t i = 0;; ++i) {
+                const int s = (int)(i % NS);
+                const int t = (int)(i % NT);
+                if (i >= NS && !mbar_wait(dempty(s), (uint32_t)((i / NS - 1) & 1), lim)) report(kDevTimeoutCopy);
+                if (i >= NT && !mbar_wait(uempty(t), (uint32_t)((i / NT - 1) & 1), lim)) report(kDevTimeoutCopy);
+                const uint32_t tk = atomicAdd(&pp.hdr->ticket, 1u);
+                if (tk >= (uint32_t)pp.U + gridDim.x) report(kDevBadWorkspace);
+                if (tk >= (uint32_t)pp.U) {
+                    *s_iend = i;
+                    slot_unit[t] = -1;
+                    for (int b = 0; b < NB; ++b) mbar_arrive(dfull(s, b));
+                    break;
+                }
+                const int64_t unit = tk;
+                WKV_TRACE_EVENT(unit, 0);
+                slot_unit[t] = unit;
+                const Geo q = geo(unit);
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    uint64_t* fb = dfull(s, b);
+                    mbar_arrive_expect_tx(fb, 2u * (uint32_t)(BR * Cg * sizeof(TIO)));
+                    tma_load_3d(ktile(s) + b * BR * Cg, &tmk, (int)q.c0, (int)(q.t0 + b * BR), (int)q.b, fb);
+                    tma_load_3d(vtile(s) + b * BR * Cg, &tmv, (int)q.c0, (int)(q.t0 + b * BR), (int)q.b, fb);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp < W_S0) {
+        // ------------------------------- look-back ------------------------------
+        const int l = warp - W_L0;
+        for (int64_t i = l;; i += kNL) {
+            const int t = (int)(i % NT);
+            const uint32_t ph = (uint32_t)((i / NT) & 1);
+            bool got = false, gone = false;
+            for (uint32_t it = 0; it <= lim; ++it) {
+                if (WKV_WAIT_HINT ? mbar_try_wait_hint(chunks_bar(t), ph, WKV_WAIT_HINT)
+                                  : mbar_try_wait(chunks_bar(t), ph)) {
+                    got = true;
+                    break;
+                }
+                if (*s_iend < i) {  // past the end (the sentinel unit itself still arrives)
+                    gone = true;
+                    break;
+                }
+                if (!WKV_WAIT_HINT) __nanosleep(32);
+            }
+            if (gone) break;
+            if (!got && lane == 0) report(kDevTimeoutCarry);
+            const int64_t unit = slot_unit[t];
+            if (unit < 0) {
+                if (lane == 0) mbar_arrive(carry_bar(t));
+                break;
+            }
+            if (lane == 0) WKV_TRACE_EVENT(unit, 3);
+            const Geo q = geo(unit);
+            const int cl = lane * V;
+            const bool lane_active = cl < q.nch;
+            float w2[V];
+#pragma unroll
+            for (int c = 0; c < V; ++c) w2[c] = lane_active ? args.w[q.c0 + cl + c] * kLog2e : 0.f;
+            // the first read of the newest predecessor's slot overlaps the scan
+            RawPair first;
+            if (q.j > 0 && lane_active) first = load_pair<Cg>(pp.slot + ((q.j - 1) * pp.G + q.g) * 4 * Cg, cl);
+            // scan the chunk summaries (exclusive prefixes for the emitters) and publish the
+            // tile aggregate for later segments
+            Rec agg[V];
+            if (lane_active) {
+                Rec* rc = recs(t);
+#pragma unroll
+                for (int c = 0; c < V; ++c) agg[c] = rec_identity();
+#pragma unroll
+                for (int w = 0; w < kNWS; ++w) {
+                    const int lw = max(0, min(LC, q.len - w * LC));
+#pragma unroll
+                    for (int c = 0; c < V; ++c) {
+                        const Rec r = rc[w * Cg + cl + c];
+                        rc[w * Cg + cl + c] = agg[c];  // exclusive prefix of chunk w
+                        if (lw > 0) agg[c] = rec_combine(agg[c], r, (float)lw, w2[c]);
+                    }
+                }
+                // (nch is even, so a lane's two channels are both in range or both out)
+                if (q.j > 0 && unit != pp.drop_unit) publish_pair<Cg>(pp.slot + unit * 4 * Cg, cl, agg[0], agg[1], tag_agg);
+            }
+            if (lane == 0) WKV_TRACE_EVENT(unit, 4);
+            Rec run[V];
+            if (q.j == 0) {
+#pragma unroll
+                for (int c = 0; c < V; ++c)
+                    run[c] = (args.state_in && lane_active) ? rec_from_state(args.state_in, q.b * C + q.c0 + cl + c, BC)
+                                                            : rec_identity();
+            } else {
+#pragma unroll
+                for (int c = 0; c < V; ++c) run[c] = rec_identity();
+                // Each lane looks back for its channel pair, kLook predecessor slots per round
+                // trip: it folds aggregates from the newest backwards and stops at the first
+                // inclusive prefix (the carry is then known) or at the first slot that is not
+                // yet published.
+                float span = 0.f;
+                int64_t hi = q.j - 1;
+                bool done = !lane_active;
+                uint32_t nap = 64;
+                bool all_done = false;
+                for (uint32_t it = 0; it <= lim && !all_done; ++it) {
+                    if (!done) {
+                        RawPair raw[kLook];
+#pragma unroll
+                        for (int d = 0; d < kLook; ++d)
+                            if (hi - d >= 0)
+                                raw[d] = (it == 0 && d == 0)
+                                             ? first
+                                             : load_pair<Cg>(pp.slot + ((hi - d) * pp.G + q.g) * 4 * Cg, cl);
+                        bool progressed = false;
+#pragma unroll
+                        for (int d = 0; d < kLook; ++d) {
+                            if (done) break;
+                            Rec r0, r1;
+                            const int kind = pair_kind(raw[d], tag_agg, tag_incl, r0, r1);
+                            if (kind == 0) break;
+                            run[0] = rec_combine(r0, run[0], span, w2[0]);
+                            run[1] = rec_combine(r1, run[1], span, w2[1]);
+                            progressed = true;
+                            if (kind == 2) {
+                                done = true;
+                            } else {
+                                span += (float)Ts;
+                                if (--hi < 0) done = true;
+                            }
+                        }
+                        if (!done && !progressed) {
+                            __nanosleep(nap);
+                            nap = nap < 1024 ? nap * 2 : 1024;
+                        } else if (progressed) {
+                            nap = 64;
+                        }
+                    }
+                    all_done = __all_sync(0xffffffffu, done);
+                }
+                if (!all_done) {
+                    report(kDevTimeoutCarry);
+                    pp.hdr->error_unit = (uint32_t)unit;
+                }
+            }
+            if (lane == 0) WKV_TRACE_EVENT(unit, 5);
+            // publish the inclusive prefix (it overwrites the aggregate), then hand the carry
+            // to the emitters
+            Rec inc[V];
+            if (lane_active) {
+#pragma unroll
+                for (int c = 0; c < V; ++c) inc[c] = rec_combine(run[c], agg[c], (float)q.len, w2[c]);
+                if (unit != pp.drop_unit) publish_pair<Cg>(pp.slot + unit * 4 * Cg, cl, inc[0], inc[1], tag_incl);
+                Rec* cs = carries(t);
+#pragma unroll
+                for (int c = 0; c < V; ++c) cs[cl + c] = run[c];
+            }
+            if (lane == 0) WKV_TRACE_EVENT(unit, 7);
+            __syncwarp();
+            if (lane == 0) {
+                WKV_TRACE_EVENT(unit, 6);
+                mbar_arrive(carry_bar(t));
+            }
+            if (lane_active && q.j == pp.S - 1 && args.state_out) {
+#pragma unroll
+                for (int c = 0; c < V; ++c) {
+                    const int64_t bc = q.b * C + q.c0 + cl + c;
+                    args.state_out[bc] = inc[c].a;
+                    args.state_out[BC + bc] = inc[c].b;
+                    args.state_out[2 * BC + bc] = rec_p(inc[c], w2[c]) * kLn2;
+                }
+            }
+        }
+    } else if (warp < W_E0) {
+        // ------------------------------- summarise ------------------------------
+        // Warp c summarises chunk c of each tile and moves its rows into tensor memory.
+        const int sw = warp - W_S0;
+        for (int64_t i = 0;; ++i) {
+            const int s = (int)(i % NS);
+            const int t = (int)(i % NT);
+            const uint32_t ph = (uint32_t)((i / NS) & 1);
+            if (!mbar_wait(dfull(s, sw * LC / BR), ph, lim) && lane == 0) report(kDevTimeoutCopy);
+            const int64_t unit = slot_unit[t];
+            if (unit < 0) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(chunks_bar(t));
+                break;
+            }
+            tc_fence_after();
+            if (sw == 0 && lane == 0) WKV_TRACE_EVENT(unit, 1);
+            const Geo q = geo(unit);
+            const int cl = lane * V;
+            const bool lane_active = cl < q.nch;
+            const int r_begin = sw * LC;
+            const int r_cnt = max(0, min(LC, q.len - r_begin));
+            if (r_cnt > 0) {
+                const float2 w2p = lane_active ? make_float2(args.w[q.c0 + cl] * kLog2e, args.w[q.c0 + cl + 1] * kLog2e)
+                                               : make_float2(0.f, 0.f);
+                const float2 L2 = make_float2(kLog2e, kLog2e);
+                const TIO* kt = ktile(s);
+                const TIO* vt = vtile(s);
+                // The TMA fills rows past T and channels past C with zeros, so every row of the
+                // chunk is read unconditionally; only the maxima and sums skip rows past the
+                // end.  A full chunk (the usual case) runs with no per-row test at all, so the
+                // rows' arithmetic interleaves freely.
+                float M0 = kPEmpty, M1 = kPEmpty;
+                float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
+                auto summarise = [&](auto full_c) {
+                    constexpr bool FULL = decltype(full_c)::value;
+                    float2 gx[LC];
+                    // pass 1: k rows -> exponents at the chunk's last row, their maximum; rows to
+                    // tensor memory
+#pragma unroll
+                    for (int h = 0; h < LC / SR; ++h) {
+                        uint32_t kw[SW];
+#pragma unroll
+                        for (int rr = 0; rr < SR; ++rr) {
+                            const int r = h * SR + rr;
+                            Pk<TIO>::load(kt + (r_begin + r) * Cg + cl, &kw[rr * W]);
+                            const float back = FULL ? -(float)(LC - 1 - r) : -(float)(r_cnt - 1 - r);
+                            gx[r] = __ffma2_rn(make_float2(back, back), w2p,
+                                               __fmul2_rn(Pk<TIO>::unpack(&kw[rr * W]), L2));
+                            if (FULL || r < r_cnt) {
+                                M0 = fmaxf(M0, gx[r].x);
+                                M1 = fmaxf(M1, gx[r].y);
+                            }
+                        }
+                        TmemIO<SW>::st(tq + tcol(t, sw, 0) + h * SW, kw);
+                        TmemIO<SW>::wait_st(kw);
+                    }
+                    // pass 2: v rows -> the chunk's sums relative to its maximum; rows to tensor
+                    // memory
+                    const float2 nM = make_float2(-M0, -M1);
+#pragma unroll
+                    for (int h = 0; h < LC / SR; ++h) {
+                        uint32_t vw[SW];
+#pragma unroll
+                        for (int rr = 0; rr < SR; ++rr) {
+                            const int r = h * SR + rr;
+                            Pk<TIO>::load(vt + (r_begin + r) * Cg + cl, &vw[rr * W]);
+                            if (FULL || r < r_cnt) {
+                                const float2 x = __fadd2_rn(gx[r], nM);
+                                const float2 e = make_float2(ex2(x.x), ex2(x.y));
+                                sa = __ffma2_rn(e, Pk<TIO>::unpack(&vw[rr * W]), sa);
+                                sb = __fadd2_rn(sb, e);
+                            }
+                        }
+                        TmemIO<SW>::st(tq + tcol(t, sw, 1) + h * SW, vw);
+                        TmemIO<SW>::wait_st(vw);
+                    }
+                };
+                if (r_cnt == LC)
+                    summarise(std::true_type{});
+                else
+                    summarise(std::false_type{});
+                if (lane_active) {
+                    Rec* rc = recs(t);
+                    rc[sw * Cg + cl] = Rec{sa.x, sb.x, M0, 0.f};
+                    rc[sw * Cg + cl + 1] = Rec{sa.y, sb.y, M1, 0.f};
+                    *reinterpret_cast<float2*>(chunk_max(t) + sw * Cg + cl) = make_float2(M0, M1);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(dempty(s));  // the stage's rows of this chunk are no longer needed
+                mbar_arrive(chunks_bar(t));
+            }
+            if (sw == 0 && lane == 0) WKV_TRACE_EVENT(unit, 2);
+        }
+    } else {
+        // --------------------------------- emit ---------------------------------
+        const int ew = warp - W_E0;  // chunk index
+        for (int64_t i = 0;; ++i) {
+            const int t = (int)(i % NT);
+            const uint32_t ph = (uint32_t)((i / NT) & 1);
+            if (!mbar_wait(carry_bar(t), ph, lim) && lane == 0) report(kDevTimeoutCarry);
+            const int64_t unit = slot_unit[t];
+            if (unit < 0) break;
+            tc_fence_after();
+            if (ew == 0 && lane == 0) WKV_TRACE_EVENT(unit, 8);
+            const Geo q = geo(unit);
+            const int cl = lane * V;
+            const bool lane_active = cl < q.nch;
+            const int r_begin = ew * LC;
+            const int r_cnt = max(0, min(LC, q.len - r_begin));
+            if (r_cnt > 0) {
+                // the first slice's rows are read while the carry is combined below
+                uint32_t kw[SW], vw[SW];
+                TmemIO<SW>::ld(tq + tcol(t, ew, 0), kw);
+                TmemIO<SW>::ld(tq + tcol(t, ew, 1), vw);
+                float w2[V], u2[V], a[V], bb[V], R[V], nn[V];
+                bool lazy_ok = true;
+#pragma unroll
+                for (int c = 0; c < V; ++c) {
+                    w2[c] = lane_active ? args.w[q.c0 + cl + c] * kLog2e : 0.f;
+                    u2[c] = lane_active ? args.u[q.c0 + cl + c] * kLog2e : 0.f;
+                    const Rec cr = lane_active
+                                       ? rec_combine(carries(t)[cl + c], recs(t)[ew * Cg + cl + c], (float)r_begin, w2[c])
+                                       : rec_identity();
+                    a[c] = cr.a;
+                    bb[c] = cr.b;
+                    R[c] = cr.anc;
+                    nn[c] = cr.n;
+                    lazy_ok = lazy_ok && fabsf(u2[c]) <= kLazyLimit && w2[c] <= kLazyLimit;
+                }
+                TIO* yg = static_cast<TIO*>(args.y) + (q.b * T + q.t0) * C + q.c0;
+                TmemIO<SW>::wait_ld(kw);
+                TmemIO<SW>::wait_ld(vw);
+                // Fixed-frame re-scan.  Seen from the chunk's last row, each token's weight
+                // e_i = 2^(k_i - (L-1-i) w - G) and the carried-in history K do not change from
+                // row to row (everything decays at the same rate), so with running sums S of
+                // K + e_i v_i and K + e_i over earlier rows and c = 2^(w - u)
+                //   y_r = (S^a + e_r v_r / c) / (S^b + e_r / c):
+                // no re-referencing and no selects, and only S is carried from row to row (the
+                // first row of a sequence without history returns v itself, as the
+                // recurrence does).  The frame G lies at most 100 above the larger of the
+                // history and the first token (so no term that matters can be flushed), at
+                // most 64 below the history (so K stays finite) and high enough that no later
+                // token's term can overflow; a chunk whose range leaves no such G takes the
+                // token-by-token step (one exp per token against a moving reference), and
+                // parameters outside that step's range take the page's two-exp step.
+                int mode = lazy_ok ? 1 : 2;
+                float2 fSa = make_float2(0.f, 0.f), fSb = fSa, fnG = fSa, fic = fSa;
+                if (WKV_PIPE_FRAME && lazy_ok) {
+                    const float2 k0 = Pk<TIO>::unpack(&kw[0]);
+                    const float k0v[2] = {k0.x, k0.y};
+                    float fa[V], fb[V], fg[V], fi[V];
+                    bool ok = true;
+                    const float fc = (float)r_cnt;
+#pragma unroll
+                    for (int c = 0; c < V; ++c) {
+                        const float M = lane_active ? chunk_max(t)[ew * Cg + cl + c] : 0.f;
+                        const float hK = fmaf(-fc, w2[c], fmaf(-nn[c], w2[c], R[c]));  // history, at the last row
+                        const float h0 = fmaf(-(fc - 1.f), w2[c], k0v[c] * kLog2e);     // first token, same
+                        const float bonus = u2[c] - w2[c];
+                        const float dom = fminf(fmaxf(hK, h0), fmaxf(hK, h0 + bonus));
+                        const float G = fmaxf(fminf(M, dom + 100.f), hK - 64.f);
+                        ok = ok && (M - G + fmaxf(bonus, 0.f) <= 100.f);
+                        const float sc = ex2(hK - G);
+                        fa[c] = a[c] * sc;
+                        fb[c] = bb[c] * sc;
+                        fg[c] = -G;
+                        fi[c] = ex2(bonus);
+                    }
+                    if (ok) {
+                        mode = 0;
+                        fSa = make_float2(fa[0], fa[1]);
+                        fSb = make_float2(fb[0], fb[1]);
+                        fnG = make_float2(fg[0], fg[1]);
+                        fic = make_float2(fi[0], fi[1]);
+                    }
+                }
+                const float back0 = 1.f - (float)r_cnt;  // -(steps from row 0 to the last row)
+                if (__all_sync(0xffffffffu, mode == 0 || !lane_active)) {
+                    // every lane in the fixed frame: one branch-free loop, the next slice's rows
+                    // read from tensor memory while this slice is computed
+                    const float2 L2 = make_float2(kLog2e, kLog2e);
+                    const float2 w2p = make_float2(w2[0], w2[1]);
+                    TIO* yrow = yg + (int64_t)r_begin * C + cl;
+                    auto emit = [&](auto full_c) {
+                        constexpr bool FULL = decltype(full_c)::value;
+#pragma unroll
+                        for (int h = 0; h < LC / SR; ++h) {
+                            uint32_t kn[SW], vn[SW];
+                            if (h + 1 < LC / SR) {
+                                TmemIO<SW>::ld(tq + tcol(t, ew, 0) + (h + 1) * SW, kn);
+                                TmemIO<SW>::ld(tq + tcol(t, ew, 1) + (h + 1) * SW, vn);
+                            }
+#pragma unroll
+                            for (int rr = 0; rr < SR; ++rr) {
+                                const int r = h * SR + rr;
+                                const float2 kp = Pk<TIO>::unpack(&kw[rr * W]);
+                                const float2 vp = Pk<TIO>::unpack(&vw[rr * W]);
+                                // k - G first: the large cancellation happens inside one rounding
+                                const float back = FULL ? (float)(r + 1 - LC) : back0 + (float)r;
+                                const float2 x = __ffma2_rn(make_float2(back, back), w2p, __ffma2_rn(kp, L2, fnG));
+                                const float2 e = make_float2(ex2(x.x), ex2(x.y));
+                                const float2 ec = __fmul2_rn(e, fic);
+                                const float2 num = __ffma2_rn(ec, vp, fSa);
+                                const float2 den = __fadd2_rn(fSb, ec);
+                                const float2 yv = __fmul2_rn(num, make_float2(rcp(den.x), rcp(den.y)));
+                                float yy[V] = {yv.x, yv.y};
+                                if (r == 0) {
+                                    if (fSb.x == 0.f) yy[0] = vp.x;
+                                    if (fSb.y == 0.f) yy[1] = vp.y;
+                                }
+                                fSa = __ffma2_rn(e, vp, fSa);
+                                fSb = __fadd2_rn(fSb, e);
+                                if (lane_active && (FULL || r < r_cnt)) Vec<TIO, V>::store(yrow + (int64_t)r * C, yy);
+                            }
+                            if (h + 1 < LC / SR) {
+                                TmemIO<SW>::wait_ld(kn);
+                                TmemIO<SW>::wait_ld(vn);
+#pragma unroll
+                                for (int x = 0; x < SW; ++x) {
+                                    kw[x] = kn[x];
+                                    vw[x] = vn[x];
+                                }
+                            }
+                        }
+                    };
+                    if (r_cnt == LC)
+                        emit(std::true_type{});
+                    else
+                        emit(std::false_type{});
+                } else {
+                const float2 L2 = make_float2(kLog2e, kLog2e), nL2 = make_float2(-kLog2e, -kLog2e);
+                const float2 w2p = make_float2(w2[0], w2[1]), u2p = make_float2(u2[0], u2[1]);
+                const float2 nu2p = make_float2(-u2[0], -u2[1]);
+                const float2 cwp = make_float2(ex2(w2[0] - u2[0]), ex2(w2[1] - u2[1]));
+                const float2 one = make_float2(1.f, 1.f);
+                float2 ap = make_float2(a[0], a[1]), bp = make_float2(bb[0], bb[1]);
+                float2 nRp = make_float2(-R[0], -R[1]), np = make_float2(nn[0], nn[1]);
+                float pp2[V] = {fmaf(-nn[0], w2[0], R[0]), fmaf(-nn[1], w2[1], R[1])};
+#pragma unroll
+                for (int h = 0; h < LC / SR; ++h) {
+                    if (h > 0) {
+                        TmemIO<SW>::ld(tq + tcol(t, ew, 0) + h * SW, kw);
+                        TmemIO<SW>::ld(tq + tcol(t, ew, 1) + h * SW, vw);
+                        TmemIO<SW>::wait_ld(kw);
+                        TmemIO<SW>::wait_ld(vw);
+                    }
+#pragma unroll
+                    for (int rr = 0; rr < SR; ++rr) {
+                        const int r = h * SR + rr;
+                        if (!lane_active || r >= r_cnt) continue;
+                        const int row = r_begin + r;
+                        const float2 kp = Pk<TIO>::unpack(&kw[rr * W]);
+                        const float2 vp = Pk<TIO>::unpack(&vw[rr * W]);
+                        float yy[V];
+                        if (mode == 0) {
+                            // k - G first: the large cancellation happens inside one rounding
+                            const float back = back0 + (float)r;
+                            const float2 x = __ffma2_rn(make_float2(back, back), w2p, __ffma2_rn(kp, L2, fnG));
+                            const float2 e = make_float2(ex2(x.x), ex2(x.y));
+                            const float2 ec = __fmul2_rn(e, fic);
+                            const float2 num = __ffma2_rn(ec, vp, fSa);
+                            const float2 den = __fadd2_rn(fSb, ec);
+                            const float2 yv = __fmul2_rn(num, make_float2(rcp(den.x), rcp(den.y)));
+                            yy[0] = (r == 0 && fSb.x == 0.f) ? vp.x : yv.x;
+                            yy[1] = (r == 0 && fSb.y == 0.f) ? vp.y : yv.y;
+                            fSa = __ffma2_rn(e, vp, fSa);
+                            fSb = __fadd2_rn(fSb, e);
+                        } else if (mode == 1) {
+                            // lazy_step on the pair; the reference is kept negated (nR = -R)
+                            const float2 uk = __ffma2_rn(kp, L2, u2p);
+                            const float2 nuk = __ffma2_rn(kp, nL2, nu2p);
+                            const float2 d = __ffma2_rn(np, w2p, __fadd2_rn(nRp, uk));  // (u + k) - (R - n w)
+                            const bool c0 = d.x > 0.f, c1 = d.y > 0.f;
+                            const float e0 = ex2(-fabsf(d.x)), e1 = ex2(-fabsf(d.y));
+                            const float2 sa = make_float2(c0 ? e0 : 1.f, c1 ? e1 : 1.f);
+                            const float2 sv = make_float2(c0 ? 1.f : e0, c1 ? 1.f : e1);
+                            const float2 tt = __fmul2_rn(sa, ap);
+                            const float2 num = __ffma2_rn(sv, vp, tt);
+                            const float2 den = __ffma2_rn(sa, bp, sv);
+                            const float2 yv = __fmul2_rn(num, make_float2(rcp(den.x), rcp(den.y)));
+                            const float2 nw = __fmul2_rn(sv, cwp);
+                            ap = __ffma2_rn(nw, vp, tt);
+                            bp = __ffma2_rn(sa, bp, nw);
+                            nRp = make_float2(c0 ? nuk.x : nRp.x, c1 ? nuk.y : nRp.y);
+                            const float2 n1 = __fadd2_rn(np, one);
+                            np = make_float2(c0 ? 1.f : n1.x, c1 ? 1.f : n1.y);
+                            yy[0] = yv.x;
+                            yy[1] = yv.y;
+                        } else {
+                            const float kv[2] = {kp.x, kp.y}, vv[2] = {vp.x, vp.y};
+#pragma unroll
+                            for (int c = 0; c < V; ++c) {
+                                const float k2 = kv[c] * kLog2e;
+                                yy[c] = wkv_output<false>(a[c], bb[c], pp2[c], u2[c] + k2, vv[c]);
+                                wkv_fold<false>(a[c], bb[c], pp2[c], pp2[c] - w2[c], k2, vv[c], w2[c]);
+                            }
+                        }
+                        Vec<TIO, V>::store(yg + (int64_t)row * C + cl, yy);
+                    }
+                }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (ew == 0 && lane == 0) WKV_TRACE_EVENT(unit, 9);
+            if (lane == 0) mbar_arrive(uempty(t));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+    if (tid == 0) {
+        __threadfence();
+        const uint32_t finished = atomicAdd(&pp.hdr->done, 1u) + 1u;
+        if (finished == gridDim.x) {
+            atomicExch(&pp.hdr->ticket, 0u);
+            atomicExch(&pp.hdr->done, 0u);
+            atomicExch(&pp.hdr->epoch, epoch30);
+        }
+    }
+}
+
+// Unit slots: as many as the tensor memory holds (at most 8); stages: as many as the rest
+// of the 227 KB of shared memory holds (at most 4).
+template <typename TIO, int LC>
+struct TmConfig {
+    static constexpr int NT0 = 512 / TmLayout<TIO, LC, 1, 1>::CPU;
+    static constexpr int NT = NT0 > 8 ? 8 : NT0;
+    static constexpr size_t fixed = TmLayout<TIO, LC, 0, NT>::total;  // everything but the stages
+    static constexpr size_t per_stage = TmLayout<TIO, LC, 1, NT>::stage + (TmLayout<TIO, LC, 1, NT>::NB + 1) * 8;
+    static constexpr int NS0 = (int)((232448 - fixed) / per_stage);
+    static constexpr int NS = NS0 > 4 ? 4 : NS0;
+};
+
+template <typename TIO, int LC>
+cudaError_t launch_tmem_t(const ForwardArgs& a, const ChunkGeom& g, const PipeParams& pp, cudaStream_t s) {
+    constexpr int NT = TmConfig<TIO, LC>::NT;
+    constexpr int NS = TmConfig<TIO, LC>::NS;
+    static_assert(NS >= 2, "fewer than two shared-memory stages");
+    // a look-back warp waits on unit i's slot only after finishing unit i - kNL, so the
+    // slot's previous phase (unit i - NT) is complete whenever NT >= kNL
+    static_assert(NT >= kNL, "fewer unit slots than look-back warps");
+    using Lay = TmLayout<TIO, LC, NS, NT>;
+    static_assert(Lay::total <= 232448, "shared memory layout over the per-CTA limit");
+    static_assert(Lay::Ts % Lay::BR == 0, "tile rows must be a multiple of the box rows");
+    static_assert(LC <= Lay::BR && Lay::BR % LC == 0, "a chunk must lie inside one box");
+    auto kern = tmem_kernel<TIO, LC, NS, NT>;
+    CUtensorMap tmk, tmv;
+    if (!make_tile_map(&tmk, a.k, a.B, a.T, a.C, a.io, Lay::Cg, Lay::BR) ||
+        !make_tile_map(&tmv, a.v, a.B, a.T, a.C, a.io, Lay::Cg, Lay::BR))
+        return cudaErrorInvalidValue;
+    static uint64_t attr_done = 0;  // per device; set once so captured launches issue no attribute call
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static int sms[64] = {0};
+    if (dev >= 64 || !(attr_done & (1ull << dev))) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::total);
+        if (e != cudaSuccess) return e;
+        int n = 0;
+        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) {
+            sms[dev] = n;
+            attr_done |= 1ull << dev;
+        }
+    }
+    const int64_t nsm = dev < 64 ? sms[dev] : 148;
+    const int64_t grid = g.U < nsm ? g.U : nsm;
+    kern<<<(unsigned)grid, kThreads, Lay::total, s>>>(a, pp, tmk, tmv);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_forward_tmem(const ForwardArgs& a, const ChunkGeom& g, void* ws, int64_t drop_unit,
+                                cudaStream_t s) {
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    PipeParams pp;
+    pp.groups_per_b = g.groups_per_b;
+    pp.G = g.G;
+    pp.S = g.S;
+    pp.U = g.U;
+    pp.hdr = reinterpret_cast<WsHeader*>(base);
+    pp.slot = reinterpret_cast<uint64_t*>(base + kWsHeaderBytes);
+    pp.drop_unit = drop_unit;
+    if (g.V != 2 || g.NW != kNWS) return cudaErrorInvalidValue;
+    if (a.io == 1) {
+        if (g.LC == 8) return launch_tmem_t<__nv_bfloat16, 8>(a, g, pp, s);
+        if (g.LC == 16) return launch_tmem_t<__nv_bfloat16, 16>(a, g, pp, s);
+        return cudaErrorInvalidValue;
+    }
+    if (g.LC == 8) return launch_tmem_t<float, 8>(a, g, pp, s);
+    if (g.LC == 16) return launch_tmem_t<float, 16>(a, g, pp, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace wkvb

@@ -70,6 +70,8 @@ cudaError_t launch_forward_chunked(const ForwardArgs& a, const ChunkGeom& g, voi
 // Persistent warp-specialised variant (bulk rows, chunk 8 or 16); same workspace layout.
 cudaError_t launch_forward_pipe(const ForwardArgs& a, const ChunkGeom& g, void* ws, int64_t drop_unit,
                                 cudaStream_t s);
+cudaError_t launch_forward_tmem(const ForwardArgs& a, const ChunkGeom& g, void* ws, int64_t drop_unit,
+                                cudaStream_t s);
 
 // ----- T == 0: state_out = state_in (or the empty state) -----
 cudaError_t launch_state_passthrough(int64_t BC, const float* state_in, float* state_out, cudaStream_t s);
