@@ -157,7 +157,8 @@ struct TmLayout {
     static constexpr size_t bars_off = slots_off + NT * slot;
     static constexpr int NBARS = NS * (NB + 1) + NT * 3;  // per stage: NB full + 1 empty; per slot: chunks, carry, empty
     static constexpr size_t misc_off = bars_off + NBARS * 8;  // slot unit ids [NT], end index, epoch, tensor memory base
-    static constexpr size_t total = misc_off + NT * 8 + 8 + 8;
+    static constexpr size_t stage_unit_off = misc_off + NT * 8 + 8 + 8;  // stage unit ids [NS]
+    static constexpr size_t total = stage_unit_off + NS * 8;
     // tensor memory: words per row per lane, columns per chunk array, per chunk, per unit and quadrant
     static constexpr int W = Pk<TIO>::W;
     static constexpr int CPA = LC * W;
@@ -177,6 +178,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int V = 2;
     constexpr int Cg = Lay::Cg, Ts = Lay::Ts, NB = Lay::NB, BR = Lay::BR, W = Lay::W, SR = Lay::SR, SW = Lay::SW;
     constexpr int W_L0 = 1, W_S0 = 1 + kNL, W_E0 = 1 + kNL + kNWS;
+    // Where a unit takes its slot.  With few slots (fp32: 4) they are the scarce resource and
+    // the summarisers take one only once the rows have landed; with more (bf16: 8) the
+    // producer takes it with the ticket, so no ticketed unit waits for a slot and holds up its
+    // successors in other CTAs.
+    constexpr bool kLateSlot = NT <= 4;
     static_assert(W_S0 % 4 == 0 && W_E0 % 4 == 0, "a chunk's summariser and emitter must share a quadrant");
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bars_off);
@@ -184,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int64_t* s_iend = reinterpret_cast<volatile int64_t*>(slot_unit + NT);
     uint32_t* s_epoch = reinterpret_cast<uint32_t*>(slot_unit + NT + 1);
     uint32_t* s_tmem = s_epoch + 1;
+    int64_t* stage_unit = reinterpret_cast<int64_t*>(smem + Lay::stage_unit_off);
     auto dfull = [&](int s, int b) { return &bars[s * (NB + 1) + b]; };
     auto dempty = [&](int s) { return &bars[s * (NB + 1) + NB]; };
     auto chunks_bar = [&](int t) { return &bars[NS * (NB + 1) + t * 3 + 0]; };
@@ -252,20 +259,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             for (int64_t i = 0;; ++i) {
                 const int s = (int)(i % NS);
-                const int t = (int)(i % NT);
                 if (i >= NS && !mbar_wait(dempty(s), (uint32_t)((i / NS - 1) & 1), lim)) report(kDevTimeoutCopy);
-                if (i >= NT && !mbar_wait(uempty(t), (uint32_t)((i / NT - 1) & 1), lim)) report(kDevTimeoutCopy);
+                const int t = (int)(i % NT);
+                if (!kLateSlot && i >= NT && !mbar_wait(uempty(t), (uint32_t)((i / NT - 1) & 1), lim))
+                    report(kDevTimeoutCopy);
                 const uint32_t tk = atomicAdd(&pp.hdr->ticket, 1u);
                 if (tk >= (uint32_t)pp.U + gridDim.x) report(kDevBadWorkspace);
                 if (tk >= (uint32_t)pp.U) {
                     *s_iend = i;
-                    slot_unit[t] = -1;
+                    stage_unit[s] = -1;
+                    if (!kLateSlot) slot_unit[t] = -1;
                     for (int b = 0; b < NB; ++b) mbar_arrive(dfull(s, b));
                     break;
                 }
                 const int64_t unit = tk;
                 WKV_TRACE_EVENT(unit, 0);
-                slot_unit[t] = unit;
+                stage_unit[s] = unit;
+                if (!kLateSlot) slot_unit[t] = unit;
                 const Geo q = geo(unit);
 #pragma unroll
                 for (int b = 0; b < NB; ++b) {
@@ -429,7 +439,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int t = (int)(i % NT);
             const uint32_t ph = (uint32_t)((i / NS) & 1);
             if (!mbar_wait(dfull(s, sw * LC / BR), ph, lim) && lane == 0) report(kDevTimeoutCopy);
-            const int64_t unit = slot_unit[t];
+            const int64_t unit = stage_unit[s];
+            // with late slots, the unit slot (tensor-memory columns and records) is taken only
+            // now that the rows are here, so a slot is held from the summaries to the re-scan's end
+            if (kLateSlot) {
+                if (i >= NT && !mbar_wait(uempty(t), (uint32_t)((i / NT - 1) & 1), lim) && lane == 0)
+                    report(kDevTimeoutCopy);
+                if (sw == 0 && lane == 0) slot_unit[t] = unit;
+            }
             if (unit < 0) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(chunks_bar(t));
