@@ -140,7 +140,8 @@ def measured_peaks():
 def kernel_source_digest():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_attention_rnn_wkv_b200", "csrc")
-    for name in ("wkv_device.cuh", "wkv_vec.cuh", "wkv_internal.h", "wkv_forward_chunked.cu", "wkv_forward_pipe.cu"):
+    for name in ("wkv_device.cuh", "wkv_vec.cuh", "wkv_internal.h", "wkv_pipe_common.cuh", "wkv_forward_chunked.cu",
+                 "wkv_forward_tmem.cu"):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -149,7 +150,7 @@ def kernel_source_digest():
 def profiled_traffic(workload):
     """DRAM bytes per launch of the forward kernel from the committed ncu summary, if it
     was taken on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", f"pipe_kernel_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"tmem_kernel_{workload}.md")
     try:
         txt = open(path).read()
     except OSError:
