@@ -138,7 +138,12 @@ struct Pk<__nv_bfloat16> {
 constexpr int kNWS = 8;   // chunks per tile (summarising warps, emitting warps)
 constexpr int kNL = 3;    // look-back warps
 constexpr int kCg = 64;   // channels per tile (a lane owns a pair)
-constexpr int kThreads = (1 + kNL + 2 * kNWS) * 32;
+// Emitting warp sets: each set has a warp per chunk index and takes every kES-th unit.
+#ifndef WKV_TMEM_EMIT_SETS
+#define WKV_TMEM_EMIT_SETS 1
+#endif
+constexpr int kES = WKV_TMEM_EMIT_SETS;
+constexpr int kThreads = (1 + kNL + (1 + kES) * kNWS) * 32;
 
 template <typename TIO, int LC, int NS, int NT>
 struct TmLayout {
@@ -536,11 +541,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // --------------------------------- emit ---------------------------------
-        const int ew = warp - W_E0;  // chunk index
-        for (int64_t i = 0;; ++i) {
+        const int ew = (warp - W_E0) % kNWS;  // chunk index (the same quadrant as its summariser)
+        const int es = (warp - W_E0) / kNWS;  // emitting set: units es, es + kES, ...
+        for (int64_t i = es;; i += kES) {
             const int t = (int)(i % NT);
             const uint32_t ph = (uint32_t)((i / NT) & 1);
-            if (!mbar_wait(carry_bar(t), ph, lim) && lane == 0) report(kDevTimeoutCarry);
+            bool got = false, gone = false;
+            for (uint32_t it = 0; it <= lim; ++it) {
+                if (WKV_WAIT_HINT ? mbar_try_wait_hint(carry_bar(t), ph, WKV_WAIT_HINT) : mbar_try_wait(carry_bar(t), ph)) {
+                    got = true;
+                    break;
+                }
+                // past the end: with several emitting sets, only one meets the sentinel unit
+                if (*s_iend < i) {
+                    gone = true;
+                    break;
+                }
+                if (!WKV_WAIT_HINT) __nanosleep(32);
+            }
+            if (gone) break;
+            if (!got && lane == 0) report(kDevTimeoutCarry);
             const int64_t unit = slot_unit[t];
             if (unit < 0) break;
             tc_fence_after();
@@ -787,6 +807,9 @@ cudaError_t launch_tmem_t(const ForwardArgs& a, const ChunkGeom& g, const PipePa
     // a look-back warp waits on unit i's slot only after finishing unit i - kNL, so the
     // slot's previous phase (unit i - NT) is complete whenever NT >= kNL
     static_assert(NT >= kNL, "fewer unit slots than look-back warps");
+    // an emitting warp waits on unit i's slot only after finishing unit i - kES; the slot's
+    // previous unit i - NT must be one it has handled, so NT is a multiple of kES
+    static_assert(NT % kES == 0, "unit slots must divide among the emitting sets");
     using Lay = TmLayout<TIO, LC, NS, NT>;
     static_assert(Lay::total <= 232448, "shared memory layout over the per-CTA limit");
     static_assert(Lay::Ts % Lay::BR == 0, "tile rows must be a multiple of the box rows");
