@@ -118,6 +118,17 @@ wkv_status wkv_workspace_init(void* workspace, size_t ws_bytes, cudaStream_t str
 wkv_status wkv_forward_status(void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * Synchronises `stream`, then reports and clears the library's device-wide error word on
+ * the current device: WKV_ERR_TIMEOUT if any forward launched on this device since the last
+ * call gave up a bounded device-side wait (its outputs are then invalid; the workspace it
+ * used also carries the error, see wkv_forward_status), else WKV_OK.  WKV_ERR_CUDA if the
+ * synchronisation or the read fails (e.g. an earlier fault).  The word is shared by all
+ * streams and workspaces of the device, so a report may concern another stream's launch.
+ * The pages have no counterpart: this is the library's failure detection for its own waits.
+ */
+wkv_status wkv_get_device_status(cudaStream_t stream);
+
+/*
  * One decode step for N sessions x L layers x C channels: for every row (n, l) and
  * channel c, emit wkv for the token (k, v) from the stored state and fold the token
  * into the state (aiwiki "RWKV": the one-token decode step; transformer-math page,

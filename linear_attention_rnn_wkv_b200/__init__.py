@@ -65,6 +65,7 @@ def lib():
                 L.wkv_forward_workspace_size.restype = sz
                 L.wkv_workspace_init.argtypes = [vp, sz, vp]
                 L.wkv_forward_status.argtypes = [vp, sz, vp]
+                L.wkv_get_device_status.argtypes = [vp]
                 L.wkv_decode_step.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp]
                 L.wkv_decode_step_fused.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
                 L.token_shift_mix.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp]
@@ -73,6 +74,7 @@ def lib():
                 L.wkv_forward_auto_path.argtypes = [i64, i64, i64, i32]
                 L.wkv_testhook_forward_drop.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, sz, i64, u32, vp]
                 for f in (L.wkv_forward, L.wkv_forward_ex, L.wkv_workspace_init, L.wkv_forward_status,
+                          L.wkv_get_device_status,
                           L.wkv_decode_step, L.wkv_decode_step_fused, L.token_shift_mix,
                           L.wkv_forward_auto_path, L.wkv_testhook_forward_drop):
                     f.restype = i32
@@ -181,6 +183,13 @@ def forward_status(workspace=None, device=None):
     dev = torch.device(device or "cuda")
     ptr, n = (workspace.data_ptr(), workspace.numel()) if workspace is not None else (None, 0)
     _check(lib().wkv_forward_status(ptr, n, _stream(dev)), "wkv_forward_status")
+
+
+def get_device_status(device=None):
+    """Synchronise the current stream and report (then clear) a device-side timeout of any
+    forward on the device since the last call (raises WkvError)."""
+    dev = torch.device(device or "cuda")
+    _check(lib().wkv_get_device_status(_stream(dev)), "wkv_get_device_status")
 
 
 def wkv_decode_step(w, u, k, v, state, y=None):

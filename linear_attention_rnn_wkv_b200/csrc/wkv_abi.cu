@@ -14,8 +14,9 @@ using namespace wkvb;
 
 thread_local int g_last_cuda_error = 0;
 
-// Library-owned status block for launches that run without a workspace (the
-// serial path): word 0 is the device error code, word 1 the failing unit.
+// Library-owned status block: words 0-1 are the error code and failing unit of launches
+// that run without a workspace (the serial path); word 2 is the device-wide error word
+// every kernel also records its first timeout in (wkv_get_device_status).
 __device__ uint32_t g_status_block[4];
 
 wkv_status cuda_fail(cudaError_t e) {
@@ -49,6 +50,15 @@ uint32_t* status_word() {
     }
     return cache[dev];
 }
+
+}  // namespace
+
+uint32_t* wkvb::device_status_word() {
+    uint32_t* w = status_word();
+    return w ? w + 2 : nullptr;
+}
+
+namespace {
 
 // Default path table: the chunked scan exposes T-parallelism and wins unless there
 // are enough independent channels to fill every SM with serial scans.
@@ -97,7 +107,8 @@ wkv_status forward_impl(int64_t B, int64_t T, int64_t C, wkv_dtype io, const flo
     if (path == WKV_PATH_AUTO) path = auto_path(B, T, C, io);
     if (path == WKV_PATH_SERIAL) {
         a.err = workspace && ws_bytes >= kWsHeaderBytes ? &static_cast<WsHeader*>(workspace)->error : status_word();
-        if (!a.err) return cuda_fail(cudaGetLastError());
+        a.dev_err = device_status_word();
+        if (!a.err || !a.dev_err) return cuda_fail(cudaGetLastError());
         const int64_t grid = B * ((C + 127) / 128);
         if (grid > INT32_MAX) return WKV_ERR_UNSUPPORTED;
         cudaError_t e = launch_forward_serial(a, stream);
@@ -108,6 +119,8 @@ wkv_status forward_impl(int64_t B, int64_t T, int64_t C, wkv_dtype io, const flo
     if (g.U > INT32_MAX) return WKV_ERR_UNSUPPORTED;
     if (!workspace || ws_bytes < g.ws_bytes) return WKV_ERR_INVALID_ARG;
     a.err = &static_cast<WsHeader*>(workspace)->error;
+    a.dev_err = device_status_word();
+    if (!a.dev_err) return cuda_fail(cudaGetLastError());
     cudaError_t e = launch_forward_chunked(a, g, workspace, drop_unit, stream);
     return e == cudaSuccess ? WKV_OK : cuda_fail(e);
 }
@@ -177,6 +190,21 @@ wkv_status wkv_forward_status(void* workspace, size_t ws_bytes, cudaStream_t str
         const uint32_t zero[2] = {0, 0};
         e = cudaMemcpy(word, zero, sizeof(zero), cudaMemcpyHostToDevice);
     }
+    if (e != cudaSuccess) return cuda_fail(e);
+    return WKV_ERR_TIMEOUT;
+}
+
+wkv_status wkv_get_device_status(cudaStream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    uint32_t* word = device_status_word();
+    if (!word) return cuda_fail(cudaGetLastError());
+    uint32_t code = 0;
+    e = cudaMemcpy(&code, word, sizeof(code), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (code == kDevOk) return WKV_OK;
+    const uint32_t zero = 0;
+    e = cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return cuda_fail(e);
     return WKV_ERR_TIMEOUT;
 }

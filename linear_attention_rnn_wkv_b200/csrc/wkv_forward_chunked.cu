@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(NW * 32) chunked_kernel(ForwardArgs args, Chun
             // the workspace was not zero-filled (or is in use by an overlapping launch):
             // stay in bounds, report it; the waits below are bounded
             atomicCAS(&cp.hdr->error, kDevOk, kDevBadWorkspace);
+            atomicCAS(args.dev_err, kDevOk, kDevBadWorkspace);
             ticket %= gridDim.x;
         }
         *s_ticket = (int64_t)ticket;
@@ -156,6 +157,7 @@ __global__ void __launch_bounds__(NW * 32) chunked_kernel(ForwardArgs args, Chun
         copy_failed = __syncthreads_or(timed_out);
         if (copy_failed && tid == 0) {
             atomicCAS(&cp.hdr->error, kDevOk, kDevTimeoutCopy);
+            atomicCAS(args.dev_err, kDevOk, kDevTimeoutCopy);
             cp.hdr->error_unit = (uint32_t)unit;
         }
     } else {
@@ -282,6 +284,7 @@ __global__ void __launch_bounds__(NW * 32) chunked_kernel(ForwardArgs args, Chun
                     // a predecessor never published: record it, take the rest of the carry as empty
                     if (lane == 0) {
                         atomicCAS(&cp.hdr->error, kDevOk, kDevTimeoutCarry);
+                        atomicCAS(args.dev_err, kDevOk, kDevTimeoutCarry);
                         cp.hdr->error_unit = (uint32_t)unit;
                     }
                     break;

@@ -100,7 +100,10 @@ __global__ void __launch_bounds__((1 + 2 * NWS + NS) * 32, 1)
     __syncthreads();
     const uint32_t epoch30 = *s_epoch;
     const uint32_t tag_agg = (epoch30 << 2) | 1u, tag_incl = (epoch30 << 2) | 2u;
-    auto report = [&](uint32_t code) { atomicCAS(&pp.hdr->error, kDevOk, code); };
+    auto report = [&](uint32_t code) {
+        atomicCAS(&pp.hdr->error, kDevOk, code);
+        atomicCAS(args.dev_err, kDevOk, code);
+    };
 
     struct Geo {
         int64_t j, g, b, c0, t0;

@@ -114,7 +114,10 @@ __global__ void __launch_bounds__(NT) serial_bulk_kernel(ForwardArgs args) {
         }
         // one CTA-wide decision, so warp 0 keeps its copies and expectations in step
         if (__syncthreads_or(timed_out)) {
-            if (tid == 0) atomicCAS(args.err, kDevOk, kDevTimeoutCopy);
+            if (tid == 0) {
+                atomicCAS(args.err, kDevOk, kDevTimeoutCopy);
+                atomicCAS(args.dev_err, kDevOk, kDevTimeoutCopy);
+            }
             failed = true;
             failed_tile = tile;
             break;

@@ -238,7 +238,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *s_tmem;
     const uint32_t epoch30 = *s_epoch;
     const uint32_t tag_agg = (epoch30 << 2) | 1u, tag_incl = (epoch30 << 2) | 2u;
-    auto report = [&](uint32_t code) { atomicCAS(&pp.hdr->error, kDevOk, code); };
+    auto report = [&](uint32_t code) {
+        atomicCAS(&pp.hdr->error, kDevOk, code);
+        atomicCAS(args.dev_err, kDevOk, code);
+    };
     // this warp's quadrant; the columns of chunk c's array a (0 k, 1 v) in unit slot t
     const uint32_t tq = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     auto tcol = [&](int t, int c, int a) { return (uint32_t)(t * Lay::CPU + (c >> 2) * Lay::CPC + a * Lay::CPA); };

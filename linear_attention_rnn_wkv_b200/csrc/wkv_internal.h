@@ -24,8 +24,14 @@ struct ForwardArgs {
     void* y;                // [B,T,C]
     float* state_out;       // [3][B][C] or null
     uint32_t* err;          // device error word (never null)
+    uint32_t* dev_err;      // the library's device-wide error word (never null)
     uint32_t spin_limit;    // bounded waits
 };
+
+// The library's device-wide error word on the current device (null if it cannot be found):
+// every kernel that gives up a bounded wait also records its code here, for
+// wkv_get_device_status.
+uint32_t* device_status_word();
 
 // ----- serial path: one thread per (b, c) -----
 cudaError_t launch_forward_serial(const ForwardArgs& a, cudaStream_t s);

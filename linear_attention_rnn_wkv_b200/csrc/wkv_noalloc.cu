@@ -99,6 +99,8 @@ extern "C" wkv_status wkv_forward_chunked_noalloc(int64_t B, int64_t T, int64_t 
     a.y = y;
     a.state_out = state_out;
     a.err = static_cast<uint32_t*>(scratch);
+    a.dev_err = device_status_word();
+    if (!a.dev_err) return WKV_ERR_CUDA;
     a.spin_limit = kSpinLimitDefault;
     e = launch_forward_chunked(a, g, scratch, -1, stream);
     return e == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;

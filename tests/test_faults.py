@@ -21,15 +21,20 @@ def test_missing_carry_times_out_and_context_survives():
     y = torch.empty_like(kg)
     ws = wkv.Workspace(nbytes=wkv.workspace_size(B, T, C))
     stream = torch.cuda.current_stream().cuda_stream
+    L.wkv_get_device_status(stream)  # start from a clear device-wide word
     # unit 5 never publishes its carry; waits give up after 20000 polls (milliseconds)
     st = L.wkv_testhook_forward_drop(B, T, C, wg.data_ptr(), ug.data_ptr(), kg.data_ptr(), vg.data_ptr(),
                                      y.data_ptr(), ws.buf.data_ptr(), ws.buf.numel(), 5, 20000, stream)
     assert st == 0
     assert L.wkv_forward_status(ws.buf.data_ptr(), ws.buf.numel(), stream) == 5  # WKV_ERR_TIMEOUT
-    # the error was cleared and the same workspace and context work again
+    # the device-wide word saw it too, independently of the workspace
+    assert L.wkv_get_device_status(stream) == 5
+    # both errors were cleared and the same workspace and context work again
     assert L.wkv_forward_status(ws.buf.data_ptr(), ws.buf.numel(), stream) == 0
+    assert L.wkv_get_device_status(stream) == 0
     y2, _ = wkv.wkv_forward(wg, ug, kg, vg, workspace=ws, path="chunked")
     wkv.forward_status(ws.buf)
+    wkv.get_device_status()
     y_ref, s_ref, _, _ = oracle.wkv_recurrent(w, u, k, v)
     assert scaled_output_error(y2.cpu().numpy(), y_ref, s_ref) <= TOL_Y["f32"]
 
@@ -43,3 +48,4 @@ def test_status_is_clean_after_normal_runs():
     import torch
     wkv.wkv_forward(*(torch.from_numpy(a).cuda() for a in (w, u, k, v)), workspace=ws)
     wkv.forward_status(ws.buf)
+    wkv.get_device_status()  # no launch on the device gave up a wait
