@@ -18,6 +18,9 @@ Functions (all inputs are converted to contiguous float64):
 * ``token_shift(mu, x, x_last=None)`` -- the two-tap lerp.
 * ``decode_step(w, u, k, v, state, sacc)`` -- one token from a given state for
   ``[N, L, C]`` rows with ``[L, C]`` parameters: the recurrence with T = 1.
+* ``gate(r, wkv)`` -- the receptance gate ``sigma(r) * wkv``, elementwise.
+* ``token_shift3(mu_r, mu_k, mu_v, x, x_last=None)`` -- the lerp with the three
+  projections' separate mu (three calls of ``token_shift``).
 
 ``s`` is the same weighted average with ``|v|`` in place of ``v`` (the error
 scale the parity tests divide by); ``sacc`` is its accumulator in the state.
@@ -59,7 +62,8 @@ def load(path: str):
     L.oracle_wkv_recurrent.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.oracle_wkv_naive.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp]
     L.oracle_token_shift.argtypes = [i64, i64, i64, vp, vp, vp, vp]
-    for f in (L.oracle_wkv_direct, L.oracle_wkv_recurrent, L.oracle_wkv_naive, L.oracle_token_shift):
+    L.oracle_gate.argtypes = [i64, vp, vp, vp]
+    for f in (L.oracle_wkv_direct, L.oracle_wkv_recurrent, L.oracle_wkv_naive, L.oracle_token_shift, L.oracle_gate):
         f.restype = None
     L.oracle_num_threads.restype = ctypes.c_int
     return L
@@ -134,6 +138,22 @@ def token_shift(mu, x, x_last=None, L=None):
     xbar = np.empty(x.shape, np.float64)
     (L or lib()).oracle_token_shift(B, T, C, _p(mu), _p(x), _p(x_last), _p(xbar))
     return xbar
+
+
+def gate(r, wkv, L=None):
+    """sigma(r) * wkv elementwise; r and wkv of one shape."""
+    r, wkv = _f64(r), _f64(wkv)
+    if r.shape != wkv.shape:
+        raise ValueError("r and wkv must have the same shape")
+    out = np.empty(r.shape, np.float64)
+    (L or lib()).oracle_gate(r.size, _p(r), _p(wkv), _p(out))
+    return out
+
+
+def token_shift3(mu_r, mu_k, mu_v, x, x_last=None, L=None):
+    """The token-shift lerp of the receptance, key and value projections, each with its
+    own mu: returns ``(xr, xk, xv)``."""
+    return tuple(token_shift(mu, x, x_last, L=L) for mu in (mu_r, mu_k, mu_v))
 
 
 def decode_step(w, u, k, v, state, sacc=None, L=None):

@@ -19,6 +19,9 @@
  *           a two-tap causal convolution" (the lerp).
  *   [WIKI]  "RWKV" (aiwiki.thehackersbrain.dev): eq. 1 and the one-token
  *           decode step in the stabilised form.
+ *           Also section "Receptance: the gate on the way out" (the output is
+ *           sigma(r) times wkv, channel by channel) and, in section "Token shift",
+ *           the separate mu_r, mu_k, mu_v of the three projections.
  *   [MULTI] "RWKV and Recurrent Models With Transformer Quality"
  *           (multigrid.ai): section "Prefill, decode, and where each form is
  *           used" (prefill yields the state after the last prompt token;
@@ -202,4 +205,20 @@ void oracle_token_shift(int64_t B, int64_t T, int64_t C, const double* mu, const
                     prev = x_last ? x_last[(size_t)b * (size_t)C + (size_t)c] : 0.0;
                 xbar[at3(b, t, c, T, C)] = mu[c] * x[at3(b, t, c, T, C)] + (1.0 - mu[c]) * prev;
             }
+}
+
+/*
+ * Receptance gate ([MATH] "Receptance: the gate on the way out"): each channel of
+ * wkv_t passes through the logistic sigmoid of r_t,
+ *   out[i] = wkv[i] * sigma(r[i]),   sigma(r) = 1 / (1 + e^{-r}),
+ * elementwise over n values (the W_o projection that follows is not part of it).
+ * For r -> -inf, e^{-r} overflows to +inf and the quotient is the limit 0.
+ */
+void oracle_gate(int64_t n, const double* r, const double* wkv, double* out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        const double sigma = 1.0 / (1.0 + exp(-r[i]));
+        out[i] = wkv[i] * sigma;
+    }
 }

@@ -357,6 +357,45 @@ def pin_token_shift(L):
     assert np.array_equal(oracle.decode_token_shift(np.ones((3, C)), xt, xp, L=L), xt)
 
 
+def pin_gate(L):
+    """The receptance gate sigma(r) * wkv ("Receptance: the gate on the way out"): sigma(0) =
+    1/2 exactly, the limits r -> +inf (pass) and r -> -inf (mute), the reflection
+    sigma(r) + sigma(-r) = 1, sigma against scipy's logistic function, and a gate that acts
+    channel by channel (each output depends only on its own r)."""
+    from scipy.special import expit
+    r = _rng(31)
+    wkv = r.normal(0, 2, (2, 9, 6))
+    assert np.array_equal(oracle.gate(np.zeros_like(wkv), wkv, L=L), wkv / 2)
+    assert np.allclose(oracle.gate(np.full_like(wkv, 60.0), wkv, L=L), wkv, rtol=1e-25, atol=0)
+    assert np.array_equal(oracle.gate(np.full_like(wkv, -800.0), wkv, L=L), np.zeros_like(wkv))
+    rr = r.normal(0, 3, wkv.shape)
+    g, gm = oracle.gate(rr, wkv, L=L), oracle.gate(-rr, wkv, L=L)
+    assert np.allclose(g + gm, wkv, rtol=1e-14, atol=1e-14)
+    assert np.allclose(g, wkv * expit(rr), rtol=1e-14, atol=1e-300)
+    # channel by channel: changing r at one position changes only that output
+    rr2 = rr.copy()
+    rr2[1, 4, 2] += 1.0
+    diff = oracle.gate(rr2, wkv, L=L) != g
+    assert diff.sum() == 1 and diff[1, 4, 2]
+
+
+def pin_token_shift3(L):
+    """The three projections' lerps ("Token shift": separate mu_r, mu_k, mu_v): each output
+    follows its own mu only (mu = 1 passes x_t, mu = 0 the previous token), in the order
+    (r, k, v)."""
+    B, T, C = 2, 6, 4
+    r = _rng(32)
+    x = r.normal(0, 1, (B, T, C))
+    xl = r.normal(0, 1, (B, C))
+    prev = np.concatenate([xl[:, None], x[:, :-1]], axis=1)
+    one, zero, half = np.ones(C), np.zeros(C), np.full(C, 0.5)
+    xr, xk, xv = oracle.token_shift3(one, zero, half, x, xl, L=L)
+    assert np.array_equal(xr, x) and np.array_equal(xk, prev) and np.array_equal(xv, (x + prev) / 2)
+    xr, xk, xv = oracle.token_shift3(zero, half, one, x, None, L=L)
+    prev0 = np.concatenate([np.zeros((B, 1, C)), x[:, :-1]], axis=1)
+    assert np.array_equal(xr, prev0) and np.array_equal(xk, (x + prev0) / 2) and np.array_equal(xv, x)
+
+
 ALL_PINS = [
     pin_worked_example,
     pin_routes_agree,
@@ -374,4 +413,6 @@ ALL_PINS = [
     pin_decode_layer_indexing,
     pin_negative_decay_convention,
     pin_token_shift,
+    pin_gate,
+    pin_token_shift3,
 ]

@@ -35,6 +35,9 @@ MUTANTS = {
     "layout_transposed": ("return ((size_t)b * (size_t)T + (size_t)t) * (size_t)C + (size_t)c;",
                           "return ((size_t)b * (size_t)C + (size_t)c) * (size_t)T + (size_t)t;"),
     "magnitude_scale_signed": ("sa = keep * sa + add * fabs(vt);", "sa = keep * sa + add * vt;"),
+    "gate_sign": ("const double sigma = 1.0 / (1.0 + exp(-r[i]));", "const double sigma = 1.0 / (1.0 + exp(r[i]));"),
+    "gate_offset": ("const double sigma = 1.0 / (1.0 + exp(-r[i]));", "const double sigma = 1.0 / (2.0 + exp(-r[i]));"),
+    "gate_divides": ("out[i] = wkv[i] * sigma;", "out[i] = wkv[i] / sigma;"),
 }
 
 
