@@ -104,6 +104,22 @@ wkv_status wkv_forward_ex(int64_t B, int64_t T, int64_t C, wkv_dtype io, const f
                           const void* k, const void* v, const float* state_in, void* y, float* state_out,
                           void* workspace, size_t ws_bytes, wkv_path path, int chunk, cudaStream_t stream);
 
+/*
+ * As wkv_forward_ex, with the receptance gate applied to the output (transformer-math page,
+ * section "Receptance: the gate on the way out"): y receives sigma(r) * wkv channel by
+ * channel, sigma the logistic function; the ungated wkv is not written.  The W_o projection
+ * that follows the gate on the page is not part of this call.
+ *   r          [B, T, C] in dtype io (required when B*T*C > 0)
+ * state_out is the recurrence state (the gate acts on the output only).  The chunked kernel
+ * for 16-byte rows applies the gate as it writes y (r is read once, y written once); other
+ * paths run the forward and then one elementwise pass y <- sigma(r) * y.  Same status codes
+ * as wkv_forward_ex; r must be 16-byte aligned.
+ */
+wkv_status wkv_forward_gated(int64_t B, int64_t T, int64_t C, wkv_dtype io, const float* w, const float* u,
+                             const void* k, const void* v, const void* r, const float* state_in, void* y,
+                             float* state_out, void* workspace, size_t ws_bytes, wkv_path path, int chunk,
+                             cudaStream_t stream);
+
 /* Workspace bytes wkv_forward needs for this shape (the largest over all paths). */
 size_t wkv_forward_workspace_size(int64_t B, int64_t T, int64_t C, wkv_dtype io);
 
@@ -150,6 +166,19 @@ wkv_status wkv_decode_step(int64_t N, int64_t L, int64_t C, const float* w, cons
  */
 wkv_status token_shift_mix(int64_t B, int64_t T, int64_t C, const float* mu, const float* x, const float* x_last,
                            float* xbar, cudaStream_t stream);
+
+/*
+ * Token shift of the three projections in one pass (transformer-math page, section "Token
+ * shift: a two-tap causal convolution": r, k and v each blend with their own mu):
+ *   xr = mu_r * x_t + (1 - mu_r) * x_{t-1}, and likewise xk with mu_k, xv with mu_v.
+ *   mu_r, mu_k, mu_v [C] fp32
+ *   x, xr, xk, xv    [B, T, C] fp32 (outputs must not alias x or each other)
+ *   x_last           [B][C] fp32, the token before t = 0, or NULL for zeros
+ * x is read once; the W_r, W_k, W_v projections that follow are not part of this call.
+ */
+wkv_status token_shift_mix3(int64_t B, int64_t T, int64_t C, const float* mu_r, const float* mu_k,
+                            const float* mu_v, const float* x, const float* x_last, float* xr, float* xk,
+                            float* xv, cudaStream_t stream);
 
 /*
  * Fused decode step: the token-shift lerp and the WKV decode step in one kernel.

@@ -66,6 +66,8 @@ def lib():
                 L.wkv_workspace_init.argtypes = [vp, sz, vp]
                 L.wkv_forward_status.argtypes = [vp, sz, vp]
                 L.wkv_get_device_status.argtypes = [vp]
+                L.wkv_forward_gated.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i32, i32, vp]
+                L.token_shift_mix3.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp]
                 L.wkv_decode_step.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp]
                 L.wkv_decode_step_fused.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
                 L.token_shift_mix.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp]
@@ -74,7 +76,7 @@ def lib():
                 L.wkv_forward_auto_path.argtypes = [i64, i64, i64, i32]
                 L.wkv_testhook_forward_drop.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, sz, i64, u32, vp]
                 for f in (L.wkv_forward, L.wkv_forward_ex, L.wkv_workspace_init, L.wkv_forward_status,
-                          L.wkv_get_device_status,
+                          L.wkv_get_device_status, L.wkv_forward_gated, L.token_shift_mix3,
                           L.wkv_decode_step, L.wkv_decode_step_fused, L.token_shift_mix,
                           L.wkv_forward_auto_path, L.wkv_testhook_forward_drop):
                     f.restype = i32
@@ -149,8 +151,9 @@ def _workspace_for(dev, B, T, C, dtype):
 
 
 def wkv_forward(w, u, k, v, state_in=None, want_state=True, path="auto", chunk=0, workspace=None, y=None,
-                state_out=None):
-    """Forward over [B, T, C].  Returns (y, state_out)."""
+                state_out=None, r=None):
+    """Forward over [B, T, C].  Returns (y, state_out).  With r ([B, T, C], k's dtype) y is the
+    gated output sigma(r) * wkv (wkv_forward_gated)."""
     if not isinstance(k, torch.Tensor) or not k.is_cuda:
         raise TypeError("k must be a CUDA tensor (no CPU path exists)")
     if k.dtype not in _DTYPE or v.dtype != k.dtype:
@@ -171,6 +174,15 @@ def wkv_forward(w, u, k, v, state_in=None, want_state=True, path="auto", chunk=0
         state_out = None
     ws = workspace.for_shape(B, T, C, k.dtype) if isinstance(workspace, Workspace) else (
         workspace if workspace is not None else _workspace_for(dev, B, T, C, k.dtype))
+    if r is not None:
+        if not isinstance(r, torch.Tensor) or not r.is_cuda or r.dtype != k.dtype or r.shape != k.shape \
+                or not r.is_contiguous():
+            raise ValueError("r must be a contiguous CUDA tensor shaped and typed like k")
+        st = lib().wkv_forward_gated(B, T, C, _DTYPE[k.dtype], w.data_ptr(), u.data_ptr(), k.data_ptr(),
+                                     v.data_ptr(), r.data_ptr(), _ptr(state_in), y.data_ptr(), _ptr(state_out),
+                                     ws.data_ptr(), ws.numel(), _PATH[path], int(chunk), _stream(dev))
+        _check(st, "wkv_forward_gated")
+        return y, state_out
     st = lib().wkv_forward_ex(B, T, C, _DTYPE[k.dtype], w.data_ptr(), u.data_ptr(), k.data_ptr(), v.data_ptr(),
                               _ptr(state_in), y.data_ptr(), _ptr(state_out), ws.data_ptr(), ws.numel(),
                               _PATH[path], int(chunk), _stream(dev))
@@ -226,6 +238,24 @@ def wkv_decode_step_fused(mu, w, u, x_t, x_prev, k, v, state, xbar=None, y=None)
                                        state.data_ptr(), y.data_ptr(), _stream(k.device)),
            "wkv_decode_step_fused")
     return xbar, y
+
+
+def token_shift_mix3(mu_r, mu_k, mu_v, x, x_last=None):
+    """The receptance, key and value lerps of x [B, T, C] in one pass, each with its own mu [C].
+    Returns (xr, xk, xv)."""
+    _cuda_f32(x, "x")
+    if x.dim() != 3:
+        raise ValueError("x must be [B, T, C]")
+    B, T, C = x.shape
+    for m, name in ((mu_r, "mu_r"), (mu_k, "mu_k"), (mu_v, "mu_v")):
+        _cuda_f32(m, name, (C,))
+    if x_last is not None:
+        _cuda_f32(x_last, "x_last", (B, C))
+    xr, xk, xv = (torch.empty_like(x) for _ in range(3))
+    _check(lib().token_shift_mix3(B, T, C, mu_r.data_ptr(), mu_k.data_ptr(), mu_v.data_ptr(), x.data_ptr(),
+                                  _ptr(x_last), xr.data_ptr(), xk.data_ptr(), xv.data_ptr(), _stream(x.device)),
+           "token_shift_mix3")
+    return xr, xk, xv
 
 
 def token_shift_mix(mu, x, x_last=None, xbar=None):

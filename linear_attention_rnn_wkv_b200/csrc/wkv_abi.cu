@@ -72,7 +72,7 @@ wkv_path auto_path(int64_t B, int64_t T, int64_t C, wkv_dtype io) {
 wkv_status forward_impl(int64_t B, int64_t T, int64_t C, wkv_dtype io, const float* w, const float* u,
                         const void* k, const void* v, const float* state_in, void* y, float* state_out,
                         void* workspace, size_t ws_bytes, wkv_path path, int chunk, uint32_t spin_limit,
-                        int64_t drop_unit, cudaStream_t stream) {
+                        int64_t drop_unit, cudaStream_t stream, const void* r = nullptr) {
     int64_t n = 0, BC = 0;
     if (!sizes_ok(B, T, C, &n) || !mul_ok(B, C, &BC) || BC > INT64_MAX / 3) return WKV_ERR_INVALID_ARG;
     if (io != WKV_F32 && io != WKV_BF16) return WKV_ERR_UNSUPPORTED;
@@ -88,7 +88,7 @@ wkv_status forward_impl(int64_t B, int64_t T, int64_t C, wkv_dtype io, const flo
         return e == cudaSuccess ? WKV_OK : cuda_fail(e);
     }
     if (!k || !v || !y) return WKV_ERR_INVALID_ARG;
-    if (!aligned16(k) || !aligned16(v) || !aligned16(y)) return WKV_ERR_MISALIGNED;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(y) || !aligned16(r)) return WKV_ERR_MISALIGNED;
 
     ForwardArgs a;
     a.B = B;
@@ -112,6 +112,7 @@ wkv_status forward_impl(int64_t B, int64_t T, int64_t C, wkv_dtype io, const flo
         const int64_t grid = B * ((C + 127) / 128);
         if (grid > INT32_MAX) return WKV_ERR_UNSUPPORTED;
         cudaError_t e = launch_forward_serial(a, stream);
+        if (e == cudaSuccess && r) e = launch_gate(n, (int)io, r, y, stream);
         return e == cudaSuccess ? WKV_OK : cuda_fail(e);
     }
     ChunkGeom g;
@@ -121,7 +122,12 @@ wkv_status forward_impl(int64_t B, int64_t T, int64_t C, wkv_dtype io, const flo
     a.err = &static_cast<WsHeader*>(workspace)->error;
     a.dev_err = device_status_word();
     if (!a.dev_err) return cuda_fail(cudaGetLastError());
+    // the tensor-memory kernel applies the gate as it writes y; other kernels are followed
+    // by an elementwise gate pass over y
+    const bool fused = r && chunked_path_fuses_gate(g);
+    a.r = fused ? r : nullptr;
     cudaError_t e = launch_forward_chunked(a, g, workspace, drop_unit, stream);
+    if (e == cudaSuccess && r && !fused) e = launch_gate(n, (int)io, r, y, stream);
     return e == cudaSuccess ? WKV_OK : cuda_fail(e);
 }
 
@@ -165,6 +171,28 @@ wkv_status wkv_forward_ex(int64_t B, int64_t T, int64_t C, wkv_dtype io, const f
                           void* workspace, size_t ws_bytes, wkv_path path, int chunk, cudaStream_t stream) {
     return forward_impl(B, T, C, io, w, u, k, v, state_in, y, state_out, workspace, ws_bytes, path, chunk,
                         kSpinLimitDefault, -1, stream);
+}
+
+wkv_status wkv_forward_gated(int64_t B, int64_t T, int64_t C, wkv_dtype io, const float* w, const float* u,
+                             const void* k, const void* v, const void* r, const float* state_in, void* y,
+                             float* state_out, void* workspace, size_t ws_bytes, wkv_path path, int chunk,
+                             cudaStream_t stream) {
+    int64_t n = 0;
+    if (!sizes_ok(B, T, C, &n)) return WKV_ERR_INVALID_ARG;
+    if (n > 0 && T > 0 && !r) return WKV_ERR_INVALID_ARG;
+    return forward_impl(B, T, C, io, w, u, k, v, state_in, y, state_out, workspace, ws_bytes, path, chunk,
+                        kSpinLimitDefault, -1, stream, r);
+}
+
+wkv_status token_shift_mix3(int64_t B, int64_t T, int64_t C, const float* mu_r, const float* mu_k, const float* mu_v,
+                            const float* x, const float* x_last, float* xr, float* xk, float* xv, cudaStream_t stream) {
+    int64_t n = 0;
+    if (!sizes_ok(B, T, C, &n)) return WKV_ERR_INVALID_ARG;
+    if (n == 0) return WKV_OK;
+    if (!mu_r || !mu_k || !mu_v || !x || !xr || !xk || !xv) return WKV_ERR_INVALID_ARG;
+    if (!f32_args_ok({mu_r, mu_k, mu_v, x, x_last, xr, xk, xv})) return WKV_ERR_MISALIGNED;
+    cudaError_t e = launch_token_shift3(B, T, C, mu_r, mu_k, mu_v, x, x_last, xr, xk, xv, stream);
+    return e == cudaSuccess ? WKV_OK : cuda_fail(e);
 }
 
 wkv_status wkv_forward_status(void* workspace, size_t ws_bytes, cudaStream_t stream) {

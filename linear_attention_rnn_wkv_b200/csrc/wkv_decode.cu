@@ -10,6 +10,7 @@
 // rows, so no per-element division is needed.  States stay in natural units.
 #include "wkv_device.cuh"
 #include "wkv_internal.h"
+#include "wkv_vec.cuh"
 
 namespace wkvb {
 namespace {
@@ -108,6 +109,61 @@ __global__ void __launch_bounds__(256) token_shift_kernel(int64_t B, int64_t T, 
     }
 }
 
+// Token shift of the three projections (transformer-math page, section "Token shift": each of
+// r, k, v has its own mu): x_t and x_{t-1} are read once and three lerps are written.
+template <int V>
+__global__ void __launch_bounds__(256) token_shift3_kernel(int64_t B, int64_t T, int64_t C, const float* __restrict__ mu_r,
+                                                           const float* __restrict__ mu_k, const float* __restrict__ mu_v,
+                                                           const float* __restrict__ x, const float* __restrict__ x_last,
+                                                           float* __restrict__ xr, float* __restrict__ xk,
+                                                           float* __restrict__ xv) {
+    const int64_t c = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * V;
+    if (c >= C) return;
+    float mr[V], mk[V], mv[V];
+    F<V>::ld_keep(mu_r + c, mr);
+    F<V>::ld_keep(mu_k + c, mk);
+    F<V>::ld_keep(mu_v + c, mv);
+    const int64_t rows = B * T;
+    for (int64_t row = blockIdx.y; row < rows; row += gridDim.y) {
+        const int64_t b = row / T, t = row % T;
+        float xt[V], xp[V], o[V];
+        F<V>::ld_keep(x + row * C + c, xt);
+        if (t > 0) {
+            F<V>::ld_keep(x + (row - 1) * C + c, xp);
+        } else if (x_last) {
+            F<V>::ld_keep(x_last + b * C + c, xp);
+        } else {
+#pragma unroll
+            for (int q = 0; q < V; ++q) xp[q] = 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < V; ++q) o[q] = fmaf(mr[q], xt[q], (1.f - mr[q]) * xp[q]);
+        F<V>::st(xr + row * C + c, o);
+#pragma unroll
+        for (int q = 0; q < V; ++q) o[q] = fmaf(mk[q], xt[q], (1.f - mk[q]) * xp[q]);
+        F<V>::st(xk + row * C + c, o);
+#pragma unroll
+        for (int q = 0; q < V; ++q) o[q] = fmaf(mv[q], xt[q], (1.f - mv[q]) * xp[q]);
+        F<V>::st(xv + row * C + c, o);
+    }
+}
+
+// The receptance gate applied in place, y <- sigma(r) * y (transformer-math page, section
+// "Receptance: the gate on the way out"), for paths whose forward kernel does not fuse it.
+// sigma(r) = 1 / (1 + 2^(-r log2 e)); for r -> -inf the exponential is +inf and the gate 0.
+template <typename TIO, int V>
+__global__ void __launch_bounds__(256) gate_kernel(int64_t n, const TIO* __restrict__ r, TIO* __restrict__ y) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x * V;
+    for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * V; i < n; i += stride) {
+        float rv[V], yv[V];
+        Vec<TIO, V>::load(r + i, rv);
+        Vec<TIO, V>::load(y + i, yv);
+#pragma unroll
+        for (int q = 0; q < V; ++q) yv[q] *= rcp(1.f + ex2(-rv[q] * kLog2e));
+        Vec<TIO, V>::store(y + i, yv);
+    }
+}
+
 __global__ void passthrough_kernel(int64_t BC, const float* in, float* out) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < 3 * BC; i += (int64_t)gridDim.x * blockDim.x)
         out[i] = in ? in[i] : (i < 2 * BC ? 0.f : kPEmpty);
@@ -156,6 +212,44 @@ cudaError_t launch_state_passthrough(int64_t BC, const float* state_in, float* s
     const int64_t n = 3 * BC;
     const int64_t blocks = (n + 255) / 256 < 148 * 16 ? (n + 255) / 256 : 148 * 16;
     passthrough_kernel<<<(unsigned)blocks, 256, 0, s>>>(BC, state_in, state_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_token_shift3(int64_t B, int64_t T, int64_t C, const float* mu_r, const float* mu_k,
+                                const float* mu_v, const float* x, const float* x_last, float* xr, float* xk, float* xv,
+                                cudaStream_t s) {
+    const bool vec = (C % 4) == 0;
+    const dim3 grid = grid2d(C, vec ? 4 : 1, B * T);
+    if (vec)
+        token_shift3_kernel<4><<<grid, 256, 0, s>>>(B, T, C, mu_r, mu_k, mu_v, x, x_last, xr, xk, xv);
+    else
+        token_shift3_kernel<1><<<grid, 256, 0, s>>>(B, T, C, mu_r, mu_k, mu_v, x, x_last, xr, xk, xv);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gate(int64_t n, int io, const void* r, void* y, cudaStream_t s) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    auto blocks = [&](int64_t units) {
+        const int64_t b = (units + 255) / 256;
+        const int64_t cap = (int64_t)sms * 8;
+        return (unsigned)(b < cap ? (b > 0 ? b : 1) : cap);
+    };
+    if (io == 1) {
+        const __nv_bfloat16* rr = static_cast<const __nv_bfloat16*>(r);
+        __nv_bfloat16* yy = static_cast<__nv_bfloat16*>(y);
+        if (n % 8 == 0)
+            gate_kernel<__nv_bfloat16, 8><<<blocks(n / 8), 256, 0, s>>>(n, rr, yy);
+        else
+            gate_kernel<__nv_bfloat16, 1><<<blocks(n), 256, 0, s>>>(n, rr, yy);
+    } else {
+        const float* rr = static_cast<const float*>(r);
+        float* yy = static_cast<float*>(y);
+        if (n % 4 == 0)
+            gate_kernel<float, 4><<<blocks(n / 4), 256, 0, s>>>(n, rr, yy);
+        else
+            gate_kernel<float, 1><<<blocks(n), 256, 0, s>>>(n, rr, yy);
+    }
     return cudaGetLastError();
 }
 

@@ -505,6 +505,8 @@ bool chunk_geometry(int64_t B, int64_t T, int64_t C, int io, int chunk, ChunkGeo
     return true;
 }
 
+bool chunked_path_fuses_gate(const ChunkGeom& g) { return g.pipe && WKV_FORWARD_TMEM; }
+
 cudaError_t launch_forward_chunked(const ForwardArgs& a, const ChunkGeom& g, void* ws, int64_t drop_unit,
                                    cudaStream_t s) {
     if (g.pipe) return WKV_FORWARD_TMEM ? launch_forward_tmem(a, g, ws, drop_unit, s) : launch_forward_pipe(a, g, ws, drop_unit, s);

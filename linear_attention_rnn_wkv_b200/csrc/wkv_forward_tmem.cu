@@ -135,6 +135,13 @@ struct Pk<__nv_bfloat16> {
     static __device__ __forceinline__ float2 unpack(const uint32_t* w) { return make_float2(bf_lo(w[0]), bf_hi(w[0])); }
 };
 
+// The receptance gate on one output pair (transformer-math page, section "Receptance: the
+// gate on the way out"): y <- sigma(r) * y with sigma(r) = 1 / (1 + 2^(-r log2 e)).
+__device__ __forceinline__ void gate_pair(float (&y)[2], const float (&r)[2]) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) y[c] *= rcp(1.f + ex2(-r[c] * kLog2e));
+}
+
 constexpr int kNWS = 8;   // chunks per tile (summarising warps, emitting warps)
 constexpr int kNL = 3;    // look-back warps
 constexpr int kCg = 64;   // channels per tile (a lane owns a pair)
@@ -145,7 +152,7 @@ constexpr int kCg = 64;   // channels per tile (a lane owns a pair)
 constexpr int kES = WKV_TMEM_EMIT_SETS;
 constexpr int kThreads = (1 + kNL + (1 + kES) * kNWS) * 32;
 
-template <typename TIO, int LC, int NS, int NT>
+template <typename TIO, int LC, int NS, int NT, bool GATE = false>
 struct TmLayout {
     static constexpr int Cg = kCg;
     static constexpr int Ts = kNWS * LC;
@@ -163,7 +170,11 @@ struct TmLayout {
     static constexpr int NBARS = NS * (NB + 1) + NT * 3;  // per stage: NB full + 1 empty; per slot: chunks, carry, empty
     static constexpr size_t misc_off = bars_off + NBARS * 8;  // slot unit ids [NT], end index, epoch, tensor memory base
     static constexpr size_t stage_unit_off = misc_off + NT * 8 + 8 + 8;  // stage unit ids [NS]
-    static constexpr size_t total = stage_unit_off + NS * 8;
+    // gated forward: each emitting warp's chunk of r (TMA box of LC rows x Cg) and its barrier
+    static constexpr size_t rbuf_bytes = align128(sizeof(TIO) * LC * Cg);
+    static constexpr size_t rbuf_off = align128(stage_unit_off + NS * 8);
+    static constexpr size_t rbar_off = rbuf_off + (GATE ? kNWS * rbuf_bytes : 0);
+    static constexpr size_t total = rbar_off + (GATE ? kNWS * 8 : 0);
     // tensor memory: words per row per lane, columns per chunk array, per chunk, per unit and quadrant
     static constexpr int W = Pk<TIO>::W;
     static constexpr int CPA = LC * W;
@@ -175,11 +186,12 @@ struct TmLayout {
     static_assert(LC % SR == 0, "slices must tile a chunk");
 };
 
-template <typename TIO, int LC, int NS, int NT>
+template <typename TIO, int LC, int NS, int NT, bool GATE>
 __global__ void __launch_bounds__(kThreads, 1)
     tmem_kernel(ForwardArgs args, PipeParams pp, const __grid_constant__ CUtensorMap tmk,
-                const __grid_constant__ CUtensorMap tmv) {
-    using Lay = TmLayout<TIO, LC, NS, NT>;
+                const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmr) {
+    using Lay = TmLayout<TIO, LC, NS, NT, GATE>;
+    static_assert(!GATE || kES == 1, "one r buffer per chunk index");
     constexpr int V = 2;
     constexpr int Cg = Lay::Cg, Ts = Lay::Ts, NB = Lay::NB, BR = Lay::BR, W = Lay::W, SR = Lay::SR, SW = Lay::SW;
     constexpr int W_L0 = 1, W_S0 = 1 + kNL, W_E0 = 1 + kNL + kNWS;
@@ -225,6 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int b = 0; b < NB; ++b) mbar_init(dfull(s, b), 1);
             mbar_init(dempty(s), kNWS);
         }
+        if (GATE)
+            for (int e = 0; e < kNWS; ++e) mbar_init(reinterpret_cast<uint64_t*>(smem + Lay::rbar_off) + e, 1);
         for (int t = 0; t < NT; ++t) {
             mbar_init(chunks_bar(t), kNWS);
             mbar_init(carry_bar(t), 1);
@@ -546,10 +560,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         // --------------------------------- emit ---------------------------------
         const int ew = (warp - W_E0) % kNWS;  // chunk index (the same quadrant as its summariser)
         const int es = (warp - W_E0) / kNWS;  // emitting set: units es, es + kES, ...
+        // gated forward: this warp's chunk of r arrives by TMA in its own buffer
+        uint64_t* rbar = reinterpret_cast<uint64_t*>(smem + Lay::rbar_off) + ew;
+        const TIO* rbuf = reinterpret_cast<const TIO*>(smem + Lay::rbuf_off + ew * Lay::rbuf_bytes);
+        uint32_t rphase = 0;
         for (int64_t i = es;; i += kES) {
             const int t = (int)(i % NT);
             const uint32_t ph = (uint32_t)((i / NT) & 1);
             bool got = false, gone = false;
+            bool r_pending = false;
+            if (GATE) {
+                // The unit is known once its summaries are in, well before its carry: fetch
+                // this chunk's r rows now (one TMA box), so they are waiting when the rows are
+                // emitted.  The buffer is free: the previous unit's rows were read before.
+                for (uint32_t it = 0; it <= lim; ++it) {
+                    if (WKV_WAIT_HINT ? mbar_try_wait_hint(chunks_bar(t), ph, WKV_WAIT_HINT) : mbar_try_wait(chunks_bar(t), ph)) {
+                        got = true;
+                        break;
+                    }
+                    if (*s_iend < i) {
+                        gone = true;
+                        break;
+                    }
+                    if (!WKV_WAIT_HINT) __nanosleep(32);
+                }
+                if (gone) break;
+                const int64_t u0 = slot_unit[t];
+                if (got && u0 >= 0) {
+                    const Geo q0 = geo(u0);
+                    if (q0.len > ew * LC) {
+                        r_pending = true;
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(rbar, (uint32_t)(LC * Cg * sizeof(TIO)));
+                            tma_load_3d(const_cast<TIO*>(rbuf), &tmr, (int)q0.c0, (int)(q0.t0 + ew * LC), (int)q0.b, rbar);
+                        }
+                    }
+                }
+                got = false;
+            }
             for (uint32_t it = 0; it <= lim; ++it) {
                 if (WKV_WAIT_HINT ? mbar_try_wait_hint(carry_bar(t), ph, WKV_WAIT_HINT) : mbar_try_wait(carry_bar(t), ph)) {
                     got = true;
@@ -596,6 +644,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 TIO* yg = static_cast<TIO*>(args.y) + (q.b * T + q.t0) * C + q.c0;
                 TmemIO<SW>::wait_ld(kw);
                 TmemIO<SW>::wait_ld(vw);
+                if (GATE && r_pending) {
+                    if (!mbar_wait(rbar, rphase, lim) && lane == 0) report(kDevTimeoutCopy);
+                    rphase ^= 1u;
+                    r_pending = false;
+                }
                 // Fixed-frame re-scan.  Seen from the chunk's last row, each token's weight
                 // e_i = 2^(k_i - (L-1-i) w - G) and the carried-in history K do not change from
                 // row to row (everything decays at the same rate), so with running sums S of
@@ -656,6 +709,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 TmemIO<SW>::ld(tq + tcol(t, ew, 0) + (h + 1) * SW, kn);
                                 TmemIO<SW>::ld(tq + tcol(t, ew, 1) + (h + 1) * SW, vn);
                             }
+
 #pragma unroll
                             for (int rr = 0; rr < SR; ++rr) {
                                 const int r = h * SR + rr;
@@ -667,12 +721,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 const float2 e = make_float2(ex2(x.x), ex2(x.y));
                                 const float2 ec = __fmul2_rn(e, fic);
                                 const float2 num = __ffma2_rn(ec, vp, fSa);
-                                const float2 den = __fadd2_rn(fSb, ec);
+                                float2 den = __fadd2_rn(fSb, ec);
+                                float2 er = make_float2(0.f, 0.f);
+                                if (GATE) {
+                                    // sigma(r) folded into the one reciprocal: y = num / (den (1 + 2^(-r log2 e)));
+                                    // for r -> -inf the product overflows and y is the limit 0
+                                    float rv[V];
+                                    Vec<TIO, V>::load(rbuf + r * Cg + cl, rv);
+                                    er = make_float2(ex2(-rv[0] * kLog2e), ex2(-rv[1] * kLog2e));
+                                    den = __ffma2_rn(den, er, den);
+                                }
                                 const float2 yv = __fmul2_rn(num, make_float2(rcp(den.x), rcp(den.y)));
                                 float yy[V] = {yv.x, yv.y};
                                 if (r == 0) {
-                                    if (fSb.x == 0.f) yy[0] = vp.x;
-                                    if (fSb.y == 0.f) yy[1] = vp.y;
+                                    // no history: the recurrence returns v itself (times the gate)
+                                    if (fSb.x == 0.f) yy[0] = GATE ? vp.x * rcp(1.f + er.x) : vp.x;
+                                    if (fSb.y == 0.f) yy[1] = GATE ? vp.y * rcp(1.f + er.y) : vp.y;
                                 }
                                 fSa = __ffma2_rn(e, vp, fSa);
                                 fSb = __fadd2_rn(fSb, e);
@@ -761,6 +825,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 wkv_fold<false>(a[c], bb[c], pp2[c], pp2[c] - w2[c], k2, vv[c], w2[c]);
                             }
                         }
+                        if (GATE) {
+                            float rv[V];
+                            Vec<TIO, V>::load(rbuf + r * Cg + cl, rv);
+                            gate_pair(yy, rv);
+                        }
                         Vec<TIO, V>::store(yg + (int64_t)row * C + cl, yy);
                     }
                 }
@@ -792,20 +861,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Unit slots: as many as the tensor memory holds (at most 8); stages: as many as the rest
 // of the 227 KB of shared memory holds (at most 4).
-template <typename TIO, int LC>
+template <typename TIO, int LC, bool GATE>
 struct TmConfig {
     static constexpr int NT0 = 512 / TmLayout<TIO, LC, 1, 1>::CPU;
     static constexpr int NT = NT0 > 8 ? 8 : NT0;
-    static constexpr size_t fixed = TmLayout<TIO, LC, 0, NT>::total;  // everything but the stages
+    static constexpr size_t fixed = TmLayout<TIO, LC, 0, NT, GATE>::total;  // everything but the stages
     static constexpr size_t per_stage = TmLayout<TIO, LC, 1, NT>::stage + (TmLayout<TIO, LC, 1, NT>::NB + 1) * 8;
     static constexpr int NS0 = (int)((232448 - fixed) / per_stage);
     static constexpr int NS = NS0 > 4 ? 4 : NS0;
 };
 
-template <typename TIO, int LC>
-cudaError_t launch_tmem_t(const ForwardArgs& a, const ChunkGeom& g, const PipeParams& pp, cudaStream_t s) {
-    constexpr int NT = TmConfig<TIO, LC>::NT;
-    constexpr int NS = TmConfig<TIO, LC>::NS;
+template <typename TIO, int LC, bool GATE>
+cudaError_t launch_tmem_g(const ForwardArgs& a, const ChunkGeom& g, const PipeParams& pp, cudaStream_t s) {
+    constexpr int NT = TmConfig<TIO, LC, GATE>::NT;
+    constexpr int NS = TmConfig<TIO, LC, GATE>::NS;
     static_assert(NS >= 2, "fewer than two shared-memory stages");
     // a look-back warp waits on unit i's slot only after finishing unit i - kNL, so the
     // slot's previous phase (unit i - NT) is complete whenever NT >= kNL
@@ -813,15 +882,17 @@ cudaError_t launch_tmem_t(const ForwardArgs& a, const ChunkGeom& g, const PipePa
     // an emitting warp waits on unit i's slot only after finishing unit i - kES; the slot's
     // previous unit i - NT must be one it has handled, so NT is a multiple of kES
     static_assert(NT % kES == 0, "unit slots must divide among the emitting sets");
-    using Lay = TmLayout<TIO, LC, NS, NT>;
+    using Lay = TmLayout<TIO, LC, NS, NT, GATE>;
     static_assert(Lay::total <= 232448, "shared memory layout over the per-CTA limit");
     static_assert(Lay::Ts % Lay::BR == 0, "tile rows must be a multiple of the box rows");
     static_assert(LC <= Lay::BR && Lay::BR % LC == 0, "a chunk must lie inside one box");
-    auto kern = tmem_kernel<TIO, LC, NS, NT>;
-    CUtensorMap tmk, tmv;
+    auto kern = tmem_kernel<TIO, LC, NS, NT, GATE>;
+    CUtensorMap tmk, tmv, tmr;
     if (!make_tile_map(&tmk, a.k, a.B, a.T, a.C, a.io, Lay::Cg, Lay::BR) ||
         !make_tile_map(&tmv, a.v, a.B, a.T, a.C, a.io, Lay::Cg, Lay::BR))
         return cudaErrorInvalidValue;
+    if (GATE ? !make_tile_map(&tmr, a.r, a.B, a.T, a.C, a.io, Lay::Cg, LC) : false) return cudaErrorInvalidValue;
+    if (!GATE) tmr = tmk;  // unused
     static uint64_t attr_done = 0;  // per device; set once so captured launches issue no attribute call
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -840,8 +911,13 @@ cudaError_t launch_tmem_t(const ForwardArgs& a, const ChunkGeom& g, const PipePa
     }
     const int64_t nsm = dev < 64 ? sms[dev] : 148;
     const int64_t grid = g.U < nsm ? g.U : nsm;
-    kern<<<(unsigned)grid, kThreads, Lay::total, s>>>(a, pp, tmk, tmv);
+    kern<<<(unsigned)grid, kThreads, Lay::total, s>>>(a, pp, tmk, tmv, tmr);
     return cudaGetLastError();
+}
+
+template <typename TIO, int LC>
+cudaError_t launch_tmem_t(const ForwardArgs& a, const ChunkGeom& g, const PipeParams& pp, cudaStream_t s) {
+    return a.r ? launch_tmem_g<TIO, LC, true>(a, g, pp, s) : launch_tmem_g<TIO, LC, false>(a, g, pp, s);
 }
 
 }  // namespace

@@ -25,6 +25,7 @@ struct ForwardArgs {
     float* state_out;       // [3][B][C] or null
     uint32_t* err;          // device error word (never null)
     uint32_t* dev_err;      // the library's device-wide error word (never null)
+    const void* r = nullptr;  // [B,T,C] receptance for a fused output gate, or null
     uint32_t spin_limit;    // bounded waits
 };
 
@@ -70,10 +71,18 @@ struct WsHeader {
 // successor's bounded wait runs out.
 // Look-back flags carry the launch's epoch (read from the workspace header on the device,
 // so a launch captured in a CUDA graph stays correct on every replay).
+// Whether the kernel this geometry selects applies a receptance gate itself (ForwardArgs::r).
+bool chunked_path_fuses_gate(const ChunkGeom& g);
 cudaError_t launch_forward_chunked(const ForwardArgs& a, const ChunkGeom& g, void* ws, int64_t drop_unit,
                                    cudaStream_t s);
 
 // Persistent warp-specialised variant (bulk rows, chunk 8 or 16); same workspace layout.
+cudaError_t launch_token_shift3(int64_t B, int64_t T, int64_t C, const float* mu_r, const float* mu_k,
+                                const float* mu_v, const float* x, const float* x_last, float* xr, float* xk, float* xv,
+                                cudaStream_t s);
+// y <- sigma(r) * y over n elements of dtype io (0 fp32, 1 bf16), in place
+cudaError_t launch_gate(int64_t n, int io, const void* r, void* y, cudaStream_t s);
+
 cudaError_t launch_forward_pipe(const ForwardArgs& a, const ChunkGeom& g, void* ws, int64_t drop_unit,
                                 cudaStream_t s);
 cudaError_t launch_forward_tmem(const ForwardArgs& a, const ChunkGeom& g, void* ws, int64_t drop_unit,

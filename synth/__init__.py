@@ -30,6 +30,7 @@ S_W, S_U, S_K, S_KSPIKE, S_V, S_MU, S_X = 1, 2, 3, 4, 5, 6, 7
 S_WARM_K, S_WARM_V, S_WARM_X = 8, 9, 10
 S_DEC_K, S_DEC_V, S_DEC_X = 11, 12, 13
 S_STATE_P, S_STATE_B, S_STATE_A = 14, 15, 16
+S_R, S_RSPIKE = 17, 18
 
 
 def build(force: bool = False) -> str:
@@ -184,6 +185,17 @@ def forward_inputs(spec: ForwardSpec):
     if spec.dtype == "bf16":
         k, v = to_bf16_exact(k), to_bf16_exact(v)
     return w, u, k, v
+
+
+def receptance(spec: ForwardSpec, r_std: float = 2.0, spike_prob: float = 0.01, spike_value: float = -40.0):
+    """Receptance r [B,T,C] for the output gate sigma(r) * wkv: N(0, r_std) with a fraction
+    of entries set to spike_value (a gate pushed shut, sigma ~ 4e-18); exact in the I/O dtype."""
+    r = normal(spec.seed, S_R, (spec.B, spec.T, spec.C), 0.0, r_std)
+    if spike_prob > 0:
+        spike(spec.seed, S_RSPIKE, r, spike_prob, spike_value)
+    if spec.dtype == "bf16":
+        r = to_bf16_exact(r)
+    return r
 
 
 def forward_inputs_at(spec: ForwardSpec, b: np.ndarray, c: np.ndarray):
