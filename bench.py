@@ -275,6 +275,7 @@ class ForwardSet:
         self.xbar1 = torch.empty_like(self.x_t)
         self.y1 = torch.empty_like(self.x_t)
         self.state4 = self.state.view(3, B, 1, C)
+        self.r = torch.from_numpy(synth.receptance(s)).to(dev)  # receptance for the gated forward
 
 
 def step(wkv, s, ws, ev=None):
@@ -296,6 +297,63 @@ def capture(torch, wkv, sets, ws, nsteps, with_events):
         for i in range(nsteps):
             step(wkv, sets[i % len(sets)], ws, evs[i])
     return g, evs
+
+
+def graph_ms(torch, fn, n_calls):
+    """Mean time of fn(i) for i in range(n_calls), captured in one CUDA graph, 10 replays."""
+    for i in range(min(n_calls, 6)):
+        fn(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n_calls):
+            fn(i)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(10):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (10 * n_calls)
+    del g
+    return ms
+
+
+def next_rows_bench(torch, wkv, sets, ws, spec, peak):
+    """The fused receptance-gated forward (y = sigma(r) * wkv: k, v, r read and y written once,
+    16 B/element fp32) and the three-mu token shift (x read, three blends written, 16
+    B/element) on the bench workload, rotating input sets, next to the plain forward timed the
+    same way."""
+    n = spec.B * spec.T * spec.C
+
+    def plain(i):
+        s = sets[i % len(sets)]
+        wkv.wkv_forward(s.w, s.u, s.k, s.v, workspace=ws, y=s.y, state_out=s.state)
+
+    def gated(i):
+        s = sets[i % len(sets)]
+        wkv.wkv_forward(s.w, s.u, s.k, s.v, workspace=ws, y=s.y, state_out=s.state, r=s.r)
+
+    mu = [torch.rand(spec.C, device=sets[0].k.device) for _ in range(3)]
+
+    def shift3(i):
+        s = sets[i % len(sets)]
+        wkv.token_shift_mix3(mu[0], mu[1], mu[2], s.k)
+
+    plain_ms = graph_ms(torch, plain, GRAPH_STEPS)
+    gated_ms = graph_ms(torch, gated, GRAPH_STEPS)
+    shift_ms = graph_ms(torch, shift3, GRAPH_STEPS)
+    g_gbs = 16 * n / (gated_ms * 1e-3) / 1e9
+    t_gbs = 16 * n / (shift_ms * 1e-3) / 1e9
+    return {
+        "gated_forward": {"launch_ms": gated_ms, "alg_bytes_per_launch": 16 * n, "achieved_gbs": g_gbs,
+                          "frac": g_gbs / peak, "plain_forward_launch_ms": plain_ms,
+                          "timing": f"graph of {GRAPH_STEPS} back-to-back launches, 10 replays, after the timed region"},
+        "token_shift3": {"launch_ms": shift_ms, "alg_bytes_per_launch": 16 * n, "achieved_gbs": t_gbs,
+                         "frac": t_gbs / peak},
+    }
 
 
 def forward_only_ms(torch, wkv, sets, ws):
@@ -485,6 +543,7 @@ def run_ours(args):
 
     del main_g, rem_g, warm_g
     dec = None if args.no_decode else decode_bench(torch, wkv, dev, 400)
+    nxt = next_rows_bench(torch, wkv, sets, ws, spec, peaks["hbm_gbs"])
     e2e = None
     if not args.no_e2e:
         ms_e2e, h2d, d2h = e2e_bench(torch, wkv, sets, ws, min(K, 240), dev)
@@ -518,6 +577,7 @@ def run_ours(args):
             "e2e": e2e,
             "gpu_launches": 2 * K,
             "decode": dec,
+            "next_rows": nxt,
             "clocks": clocks.summary(t_wall0, t_wall1) if rank == 0 else None,
         }
         print(json.dumps(line), flush=True)
