@@ -19,6 +19,10 @@ Functions (all inputs are converted to contiguous float64):
 * ``decode_step(w, u, k, v, state, sacc)`` -- one token from a given state for
   ``[N, L, C]`` rows with ``[L, C]`` parameters: the recurrence with T = 1.
 * ``gate(r, wkv)`` -- the receptance gate ``sigma(r) * wkv``, elementwise.
+* ``wkv_backward(w, u, k, v, gy)`` -- the gradient of ``sum(gy * y)`` with respect to
+  k, v (per element) and w, u (per channel, summed over batch and time), the
+  wkv_t equation differentiated as written (O(T^2)).  Returns
+  ``(gk, gv, gw, gu, (sk, sv, sw, su))`` with the terms' magnitude scales.
 * ``token_shift3(mu_r, mu_k, mu_v, x, x_last=None)`` -- the lerp with the three
   projections' separate mu (three calls of ``token_shift``).
 
@@ -63,7 +67,9 @@ def load(path: str):
     L.oracle_wkv_naive.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp]
     L.oracle_token_shift.argtypes = [i64, i64, i64, vp, vp, vp, vp]
     L.oracle_gate.argtypes = [i64, vp, vp, vp]
-    for f in (L.oracle_wkv_direct, L.oracle_wkv_recurrent, L.oracle_wkv_naive, L.oracle_token_shift, L.oracle_gate):
+    L.oracle_wkv_backward_direct.argtypes = [i64, i64, i64] + [vp] * 13
+    for f in (L.oracle_wkv_direct, L.oracle_wkv_recurrent, L.oracle_wkv_naive, L.oracle_token_shift, L.oracle_gate,
+              L.oracle_wkv_backward_direct):
         f.restype = None
     L.oracle_num_threads.restype = ctypes.c_int
     return L
@@ -148,6 +154,16 @@ def gate(r, wkv, L=None):
     out = np.empty(r.shape, np.float64)
     (L or lib()).oracle_gate(r.size, _p(r), _p(wkv), _p(out))
     return out
+
+
+def wkv_backward(w, u, k, v, gy, L=None):
+    w, u, k, v, gy = _f64(w), _f64(u), _f64(k), _f64(v), _f64(gy)
+    B, T, C = _btc(k)
+    gk, gv, sk, sv = (np.empty(k.shape, np.float64) for _ in range(4))
+    gw, gu, sw, su = (np.empty(C, np.float64) for _ in range(4))
+    (L or lib()).oracle_wkv_backward_direct(B, T, C, _p(w), _p(u), _p(k), _p(v), _p(gy), _p(gk), _p(gv), _p(gw),
+                                            _p(gu), _p(sk), _p(sv), _p(sw), _p(su))
+    return gk, gv, gw, gu, (sk, sv, sw, su)
 
 
 def token_shift3(mu_r, mu_k, mu_v, x, x_last=None, L=None):

@@ -222,3 +222,73 @@ void oracle_gate(int64_t n, const double* r, const double* wkv, double* out)
         out[i] = wkv[i] * sigma;
     }
 }
+
+/*
+ * Gradient of the wkv_t equation ([MATH] "The WKV operator: attention with a fixed decay";
+ * [WIKI] eq. 1), differentiated as written; the pages give no gradient.  For a loss
+ * L = sum_{b,t,c} gy[b,t,c] * y[b,t,c], with y_t = N_t / D_t,
+ *   N_t = sum_{i<t} beta_{t,i} v_i + alpha_t v_t,   D_t = sum_{i<t} beta_{t,i} + alpha_t,
+ *   beta_{t,i} = e^{-(t-1-i) w + k_i},   alpha_t = e^{u + k_t},
+ * each term contributes (dy_t/dN_t = 1/D_t, dy_t/dD_t = -y_t/D_t):
+ *   current token:  dy_t/dv_t = alpha_t / D_t;   dy_t/dk_t = dy_t/du = alpha_t (v_t - y_t) / D_t
+ *   past token i:   dy_t/dv_i = beta_{t,i} / D_t;  dy_t/dk_i = beta_{t,i} (v_i - y_t) / D_t;
+ *                   dy_t/dw  += -(t-1-i) beta_{t,i} (v_i - y_t) / D_t
+ * gk, gv are [B][T][C]; gw, gu are [C], summed over b and t.  O(T^2) per channel, valid
+ * while every exponent stays below ~709.  The optional s* outputs add up the same terms'
+ * magnitudes (|gy| and |v - y| in place of gy and v - y): the scales the tests divide by.
+ */
+void oracle_wkv_backward_direct(int64_t B, int64_t T, int64_t C, const double* w, const double* u,
+                                const double* k, const double* v, const double* gy, double* gk, double* gv,
+                                double* gw, double* gu, double* sk, double* sv, double* sw, double* su)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t c = 0; c < C; ++c) {
+        double gwc = 0.0, guc = 0.0, swc = 0.0, suc = 0.0;
+        for (int64_t b = 0; b < B; ++b) {
+            for (int64_t t = 0; t < T; ++t) {
+                gk[at3(b, t, c, T, C)] = 0.0;
+                gv[at3(b, t, c, T, C)] = 0.0;
+                if (sk) sk[at3(b, t, c, T, C)] = 0.0;
+                if (sv) sv[at3(b, t, c, T, C)] = 0.0;
+            }
+            for (int64_t t = 0; t < T; ++t) {
+                /* forward value of position t */
+                double num = 0.0, den = 0.0;
+                for (int64_t i = 0; i < t; ++i) {
+                    double beta = exp(-(double)(t - 1 - i) * w[c] + k[at3(b, i, c, T, C)]);
+                    num += beta * v[at3(b, i, c, T, C)];
+                    den += beta;
+                }
+                double alpha = exp(u[c] + k[at3(b, t, c, T, C)]);
+                num += alpha * v[at3(b, t, c, T, C)];
+                den += alpha;
+                double yt = num / den;
+                double g = gy[at3(b, t, c, T, C)] / den;
+                double gm = fabs(gy[at3(b, t, c, T, C)]) / den;
+                /* current token */
+                double vt = v[at3(b, t, c, T, C)];
+                gv[at3(b, t, c, T, C)] += g * alpha;
+                gk[at3(b, t, c, T, C)] += g * alpha * (vt - yt);
+                guc += g * alpha * (vt - yt);
+                if (sv) sv[at3(b, t, c, T, C)] += gm * alpha;
+                if (sk) sk[at3(b, t, c, T, C)] += gm * alpha * fabs(vt - yt);
+                suc += gm * alpha * fabs(vt - yt);
+                /* past tokens */
+                for (int64_t i = 0; i < t; ++i) {
+                    double beta = exp(-(double)(t - 1 - i) * w[c] + k[at3(b, i, c, T, C)]);
+                    double vi = v[at3(b, i, c, T, C)];
+                    gv[at3(b, i, c, T, C)] += g * beta;
+                    gk[at3(b, i, c, T, C)] += g * beta * (vi - yt);
+                    gwc += -g * (double)(t - 1 - i) * beta * (vi - yt);
+                    if (sv) sv[at3(b, i, c, T, C)] += gm * beta;
+                    if (sk) sk[at3(b, i, c, T, C)] += gm * beta * fabs(vi - yt);
+                    swc += gm * (double)(t - 1 - i) * beta * fabs(vi - yt);
+                }
+            }
+        }
+        gw[c] = gwc;
+        gu[c] = guc;
+        if (sw) sw[c] = swc;
+        if (su) su[c] = suc;
+    }
+}

@@ -396,6 +396,51 @@ def pin_token_shift3(L):
     assert np.array_equal(xr, prev0) and np.array_equal(xk, (x + prev0) / 2) and np.array_equal(xv, x)
 
 
+def _loss(L, w, u, k, v, gy):
+    return float((oracle.wkv_direct(w, u, k, v, L=L)[0] * gy).sum())
+
+
+def pin_backward_finite_differences(L):
+    """The gradient of L = sum(gy * y) against central finite differences of the (pinned)
+    direct forward, for every k and v element and every channel's w and u."""
+    for seed, (B, T, C) in ((41, (1, 6, 2)), (42, (2, 4, 3))):
+        w, u, k, v = _rand_case(seed, B, T, C)
+        gy = _rng(seed + 100).normal(0, 1, k.shape)
+        gk, gv, gw, gu, (sk, sv, sw, su) = oracle.wkv_backward(w, u, k, v, gy, L=L)
+        h = 1e-6
+
+        def fd(arr, idx, fn):
+            a1, a0 = arr.copy(), arr.copy()
+            a1[idx] += h
+            a0[idx] -= h
+            return (fn(a1) - fn(a0)) / (2 * h)
+
+        for idx in np.ndindex(k.shape):
+            assert abs(fd(k, idx, lambda x: _loss(L, w, u, x, v, gy)) - gk[idx]) <= 1e-7 * (sk[idx] + 1e-12)
+            assert abs(fd(v, idx, lambda x: _loss(L, w, u, k, x, gy)) - gv[idx]) <= 1e-7 * (sv[idx] + 1e-12)
+        for c in range(C):
+            assert abs(fd(w, (c,), lambda x: _loss(L, x, u, k, v, gy)) - gw[c]) <= 1e-7 * (sw[c] + 1e-12)
+            assert abs(fd(u, (c,), lambda x: _loss(L, w, x, k, v, gy)) - gu[c]) <= 1e-7 * (su[c] + 1e-12)
+
+
+def pin_backward_closed_forms(L):
+    """T = 1: y = v exactly, so gv = gy and every other gradient is zero.  Key shift: y does not
+    change when every key of a channel moves by the same amount, so the k-gradients of each
+    (b, c) sum to zero.  Value shift: y moves by exactly the shift (a convex combination), so
+    the v-gradients of each (b, c) sum to the sum of gy."""
+    w, u, k, v = _rand_case(43, 2, 1, 4)
+    gy = _rng(143).normal(0, 1, k.shape)
+    gk, gv, gw, gu, _ = oracle.wkv_backward(w, u, k, v, gy, L=L)
+    tiny = 1e-15 * np.abs(gy * v)  # y = (alpha v) / alpha is v up to one rounding
+    assert np.allclose(gv, gy, rtol=1e-15, atol=0) and np.all(gw == 0)
+    assert np.all(np.abs(gk) <= tiny) and np.all(np.abs(gu) <= tiny.sum(axis=(0, 1)))
+    w, u, k, v = _rand_case(44, 2, 9, 3)
+    gy = _rng(144).normal(0, 1, k.shape)
+    gk, gv, gw, gu, (sk, sv, _, _) = oracle.wkv_backward(w, u, k, v, gy, L=L)
+    assert np.all(np.abs(gk.sum(axis=1)) <= 1e-12 * sk.sum(axis=1))
+    assert np.allclose(gv.sum(axis=1), gy.sum(axis=1), rtol=1e-12, atol=1e-12)
+
+
 ALL_PINS = [
     pin_worked_example,
     pin_routes_agree,
@@ -415,4 +460,6 @@ ALL_PINS = [
     pin_token_shift,
     pin_gate,
     pin_token_shift3,
+    pin_backward_finite_differences,
+    pin_backward_closed_forms,
 ]

@@ -38,6 +38,12 @@ MUTANTS = {
     "gate_sign": ("const double sigma = 1.0 / (1.0 + exp(-r[i]));", "const double sigma = 1.0 / (1.0 + exp(r[i]));"),
     "gate_offset": ("const double sigma = 1.0 / (1.0 + exp(-r[i]));", "const double sigma = 1.0 / (2.0 + exp(-r[i]));"),
     "gate_divides": ("out[i] = wkv[i] * sigma;", "out[i] = wkv[i] / sigma;"),
+    "backward_drops_current_value": ("gv[at3(b, t, c, T, C)] += g * alpha;", "gv[at3(b, t, c, T, C)] += 0.0 * alpha;"),
+    "backward_key_uses_own_output": ("gk[at3(b, i, c, T, C)] += g * beta * (vi - yt);",
+                                     "gk[at3(b, i, c, T, C)] += g * beta * vi;"),
+    "backward_decay_count_off_by_one": ("gwc += -g * (double)(t - 1 - i) * beta * (vi - yt);",
+                                        "gwc += -g * (double)(t - i) * beta * (vi - yt);"),
+    "backward_bonus_sign": ("guc += g * alpha * (vt - yt);", "guc += g * alpha * (yt - vt);"),
 }
 
 
