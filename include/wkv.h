@@ -120,6 +120,30 @@ wkv_status wkv_forward_gated(int64_t B, int64_t T, int64_t C, wkv_dtype io, cons
                              float* state_out, void* workspace, size_t ws_bytes, wkv_path path, int chunk,
                              cudaStream_t stream);
 
+/*
+ * Backward of the forward from the empty state: for a loss L = sum(gy * y) over [B, T, C],
+ * the gradients of L with respect to k and v (per element) and w and u (per channel, summed
+ * over batch and time).  The pages give no gradient; this is the wkv_t equation above
+ * differentiated as written (with D_t its denominator, alpha_t = e^{u+k_t},
+ * beta_{t,i} = e^{-(t-1-i) w + k_i}: dy_t/dv_i = beta_{t,i} / D_t, dy_t/dk_i =
+ * beta_{t,i} (v_i - y_t) / D_t, dy_t/dw = -sum_i (t-1-i) beta_{t,i} (v_i - y_t) / D_t, and the
+ * current token's alpha_t terms for v_t, k_t and u).
+ *   w, u          [C] fp32
+ *   k, v, gy      [B, T, C] fp32
+ *   gk, gv        [B, T, C] fp32 (written)
+ *   gw, gu        [C] fp32 (written: zeroed, then accumulated on the device)
+ *   workspace     caller-owned device scratch of ws_bytes >= wkv_backward_workspace_size()
+ *                 (per position the output's reference exponent, denominator and value)
+ * One thread per (b, c) runs the recurrence forward and the adjoint recurrence back over T.
+ * Status codes as wkv_forward; B must be <= 65535.
+ */
+wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
+                        const float* v, const float* gy, float* gk, float* gv, float* gw, float* gu,
+                        void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Workspace bytes wkv_backward needs (12 bytes per element). */
+size_t wkv_backward_workspace_size(int64_t B, int64_t T, int64_t C);
+
 /* Workspace bytes wkv_forward needs for this shape (the largest over all paths). */
 size_t wkv_forward_workspace_size(int64_t B, int64_t T, int64_t C, wkv_dtype io);
 

@@ -68,6 +68,9 @@ def lib():
                 L.wkv_get_device_status.argtypes = [vp]
                 L.wkv_forward_gated.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i32, i32, vp]
                 L.token_shift_mix3.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+                L.wkv_backward.argtypes = [i64, i64, i64] + [vp] * 10 + [sz, vp]
+                L.wkv_backward_workspace_size.argtypes = [i64, i64, i64]
+                L.wkv_backward_workspace_size.restype = sz
                 L.wkv_decode_step.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp]
                 L.wkv_decode_step_fused.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
                 L.token_shift_mix.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp]
@@ -76,7 +79,7 @@ def lib():
                 L.wkv_forward_auto_path.argtypes = [i64, i64, i64, i32]
                 L.wkv_testhook_forward_drop.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, sz, i64, u32, vp]
                 for f in (L.wkv_forward, L.wkv_forward_ex, L.wkv_workspace_init, L.wkv_forward_status,
-                          L.wkv_get_device_status, L.wkv_forward_gated, L.token_shift_mix3,
+                          L.wkv_get_device_status, L.wkv_forward_gated, L.token_shift_mix3, L.wkv_backward,
                           L.wkv_decode_step, L.wkv_decode_step_fused, L.token_shift_mix,
                           L.wkv_forward_auto_path, L.wkv_testhook_forward_drop):
                     f.restype = i32
@@ -188,6 +191,28 @@ def wkv_forward(w, u, k, v, state_in=None, want_state=True, path="auto", chunk=0
                               _PATH[path], int(chunk), _stream(dev))
     _check(st, "wkv_forward")
     return y, state_out
+
+
+def wkv_backward(w, u, k, v, gy, workspace=None):
+    """Gradients of sum(gy * y) for the forward from the empty state over fp32 [B, T, C]:
+    returns (gk, gv, gw, gu) with gk, gv [B, T, C] and gw, gu [C]."""
+    for t, name in ((k, "k"), (v, "v"), (gy, "gy")):
+        _cuda_f32(t, name)
+    if k.dim() != 3 or v.shape != k.shape or gy.shape != k.shape:
+        raise ValueError("k, v, gy must be [B, T, C] tensors of one shape")
+    B, T, C = k.shape
+    _cuda_f32(w, "w", (C,))
+    _cuda_f32(u, "u", (C,))
+    gk, gv = torch.empty_like(k), torch.empty_like(v)
+    gw = torch.empty(C, dtype=torch.float32, device=k.device)
+    gu = torch.empty_like(gw)
+    nbytes = int(lib().wkv_backward_workspace_size(B, T, C))
+    ws = workspace if workspace is not None and workspace.numel() >= nbytes else \
+        torch.empty(max(nbytes, 16), dtype=torch.uint8, device=k.device)
+    _check(lib().wkv_backward(B, T, C, w.data_ptr(), u.data_ptr(), k.data_ptr(), v.data_ptr(), gy.data_ptr(),
+                              gk.data_ptr(), gv.data_ptr(), gw.data_ptr(), gu.data_ptr(), ws.data_ptr(), ws.numel(),
+                              _stream(k.device)), "wkv_backward")
+    return gk, gv, gw, gu
 
 
 def forward_status(workspace=None, device=None):

@@ -83,6 +83,12 @@ cudaError_t launch_token_shift3(int64_t B, int64_t T, int64_t C, const float* mu
 // y <- sigma(r) * y over n elements of dtype io (0 fp32, 1 bf16), in place
 cudaError_t launch_gate(int64_t n, int io, const void* r, void* y, cudaStream_t s);
 
+// WKV backward (fp32): gk, gv [B,T,C]; gw, gu [C] (zeroed here, then accumulated); ws holds
+// 3 * B*T*C floats
+cudaError_t launch_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
+                            const float* v, const float* gy, float* gk, float* gv, float* gw, float* gu, void* ws,
+                            cudaStream_t s);
+
 cudaError_t launch_forward_pipe(const ForwardArgs& a, const ChunkGeom& g, void* ws, int64_t drop_unit,
                                 cudaStream_t s);
 cudaError_t launch_forward_tmem(const ForwardArgs& a, const ChunkGeom& g, void* ws, int64_t drop_unit,

@@ -22,7 +22,8 @@ Functions (all inputs are converted to contiguous float64):
 * ``wkv_backward(w, u, k, v, gy)`` -- the gradient of ``sum(gy * y)`` with respect to
   k, v (per element) and w, u (per channel, summed over batch and time), the
   wkv_t equation differentiated as written (O(T^2)).  Returns
-  ``(gk, gv, gw, gu, (sk, sv, sw, su))`` with the terms' magnitude scales.
+  ``(gk, gv, gw, gu, (sk, sv, sw, su))`` with the terms' magnitude scales (|gy|,
+  and |v| + |y| in place of v - y).
 * ``token_shift3(mu_r, mu_k, mu_v, x, x_last=None)`` -- the lerp with the three
   projections' separate mu (three calls of ``token_shift``).
 

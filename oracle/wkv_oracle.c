@@ -235,7 +235,9 @@ void oracle_gate(int64_t n, const double* r, const double* wkv, double* out)
  *                   dy_t/dw  += -(t-1-i) beta_{t,i} (v_i - y_t) / D_t
  * gk, gv are [B][T][C]; gw, gu are [C], summed over b and t.  O(T^2) per channel, valid
  * while every exponent stays below ~709.  The optional s* outputs add up the same terms'
- * magnitudes (|gy| and |v - y| in place of gy and v - y): the scales the tests divide by.
+ * magnitudes with |gy| in place of gy and |v| + |y| in place of v - y: the scales the tests
+ * divide by (y_t is only known to its own rounding, so v - y_t is only known to within a
+ * fraction of |v| + |y_t|, whatever the arithmetic that follows).
  */
 void oracle_wkv_backward_direct(int64_t B, int64_t T, int64_t C, const double* w, const double* u,
                                 const double* k, const double* v, const double* gy, double* gk, double* gv,
@@ -271,8 +273,8 @@ void oracle_wkv_backward_direct(int64_t B, int64_t T, int64_t C, const double* w
                 gk[at3(b, t, c, T, C)] += g * alpha * (vt - yt);
                 guc += g * alpha * (vt - yt);
                 if (sv) sv[at3(b, t, c, T, C)] += gm * alpha;
-                if (sk) sk[at3(b, t, c, T, C)] += gm * alpha * fabs(vt - yt);
-                suc += gm * alpha * fabs(vt - yt);
+                if (sk) sk[at3(b, t, c, T, C)] += gm * alpha * (fabs(vt) + fabs(yt));
+                suc += gm * alpha * (fabs(vt) + fabs(yt));
                 /* past tokens */
                 for (int64_t i = 0; i < t; ++i) {
                     double beta = exp(-(double)(t - 1 - i) * w[c] + k[at3(b, i, c, T, C)]);
@@ -281,8 +283,8 @@ void oracle_wkv_backward_direct(int64_t B, int64_t T, int64_t C, const double* w
                     gk[at3(b, i, c, T, C)] += g * beta * (vi - yt);
                     gwc += -g * (double)(t - 1 - i) * beta * (vi - yt);
                     if (sv) sv[at3(b, i, c, T, C)] += gm * beta;
-                    if (sk) sk[at3(b, i, c, T, C)] += gm * beta * fabs(vi - yt);
-                    swc += gm * (double)(t - 1 - i) * beta * fabs(vi - yt);
+                    if (sk) sk[at3(b, i, c, T, C)] += gm * beta * (fabs(vi) + fabs(yt));
+                    swc += gm * (double)(t - 1 - i) * beta * (fabs(vi) + fabs(yt));
                 }
             }
         }

@@ -31,6 +31,7 @@ S_WARM_K, S_WARM_V, S_WARM_X = 8, 9, 10
 S_DEC_K, S_DEC_V, S_DEC_X = 11, 12, 13
 S_STATE_P, S_STATE_B, S_STATE_A = 14, 15, 16
 S_R, S_RSPIKE = 17, 18
+S_GY = 19
 
 
 def build(force: bool = False) -> str:
@@ -196,6 +197,11 @@ def receptance(spec: ForwardSpec, r_std: float = 2.0, spike_prob: float = 0.01, 
     if spec.dtype == "bf16":
         r = to_bf16_exact(r)
     return r
+
+
+def grad_output(spec: ForwardSpec, std: float = 1.0):
+    """Upstream gradient gy [B,T,C] for the backward: N(0, std), fp32."""
+    return normal(spec.seed, S_GY, (spec.B, spec.T, spec.C), 0.0, std)
 
 
 def forward_inputs_at(spec: ForwardSpec, b: np.ndarray, c: np.ndarray):

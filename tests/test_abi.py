@@ -92,3 +92,31 @@ def test_binding_refuses_cpu_tensors():
         wkv.wkv_forward(torch.ones(4), torch.zeros(4), k, k)
     with pytest.raises(TypeError):
         wkv.token_shift_mix(torch.ones(4), k)
+
+
+def test_backward_validation_without_launch():
+    """wkv_backward checks its arguments before touching the device (through the binding's
+    argument types, so a wrong argument count fails here too)."""
+    L = wkv.lib()
+
+    def bwd(B, T, C, w=FAKE, k=FAKE, gk=FAKE, ws=FAKE, nbytes=1 << 30):
+        return L.wkv_backward(B, T, C, w, FAKE, k, FAKE, FAKE, gk, FAKE, FAKE, FAKE, ws, nbytes, None)
+
+    assert bwd(-1, 4, 4) == 1                    # negative size
+    assert bwd(1, 4, 4, w=None) == 1             # null parameter
+    assert bwd(1, 4, 4, k=None) == 1             # null input
+    assert bwd(1, 4, 4, gk=FAKE + 4) == 2        # misaligned output
+    assert bwd(1, 4, 4, nbytes=16) == 1          # workspace too small (12 B per element)
+    assert bwd(70000, 1, 4) == 3                 # batch above the grid's y limit
+    assert L.wkv_backward_workspace_size(2, 3, 5) == 2 * 3 * 5 * 12
+
+
+def test_gated_and_shift3_validation_without_launch():
+    L = wkv.lib()
+    gated = lambda r, y=FAKE: L.wkv_forward_gated(1, 4, 4, 0, FAKE, FAKE, FAKE, FAKE, r, None, y, None, FAKE,
+                                                   1 << 30, 0, 0, None)
+    assert gated(None) == 1                      # r is required
+    assert gated(FAKE + 8) == 2                  # misaligned r
+    shift3 = lambda x=FAKE, xr=FAKE: L.token_shift_mix3(1, 4, 4, FAKE, FAKE, FAKE, x, None, xr, FAKE, FAKE, None)
+    assert shift3(x=None) == 1
+    assert shift3(xr=FAKE + 4) == 2

@@ -1,0 +1,72 @@
+"""The WKV backward against the oracle (GPU).
+
+Gradients of L = sum(gy * y) with respect to k, v (per element) and w, u (per channel),
+for the forward from the empty state.  Each error is divided by the magnitude of the terms
+that make up that gradient (the oracle adds them up with |gy| and |v - y|): gradients that
+cancel to near zero are not judged relative to themselves.  Bar: 2e-4 of that scale (fp32
+throughout; the reverse scan compounds the forward's rounding over T steps).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from parity_util import to_gpu
+
+pytestmark = pytest.mark.gpu
+
+TOL_GRAD = 2e-4
+SHAPES = [(1, 1, 4), (2, 5, 3), (1, 64, 64), (3, 200, 96), (1, 1000, 32), (2, 130, 129)]
+
+
+def _case(B, T, C, base, seed, k_shift=0.0):
+    spec = synth.forward_spec_like(base, B, T, C, seed=seed)
+    w, u, k, v = synth.forward_inputs(spec)
+    return w, u, k + np.float32(k_shift), v, synth.grad_output(spec)
+
+
+def _gpu_backward(w, u, k, v, gy):
+    import torch
+    import linear_attention_rnn_wkv_b200 as wkv
+    gk, gv, gw, gu = wkv.wkv_backward(to_gpu(w), to_gpu(u), to_gpu(k), to_gpu(v), to_gpu(gy))
+    torch.cuda.synchronize()
+    return gk.cpu().numpy(), gv.cpu().numpy(), gw.cpu().numpy(), gu.cpu().numpy()
+
+
+def _check(w, u, k, v, gy):
+    gk, gv, gw, gu = _gpu_backward(w, u, k, v, gy)
+    rk, rv, rw, ru, (sk, sv, sw, su) = oracle.wkv_backward(w, u, k, v, gy)
+    for name, g, r, s in (("gk", gk, rk, sk), ("gv", gv, rv, sv), ("gw", gw, rw, sw), ("gu", gu, ru, su)):
+        err = np.abs(g - r) / np.maximum(s, 1e-30)
+        assert np.all(np.isfinite(g)), name
+        assert err.max() <= TOL_GRAD, f"{name}: {err.max():.3e}"
+
+
+@pytest.mark.parametrize("base", ["fwd_64x64", "fwd_8x1024x768"])
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_backward_matches_oracle(shape, base):
+    B, T, C = shape
+    _check(*_case(B, T, C, base, seed=9500 + B * 131 + T * 17 + C))
+
+
+def test_backward_key_shift():
+    """Keys shifted by +100 (exponents near 144 in base 2): the gradients do not change."""
+    _check(*_case(2, 300, 64, "fwd_8x1024x768", seed=9601, k_shift=100.0))
+
+
+def test_backward_full_width_sampled():
+    """fwd_8x1024x768's shape (B=8, T=1024, C=768) through the GPU, sampled channels against
+    the oracle (channels are independent; gw and gu of a channel sum over the whole batch)."""
+    import torch
+    import linear_attention_rnn_wkv_b200 as wkv
+    spec = synth.FORWARD["fwd_8x1024x768"]
+    w, u, k, v = synth.forward_inputs(spec)
+    gy = synth.grad_output(spec)
+    gk, gv, gw, gu = (t.cpu().numpy() for t in wkv.wkv_backward(*(to_gpu(a) for a in (w, u, k, v, gy))))
+    for c in np.random.default_rng(11).choice(spec.C, 6, replace=False):
+        sl = np.s_[:, :, c:c + 1]
+        rk, rv, rw, ru, (sk, sv, sw, su) = oracle.wkv_backward(w[c:c + 1], u[c:c + 1], k[sl], v[sl], gy[sl])
+        assert np.max(np.abs(gk[sl] - rk) / np.maximum(sk, 1e-30)) <= TOL_GRAD
+        assert np.max(np.abs(gv[sl] - rv) / np.maximum(sv, 1e-30)) <= TOL_GRAD
+        assert abs(gw[c] - rw[0]) <= TOL_GRAD * sw[0]
+        assert abs(gu[c] - ru[0]) <= TOL_GRAD * su[0]
