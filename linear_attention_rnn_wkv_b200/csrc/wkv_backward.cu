@@ -43,11 +43,13 @@ __global__ void __launch_bounds__(128) backward_kernel(int64_t B, int64_t T, int
     const float w2 = w[c] * kLog2e, u2 = u[c] * kLog2e;
     const int64_t base = b * T * C + c;
 
+    // Both passes walk T in blocks of kBlk steps: a block's loads are all issued before its
+    // first step is computed, so the recurrence waits for memory once per block, not per step.
+    constexpr int kBlk = 8;
+
     // ---- pass 1: forward, anchored reference p = anc - n w (no drift from rounding p - w)
     float a = 0.f, bb = 0.f, anc = kPEmpty, n = 0.f;
-    for (int64_t t = 0; t < T; ++t) {
-        const int64_t at = base + t * C;
-        const float k2 = k[at] * kLog2e, vt = v[at];
+    auto fwd_step = [&](int64_t at, float k2, float vt) {
         const float p = fmaf(-n, w2, anc);
         const float uk = u2 + k2;
         const float q = fmaxf(p, uk);
@@ -72,16 +74,26 @@ __global__ void __launch_bounds__(128) backward_kernel(int64_t B, int64_t T, int
             bb += f;
             n += 1.f;
         }
+    };
+    int64_t t = 0;
+    for (; t + kBlk <= T; t += kBlk) {
+        float kb[kBlk], vb[kBlk];
+#pragma unroll
+        for (int j = 0; j < kBlk; ++j) {
+            kb[j] = k[base + (t + j) * C];
+            vb[j] = v[base + (t + j) * C];
+        }
+#pragma unroll
+        for (int j = 0; j < kBlk; ++j) fwd_step(base + (t + j) * C, kb[j] * kLog2e, vb[j]);
     }
+    for (; t < T; ++t) fwd_step(base + t * C, k[base + t * C] * kLog2e, v[base + t * C]);
 
     // ---- pass 2: reverse
     float x = 0.f, ya = 0.f, xp = 0.f, yp = 0.f;  // X, Y, X', Y' relative to 2^{-r}
     float r = 3.0e38f;                            // no later output yet
     float sgw = 0.f, sgu = 0.f;
-    for (int64_t t = T - 1; t >= 0; --t) {
-        const int64_t at = base + t * C;
-        const float k2 = k[at] * kLog2e, vt = v[at], g = gy[at];
-        const float q = wq[at], rd = rcp(wd[at]), yt = wy[at];
+    auto rev_step = [&](int64_t at, float k2, float vt, float g, float q, float dn, float yt) {
+        const float rd = rcp(dn);
         const float cur = ex2(u2 + k2 - q) * rd;          // alpha_t / D_t
         const float ek = ex2(k2 - r);                     // e^{k_t} 2^{-r} (0 while r is the sentinel)
         const float gc = g * cur;
@@ -98,6 +110,27 @@ __global__ void __launch_bounds__(128) backward_kernel(int64_t B, int64_t T, int
         x = fmaf(x, so, sn);
         ya = fmaf(ya, so, sn * yt);
         r = rn;
+    };
+    t = T;
+    for (; t - kBlk >= 0; t -= kBlk) {
+        float kb[kBlk], vb[kBlk], gb[kBlk], qb[kBlk], db[kBlk], yb[kBlk];
+#pragma unroll
+        for (int j = 0; j < kBlk; ++j) {
+            const int64_t at = base + (t - 1 - j) * C;
+            kb[j] = k[at];
+            vb[j] = v[at];
+            gb[j] = gy[at];
+            qb[j] = wq[at];
+            db[j] = wd[at];
+            yb[j] = wy[at];
+        }
+#pragma unroll
+        for (int j = 0; j < kBlk; ++j)
+            rev_step(base + (t - 1 - j) * C, kb[j] * kLog2e, vb[j], gb[j], qb[j], db[j], yb[j]);
+    }
+    for (; t > 0; --t) {
+        const int64_t at = base + (t - 1) * C;
+        rev_step(at, k[at] * kLog2e, v[at], gy[at], wq[at], wd[at], wy[at]);
     }
     atomicAdd(&gw[c], sgw);
     atomicAdd(&gu[c], sgu);
