@@ -323,9 +323,9 @@ def graph_ms(torch, fn, n_calls):
 
 def next_rows_bench(torch, wkv, sets, ws, spec, peak):
     """The fused receptance-gated forward (y = sigma(r) * wkv: k, v, r read and y written once,
-    16 B/element fp32) and the three-mu token shift (x read, three blends written, 16
-    B/element) on the bench workload, rotating input sets, next to the plain forward timed the
-    same way."""
+    16 B/element fp32), the three-mu token shift (x read, three blends written, 16 B/element)
+    and the backward (k, v, gy read, gk, gv written: 20 B/element) on the bench workload,
+    rotating input sets, next to the plain forward timed the same way."""
     n = spec.B * spec.T * spec.C
 
     def plain(i):
@@ -342,9 +342,19 @@ def next_rows_bench(torch, wkv, sets, ws, spec, peak):
         s = sets[i % len(sets)]
         wkv.token_shift_mix3(mu[0], mu[1], mu[2], s.k)
 
+    gy = torch.randn_like(sets[0].k)
+    bws = torch.empty(int(wkv.lib().wkv_backward_workspace_size(spec.B, spec.T, spec.C)), dtype=torch.uint8,
+                      device=sets[0].k.device)
+
+    def backward(i):
+        s = sets[i % len(sets)]
+        wkv.wkv_backward(s.w, s.u, s.k, s.v, gy, workspace=bws)
+
     plain_ms = graph_ms(torch, plain, GRAPH_STEPS)
     gated_ms = graph_ms(torch, gated, GRAPH_STEPS)
     shift_ms = graph_ms(torch, shift3, GRAPH_STEPS)
+    bwd_ms = graph_ms(torch, backward, 6)
+    b_gbs = 20 * n / (bwd_ms * 1e-3) / 1e9
     g_gbs = 16 * n / (gated_ms * 1e-3) / 1e9
     t_gbs = 16 * n / (shift_ms * 1e-3) / 1e9
     return {
@@ -353,6 +363,10 @@ def next_rows_bench(torch, wkv, sets, ws, spec, peak):
                           "timing": f"graph of {GRAPH_STEPS} back-to-back launches, 10 replays, after the timed region"},
         "token_shift3": {"launch_ms": shift_ms, "alg_bytes_per_launch": 16 * n, "achieved_gbs": t_gbs,
                          "frac": t_gbs / peak},
+        "backward": {"launch_ms": bwd_ms, "alg_bytes_per_launch": 20 * n, "achieved_gbs": b_gbs,
+                     "frac": b_gbs / peak,
+                     "note": "k, v, gy read and gk, gv written once (20 B/element); the kernel also writes and "
+                             "reads back 12 B/element of per-position forward values"},
     }
 
 
