@@ -134,14 +134,15 @@ wkv_status wkv_forward_gated(int64_t B, int64_t T, int64_t C, wkv_dtype io, cons
  *   gw, gu        [C] fp32 (written: zeroed, then accumulated on the device)
  *   workspace     caller-owned device scratch of ws_bytes >= wkv_backward_workspace_size()
  *                 (per position the output's reference exponent, denominator and value)
- * One thread per (b, c) runs the recurrence forward and the adjoint recurrence back over T.
- * Status codes as wkv_forward; B must be <= 65535.
+ * Time-parallel over segments of 64 steps: the segments' forward states and adjoint sums are
+ * each combined by one scan per channel, then every segment writes its gradients.
+ * Status codes as wkv_forward; B and ceil(T / 64) must be <= 65535.
  */
 wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
                         const float* v, const float* gy, float* gk, float* gv, float* gw, float* gu,
                         void* workspace, size_t ws_bytes, cudaStream_t stream);
 
-/* Workspace bytes wkv_backward needs (12 bytes per element). */
+/* Workspace bytes wkv_backward needs (12 bytes per element, plus 36 per channel and 64 steps). */
 size_t wkv_backward_workspace_size(int64_t B, int64_t T, int64_t C);
 
 /* Workspace bytes wkv_forward needs for this shape (the largest over all paths). */

@@ -197,21 +197,23 @@ wkv_status token_shift_mix3(int64_t B, int64_t T, int64_t C, const float* mu_r, 
 
 size_t wkv_backward_workspace_size(int64_t B, int64_t T, int64_t C) {
     int64_t n = 0;
-    if (!sizes_ok(B, T, C, &n) || n > INT64_MAX / 12) return 0;
-    return (size_t)n * 3 * sizeof(float);
+    if (!sizes_ok(B, T, C, &n) || n > INT64_MAX / 64) return 0;
+    // per element: the output's reference exponent, denominator and value; per (b, segment, c):
+    // a forward state record (4 floats) and the adjoint sums with their reference (5 floats)
+    return ((size_t)n * 3 + (size_t)B * (size_t)backward_segments(T) * (size_t)C * 9) * sizeof(float);
 }
 
 wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
                         const float* v, const float* gy, float* gk, float* gv, float* gw, float* gu, void* workspace,
                         size_t ws_bytes, cudaStream_t stream) {
     int64_t n = 0;
-    if (!sizes_ok(B, T, C, &n) || n > INT64_MAX / 12) return WKV_ERR_INVALID_ARG;
+    if (!sizes_ok(B, T, C, &n) || n > INT64_MAX / 64) return WKV_ERR_INVALID_ARG;
     if (C == 0) return WKV_OK;
     if (!w || !u || !gw || !gu) return WKV_ERR_INVALID_ARG;
     if (n > 0 && (!k || !v || !gy || !gk || !gv)) return WKV_ERR_INVALID_ARG;
     if (!f32_args_ok({w, u, k, v, gy, gk, gv, gw, gu, workspace})) return WKV_ERR_MISALIGNED;
-    if (n > 0 && (!workspace || ws_bytes < (size_t)n * 3 * sizeof(float))) return WKV_ERR_INVALID_ARG;
-    if (B > 65535) return WKV_ERR_UNSUPPORTED;
+    if (n > 0 && (!workspace || ws_bytes < wkv_backward_workspace_size(B, T, C))) return WKV_ERR_INVALID_ARG;
+    if (B > 65535 || backward_segments(T) > 65535) return WKV_ERR_UNSUPPORTED;
     cudaError_t e = launch_backward(B, T, C, w, u, k, v, gy, gk, gv, gw, gu, workspace, stream);
     return e == cudaSuccess ? WKV_OK : cuda_fail(e);
 }

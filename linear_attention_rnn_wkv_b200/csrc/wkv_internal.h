@@ -84,7 +84,8 @@ cudaError_t launch_token_shift3(int64_t B, int64_t T, int64_t C, const float* mu
 cudaError_t launch_gate(int64_t n, int io, const void* r, void* y, cudaStream_t s);
 
 // WKV backward (fp32): gk, gv [B,T,C]; gw, gu [C] (zeroed here, then accumulated); ws holds
-// 3 * B*T*C floats
+// 3 * B*T*C + 9 * B*P*C floats, P = backward_segments(T)
+int64_t backward_segments(int64_t T);
 cudaError_t launch_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
                             const float* v, const float* gy, float* gk, float* gv, float* gw, float* gu, void* ws,
                             cudaStream_t s);

@@ -106,9 +106,11 @@ def test_backward_validation_without_launch():
     assert bwd(1, 4, 4, w=None) == 1             # null parameter
     assert bwd(1, 4, 4, k=None) == 1             # null input
     assert bwd(1, 4, 4, gk=FAKE + 4) == 2        # misaligned output
-    assert bwd(1, 4, 4, nbytes=16) == 1          # workspace too small (12 B per element)
-    assert bwd(70000, 1, 4) == 3                 # batch above the grid's y limit
-    assert L.wkv_backward_workspace_size(2, 3, 5) == 2 * 3 * 5 * 12
+    assert bwd(1, 4, 4, nbytes=16) == 1          # workspace too small
+    assert bwd(70000, 1, 4) == 3                 # batch above the grid's z limit
+    # 12 B per element plus 36 B per (b, 64-step segment, c)
+    assert L.wkv_backward_workspace_size(2, 3, 5) == 2 * 3 * 5 * 12 + 2 * 1 * 5 * 36
+    assert L.wkv_backward_workspace_size(1, 130, 2) == 130 * 2 * 12 + 3 * 2 * 36
 
 
 def test_gated_and_shift3_validation_without_launch():
