@@ -365,8 +365,8 @@ def next_rows_bench(torch, wkv, sets, ws, spec, peak):
                          "frac": t_gbs / peak},
         "backward": {"launch_ms": bwd_ms, "alg_bytes_per_launch": 20 * n, "achieved_gbs": b_gbs,
                      "frac": b_gbs / peak,
-                     "note": "k, v, gy read and gk, gv written once (20 B/element); the kernel also writes and "
-                             "reads back 12 B/element of per-position forward values"},
+                     "note": "k, v, gy read and gk, gv written once (20 B/element); the five kernels read k, v "
+                             "three times and gy twice (40 B/element moved)"},
     }
 
 

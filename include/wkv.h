@@ -130,19 +130,20 @@ wkv_status wkv_forward_gated(int64_t B, int64_t T, int64_t C, wkv_dtype io, cons
  * current token's alpha_t terms for v_t, k_t and u).
  *   w, u          [C] fp32
  *   k, v, gy      [B, T, C] fp32
- *   gk, gv        [B, T, C] fp32 (written)
+ *   gk, gv        [B, T, C] fp32 (written; must not overlap the inputs)
  *   gw, gu        [C] fp32 (written: zeroed, then accumulated on the device)
  *   workspace     caller-owned device scratch of ws_bytes >= wkv_backward_workspace_size()
- *                 (per position the output's reference exponent, denominator and value)
- * Time-parallel over segments of 64 steps: the segments' forward states and adjoint sums are
- * each combined by one scan per channel, then every segment writes its gradients.
- * Status codes as wkv_forward; B and ceil(T / 64) must be <= 65535.
+ *                 (per channel and segment: a forward state record and the adjoint sums)
+ * Time-parallel over segments of 32 steps: the segments' forward states and adjoint sums are
+ * each combined by one scan per channel, then every segment recomputes its outputs and writes
+ * its gradients; nothing per position is kept in global memory.
+ * Status codes as wkv_forward; B and ceil(T / 32) must be <= 65535.
  */
 wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
                         const float* v, const float* gy, float* gk, float* gv, float* gw, float* gu,
                         void* workspace, size_t ws_bytes, cudaStream_t stream);
 
-/* Workspace bytes wkv_backward needs (12 bytes per element, plus 36 per channel and 64 steps). */
+/* Workspace bytes wkv_backward needs (36 per batch row, channel and 32 steps). */
 size_t wkv_backward_workspace_size(int64_t B, int64_t T, int64_t C);
 
 /* Workspace bytes wkv_forward needs for this shape (the largest over all paths). */

@@ -198,9 +198,9 @@ wkv_status token_shift_mix3(int64_t B, int64_t T, int64_t C, const float* mu_r, 
 size_t wkv_backward_workspace_size(int64_t B, int64_t T, int64_t C) {
     int64_t n = 0;
     if (!sizes_ok(B, T, C, &n) || n > INT64_MAX / 64) return 0;
-    // per element: the output's reference exponent, denominator and value; per (b, segment, c):
-    // a forward state record (4 floats) and the adjoint sums with their reference (5 floats)
-    return ((size_t)n * 3 + (size_t)B * (size_t)backward_segments(T) * (size_t)C * 9) * sizeof(float);
+    // per (b, segment, c): a forward state record (4 floats) and the adjoint sums with their
+    // reference (5 floats)
+    return (size_t)B * (size_t)backward_segments(T) * (size_t)C * 9 * sizeof(float);
 }
 
 wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,

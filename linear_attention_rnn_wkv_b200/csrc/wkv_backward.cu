@@ -13,30 +13,41 @@
 // same sums weighted by (t-1-i).  They obey the reverse (adjoint) recurrences
 //   X_{i-1} = gy_i / D_i + e^{-w} X_i,   X'_{i-1} = e^{-w} (X'_i + X_i)   (likewise Y, Y'),
 // so over a span of len positions entered with (X, X') from its right they compose as
-//   X_start = X_local + e^{-w len} X,   X'_start = X'_local + e^{-w len} (X' + len X).
+//   X_start = X_local + e^{-w len} X,   X'_start = X'_local + e^{-w len} (X' + len X),
+// and a span's local sums at its left edge t0 - 1 are the plain weighted sums
+//   X_local = sum_{t in span} e^{-(t-t0) w} gy_t / D_t,  X'_local = the same weighted by (t - t0),
+// which can be accumulated walking left to right.
 //
 // Time-parallel in segments of kSeg steps, one thread per (b, c, segment), five launches:
 //   A  each segment's forward recurrence from the empty state -> its state record;
-//   B  per channel, the records combined in time order -> each segment's starting state;
-//   C  each segment's forward from its starting state, keeping per position the output's
-//      reference exponent q_t, normalised denominator Dn_t (D_t = Dn_t 2^{q_t}) and y_t, then
-//      its adjoint recurrence from zero -> the segment's local (X, Y, X', Y');
+//   B  per channel, the records combined in time order -> each segment's starting state
+//      (and gw, gu zeroed for the atomics of E);
+//   C  each segment's forward from its starting state, accumulating its local (X, Y, X', Y')
+//      left to right as each D_t and y_t appears;
 //   D  per channel, the local sums composed right to left -> each segment's incoming sums;
-//   E  each segment's adjoint recurrence from its incoming sums -> gk, gv, and gw, gu
-//      partials added into the zeroed outputs with atomics.
+//   E  each segment's forward again, keeping per position the output's reference exponent q_t,
+//      1 / Dn_t (D_t = Dn_t 2^{q_t}) and y_t in shared memory, then its adjoint recurrence from
+//      the incoming sums -> gk, gv, and gw, gu partials added with atomics.
+// k, v are read three times and gy twice (40 B per element with gk, gv written); nothing per
+// position is stored in global memory.
 // Numerics: the forward keeps an anchored reference p = anc - n w (no drift from rounding
-// p - w); the adjoint sums are held relative to a running reference r (X = x 2^{-r}) chosen so
-// every rescaling exponent is <= 0, and e^{k_i} X_i = x 2^{k_i log2 e - r} <= x because k_i
-// never exceeds the reference of a later output.
+// p - w); the adjoint sums are held relative to a reference r (X = x 2^{-r}) chosen so every
+// rescaling exponent is <= 0, and e^{k_i} X_i = x 2^{k_i log2 e - r} <= x because k_i never
+// exceeds the reference of a later output.
 #include "wkv_device.cuh"
 #include "wkv_internal.h"
 
 namespace wkvb {
 namespace {
 
-constexpr int kSeg = 64;      // time steps per segment
-constexpr int kBlk = 8;       // steps whose loads are issued together
+constexpr int kSeg = 32;           // time steps per segment
+constexpr int kBlk = 16;           // steps whose loads are issued together
+constexpr int kScanBlk = 8;        // segment records loaded together by the per-channel scans
+constexpr int kThreads = 128;      // threads per block (channels of one (b, segment))
 constexpr float kRNone = 3.0e38f;  // reference of an empty adjoint sum
+// E's per-position values: [kSeg][3][kThreads] floats, each thread its own column
+constexpr size_t kGradSmem = (size_t)kSeg * 3 * kThreads * sizeof(float);
+static_assert(kGradSmem <= 48 * 1024, "fits the default dynamic shared memory limit");
 
 struct Adj {
     float x, y, xp, yp, r;  // X, Y, X', Y' relative to 2^{-r}
@@ -49,95 +60,151 @@ struct FwdState {
     float a, bb, anc, n;
 };
 
-// One forward step at position `at`: the output's (q, Dn, y) into the scratch planes, then the
-// token folded in (decay by counting, re-anchor on a new maximum).
-__device__ __forceinline__ void fwd_step(FwdState& s, float k2, float vt, float u2, float w2, float* q_out,
-                                         float* d_out, float* y_out) {
-    const float p = fmaf(-s.n, w2, s.anc);
-    const float uk = u2 + k2;
-    if (q_out) {
+// What the adjoint needs of one output: its reference exponent q (base 2), 1 / Dn with
+// D = Dn 2^q, and y.
+struct FwdOut {
+    float q, rd, y;
+};
+
+// One forward step: the output (when OUT) from the state before the token, then the token
+// folded in (decay by counting, re-anchor on a new maximum).
+template <bool OUT>
+__device__ __forceinline__ void fwd_step(FwdState& s, float k2, float vt, float u2, float w2, FwdOut& o) {
+    if (OUT) {
+        const float p = fmaf(-s.n, w2, s.anc);
+        const float uk = u2 + k2;
         const float e = ex2(-fabsf(p - uk));  // the other weight is exactly 1
         const bool cur = uk > p;
         const float e1 = cur ? e : 1.f, e2 = cur ? 1.f : e;
-        const float dn = fmaf(e1, s.bb, e2);
-        *q_out = fmaxf(p, uk);
-        *d_out = dn;
-        *y_out = fmaf(e1, s.a, e2 * vt) * rcp(dn);
+        o.q = fmaxf(p, uk);
+        o.rd = rcp(fmaf(e1, s.bb, e2));
+        o.y = fmaf(e1, s.a, e2 * vt) * o.rd;
     }
+    // fold the token in without a branch (the loads of later steps stay ahead of this):
+    // a new maximum re-anchors on k2 and scales the history, else the token is scaled
     const float pn = fmaf(-(s.n + 1.f), w2, s.anc);
-    if (k2 > pn) {
-        const float f = ex2(pn - k2);
-        s.a = fmaf(f, s.a, vt);
-        s.bb = fmaf(f, s.bb, 1.f);
-        s.anc = k2;
-        s.n = 0.f;
-    } else {
-        const float f = ex2(k2 - pn);
-        s.a = fmaf(f, vt, s.a);
-        s.bb += f;
-        s.n += 1.f;
-    }
+    const bool nw = k2 > pn;
+    const float f = ex2(-fabsf(pn - k2));
+    s.a = fmaf(f, nw ? s.a : vt, nw ? vt : s.a);
+    s.bb = fmaf(f, nw ? s.bb : 1.f, nw ? 1.f : s.bb);
+    s.anc = nw ? k2 : s.anc;
+    s.n = nw ? 0.f : s.n + 1.f;
 }
 
-// One adjoint step at a position (walking right to left): the position's gradients (if asked
-// for) from the sums over later outputs, then its own output's terms added and the rest decayed.
-template <bool OUT>
-__device__ __forceinline__ void adj_step(Adj& s, float k2, float vt, float g, float q, float dn, float yt, float u2,
-                                         float w2, float* gk_out, float* gv_out, float& sgw, float& sgu) {
-    const float rd = rcp(dn);
-    if (OUT) {
-        const float cur = ex2(u2 + k2 - q) * rd;  // alpha_t / D_t
-        const float ek = ex2(k2 - s.r);           // e^{k_t} 2^{-r} (0 for an empty sum)
-        const float gc = g * cur;
-        *gv_out = fmaf(ek, s.x, gc);
-        *gk_out = fmaf(ek, fmaf(vt, s.x, -s.y), gc * (vt - yt));
-        sgu = fmaf(gc, vt - yt, sgu);
-        sgw = fmaf(-ek, fmaf(vt, s.xp, -s.yp), sgw);
-    }
-    const float rn = fminf(q, s.r + w2);
-    const float sn = ex2(rn - q) * rd * g;  // gy_t / D_t in the new frame
-    const float so = ex2(rn - s.r - w2);    // e^{-w} and the change of frame
+// One adjoint step at a position (walking right to left): the position's gradients from the
+// sums over later outputs, then its own output's terms added and the rest decayed.
+__device__ __forceinline__ void adj_step(Adj& s, float k2, float vt, float g, const FwdOut& o, float u2, float w2,
+                                         float& gk_out, float& gv_out, float& sgw, float& sgu) {
+    const float cur = ex2(u2 + k2 - o.q) * o.rd;  // alpha_t / D_t
+    const float ek = ex2(k2 - s.r);               // e^{k_t} 2^{-r} (0 for an empty sum)
+    const float gc = g * cur;
+    gv_out = fmaf(ek, s.x, gc);
+    gk_out = fmaf(ek, fmaf(vt, s.x, -s.y), gc * (vt - o.y));
+    sgu = fmaf(gc, vt - o.y, sgu);
+    sgw = fmaf(-ek, fmaf(vt, s.xp, -s.yp), sgw);
+    const float rn = fminf(o.q, s.r + w2);
+    const float sn = ex2(rn - o.q) * o.rd * g;  // gy_t / D_t in the new frame
+    const float so = ex2(rn - s.r - w2);        // e^{-w} and the change of frame
     s.xp = (s.xp + s.x) * so;
     s.yp = (s.yp + s.y) * so;
     s.x = fmaf(s.x, so, sn);
-    s.y = fmaf(s.y, so, sn * yt);
+    s.y = fmaf(s.y, so, sn * o.y);
     s.r = rn;
 }
+
+// A segment's local adjoint sums at its left edge, accumulated left to right.  Term j (the
+// segment's j-th output) is gy/D e^{-j w} = (g rd) 2^{-(q + j w2)}; the sums are held relative
+// to 2^{-R} with R = Rq + Rj w2 the smallest term exponent so far, so each rescaling factor
+// is <= 1 and the exponent difference is formed without the large j w2 rounded on its own.
+struct LocalSums {
+    float x, y, xp, yp, Rq, Rj;
+    __device__ __forceinline__ void add(float jf, float g, const FwdOut& o, float w2) {
+        const float d = fmaf(jf - Rj, w2, o.q - Rq);  // this term's exponent minus R
+        const float e = ex2(-fabsf(d));
+        const bool lower = d < 0.f;                   // the new term is the larger: new frame
+        const float fo = lower ? e : 1.f, fn = lower ? 1.f : e;
+        Rq = lower ? o.q : Rq;
+        Rj = lower ? jf : Rj;
+        const float m = g * o.rd * fn;
+        const float my = m * o.y;
+        x = fmaf(x, fo, m);
+        y = fmaf(y, fo, my);
+        xp = fmaf(xp, fo, jf * m);
+        yp = fmaf(yp, fo, jf * my);
+    }
+};
+
+// A block's loads are volatile asm (kept in program order) and each loaded value passes through
+// an empty volatile asm after the last of them, so all of a block's loads are in flight before
+// its first step is computed.  The inputs are read-only for the whole launch.
+__device__ __forceinline__ float ld_in(const float* p) {
+    float x;
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(x) : "l"(p));
+    return x;
+}
+__device__ __forceinline__ void hold(float& x) { asm volatile("" : "+f"(x)); }
 
 struct BwdArgs {
     int64_t B, T, C, P;  // P segments of kSeg steps (the last may be shorter)
     const float *w, *u, *k, *v, *gy;
     float *gk, *gv, *gw, *gu;
-    float *q, *dn, *y;   // [B][T][C] per-position forward values
-    float* fs;           // [4][B][P][C] segment records, then starting states
-    float* as;           // [5][B][P][C] local adjoint sums, then incoming sums
+    float* fs;  // [4][B][P][C] segment records, then starting states
+    float* as;  // [5][B][P][C] local adjoint sums, then incoming sums
 };
 
 __device__ __forceinline__ int64_t seg_index(const BwdArgs& a, int64_t b, int64_t j, int64_t c) {
     return (b * a.P + j) * a.C + c;
 }
 
+__device__ __forceinline__ FwdState load_state(const BwdArgs& a, int64_t si) {
+    const int64_t SP = a.B * a.P * a.C;
+    return FwdState{a.fs[si], a.fs[SP + si], a.fs[2 * SP + si], a.fs[3 * SP + si]};
+}
+
+// Runs the forward over positions [t0, t1) of one channel (element offset `base` + t C),
+// loads issued kBlk steps at a time; `visit(i, out, g)` sees each output (i = t - t0) with its
+// gy when WITH_G.
+template <bool OUT, bool WITH_G, class Visit>
+__device__ __forceinline__ void forward_span(const BwdArgs& a, int64_t base, int64_t t0, int64_t t1, FwdState& s,
+                                             float u2, float w2, Visit&& visit) {
+    FwdOut o{0.f, 0.f, 0.f};
+    int64_t t = t0;
+    for (; t + kBlk <= t1; t += kBlk) {
+        float kb[kBlk], vb[kBlk], gb[kBlk];
+#pragma unroll
+        for (int i = 0; i < kBlk; ++i) {
+            kb[i] = ld_in(a.k + base + (t + i) * a.C);
+            vb[i] = ld_in(a.v + base + (t + i) * a.C);
+            if (WITH_G) gb[i] = ld_in(a.gy + base + (t + i) * a.C);
+        }
+#pragma unroll
+        for (int i = 0; i < kBlk; ++i) {
+            hold(kb[i]);
+            hold(vb[i]);
+            if (WITH_G) hold(gb[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < kBlk; ++i) {
+            fwd_step<OUT>(s, kb[i] * kLog2e, vb[i], u2, w2, o);
+            if (OUT) visit((int)(t - t0) + i, o, WITH_G ? gb[i] : 0.f);
+        }
+    }
+    for (; t < t1; ++t) {
+        const int64_t at = base + t * a.C;
+        fwd_step<OUT>(s, a.k[at] * kLog2e, a.v[at], u2, w2, o);
+        if (OUT) visit((int)(t - t0), o, WITH_G ? a.gy[at] : 0.f);
+    }
+}
+
 // A: each segment's forward from the empty state -> its record
-__global__ void __launch_bounds__(128) bwd_seg_forward(BwdArgs a) {
-    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+__global__ void __launch_bounds__(kThreads) bwd_seg_forward(BwdArgs a) {
+    const int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     const int64_t j = blockIdx.y, b = blockIdx.z;
     if (c >= a.C) return;
     const float w2 = a.w[c] * kLog2e, u2 = a.u[c] * kLog2e;
     const int64_t t0 = j * kSeg, t1 = min64(a.T, t0 + kSeg);
-    const int64_t base = b * a.T * a.C + c;
     FwdState s{0.f, 0.f, kPEmpty, 0.f};
-    int64_t t = t0;
-    for (; t + kBlk <= t1; t += kBlk) {
-        float kb[kBlk], vb[kBlk];
-#pragma unroll
-        for (int i = 0; i < kBlk; ++i) {
-            kb[i] = a.k[base + (t + i) * a.C];
-            vb[i] = a.v[base + (t + i) * a.C];
-        }
-#pragma unroll
-        for (int i = 0; i < kBlk; ++i) fwd_step(s, kb[i] * kLog2e, vb[i], u2, w2, nullptr, nullptr, nullptr);
-    }
-    for (; t < t1; ++t) fwd_step(s, a.k[base + t * a.C] * kLog2e, a.v[base + t * a.C], u2, w2, nullptr, nullptr, nullptr);
+    forward_span<false, false>(a, b * a.T * a.C + c, t0, t1, s, u2, w2, [](int, const FwdOut&, float) {});
     const int64_t si = seg_index(a, b, j, c), SP = a.B * a.P * a.C;
     a.fs[si] = s.a;
     a.fs[SP + si] = s.bb;
@@ -145,136 +212,155 @@ __global__ void __launch_bounds__(128) bwd_seg_forward(BwdArgs a) {
     a.fs[3 * SP + si] = s.n;
 }
 
-// B: per channel, segment records combined left to right -> each segment's starting state
-__global__ void __launch_bounds__(128) bwd_seg_carry(BwdArgs a) {
-    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+// B: per channel, segment records combined left to right -> each segment's starting state.
+// The records of kScanBlk segments are loaded before any is overwritten, so the serial chain
+// waits on memory once per kScanBlk segments.
+__global__ void __launch_bounds__(kThreads) bwd_seg_carry(BwdArgs a) {
+    const int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     const int64_t b = blockIdx.y;
     if (c >= a.C) return;
+    if (b == 0) {  // E accumulates into these
+        a.gw[c] = 0.f;
+        a.gu[c] = 0.f;
+    }
     const float w2 = a.w[c] * kLog2e;
     const int64_t SP = a.B * a.P * a.C;
     Rec run = rec_identity();
-    for (int64_t j = 0; j < a.P; ++j) {
-        const int64_t si = seg_index(a, b, j, c);
-        const Rec seg{a.fs[si], a.fs[SP + si], a.fs[2 * SP + si], a.fs[3 * SP + si]};
-        a.fs[si] = run.a;
-        a.fs[SP + si] = run.b;
-        a.fs[2 * SP + si] = run.anc;
-        a.fs[3 * SP + si] = run.n;
-        const float len = (float)(min64(a.T, (j + 1) * kSeg) - j * kSeg);
-        run = rec_combine(run, seg, len, w2);
+    for (int64_t j0 = 0; j0 < a.P; j0 += kScanBlk) {
+        const int nb = (int)min64(kScanBlk, a.P - j0);
+        Rec seg[kScanBlk];
+#pragma unroll
+        for (int i = 0; i < kScanBlk; ++i) {
+            if (i < nb) {
+                const int64_t si = seg_index(a, b, j0 + i, c);
+                seg[i] = Rec{a.fs[si], a.fs[SP + si], a.fs[2 * SP + si], a.fs[3 * SP + si]};
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kScanBlk; ++i) {
+            if (i < nb) {
+                const int64_t j = j0 + i, si = seg_index(a, b, j, c);
+                a.fs[si] = run.a;
+                a.fs[SP + si] = run.b;
+                a.fs[2 * SP + si] = run.anc;
+                a.fs[3 * SP + si] = run.n;
+                const float len = (float)(min64(a.T, (j + 1) * kSeg) - j * kSeg);
+                run = rec_combine(run, seg[i], len, w2);
+            }
+        }
     }
 }
 
-// C: each segment's forward from its starting state (per-position values kept), then its
-// adjoint recurrence from zero -> the segment's local sums
-__global__ void __launch_bounds__(128) bwd_seg_values(BwdArgs a) {
-    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+// C: each segment's forward from its starting state -> its local adjoint sums
+__global__ void __launch_bounds__(kThreads) bwd_seg_local(BwdArgs a) {
+    const int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     const int64_t j = blockIdx.y, b = blockIdx.z;
     if (c >= a.C) return;
     const float w2 = a.w[c] * kLog2e, u2 = a.u[c] * kLog2e;
     const int64_t t0 = j * kSeg, t1 = min64(a.T, t0 + kSeg);
     const int64_t base = b * a.T * a.C + c;
     const int64_t si = seg_index(a, b, j, c), SP = a.B * a.P * a.C;
-    FwdState s{a.fs[si], a.fs[SP + si], a.fs[2 * SP + si], a.fs[3 * SP + si]};
-    int64_t t = t0;
-    for (; t + kBlk <= t1; t += kBlk) {
-        float kb[kBlk], vb[kBlk];
-#pragma unroll
-        for (int i = 0; i < kBlk; ++i) {
-            kb[i] = a.k[base + (t + i) * a.C];
-            vb[i] = a.v[base + (t + i) * a.C];
-        }
-#pragma unroll
-        for (int i = 0; i < kBlk; ++i) {
-            const int64_t at = base + (t + i) * a.C;
-            fwd_step(s, kb[i] * kLog2e, vb[i], u2, w2, a.q + at, a.dn + at, a.y + at);
-        }
-    }
-    for (; t < t1; ++t) {
-        const int64_t at = base + t * a.C;
-        fwd_step(s, a.k[at] * kLog2e, a.v[at], u2, w2, a.q + at, a.dn + at, a.y + at);
-    }
-    Adj r = adj_empty();
-    float dummy_w = 0.f, dummy_u = 0.f;
-    for (t = t1; t > t0; --t) {
-        const int64_t at = base + (t - 1) * a.C;
-        adj_step<false>(r, 0.f, 0.f, a.gy[at], a.q[at], a.dn[at], a.y[at], u2, w2, nullptr, nullptr, dummy_w,
-                        dummy_u);
-    }
-    a.as[si] = r.x;
-    a.as[SP + si] = r.y;
-    a.as[2 * SP + si] = r.xp;
-    a.as[3 * SP + si] = r.yp;
-    a.as[4 * SP + si] = r.r;
+    FwdState s = load_state(a, si);
+    LocalSums ls{0.f, 0.f, 0.f, 0.f, kRNone, 0.f};
+    forward_span<true, true>(a, base, t0, t1, s, u2, w2,
+                             [&](int i, const FwdOut& o, float g) { ls.add((float)i, g, o, w2); });
+    a.as[si] = ls.x;
+    a.as[SP + si] = ls.y;
+    a.as[2 * SP + si] = ls.xp;
+    a.as[3 * SP + si] = ls.yp;
+    a.as[4 * SP + si] = fmaf(ls.Rj, w2, ls.Rq);
 }
 
 // D: per channel, local sums composed right to left -> each segment's incoming sums
-__global__ void __launch_bounds__(128) bwd_seg_adjoint_carry(BwdArgs a) {
-    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+__global__ void __launch_bounds__(kThreads) bwd_seg_adjoint_carry(BwdArgs a) {
+    const int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     const int64_t b = blockIdx.y;
     if (c >= a.C) return;
     const float w2 = a.w[c] * kLog2e;
     const int64_t SP = a.B * a.P * a.C;
     Adj in = adj_empty();  // entering the last segment from its right: nothing
-    for (int64_t j = a.P - 1; j >= 0; --j) {
-        const int64_t si = seg_index(a, b, j, c);
-        const Adj loc{a.as[si], a.as[SP + si], a.as[2 * SP + si], a.as[3 * SP + si], a.as[4 * SP + si]};
-        a.as[si] = in.x;
-        a.as[SP + si] = in.y;
-        a.as[2 * SP + si] = in.xp;
-        a.as[3 * SP + si] = in.yp;
-        a.as[4 * SP + si] = in.r;
-        // what leaves this segment to its left: the local sums plus the incoming ones carried
-        // across the segment's len steps
-        const float len = (float)(min64(a.T, (j + 1) * kSeg) - j * kSeg);
-        const float rin = in.r + len * w2;
-        const float rn = fminf(loc.r, rin);
-        const float fl = ex2(rn - loc.r), fi = ex2(rn - rin);
-        Adj out;
-        out.x = fmaf(in.x, fi, loc.x * fl);
-        out.y = fmaf(in.y, fi, loc.y * fl);
-        out.xp = fmaf(fmaf(len, in.x, in.xp), fi, loc.xp * fl);
-        out.yp = fmaf(fmaf(len, in.y, in.yp), fi, loc.yp * fl);
-        out.r = rn;
-        in = out;
+    for (int64_t j1 = a.P; j1 > 0; j1 -= kScanBlk) {
+        const int nb = (int)min64(kScanBlk, j1);
+        Adj loc[kScanBlk];
+#pragma unroll
+        for (int i = 0; i < kScanBlk; ++i) {
+            if (i < nb) {
+                const int64_t si = seg_index(a, b, j1 - 1 - i, c);
+                loc[i] = Adj{a.as[si], a.as[SP + si], a.as[2 * SP + si], a.as[3 * SP + si], a.as[4 * SP + si]};
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kScanBlk; ++i) {
+            if (i < nb) {
+                const int64_t j = j1 - 1 - i, si = seg_index(a, b, j, c);
+                a.as[si] = in.x;
+                a.as[SP + si] = in.y;
+                a.as[2 * SP + si] = in.xp;
+                a.as[3 * SP + si] = in.yp;
+                a.as[4 * SP + si] = in.r;
+                // what leaves this segment to its left: the local sums plus the incoming ones
+                // carried across the segment's len steps
+                const float len = (float)(min64(a.T, (j + 1) * kSeg) - j * kSeg);
+                const float rin = in.r + len * w2;
+                const float rn = fminf(loc[i].r, rin);
+                const float fl = ex2(rn - loc[i].r), fi = ex2(rn - rin);
+                Adj out;
+                out.x = fmaf(in.x, fi, loc[i].x * fl);
+                out.y = fmaf(in.y, fi, loc[i].y * fl);
+                out.xp = fmaf(fmaf(len, in.x, in.xp), fi, loc[i].xp * fl);
+                out.yp = fmaf(fmaf(len, in.y, in.yp), fi, loc[i].yp * fl);
+                out.r = rn;
+                in = out;
+            }
+        }
     }
 }
 
-// E: each segment's adjoint recurrence from its incoming sums -> gradients
-__global__ void __launch_bounds__(128) bwd_seg_grads(BwdArgs a) {
-    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+// E: each segment's forward again (per-position values into shared memory), then its adjoint
+// recurrence from its incoming sums -> gradients
+__global__ void __launch_bounds__(kThreads) bwd_seg_grads(BwdArgs a) {
+    extern __shared__ float sm[];  // [kSeg][3][kThreads]
+    const int tid = threadIdx.x;
+    const int64_t c = (int64_t)blockIdx.x * kThreads + tid;
     const int64_t j = blockIdx.y, b = blockIdx.z;
-    if (c >= a.C) return;
+    if (c >= a.C) return;  // no block-wide synchronisation below: each thread uses its own column
     const float w2 = a.w[c] * kLog2e, u2 = a.u[c] * kLog2e;
     const int64_t t0 = j * kSeg, t1 = min64(a.T, t0 + kSeg);
     const int64_t base = b * a.T * a.C + c;
     const int64_t si = seg_index(a, b, j, c), SP = a.B * a.P * a.C;
+    FwdState fsd = load_state(a, si);
+    forward_span<true, false>(a, base, t0, t1, fsd, u2, w2, [&](int i, const FwdOut& o, float) {
+        sm[(i * 3 + 0) * kThreads + tid] = o.q;
+        sm[(i * 3 + 1) * kThreads + tid] = o.rd;
+        sm[(i * 3 + 2) * kThreads + tid] = o.y;
+    });
     Adj s{a.as[si], a.as[SP + si], a.as[2 * SP + si], a.as[3 * SP + si], a.as[4 * SP + si]};
     float sgw = 0.f, sgu = 0.f;
+    auto step = [&](int64_t t, float kt, float vt, float g) {
+        const int i = (int)(t - t0);
+        const FwdOut o{sm[(i * 3 + 0) * kThreads + tid], sm[(i * 3 + 1) * kThreads + tid],
+                       sm[(i * 3 + 2) * kThreads + tid]};
+        float gk, gv;
+        adj_step(s, kt * kLog2e, vt, g, o, u2, w2, gk, gv, sgw, sgu);
+        a.gk[base + t * a.C] = gk;
+        a.gv[base + t * a.C] = gv;
+    };
     int64_t t = t1;
     for (; t - kBlk >= t0; t -= kBlk) {
-        float kb[kBlk], vb[kBlk], gb[kBlk], qb[kBlk], db[kBlk], yb[kBlk];
+        float kb[kBlk], vb[kBlk], gb[kBlk];
 #pragma unroll
         for (int i = 0; i < kBlk; ++i) {
             const int64_t at = base + (t - 1 - i) * a.C;
             kb[i] = a.k[at];
             vb[i] = a.v[at];
             gb[i] = a.gy[at];
-            qb[i] = a.q[at];
-            db[i] = a.dn[at];
-            yb[i] = a.y[at];
         }
 #pragma unroll
-        for (int i = 0; i < kBlk; ++i) {
-            const int64_t at = base + (t - 1 - i) * a.C;
-            adj_step<true>(s, kb[i] * kLog2e, vb[i], gb[i], qb[i], db[i], yb[i], u2, w2, a.gk + at, a.gv + at, sgw,
-                           sgu);
-        }
+        for (int i = 0; i < kBlk; ++i) step(t - 1 - i, kb[i], vb[i], gb[i]);
     }
     for (; t > t0; --t) {
         const int64_t at = base + (t - 1) * a.C;
-        adj_step<true>(s, a.k[at] * kLog2e, a.v[at], a.gy[at], a.q[at], a.dn[at], a.y[at], u2, w2, a.gk + at,
-                       a.gv + at, sgw, sgu);
+        step(t - 1, a.k[at], a.v[at], a.gy[at]);
     }
     atomicAdd(&a.gw[c], sgw);
     atomicAdd(&a.gu[c], sgu);
@@ -287,11 +373,11 @@ int64_t backward_segments(int64_t T) { return (T + kSeg - 1) / kSeg; }
 cudaError_t launch_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
                             const float* v, const float* gy, float* gk, float* gv, float* gw, float* gu, void* ws,
                             cudaStream_t s) {
-    cudaError_t e = cudaMemsetAsync(gw, 0, (size_t)C * sizeof(float), s);
-    if (e != cudaSuccess) return e;
-    e = cudaMemsetAsync(gu, 0, (size_t)C * sizeof(float), s);
-    if (e != cudaSuccess) return e;
-    if (B == 0 || T == 0) return cudaSuccess;
+    if (B == 0 || T == 0) {  // no position: the per-channel gradients are zero
+        cudaError_t e = cudaMemsetAsync(gw, 0, (size_t)C * sizeof(float), s);
+        if (e != cudaSuccess) return e;
+        return cudaMemsetAsync(gu, 0, (size_t)C * sizeof(float), s);
+    }
     BwdArgs a;
     a.B = B;
     a.T = T;
@@ -306,20 +392,16 @@ cudaError_t launch_backward(int64_t B, int64_t T, int64_t C, const float* w, con
     a.gv = gv;
     a.gw = gw;
     a.gu = gu;
-    float* f = static_cast<float*>(ws);
-    const int64_t n = B * T * C, SP = B * a.P * C;
-    a.q = f;
-    a.dn = f + n;
-    a.y = f + 2 * n;
-    a.fs = f + 3 * n;
+    const int64_t SP = B * a.P * C;
+    a.fs = static_cast<float*>(ws);
     a.as = a.fs + 4 * SP;
-    const unsigned cx = (unsigned)((C + 127) / 128);
+    const unsigned cx = (unsigned)((C + kThreads - 1) / kThreads);
     const dim3 seg_grid(cx, (unsigned)a.P, (unsigned)B), chan_grid(cx, (unsigned)B);
-    bwd_seg_forward<<<seg_grid, 128, 0, s>>>(a);
-    bwd_seg_carry<<<chan_grid, 128, 0, s>>>(a);
-    bwd_seg_values<<<seg_grid, 128, 0, s>>>(a);
-    bwd_seg_adjoint_carry<<<chan_grid, 128, 0, s>>>(a);
-    bwd_seg_grads<<<seg_grid, 128, 0, s>>>(a);
+    bwd_seg_forward<<<seg_grid, kThreads, 0, s>>>(a);
+    bwd_seg_carry<<<chan_grid, kThreads, 0, s>>>(a);
+    bwd_seg_local<<<seg_grid, kThreads, 0, s>>>(a);
+    bwd_seg_adjoint_carry<<<chan_grid, kThreads, 0, s>>>(a);
+    bwd_seg_grads<<<seg_grid, kThreads, kGradSmem, s>>>(a);
     return cudaGetLastError();
 }
 

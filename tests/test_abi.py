@@ -108,9 +108,11 @@ def test_backward_validation_without_launch():
     assert bwd(1, 4, 4, gk=FAKE + 4) == 2        # misaligned output
     assert bwd(1, 4, 4, nbytes=16) == 1          # workspace too small
     assert bwd(70000, 1, 4) == 3                 # batch above the grid's z limit
-    # 12 B per element plus 36 B per (b, 64-step segment, c)
-    assert L.wkv_backward_workspace_size(2, 3, 5) == 2 * 3 * 5 * 12 + 2 * 1 * 5 * 36
-    assert L.wkv_backward_workspace_size(1, 130, 2) == 130 * 2 * 12 + 3 * 2 * 36
+    assert bwd(1, 32 * 65535 + 1, 4) == 3        # more 32-step segments than the grid's y limit
+    # 36 B per (b, 32-step segment, c)
+    assert L.wkv_backward_workspace_size(2, 3, 5) == 2 * 1 * 5 * 36
+    assert L.wkv_backward_workspace_size(1, 130, 2) == 1 * 5 * 2 * 36
+    assert L.wkv_backward_workspace_size(1, 128, 2) == 1 * 4 * 2 * 36
 
 
 def test_gated_and_shift3_validation_without_launch():
