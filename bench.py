@@ -57,6 +57,9 @@ def parse():
     ap.add_argument("--profile-forward", metavar="WORKLOAD", default=None,
                     help="only run 2 + 3 eager forward launches of a forward workload (e.g. fwd_1x16384x4096) "
                          "and exit: a short, self-contained command to capture under a profiler")
+    ap.add_argument("--profile-backward", metavar="WORKLOAD", default=None,
+                    help="only run 2 + 3 eager backward calls (five launches each) on a forward workload's shape "
+                         "(fp32) and exit, for a profiler")
     return ap.parse_args()
 
 
@@ -623,10 +626,32 @@ def profile_forward(name):
                       "io": spec.dtype}))
 
 
+def profile_backward(name):
+    """Two warm-up and three profiled eager backward calls on one forward workload's shape, in
+    fp32 (the backward's only I/O type)."""
+    import torch
+    import linear_attention_rnn_wkv_b200 as wkv
+    import synth
+    spec = synth.FORWARD[name]
+    dev = torch.device("cuda", 0)
+    w, u, k, v = synth.forward_inputs(spec)
+    gy = synth.grad_output(spec)
+    t = [torch.from_numpy(a.astype("float32")).to(dev) for a in (w, u, k, v, gy)]
+    ws = torch.empty(int(wkv.lib().wkv_backward_workspace_size(spec.B, spec.T, spec.C)), dtype=torch.uint8,
+                     device=dev)
+    for _ in range(5):
+        wkv.wkv_backward(*t, workspace=ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_backward": name, "calls": 5, "B": spec.B, "T": spec.T, "C": spec.C}))
+
+
 def main():
     args = parse()
     if args.profile_forward:
         profile_forward(args.profile_forward)
+        return
+    if args.profile_backward:
+        profile_backward(args.profile_backward)
         return
     if args.impl == "reference":
         run_reference(args)
