@@ -26,6 +26,11 @@ Functions (all inputs are converted to contiguous float64):
   and |v| + |y| in place of v - y).
 * ``token_shift3(mu_r, mu_k, mu_v, x, x_last=None)`` -- the lerp with the three
   projections' separate mu (three calls of ``token_shift``).
+* ``eagle_recurrent(w, r, k, v, N=64, state_in=None)`` -- the Eagle (RWKV-5)
+  matrix-state recurrence ``S_t = diag(e^{-w}) S_{t-1} + k_t v_t^T``, ``y_t = r_t^T S_t``
+  per head of N channels.  Returns ``(y, s, state_out)`` (state ``[B, H, N, N]``).
+* ``eagle_direct(w, r, k, v, N=64, state_in=None)`` -- the same outputs summed
+  directly over the past (O(T^2 N^2) per head).
 
 ``s`` is the same weighted average with ``|v|`` in place of ``v`` (the error
 scale the parity tests divide by); ``sacc`` is its accumulator in the state.
@@ -69,8 +74,10 @@ def load(path: str):
     L.oracle_token_shift.argtypes = [i64, i64, i64, vp, vp, vp, vp]
     L.oracle_gate.argtypes = [i64, vp, vp, vp]
     L.oracle_wkv_backward_direct.argtypes = [i64, i64, i64] + [vp] * 13
+    L.oracle_eagle_recurrent.argtypes = [i64, i64, i64, i64] + [vp] * 8
+    L.oracle_eagle_direct.argtypes = [i64, i64, i64, i64] + [vp] * 6
     for f in (L.oracle_wkv_direct, L.oracle_wkv_recurrent, L.oracle_wkv_naive, L.oracle_token_shift, L.oracle_gate,
-              L.oracle_wkv_backward_direct):
+              L.oracle_wkv_backward_direct, L.oracle_eagle_recurrent, L.oracle_eagle_direct):
         f.restype = None
     L.oracle_num_threads.restype = ctypes.c_int
     return L
@@ -193,3 +200,31 @@ def decode_token_shift(mu, x_t, x_prev, L=None):
     LC = x_t[0].size
     xb = token_shift(_f64(mu).reshape(LC), x_t.reshape(N, 1, LC), _f64(x_prev).reshape(N, LC), L=L)
     return xb.reshape(x_t.shape)
+
+
+def _eagle_shapes(k, N, state_in):
+    B, T, C = _btc(k)
+    if C % N:
+        raise ValueError(f"C = {C} is not a multiple of the head size {N}")
+    H = C // N
+    state_in = None if state_in is None else _f64(state_in).reshape(B, H, N, N)
+    return B, T, C, H, state_in
+
+
+def eagle_recurrent(w, r, k, v, N=64, state_in=None, L=None):
+    w, r, k, v = _f64(w), _f64(r), _f64(k), _f64(v)
+    B, T, C, H, state_in = _eagle_shapes(k, N, state_in)
+    y = np.empty(k.shape, np.float64)
+    s = np.empty(k.shape, np.float64)
+    st = np.empty((B, H, N, N), np.float64)
+    (L or lib()).oracle_eagle_recurrent(B, T, H, N, _p(w), _p(r), _p(k), _p(v), _p(state_in), _p(y), _p(s),
+                                        _p(st))
+    return y, s, st
+
+
+def eagle_direct(w, r, k, v, N=64, state_in=None, L=None):
+    w, r, k, v = _f64(w), _f64(r), _f64(k), _f64(v)
+    B, T, C, H, state_in = _eagle_shapes(k, N, state_in)
+    y = np.empty(k.shape, np.float64)
+    (L or lib()).oracle_eagle_direct(B, T, H, N, _p(w), _p(r), _p(k), _p(v), _p(state_in), _p(y))
+    return y

@@ -22,6 +22,12 @@
  *           Also section "Receptance: the gate on the way out" (the output is
  *           sigma(r) times wkv, channel by channel) and, in section "Token shift",
  *           the separate mu_r, mu_k, mu_v of the three projections.
+ *   [VANOS] "RWKV (Attention-RNN Hybrid)" (vanos001.github.io): section
+ *           "Versions: RWKV-4 -> Eagle -> Finch" (the Eagle matrix-state
+ *           recurrence S_t = diag(d) S_{t-1} + k_t v_t^T read out as
+ *           y_t = r_t^T S_t, one 64 x 64 state per head) and section
+ *           "O(N) Inference Characteristics" (decode is one matrix-vector
+ *           product against the state).
  *   [MULTI] "RWKV and Recurrent Models With Transformer Quality"
  *           (multigrid.ai): section "Prefill, decode, and where each form is
  *           used" (prefill yields the state after the last prompt token;
@@ -41,6 +47,7 @@
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <stdlib.h>
 #ifdef _OPENMP
 #include <omp.h>
 #endif
@@ -293,4 +300,97 @@ void oracle_wkv_backward_direct(int64_t B, int64_t T, int64_t C, const double* w
         if (sw) sw[c] = swc;
         if (su) su[c] = suc;
     }
+}
+
+/*
+ * Eagle (RWKV-5) matrix-state WKV ([VANOS] "Versions: RWKV-4 -> Eagle -> Finch"),
+ * per sequence b and head h of N channels, token after token:
+ *   S_t = diag(d) S_{t-1} + k_t v_t^T     S is N x N: row m a key channel, column j a value channel
+ *   y_t = r_t^T S_t                       y_t[j] = sum_m r_t[m] S_t[m][j]
+ * with d[m] = exp(-w[h N + m]) (w > 0: the per-channel decay rate, as in RWKV-4)
+ * and S_{-1} = state_in (zero when NULL).
+ *
+ * r, k, v, y, s: [B][T][C] with C = H N, head h owning channels h N .. h N + N - 1.
+ * w: [C].  state_in, state_out: [B][H][N][N] (m, j), either may be NULL.
+ * s (may be NULL): the same read-out with |r|, |k|, |v| and |state_in|, the
+ * magnitude scale that errors are measured against.
+ * With T = 1 this is one decode step from the given state ([VANOS] "O(N) Inference
+ * Characteristics").
+ */
+void oracle_eagle_recurrent(int64_t B, int64_t T, int64_t H, int64_t N, const double* w,
+                            const double* r, const double* k, const double* v,
+                            const double* state_in, double* y, double* s, double* state_out)
+{
+    const int64_t C = H * N;
+    const size_t NN = (size_t)N * (size_t)N;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t h = 0; h < H; ++h) {
+            const size_t sb = ((size_t)b * (size_t)H + (size_t)h) * NN;
+            double* S = (double*)malloc(NN * sizeof(double));
+            double* Sa = (double*)malloc(NN * sizeof(double));
+            for (size_t e = 0; e < NN; ++e) {
+                S[e] = state_in ? state_in[sb + e] : 0.0;
+                Sa[e] = fabs(S[e]);
+            }
+            for (int64_t t = 0; t < T; ++t) {
+                /* update: S <- diag(d) S + k_t v_t^T */
+                for (int64_t m = 0; m < N; ++m) {
+                    const double d = exp(-w[h * N + m]);
+                    const double km = k[at3(b, t, h * N + m, T, C)];
+                    for (int64_t j = 0; j < N; ++j) {
+                        const double vj = v[at3(b, t, h * N + j, T, C)];
+                        S[m * N + j] = d * S[m * N + j] + km * vj;
+                        Sa[m * N + j] = d * Sa[m * N + j] + fabs(km) * fabs(vj);
+                    }
+                }
+                /* read-out: y_t = r_t^T S_t */
+                for (int64_t j = 0; j < N; ++j) {
+                    double acc = 0.0, acc_s = 0.0;
+                    for (int64_t m = 0; m < N; ++m) {
+                        const double rm = r[at3(b, t, h * N + m, T, C)];
+                        acc += rm * S[m * N + j];
+                        acc_s += fabs(rm) * Sa[m * N + j];
+                    }
+                    y[at3(b, t, h * N + j, T, C)] = acc;
+                    if (s) s[at3(b, t, h * N + j, T, C)] = acc_s;
+                }
+            }
+            if (state_out)
+                for (size_t e = 0; e < NN; ++e) state_out[sb + e] = S[e];
+            free(S);
+            free(Sa);
+        }
+}
+
+/*
+ * The same outputs summed directly instead of carried: unrolling the recurrence gives
+ * S_t = sum_{i<=t} diag(d)^{t-i} k_i v_i^T + diag(d)^{t+1} S_{-1}, so
+ *   y_t[j] = sum_{i<=t} sum_m r_t[m] exp(-(t-i) w[m]) k_i[m] v_i[j]
+ *          + sum_m r_t[m] exp(-(t+1) w[m]) state_in[m][j].
+ * O(T^2 N^2) per head: for small cases only.
+ */
+void oracle_eagle_direct(int64_t B, int64_t T, int64_t H, int64_t N, const double* w,
+                         const double* r, const double* k, const double* v,
+                         const double* state_in, double* y)
+{
+    const int64_t C = H * N;
+    const size_t NN = (size_t)N * (size_t)N;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t h = 0; h < H; ++h) {
+            const size_t sb = ((size_t)b * (size_t)H + (size_t)h) * NN;
+            for (int64_t t = 0; t < T; ++t)
+                for (int64_t j = 0; j < N; ++j) {
+                    double acc = 0.0;
+                    for (int64_t m = 0; m < N; ++m) {
+                        const double rm = r[at3(b, t, h * N + m, T, C)];
+                        for (int64_t i = 0; i <= t; ++i)
+                            acc += rm * exp(-(double)(t - i) * w[h * N + m]) * k[at3(b, i, h * N + m, T, C)] *
+                                   v[at3(b, i, h * N + j, T, C)];
+                        if (state_in) acc += rm * exp(-(double)(t + 1) * w[h * N + m]) * state_in[sb + m * N + j];
+                    }
+                    y[at3(b, t, h * N + j, T, C)] = acc;
+                }
+        }
 }

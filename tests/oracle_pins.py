@@ -441,6 +441,121 @@ def pin_backward_closed_forms(L):
     assert np.allclose(gv.sum(axis=1), gy.sum(axis=1), rtol=1e-12, atol=1e-12)
 
 
+# ----------------------------------------------------------------------------
+# Eagle (RWKV-5) matrix-state WKV ("RWKV (Attention-RNN Hybrid)", section
+# "Versions: RWKV-4 -> Eagle -> Finch"): S_t = diag(d) S_{t-1} + k_t v_t^T,
+# y_t = r_t^T S_t per head, d = exp(-w) on the key index
+# ----------------------------------------------------------------------------
+
+EAGLE_GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "eagle_hand_example.txt")
+
+
+def _eagle_case(seed, B=2, T=9, H=2, N=4, w_lo=-3.0, w_hi=1.0):
+    g = _rng(seed)
+    C = H * N
+    w = np.exp(g.uniform(w_lo, w_hi, C))
+    r, k, v = (g.normal(0.0, 1.0, (B, T, C)) for _ in range(3))
+    return w, r, k, v
+
+
+def pin_eagle_hand_example(L):
+    """One head of two channels over three tokens, worked by hand (exact in binary)."""
+    g = read_golden(EAGLE_GOLDEN)
+    w = -np.log(np.array(g["d"]))
+    r, k, v = (np.array(g[x]).reshape(1, 3, 2) for x in "rkv")
+    y, s, st = oracle.eagle_recurrent(w, r, k, v, N=2, L=L)
+    assert np.allclose(y.ravel(), g["y"], rtol=0, atol=1e-14)
+    assert np.allclose(st.ravel(), g["S"], rtol=0, atol=1e-14)
+    assert np.allclose(oracle.eagle_direct(w, r, k, v, N=2, L=L).ravel(), g["y"], rtol=0, atol=1e-14)
+
+
+def pin_eagle_linear_attention(L):
+    """No decay (w = 0, d = 1): the state is the running sum of k_i v_i^T, so each head's
+    output is causal linear attention, tril(R K^T) V, here by matrix products."""
+    B, T, H, N = 2, 11, 3, 4
+    w, r, k, v = _eagle_case(50, B, T, H, N)
+    w = np.zeros_like(w)
+    y, s, _ = oracle.eagle_recurrent(w, r, k, v, N=N, L=L)
+    yd = oracle.eagle_direct(w, r, k, v, N=N, L=L)
+    mask = np.tril(np.ones((T, T)))
+    for b in range(B):
+        for h in range(H):
+            sl = slice(h * N, (h + 1) * N)
+            ref = ((r[b, :, sl] @ k[b, :, sl].T) * mask) @ v[b, :, sl]
+            assert np.allclose(y[b, :, sl], ref, rtol=1e-12, atol=1e-12)
+            assert np.allclose(yd[b, :, sl], ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_eagle_no_memory(L):
+    """Total decay (w = 1e4: exp(-1e4) is exactly 0): only the current token survives, so
+    y_t = (r_t . k_t) v_t per head, and the state is k_{T-1} v_{T-1}^T."""
+    B, T, H, N = 2, 5, 2, 3
+    w, r, k, v = _eagle_case(51, B, T, H, N)
+    w = np.full_like(w, 1e4)
+    y, _, st = oracle.eagle_recurrent(w, r, k, v, N=N, L=L)
+    for h in range(H):
+        sl = slice(h * N, (h + 1) * N)
+        dot = (r[:, :, sl] * k[:, :, sl]).sum(-1, keepdims=True)
+        assert np.allclose(y[:, :, sl], dot * v[:, :, sl], rtol=1e-13, atol=1e-13)
+        assert np.allclose(st[:, h], k[:, -1, sl][:, :, None] * v[:, -1, sl][:, None, :], rtol=0, atol=0)
+
+
+def pin_eagle_one_token_from_state(L):
+    """One token from a given state S: y = r^T (diag(d) S + k v^T) written out per element, and
+    the state that comes back is that matrix."""
+    B, H, N = 2, 2, 3
+    w, r, k, v = _eagle_case(52, B, 1, H, N)
+    S0 = _rng(152).normal(0, 1, (B, H, N, N))
+    y, _, st = oracle.eagle_recurrent(w, r, k, v, N=N, state_in=S0, L=L)
+    for b in range(B):
+        for h in range(H):
+            sl = slice(h * N, (h + 1) * N)
+            d = np.exp(-w[sl])
+            S1 = np.array([[d[m] * S0[b, h, m, j] + k[b, 0, sl][m] * v[b, 0, sl][j] for j in range(N)]
+                           for m in range(N)])
+            assert np.allclose(st[b, h], S1, rtol=1e-14, atol=1e-14)
+            yj = [sum(r[b, 0, sl][m] * S1[m, j] for m in range(N)) for j in range(N)]
+            assert np.allclose(y[b, 0, sl], yj, rtol=1e-13, atol=1e-13)
+
+
+def pin_eagle_routes_and_split(L):
+    """The recurrence and the direct sum agree (the same arithmetic regrouped), also from a
+    given state; running T1 tokens, then the rest from the returned state, gives the whole."""
+    B, T, H, N = 2, 13, 2, 4
+    w, r, k, v = _eagle_case(53, B, T, H, N)
+    S0 = _rng(153).normal(0, 1, (B, H, N, N))
+    for st_in in (None, S0):
+        y, s, st = oracle.eagle_recurrent(w, r, k, v, N=N, state_in=st_in, L=L)
+        yd = oracle.eagle_direct(w, r, k, v, N=N, state_in=st_in, L=L)
+        assert np.all(np.abs(y - yd) <= 1e-12 * s)
+        assert np.all(s >= np.abs(y) * (1 - 1e-12))
+    y, s, st = oracle.eagle_recurrent(w, r, k, v, N=N, L=L)
+    cut = 6
+    y1, _, st1 = oracle.eagle_recurrent(w, r[:, :cut], k[:, :cut], v[:, :cut], N=N, L=L)
+    y2, _, st2 = oracle.eagle_recurrent(w, r[:, cut:], k[:, cut:], v[:, cut:], N=N, state_in=st1, L=L)
+    assert np.all(np.abs(np.concatenate([y1, y2], axis=1) - y) <= 1e-13 * s)
+    assert np.allclose(st2, st, rtol=1e-13, atol=1e-13)
+
+
+def pin_eagle_bilinear_and_heads(L):
+    """y is linear in v and in r (each alone), and a head's output depends on its own
+    channels only: changing one head's inputs leaves every other head's outputs as they were."""
+    B, T, H, N = 1, 7, 3, 4
+    w, r, k, v = _eagle_case(54, B, T, H, N)
+    _, _, v2 = (x for x in _eagle_case(55, B, T, H, N)[1:])
+    y1 = oracle.eagle_recurrent(w, r, k, v, N=N, L=L)[0]
+    y2, s2, _ = oracle.eagle_recurrent(w, r, k, v2, N=N, L=L)
+    y12, s12, _ = oracle.eagle_recurrent(w, r, k, 2 * v - 3 * v2, N=N, L=L)
+    assert np.all(np.abs(y12 - (2 * y1 - 3 * y2)) <= 1e-12 * (s12 + s2))
+    yr = oracle.eagle_recurrent(w, -0.5 * r, k, v, N=N, L=L)[0]
+    assert np.allclose(yr, -0.5 * y1, rtol=1e-14, atol=0)
+    k3 = k.copy()
+    k3[:, :, N:2 * N] += 1.0  # head 1's keys only
+    y3 = oracle.eagle_recurrent(w, r, k3, v, N=N, L=L)[0]
+    assert np.array_equal(y3[:, :, :N], y1[:, :, :N]) and np.array_equal(y3[:, :, 2 * N:], y1[:, :, 2 * N:])
+    assert not np.allclose(y3[:, :, N:2 * N], y1[:, :, N:2 * N])
+
+
 ALL_PINS = [
     pin_worked_example,
     pin_routes_agree,
@@ -462,4 +577,10 @@ ALL_PINS = [
     pin_token_shift3,
     pin_backward_finite_differences,
     pin_backward_closed_forms,
+    pin_eagle_hand_example,
+    pin_eagle_linear_attention,
+    pin_eagle_no_memory,
+    pin_eagle_one_token_from_state,
+    pin_eagle_routes_and_split,
+    pin_eagle_bilinear_and_heads,
 ]

@@ -44,6 +44,20 @@ MUTANTS = {
     "backward_decay_count_off_by_one": ("gwc += -g * (double)(t - 1 - i) * beta * (vi - yt);",
                                         "gwc += -g * (double)(t - i) * beta * (vi - yt);"),
     "backward_bonus_sign": ("guc += g * alpha * (vt - yt);", "guc += g * alpha * (yt - vt);"),
+    "eagle_decay_on_value_index": ("const double d = exp(-w[h * N + m]);\n                    const double km",
+                                   "const double d = exp(-w[h * N]);\n                    const double km"),
+    "eagle_outer_product_transposed": ("S[m * N + j] = d * S[m * N + j] + km * vj;",
+                                       "S[j * N + m] = d * S[j * N + m] + km * vj;"),
+    "eagle_drops_current_token": ("S[m * N + j] = d * S[m * N + j] + km * vj;", "S[m * N + j] = d * S[m * N + j];"),
+    "eagle_readout_transposed": ("acc += rm * S[m * N + j];", "acc += rm * S[j * N + m];"),
+    "eagle_decay_sign": ("const double d = exp(-w[h * N + m]);", "const double d = exp(w[h * N + m]);"),
+    "eagle_head_offset": ("const double rm = r[at3(b, t, h * N + m, T, C)];\n                        acc += rm * S",
+                          "const double rm = r[at3(b, t, m, T, C)];\n                        acc += rm * S"),
+    "eagle_state_in_transposed": ("S[e] = state_in ? state_in[sb + e] : 0.0;",
+                                  "S[e] = state_in ? state_in[sb + (e % N) * N + e / N] : 0.0;"),
+    "eagle_direct_decay_off_by_one": ("exp(-(double)(t - i) * w[h * N + m])", "exp(-(double)(t - 1 - i) * w[h * N + m])"),
+    "eagle_direct_state_in_undecayed": ("exp(-(double)(t + 1) * w[h * N + m]) * state_in",
+                                        "exp(-(double)t * w[h * N + m]) * state_in"),
 }
 
 
