@@ -373,6 +373,59 @@ def next_rows_bench(torch, wkv, sets, ws, spec, peak):
     }
 
 
+def eagle_bench(torch, wkv, dev, peak, decode=True):
+    """Eagle (RWKV-5) matrix-state WKV: the prefill on eagle_8x1024x768 (r, k, v read and y
+    written once: 16 B/element, plus the final state, 16 KiB per sequence-head) over three
+    rotating input sets (> 2x L2), and the decode step for 256 sessions x 32 layers x 4096
+    channels (each 64 x 64 state read and written once, r, k, v read and y written)."""
+    import synth
+    spec = synth.EAGLE["eagle_8x1024x768"]
+    B, T, C = spec.B, spec.T, spec.C
+    H = C // 64
+    g = torch.Generator(device=dev)
+    g.manual_seed(spec.seed)
+    w = torch.exp(torch.rand(C, generator=g, device=dev) * (spec.w_hi - spec.w_lo) + spec.w_lo)
+    sets = [[torch.randn((B, T, C), generator=g, device=dev) for _ in range(3)] for _ in range(3)]
+    y = torch.empty((B, T, C), device=dev)
+    st = torch.empty((B, H, 64, 64), device=dev)
+    ws = torch.empty(int(wkv.lib().eagle_forward_workspace_size(B, T, C)), dtype=torch.uint8, device=dev)
+
+    def fwd(i):
+        r, k, v = sets[i % 3]
+        wkv.eagle_forward(w, r, k, v, y=y, state_out=st, workspace=ws)
+
+    n = B * T * C
+    alg = 16 * n + B * H * 64 * 64 * 4
+    f_ms = graph_ms(torch, fwd, 12)
+    out = {"eagle_forward": {"workload": spec.name, "launch_ms": f_ms, "alg_bytes_per_launch": alg,
+                             "achieved_gbs": alg / (f_ms * 1e-3) / 1e9, "frac": alg / (f_ms * 1e-3) / 1e9 / peak,
+                             "elements_per_s": n / (f_ms * 1e-3),
+                             "note": "three launches (chunk sums, scan over chunks, chunk outputs), fp32 on "
+                                     "CUDA cores"}}
+    del sets, ws
+    if decode:
+        N, L, Cd = 256, 32, 4096
+        Hd = Cd // 64
+        wd = torch.exp(torch.rand((L, Cd), generator=g, device=dev) * 6 - 5)
+        S = torch.randn((N, L, Hd, 64, 64), generator=g, device=dev)
+        dsets = [[torch.randn((N, L, Cd), generator=g, device=dev) for _ in range(3)] for _ in range(2)]
+        yd = torch.empty((N, L, Cd), device=dev)
+
+        def dec(i):
+            r, k, v = dsets[i % 2]
+            wkv.eagle_decode_step(wd, r, k, v, S, y=yd)
+
+        d_ms = graph_ms(torch, dec, 4)
+        d_alg = 2 * S.numel() * 4 + 4 * N * L * Cd * 4
+        out["eagle_decode"] = {"workload": "eagle_decode_256x32x4096", "ms_per_step": d_ms,
+                               "tokens_per_s": N / (d_ms * 1e-3), "alg_bytes_per_step": d_alg,
+                               "achieved_gbs": d_alg / (d_ms * 1e-3) / 1e9,
+                               "frac": d_alg / (d_ms * 1e-3) / 1e9 / peak}
+        del S, dsets
+    torch.cuda.empty_cache()
+    return out
+
+
 def forward_only_ms(torch, wkv, sets, ws):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
@@ -561,6 +614,7 @@ def run_ours(args):
     del main_g, rem_g, warm_g
     dec = None if args.no_decode else decode_bench(torch, wkv, dev, 400)
     nxt = next_rows_bench(torch, wkv, sets, ws, spec, peaks["hbm_gbs"])
+    nxt.update(eagle_bench(torch, wkv, dev, peaks["hbm_gbs"], decode=not args.no_decode))
     e2e = None
     if not args.no_e2e:
         ms_e2e, h2d, d2h = e2e_bench(torch, wkv, sets, ws, min(K, 240), dev)

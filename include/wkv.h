@@ -1,5 +1,6 @@
 /*
- * wkv.h -- C ABI of the B200 (sm_100a) RWKV-4 WKV library (libwkv_b200.so).
+ * wkv.h -- C ABI of the B200 (sm_100a) RWKV-4 WKV library (libwkv_b200.so), with the
+ * Eagle (RWKV-5) matrix-state operator at the end.
  *
  * The operator ("RWKV" transformer-math page, aicassindra.com, section "The WKV
  * operator: attention with a fixed decay"; aiwiki "RWKV", eq. 1), per channel c,
@@ -245,6 +246,49 @@ wkv_status wkv_decode_step_fused(int64_t N, int64_t L, int64_t C, const float* m
 wkv_status wkv_forward_chunked_noalloc(int64_t B, int64_t T, int64_t C, wkv_dtype io, const float* w,
                                        const float* u, const void* k, const void* v, const float* state_in,
                                        void* y, float* state_out, cudaStream_t stream);
+
+/*
+ * Eagle (RWKV-5) matrix-state WKV ("RWKV (Attention-RNN Hybrid)", vanos001.github.io,
+ * section "Versions: RWKV-4 -> Eagle -> Finch"), per sequence b and head h of 64 channels
+ * (channels h*64 .. h*64+63), token after token:
+ *
+ *   S_t = diag(d) S_{t-1} + k_t v_t^T,     y_t = r_t^T S_t   (y_t[j] = sum_m r_t[m] S_t[m][j])
+ *
+ * S is 64 x 64 per head (row m a key channel, column j a value channel), d[m] = e^{-w[m]}
+ * with w >= 0 the per-channel decay rate as for RWKV-4.  The read-out follows the update (the
+ * current token enters with weight 1; the pages give Eagle no bonus term and no
+ * normalisation).  A state buffer is [B][C / 64][64][64] fp32 (m, j), the empty state zeros.
+ *
+ * eagle_forward: prefill over [B, T, C].
+ *   w              [C] fp32
+ *   r, k, v        [B, T, C] fp32
+ *   state_in       [B][C/64][64][64] fp32, or NULL for the empty state
+ *   y              [B, T, C] fp32 (written; must not alias the inputs)
+ *   state_out      [B][C/64][64][64] fp32, the state after the last token, or NULL
+ *   workspace      caller-owned device scratch, ws_bytes >= eagle_forward_workspace_size()
+ * C must be a multiple of 64 (else WKV_ERR_UNSUPPORTED), C/64 and B at most 65535.  T = 0
+ * writes state_out only (state_in, or zeros).  Time-parallel over 64-token chunks: each
+ * chunk's own state contribution, a scan over the chunks per state entry, then each chunk's
+ * outputs from its starting state.  Status codes as wkv_forward.
+ */
+wkv_status eagle_forward(int64_t B, int64_t T, int64_t C, const float* w, const float* r, const float* k,
+                         const float* v, const float* state_in, float* y, float* state_out, void* workspace,
+                         size_t ws_bytes, cudaStream_t stream);
+
+/* Workspace bytes eagle_forward needs: 16 KiB per sequence, head and 64-token chunk. */
+size_t eagle_forward_workspace_size(int64_t B, int64_t T, int64_t C);
+
+/*
+ * Eagle decode: one token for N sessions x L layers (section "O(N) Inference
+ * Characteristics": one matrix-vector product against the fixed-size state per token).
+ *   w              [L][C] fp32 (layer l's decay rates)
+ *   r, k, v, y     [N][L][C] fp32 (y written)
+ *   state_inout    [N][L][C/64][64][64] fp32, updated in place
+ * C must be a multiple of 64.  With L = 1 and N = B, state_out of eagle_forward continues
+ * the same sequences.
+ */
+wkv_status eagle_decode_step(int64_t N, int64_t L, int64_t C, const float* w, const float* r, const float* k,
+                             const float* v, float* state_inout, float* y, cudaStream_t stream);
 
 /* Human-readable name of a status code (static string). */
 const char* wkv_status_string(wkv_status status);

@@ -72,6 +72,10 @@ def lib():
                 L.wkv_backward_workspace_size.argtypes = [i64, i64, i64]
                 L.wkv_backward_workspace_size.restype = sz
                 L.wkv_decode_step.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp]
+                L.eagle_forward.argtypes = [i64, i64, i64] + [vp] * 8 + [sz, vp]
+                L.eagle_forward_workspace_size.argtypes = [i64, i64, i64]
+                L.eagle_forward_workspace_size.restype = sz
+                L.eagle_decode_step.argtypes = [i64, i64, i64] + [vp] * 7
                 L.wkv_decode_step_fused.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
                 L.token_shift_mix.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp]
                 L.wkv_status_string.argtypes = [i32]
@@ -213,6 +217,47 @@ def wkv_backward(w, u, k, v, gy, workspace=None):
                               gk.data_ptr(), gv.data_ptr(), gw.data_ptr(), gu.data_ptr(), ws.data_ptr(), ws.numel(),
                               _stream(k.device)), "wkv_backward")
     return gk, gv, gw, gu
+
+
+def eagle_forward(w, r, k, v, state_in=None, want_state=True, y=None, state_out=None, workspace=None):
+    """Eagle (RWKV-5) matrix-state prefill over fp32 [B, T, C] (C a multiple of 64): returns
+    (y, state_out) with state [B, C // 64, 64, 64] (None unless want_state or state_out)."""
+    for t, name in ((r, "r"), (k, "k"), (v, "v")):
+        _cuda_f32(t, name)
+    if k.dim() != 3 or r.shape != k.shape or v.shape != k.shape:
+        raise ValueError("r, k, v must be [B, T, C] tensors of one shape")
+    B, T, C = k.shape
+    _cuda_f32(w, "w", (C,))
+    H = C // 64
+    if state_in is not None:
+        _cuda_f32(state_in, "state_in", (B, H, 64, 64))
+    y = torch.empty_like(k) if y is None else y
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, 64, 64), dtype=torch.float32, device=k.device)
+    nbytes = int(lib().eagle_forward_workspace_size(B, T, C))
+    ws = workspace if workspace is not None and workspace.numel() >= nbytes else \
+        torch.empty(max(nbytes, 16), dtype=torch.uint8, device=k.device)
+    _check(lib().eagle_forward(B, T, C, w.data_ptr(), r.data_ptr(), k.data_ptr(), v.data_ptr(),
+                               _ptr(state_in), y.data_ptr(), _ptr(state_out), ws.data_ptr(), ws.numel(),
+                               _stream(k.device)), "eagle_forward")
+    return y, state_out
+
+
+def eagle_decode_step(w, r, k, v, state, y=None):
+    """One Eagle token for [N, L, C] rows with [L, C] decay rates; state [N, L, C // 64, 64, 64]
+    updated in place.  Returns y [N, L, C]."""
+    _cuda_f32(k, "k")
+    if k.dim() != 3:
+        raise ValueError("k must be [N, L, C]")
+    N, L, C = k.shape
+    _cuda_f32(r, "r", (N, L, C))
+    _cuda_f32(v, "v", (N, L, C))
+    _cuda_f32(w, "w", (L, C))
+    _cuda_f32(state, "state", (N, L, C // 64, 64, 64))
+    y = torch.empty_like(k) if y is None else y
+    _check(lib().eagle_decode_step(N, L, C, w.data_ptr(), r.data_ptr(), k.data_ptr(), v.data_ptr(), state.data_ptr(),
+                                   y.data_ptr(), _stream(k.device)), "eagle_decode_step")
+    return y
 
 
 def forward_status(workspace=None, device=None):

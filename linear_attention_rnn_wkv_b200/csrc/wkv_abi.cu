@@ -6,6 +6,7 @@
 
 #include "wkv.h"
 #include "wkv_device.cuh"
+#include "wkv_eagle_internal.h"
 #include "wkv_internal.h"
 
 namespace {
@@ -215,6 +216,46 @@ wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float* w, const f
     if (n > 0 && (!workspace || ws_bytes < wkv_backward_workspace_size(B, T, C))) return WKV_ERR_INVALID_ARG;
     if (B > 65535 || backward_segments(T) > 65535) return WKV_ERR_UNSUPPORTED;
     cudaError_t e = launch_backward(B, T, C, w, u, k, v, gy, gk, gv, gw, gu, workspace, stream);
+    return e == cudaSuccess ? WKV_OK : cuda_fail(e);
+}
+
+size_t eagle_forward_workspace_size(int64_t B, int64_t T, int64_t C) {
+    int64_t n = 0;
+    if (!sizes_ok(B, T, C, &n) || C % 64 != 0) return 0;
+    // per (b, head, chunk): one 64 x 64 fp32 state (the chunk's sum, then its starting state)
+    const int64_t heads = B * (C / 64), chunks = eagle_chunks(T);
+    if (chunks != 0 && heads > INT64_MAX / 16384 / chunks) return 0;
+    return (size_t)heads * (size_t)chunks * 64 * 64 * sizeof(float);
+}
+
+wkv_status eagle_forward(int64_t B, int64_t T, int64_t C, const float* w, const float* r, const float* k,
+                         const float* v, const float* state_in, float* y, float* state_out, void* workspace,
+                         size_t ws_bytes, cudaStream_t stream) {
+    int64_t n = 0;
+    if (!sizes_ok(B, T, C, &n) || n > INT64_MAX / 64) return WKV_ERR_INVALID_ARG;
+    if (C % 64 != 0) return WKV_ERR_UNSUPPORTED;
+    if (B == 0 || C == 0) return WKV_OK;
+    if (!w) return WKV_ERR_INVALID_ARG;
+    if (n > 0 && (!r || !k || !v || !y)) return WKV_ERR_INVALID_ARG;
+    if (!f32_args_ok({w, r, k, v, state_in, y, state_out, workspace})) return WKV_ERR_MISALIGNED;
+    // grids: (chunks, heads, B) for the chunk kernels, 16 blocks of 256 per head for the scan
+    if (B > 65535 || C / 64 > 65535 || eagle_chunks(T) > INT32_MAX || B * (C / 64) > INT32_MAX / 16)
+        return WKV_ERR_UNSUPPORTED;
+    if (n > 0 && (!workspace || ws_bytes < eagle_forward_workspace_size(B, T, C))) return WKV_ERR_INVALID_ARG;
+    cudaError_t e = launch_eagle_forward(B, T, C, w, r, k, v, state_in, y, state_out, workspace, stream);
+    return e == cudaSuccess ? WKV_OK : cuda_fail(e);
+}
+
+wkv_status eagle_decode_step(int64_t N, int64_t L, int64_t C, const float* w, const float* r, const float* k,
+                             const float* v, float* state_inout, float* y, cudaStream_t stream) {
+    int64_t n = 0;
+    if (!sizes_ok(N, L, C, &n) || n > INT64_MAX / 64) return WKV_ERR_INVALID_ARG;
+    if (C % 64 != 0) return WKV_ERR_UNSUPPORTED;
+    if (n == 0) return WKV_OK;
+    if (!w || !r || !k || !v || !state_inout || !y) return WKV_ERR_INVALID_ARG;
+    if (!f32_args_ok({w, r, k, v, state_inout, y})) return WKV_ERR_MISALIGNED;
+    if (n / 64 > INT32_MAX) return WKV_ERR_UNSUPPORTED;  // one block per (row, head)
+    cudaError_t e = launch_eagle_decode(N, L, C, w, r, k, v, state_inout, y, stream);
     return e == cudaSuccess ? WKV_OK : cuda_fail(e);
 }
 

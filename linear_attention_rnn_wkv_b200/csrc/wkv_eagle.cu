@@ -1,0 +1,237 @@
+// Eagle (RWKV-5) matrix-state WKV: per sequence and head of 64 channels
+//   S_t = diag(d) S_{t-1} + k_t v_t^T,   y_t = r_t^T S_t,   d = e^{-w} per key channel
+// ("RWKV (Attention-RNN Hybrid)", vanos001.github.io, section "Versions: RWKV-4 -> Eagle ->
+// Finch": the matrix form of the recurrence and its read-out; one 64 x 64 state per head,
+// section "O(N) Inference Characteristics").  Row m of S is a key channel, column j a value
+// channel; columns never mix, so each (sequence, head, column) is an independent scan whose
+// state is a 64-vector.
+//
+// Prefill, time-parallel in chunks of kEL tokens (three launches):
+//   1 eagle_chunk_sum   each chunk's own contribution to the state at its end, from zero:
+//                       U_c = sum_l diag(d)^{len-1-l} k_l v_l^T (decayed keys formed once per
+//                       chunk in shared memory, then one fused multiply-add per state entry
+//                       and token);
+//   2 eagle_state_scan  per state entry, the chunks in time order: S_start(c) and, after the
+//                       last chunk, the final state (S <- d^len S + U_c);
+//   3 eagle_chunk_out   each chunk's tokens again from its S_start: update, then read-out.
+// Decode (eagle_decode): one token of the recurrence per (row, head), the state read and
+// written once (section "O(N) Inference Characteristics": one matrix-vector product per token).
+//
+// Arithmetic is fp32 on the CUDA cores (packed f32x2 where a lane holds two key rows); the
+// decay powers are single exponentials 2^{-n w log2 e} of exact integer n, so no rounding
+// accumulates in them.
+#include <cuda_runtime.h>
+
+#include "wkv_device.cuh"
+#include "wkv_eagle_internal.h"
+
+namespace wkvb {
+namespace {
+
+constexpr int kHead = 64;  // channels per head
+constexpr int kEL = 64;    // tokens per chunk
+constexpr int kSS = kHead * kHead;
+
+struct EagleArgs {
+    int64_t B, T, C, H, P;  // P chunks of kEL tokens (the last may be shorter)
+    const float *w, *r, *k, *v, *state_in;
+    float *y, *state_out;
+    float* ch;  // [B][H][P][64][64]: chunk sums U_c, then chunk starting states
+};
+
+__device__ __forceinline__ float* chunk_state(const EagleArgs& a, int64_t b, int64_t h, int64_t c) {
+    return a.ch + ((b * a.H + h) * a.P + c) * kSS;
+}
+
+// 1: U_c[m][j] = sum_{l < len} e^{-(len-1-l) w_m} k_l[m] v_l[j]
+__global__ void __launch_bounds__(kHead) eagle_chunk_sum(EagleArgs a) {
+    __shared__ __align__(16) float kp[kEL][kHead];
+    __shared__ float vs[kEL][kHead];
+    const int j = threadIdx.x;
+    const int64_t c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int64_t t0 = c * kEL;
+    const int len = (int)min64(kEL, a.T - t0);
+    const int64_t row0 = (b * a.T + t0) * a.C + h * kHead;
+    {
+        const float w2 = a.w[h * kHead + j] * kLog2e;  // here thread j forms key row m = j
+#pragma unroll 8
+        for (int l = 0; l < len; ++l) {
+            kp[l][j] = a.k[row0 + l * a.C + j] * ex2(-(float)(len - 1 - l) * w2);
+            vs[l][j] = a.v[row0 + l * a.C + j];
+        }
+    }
+    __syncthreads();
+    float2 S[kHead / 2];
+#pragma unroll
+    for (int i = 0; i < kHead / 2; ++i) S[i] = make_float2(0.f, 0.f);
+    for (int l = 0; l < len; ++l) {
+        const float vj = vs[l][j];
+        const float2 vv = make_float2(vj, vj);
+#pragma unroll
+        for (int i = 0; i < kHead / 2; i += 2) {
+            const float4 kk = *reinterpret_cast<const float4*>(&kp[l][2 * i]);
+            S[i] = __ffma2_rn(make_float2(kk.x, kk.y), vv, S[i]);
+            S[i + 1] = __ffma2_rn(make_float2(kk.z, kk.w), vv, S[i + 1]);
+        }
+    }
+    float* out = chunk_state(a, b, h, c) + j;
+#pragma unroll
+    for (int i = 0; i < kHead / 2; ++i) {
+        out[(2 * i) * kHead] = S[i].x;
+        out[(2 * i + 1) * kHead] = S[i].y;
+    }
+}
+
+constexpr int kScanThreads = 256;
+constexpr int kScanBlk = 8;  // chunk sums loaded before any is overwritten
+
+// 2: per state entry (b, h, m, j), in time order: the slot of chunk c receives S_start(c),
+// then S <- e^{-len_c w_m} S + U_c; the state after the last chunk is the final state.
+__global__ void __launch_bounds__(kScanThreads) eagle_state_scan(EagleArgs a) {
+    const int64_t e = (int64_t)blockIdx.x * kScanThreads + threadIdx.x;
+    if (e >= a.B * a.H * kSS) return;
+    const int64_t bh = e / kSS;
+    const int mj = (int)(e % kSS), m = mj / kHead;
+    const int64_t h = bh % a.H;
+    const float w2 = a.w[h * kHead + m] * kLog2e;
+    const float d_full = ex2(-(float)kEL * w2);
+    float S = a.state_in ? a.state_in[bh * kSS + mj] : 0.f;
+    float* p = a.ch + bh * a.P * kSS + mj;
+    for (int64_t c0 = 0; c0 < a.P; c0 += kScanBlk) {
+        const int nb = (int)min64(kScanBlk, a.P - c0);
+        float u[kScanBlk];
+#pragma unroll
+        for (int i = 0; i < kScanBlk; ++i)
+            if (i < nb) u[i] = p[(c0 + i) * kSS];
+#pragma unroll
+        for (int i = 0; i < kScanBlk; ++i) {
+            if (i < nb) {
+                const int64_t c = c0 + i;
+                p[c * kSS] = S;
+                const int64_t len = min64(kEL, a.T - c * kEL);
+                const float d = len == kEL ? d_full : ex2(-(float)len * w2);
+                S = fmaf(d, S, u[i]);
+            }
+        }
+    }
+    if (a.state_out) a.state_out[bh * kSS + mj] = S;
+}
+
+// 3: each chunk's tokens from its starting state: S <- diag(d) S + k_l v_l^T, y_l = r_l^T S
+__global__ void __launch_bounds__(kHead) eagle_chunk_out(EagleArgs a) {
+    __shared__ __align__(16) float rs[kEL][kHead];
+    __shared__ __align__(16) float ks[kEL][kHead];
+    __shared__ float vs[kEL][kHead];
+    const int j = threadIdx.x;
+    const int64_t c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int64_t t0 = c * kEL;
+    const int len = (int)min64(kEL, a.T - t0);
+    const int64_t row0 = (b * a.T + t0) * a.C + h * kHead;
+#pragma unroll 8
+    for (int l = 0; l < len; ++l) {
+        rs[l][j] = a.r[row0 + l * a.C + j];
+        ks[l][j] = a.k[row0 + l * a.C + j];
+        vs[l][j] = a.v[row0 + l * a.C + j];
+    }
+    const float* st = chunk_state(a, b, h, c) + j;
+    float2 S[kHead / 2], d[kHead / 2];
+#pragma unroll
+    for (int i = 0; i < kHead / 2; ++i) {
+        S[i] = make_float2(st[(2 * i) * kHead], st[(2 * i + 1) * kHead]);
+        d[i] = make_float2(ex2(-a.w[h * kHead + 2 * i] * kLog2e), ex2(-a.w[h * kHead + 2 * i + 1] * kLog2e));
+    }
+    __syncthreads();
+    for (int l = 0; l < len; ++l) {
+        const float vj = vs[l][j];
+        const float2 vv = make_float2(vj, vj);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int i = 0; i < kHead / 2; i += 2) {
+            const float4 kk = *reinterpret_cast<const float4*>(&ks[l][2 * i]);
+            const float4 rr = *reinterpret_cast<const float4*>(&rs[l][2 * i]);
+            S[i] = __ffma2_rn(d[i], S[i], __fmul2_rn(make_float2(kk.x, kk.y), vv));
+            S[i + 1] = __ffma2_rn(d[i + 1], S[i + 1], __fmul2_rn(make_float2(kk.z, kk.w), vv));
+            acc[(i / 2) & 3] = __ffma2_rn(make_float2(rr.x, rr.y), S[i], acc[(i / 2) & 3]);
+            acc[(i / 2) & 3] = __ffma2_rn(make_float2(rr.z, rr.w), S[i + 1], acc[(i / 2) & 3]);
+        }
+        const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
+        const float2 s = __fadd2_rn(s01, s23);
+        a.y[row0 + l * a.C + j] = s.x + s.y;
+    }
+}
+
+// One token per (row, head): rows = N L, w [L][C] by the row's layer, state [rows][H][64][64].
+__global__ void __launch_bounds__(kHead) eagle_decode(int64_t L, int64_t C, int64_t H, const float* w,
+                                                      const float* r, const float* k, const float* v,
+                                                      float* state, float* y) {
+    __shared__ float rs[kHead], ks[kHead], ds[kHead];
+    const int j = threadIdx.x;
+    const int64_t idx = blockIdx.x, row = idx / H, h = idx % H, layer = row % L;
+    const int64_t base = row * C + h * kHead;
+    rs[j] = r[base + j];
+    ks[j] = k[base + j];
+    ds[j] = ex2(-w[layer * C + h * kHead + j] * kLog2e);
+    const float vj = v[base + j];
+    float* S = state + idx * kSS + j;
+    float s[kHead];
+#pragma unroll
+    for (int m = 0; m < kHead; ++m) s[m] = S[m * kHead];
+    __syncthreads();
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+    for (int m = 0; m < kHead; m += 2) {
+        s[m] = fmaf(ds[m], s[m], ks[m] * vj);
+        s[m + 1] = fmaf(ds[m + 1], s[m + 1], ks[m + 1] * vj);
+        acc0 = fmaf(rs[m], s[m], acc0);
+        acc1 = fmaf(rs[m + 1], s[m + 1], acc1);
+    }
+#pragma unroll
+    for (int m = 0; m < kHead; ++m) S[m * kHead] = s[m];
+    y[base + j] = acc0 + acc1;
+}
+
+}  // namespace
+
+int64_t eagle_chunks(int64_t T) { return (T + kEL - 1) / kEL; }
+
+cudaError_t launch_eagle_forward(int64_t B, int64_t T, int64_t C, const float* w, const float* r, const float* k,
+                                 const float* v, const float* state_in, float* y, float* state_out, void* ws,
+                                 cudaStream_t s) {
+    const int64_t H = C / kHead;
+    if (T == 0) {  // no token: the state passes through (zero without one)
+        if (!state_out) return cudaSuccess;
+        const size_t bytes = (size_t)B * (size_t)H * kSS * sizeof(float);
+        if (state_in) return cudaMemcpyAsync(state_out, state_in, bytes, cudaMemcpyDeviceToDevice, s);
+        return cudaMemsetAsync(state_out, 0, bytes, s);
+    }
+    EagleArgs a;
+    a.B = B;
+    a.T = T;
+    a.C = C;
+    a.H = H;
+    a.P = eagle_chunks(T);
+    a.w = w;
+    a.r = r;
+    a.k = k;
+    a.v = v;
+    a.state_in = state_in;
+    a.y = y;
+    a.state_out = state_out;
+    a.ch = static_cast<float*>(ws);
+    const dim3 grid((unsigned)a.P, (unsigned)H, (unsigned)B);
+    eagle_chunk_sum<<<grid, kHead, 0, s>>>(a);
+    const int64_t entries = B * H * kSS;
+    eagle_state_scan<<<(unsigned)((entries + kScanThreads - 1) / kScanThreads), kScanThreads, 0, s>>>(a);
+    eagle_chunk_out<<<grid, kHead, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_eagle_decode(int64_t N, int64_t L, int64_t C, const float* w, const float* r, const float* k,
+                                const float* v, float* state, float* y, cudaStream_t s) {
+    const int64_t H = C / kHead;
+    eagle_decode<<<(unsigned)(N * L * H), kHead, 0, s>>>(L, C, H, w, r, k, v, state, y);
+    return cudaGetLastError();
+}
+
+}  // namespace wkvb

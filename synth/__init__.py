@@ -32,6 +32,7 @@ S_DEC_K, S_DEC_V, S_DEC_X = 11, 12, 13
 S_STATE_P, S_STATE_B, S_STATE_A = 14, 15, 16
 S_R, S_RSPIKE = 17, 18
 S_GY = 19
+S_EAGLE_W, S_EAGLE_R, S_EAGLE_K, S_EAGLE_V, S_EAGLE_STATE = 20, 21, 22, 23, 24
 
 
 def build(force: bool = False) -> str:
@@ -301,3 +302,48 @@ def filler_state(spec: DecodeSpec):
     an = normal(spec.seed, S_STATE_A, shape)
     np.multiply(an, bn, out=st[0])
     return st
+
+
+# --------------------------------------------------------------------------
+# Eagle (RWKV-5) matrix-state workloads: heads of 64 channels.  The pages give no
+# distributions for it; these take the RWKV-4 forward workloads' decay range
+# (w = exp(U(-5, 1))) and r, k, v ~ N(0, 1).
+# --------------------------------------------------------------------------
+
+@dataclass(frozen=True)
+class EagleSpec:
+    name: str
+    B: int
+    T: int
+    C: int                # a multiple of 64: C / 64 heads
+    seed: int
+    w_lo: float = -5.0
+    w_hi: float = 1.0
+
+
+EAGLE = {
+    # the headline forward shape read as 12 heads of 64 channels
+    "eagle_8x1024x768": EagleSpec("eagle_8x1024x768", 8, 1024, 768, 2001),
+    # the long bf16 forward shape's size, fp32, 32 heads
+    "eagle_4x4096x2048": EagleSpec("eagle_4x4096x2048", 4, 4096, 2048, 2002),
+}
+
+
+def eagle_spec_like(base: str, B: int, T: int, C: int, seed: int | None = None) -> EagleSpec:
+    s = EAGLE[base]
+    return EagleSpec(f"{base}@{B}x{T}x{C}", B, T, C, s.seed if seed is None else seed, s.w_lo, s.w_hi)
+
+
+def eagle_inputs(spec: EagleSpec):
+    """(w, r, k, v): w fp32 [C] (> 0), r, k, v fp32 [B, T, C]."""
+    w = exp_uniform(spec.seed, S_EAGLE_W, (spec.C,), spec.w_lo, spec.w_hi)
+    shape = (spec.B, spec.T, spec.C)
+    r = normal(spec.seed, S_EAGLE_R, shape)
+    k = normal(spec.seed, S_EAGLE_K, shape)
+    v = normal(spec.seed, S_EAGLE_V, shape)
+    return w, r, k, v
+
+
+def eagle_state(spec: EagleSpec, std: float = 1.0):
+    """A given starting state [B, C / 64, 64, 64], N(0, std)."""
+    return normal(spec.seed, S_EAGLE_STATE, (spec.B, spec.C // 64, 64, 64), 0.0, std)

@@ -124,3 +124,32 @@ def test_gated_and_shift3_validation_without_launch():
     shift3 = lambda x=FAKE, xr=FAKE: L.token_shift_mix3(1, 4, 4, FAKE, FAKE, FAKE, x, None, xr, FAKE, FAKE, None)
     assert shift3(x=None) == 1
     assert shift3(xr=FAKE + 4) == 2
+
+
+def test_eagle_validation_without_launch():
+    """eagle_forward / eagle_decode_step check their arguments before touching the device."""
+    L = wkv.lib()
+
+    def fwd(B, T, C, r=FAKE, y=FAKE, ws=FAKE, nbytes=1 << 30, state_in=None):
+        return L.eagle_forward(B, T, C, FAKE, r, FAKE, FAKE, state_in, y, None, ws, nbytes, None)
+
+    assert fwd(-1, 4, 64) == 1                   # negative size
+    assert fwd(1, 4, 96) == 3                    # C not a multiple of the head size
+    assert fwd(1, 4, 64, r=None) == 1            # null input
+    assert fwd(1, 4, 64, y=FAKE + 4) == 2        # misaligned output
+    assert fwd(1, 4, 64, state_in=FAKE + 8) == 2  # misaligned optional state
+    assert fwd(1, 4, 64, nbytes=16) == 1         # workspace too small
+    assert fwd(70000, 1, 64) == 3                # batch above the grid's z limit
+    assert fwd(0, 4, 64) == 0 and fwd(1, 4, 0) == 0  # empty calls
+    # one 64 x 64 fp32 state per (sequence, head, 64-token chunk)
+    assert L.eagle_forward_workspace_size(2, 65, 128) == 2 * 2 * 2 * 64 * 64 * 4
+    assert L.eagle_forward_workspace_size(1, 64, 64) == 64 * 64 * 4
+    assert L.eagle_forward_workspace_size(1, 4, 96) == 0
+
+    def dec(N, L_, C, state=FAKE, y=FAKE):
+        return L.eagle_decode_step(N, L_, C, FAKE, FAKE, FAKE, FAKE, state, y, None)
+
+    assert dec(2, 1, 100) == 3
+    assert dec(2, 1, 64, state=None) == 1
+    assert dec(2, 1, 64, y=FAKE + 4) == 2
+    assert dec(0, 1, 64) == 0
