@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--profile-forward", metavar="WORKLOAD", default=None,
                     help="only run 2 + 3 eager forward launches of a forward workload (e.g. fwd_1x16384x4096) "
                          "and exit: a short, self-contained command to capture under a profiler")
+    ap.add_argument("--profile-eagle", action="store_true",
+                    help="only run 2 + 3 eager Eagle prefills on eagle_8x1024x768 and exit, for a profiler")
     ap.add_argument("--profile-backward", metavar="WORKLOAD", default=None,
                     help="only run 2 + 3 eager backward calls (five launches each) on a forward workload's shape "
                          "(fp32) and exit, for a profiler")
@@ -699,6 +701,22 @@ def profile_backward(name):
     print(json.dumps({"profile_backward": name, "calls": 5, "B": spec.B, "T": spec.T, "C": spec.C}))
 
 
+def profile_eagle():
+    """Two warm-up and three profiled eager Eagle prefills (with the final state) on
+    eagle_8x1024x768."""
+    import torch
+    import linear_attention_rnn_wkv_b200 as wkv
+    import synth
+    spec = synth.EAGLE["eagle_8x1024x768"]
+    dev = torch.device("cuda", 0)
+    w, r, k, v = (torch.from_numpy(a).to(dev) for a in synth.eagle_inputs(spec))
+    for _ in range(5):
+        wkv.eagle_forward(w, r, k, v)
+    torch.cuda.synchronize()
+    wkv.get_device_status()
+    print(json.dumps({"profile_eagle": spec.name, "calls": 5}))
+
+
 def main():
     args = parse()
     if args.profile_forward:
@@ -706,6 +724,9 @@ def main():
         return
     if args.profile_backward:
         profile_backward(args.profile_backward)
+        return
+    if args.profile_eagle:
+        profile_eagle()
         return
     if args.impl == "reference":
         run_reference(args)

@@ -239,7 +239,8 @@ wkv_status eagle_forward(int64_t B, int64_t T, int64_t C, const float* w, const 
     if (n > 0 && (!r || !k || !v || !y)) return WKV_ERR_INVALID_ARG;
     if (!f32_args_ok({w, r, k, v, state_in, y, state_out, workspace})) return WKV_ERR_MISALIGNED;
     // grids: (chunks, heads, B) for the chunk kernels, 16 blocks of 256 per head for the scan
-    if (B > 65535 || C / 64 > 65535 || eagle_chunks(T) > INT32_MAX || B * (C / 64) > INT32_MAX / 16)
+    // TMA coordinates are 32-bit
+    if (B > 65535 || C / 64 > 65535 || T > INT32_MAX || C > INT32_MAX || B * (C / 64) > INT32_MAX / 16)
         return WKV_ERR_UNSUPPORTED;
     if (n > 0 && (!workspace || ws_bytes < eagle_forward_workspace_size(B, T, C))) return WKV_ERR_INVALID_ARG;
     cudaError_t e = launch_eagle_forward(B, T, C, w, r, k, v, state_in, y, state_out, workspace, stream);

@@ -24,6 +24,8 @@
 
 #include "wkv_device.cuh"
 #include "wkv_eagle_internal.h"
+#include "wkv_internal.h"
+#include "wkv_pipe_common.cuh"
 
 namespace wkvb {
 namespace {
@@ -36,30 +38,45 @@ struct EagleArgs {
     int64_t B, T, C, H, P;  // P chunks of kEL tokens (the last may be shorter)
     const float *w, *r, *k, *v, *state_in;
     float *y, *state_out;
-    float* ch;  // [B][H][P][64][64]: chunk sums U_c, then chunk starting states
+    float* ch;          // [B][H][P][64][64]: chunk sums U_c, then chunk starting states
+    uint32_t* dev_err;  // the library's device-wide error word
+    uint32_t spin_limit;
 };
+
+constexpr uint32_t kTileBytes = kEL * kHead * sizeof(float);  // one [64 tokens][64 channels] box
+
+// The chunk's rows of r, k, v arrive by TMA tensor copies (rows past T read as zeros); every
+// thread waits on the barrier, bounded: a copy that never lands is recorded in the error word
+// and the block goes on with what it has (its outputs are then invalid).
+__device__ __forceinline__ void wait_tiles(const EagleArgs& a, uint64_t* bar) {
+    if (!mbar_wait(bar, 0, a.spin_limit) && threadIdx.x == 0) atomicCAS(a.dev_err, kDevOk, (uint32_t)kDevTimeoutCopy);
+}
 
 __device__ __forceinline__ float* chunk_state(const EagleArgs& a, int64_t b, int64_t h, int64_t c) {
     return a.ch + ((b * a.H + h) * a.P + c) * kSS;
 }
 
 // 1: U_c[m][j] = sum_{l < len} e^{-(len-1-l) w_m} k_l[m] v_l[j]
-__global__ void __launch_bounds__(kHead) eagle_chunk_sum(EagleArgs a) {
-    __shared__ __align__(16) float kp[kEL][kHead];
-    __shared__ float vs[kEL][kHead];
+__global__ void __launch_bounds__(kHead) eagle_chunk_sum(EagleArgs a, const __grid_constant__ CUtensorMap tmk,
+                                                         const __grid_constant__ CUtensorMap tmv) {
+    __shared__ __align__(128) float kp[kEL][kHead];
+    __shared__ __align__(128) float vs[kEL][kHead];
+    __shared__ uint64_t bar;
     const int j = threadIdx.x;
     const int64_t c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int64_t t0 = c * kEL;
     const int len = (int)min64(kEL, a.T - t0);
-    const int64_t row0 = (b * a.T + t0) * a.C + h * kHead;
-    {
-        const float w2 = a.w[h * kHead + j] * kLog2e;  // here thread j forms key row m = j
-#pragma unroll 8
-        for (int l = 0; l < len; ++l) {
-            kp[l][j] = a.k[row0 + l * a.C + j] * ex2(-(float)(len - 1 - l) * w2);
-            vs[l][j] = a.v[row0 + l * a.C + j];
-        }
+    if (j == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(&bar, 2 * kTileBytes);
+        tma_load_3d(&kp[0][0], &tmk, (int)(h * kHead), (int)t0, (int)b, &bar);
+        tma_load_3d(&vs[0][0], &tmv, (int)(h * kHead), (int)t0, (int)b, &bar);
     }
+    const float w2 = a.w[h * kHead + j] * kLog2e;  // here thread j scales key row m = j
+    __syncthreads();                                // the barrier is initialised
+    wait_tiles(a, &bar);
+    for (int l = 0; l < len; ++l) kp[l][j] *= ex2(-(float)(len - 1 - l) * w2);
     __syncthreads();
     float2 S[kHead / 2];
 #pragma unroll
@@ -118,21 +135,29 @@ __global__ void __launch_bounds__(kScanThreads) eagle_state_scan(EagleArgs a) {
 }
 
 // 3: each chunk's tokens from its starting state: S <- diag(d) S + k_l v_l^T, y_l = r_l^T S
-__global__ void __launch_bounds__(kHead) eagle_chunk_out(EagleArgs a) {
-    __shared__ __align__(16) float rs[kEL][kHead];
-    __shared__ __align__(16) float ks[kEL][kHead];
-    __shared__ float vs[kEL][kHead];
+constexpr size_t kOutSmem = 3 * (size_t)kTileBytes + 128;  // r, k, v tiles and the barrier
+
+__global__ void __launch_bounds__(kHead) eagle_chunk_out(EagleArgs a, const __grid_constant__ CUtensorMap tmr,
+                                                         const __grid_constant__ CUtensorMap tmk,
+                                                         const __grid_constant__ CUtensorMap tmv) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    float(*rs)[kHead] = reinterpret_cast<float(*)[kHead]>(smem);
+    float(*ks)[kHead] = reinterpret_cast<float(*)[kHead]>(smem + kTileBytes);
+    float(*vs)[kHead] = reinterpret_cast<float(*)[kHead]>(smem + 2 * kTileBytes);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 3 * kTileBytes);
     const int j = threadIdx.x;
     const int64_t c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int64_t t0 = c * kEL;
     const int len = (int)min64(kEL, a.T - t0);
-    const int64_t row0 = (b * a.T + t0) * a.C + h * kHead;
-#pragma unroll 8
-    for (int l = 0; l < len; ++l) {
-        rs[l][j] = a.r[row0 + l * a.C + j];
-        ks[l][j] = a.k[row0 + l * a.C + j];
-        vs[l][j] = a.v[row0 + l * a.C + j];
+    if (j == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(bar, 3 * kTileBytes);
+        tma_load_3d(&rs[0][0], &tmr, (int)(h * kHead), (int)t0, (int)b, bar);
+        tma_load_3d(&ks[0][0], &tmk, (int)(h * kHead), (int)t0, (int)b, bar);
+        tma_load_3d(&vs[0][0], &tmv, (int)(h * kHead), (int)t0, (int)b, bar);
     }
+    // the starting state and the decays while the tiles are in flight
     const float* st = chunk_state(a, b, h, c) + j;
     float2 S[kHead / 2], d[kHead / 2];
 #pragma unroll
@@ -140,7 +165,8 @@ __global__ void __launch_bounds__(kHead) eagle_chunk_out(EagleArgs a) {
         S[i] = make_float2(st[(2 * i) * kHead], st[(2 * i + 1) * kHead]);
         d[i] = make_float2(ex2(-a.w[h * kHead + 2 * i] * kLog2e), ex2(-a.w[h * kHead + 2 * i + 1] * kLog2e));
     }
-    __syncthreads();
+    __syncthreads();  // the barrier is initialised
+    wait_tiles(a, bar);
     for (int l = 0; l < len; ++l) {
         const float vj = vs[l][j];
         const float2 vv = make_float2(vj, vj);
@@ -157,7 +183,7 @@ __global__ void __launch_bounds__(kHead) eagle_chunk_out(EagleArgs a) {
         }
         const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
         const float2 s = __fadd2_rn(s01, s23);
-        a.y[row0 + l * a.C + j] = s.x + s.y;
+        a.y[(b * a.T + t0 + l) * a.C + h * kHead + j] = s.x + s.y;
     }
 }
 
@@ -205,6 +231,19 @@ cudaError_t launch_eagle_forward(int64_t B, int64_t T, int64_t C, const float* w
         if (state_in) return cudaMemcpyAsync(state_out, state_in, bytes, cudaMemcpyDeviceToDevice, s);
         return cudaMemsetAsync(state_out, 0, bytes, s);
     }
+    CUtensorMap tmr, tmk, tmv;
+    if (!make_tile_map(&tmr, r, B, T, C, 0, kHead, kEL) || !make_tile_map(&tmk, k, B, T, C, 0, kHead, kEL) ||
+        !make_tile_map(&tmv, v, B, T, C, 0, kHead, kEL))
+        return cudaErrorInvalidValue;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static uint64_t attr_done = 0;
+    if (dev >= 64 || !(attr_done & (1ull << dev))) {
+        e = cudaFuncSetAttribute(eagle_chunk_out, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kOutSmem);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) attr_done |= 1ull << dev;
+    }
     EagleArgs a;
     a.B = B;
     a.T = T;
@@ -219,11 +258,14 @@ cudaError_t launch_eagle_forward(int64_t B, int64_t T, int64_t C, const float* w
     a.y = y;
     a.state_out = state_out;
     a.ch = static_cast<float*>(ws);
+    a.dev_err = device_status_word();
+    a.spin_limit = kSpinLimitDefault;
+    if (!a.dev_err) return cudaErrorInvalidValue;
     const dim3 grid((unsigned)a.P, (unsigned)H, (unsigned)B);
-    eagle_chunk_sum<<<grid, kHead, 0, s>>>(a);
+    eagle_chunk_sum<<<grid, kHead, 0, s>>>(a, tmk, tmv);
     const int64_t entries = B * H * kSS;
     eagle_state_scan<<<(unsigned)((entries + kScanThreads - 1) / kScanThreads), kScanThreads, 0, s>>>(a);
-    eagle_chunk_out<<<grid, kHead, 0, s>>>(a);
+    eagle_chunk_out<<<grid, kHead, kOutSmem, s>>>(a, tmr, tmk, tmv);
     return cudaGetLastError();
 }
 
