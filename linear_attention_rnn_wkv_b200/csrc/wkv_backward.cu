@@ -21,10 +21,11 @@
 // Time-parallel in segments of kSeg steps, one thread per (b, c, segment), five launches:
 //   A  each segment's forward recurrence from the empty state -> its state record;
 //   B  per channel, the records combined in time order -> each segment's starting state
-//      (and gw, gu zeroed for the atomics of E);
+//      (and gw, gu zeroed for the atomics of E), two-level over groups of segments;
 //   C  each segment's forward from its starting state, accumulating its local (X, Y, X', Y')
 //      left to right as each D_t and y_t appears;
-//   D  per channel, the local sums composed right to left -> each segment's incoming sums;
+//   D  per channel, the local sums composed right to left -> each segment's incoming sums,
+//      two-level like B;
 //   E  each segment's forward again, keeping per position the output's reference exponent q_t,
 //      1 / Dn_t (D_t = Dn_t 2^{q_t}) and y_t in shared memory, then its adjoint recurrence from
 //      the incoming sums -> gk, gv, and gw, gu partials added with atomics.
@@ -212,40 +213,85 @@ __global__ void __launch_bounds__(kThreads) bwd_seg_forward(BwdArgs a) {
     a.fs[3 * SP + si] = s.n;
 }
 
-// B: per channel, segment records combined left to right -> each segment's starting state.
-// The records of kScanBlk segments are loaded before any is overwritten, so the serial chain
-// waits on memory once per kScanBlk segments.
-__global__ void __launch_bounds__(kThreads) bwd_seg_carry(BwdArgs a) {
-    const int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    const int64_t b = blockIdx.y;
-    if (c >= a.C) return;
-    if (b == 0) {  // E accumulates into these
-        a.gw[c] = 0.f;
-        a.gu[c] = 0.f;
-    }
-    const float w2 = a.w[c] * kLog2e;
+// The two per-channel scans (B, D) split a channel's segments into kGroups consecutive groups:
+// every group folds its own segments (in parallel with the others), each group then combines
+// the aggregates of the groups before it (B) or after it (D), and walks its segments again from
+// that carry, writing each segment's carry.  The serial chain per channel is one group long.
+constexpr int kGroups = 8;
+constexpr int kScanCh = 32;  // channels per scan block: one warp per group
+constexpr int kScanThreadsB = kScanCh * kGroups;
+
+struct GroupSpan {
+    int64_t j0, j1;  // the group's segments [j0, j1) (possibly empty)
+};
+
+__device__ __forceinline__ GroupSpan group_span(const BwdArgs& a, int g) {
+    const int64_t per = (a.P + kGroups - 1) / kGroups;
+    const int64_t j0 = min64(a.P, g * per);
+    return GroupSpan{j0, min64(a.P, j0 + per)};
+}
+
+__device__ __forceinline__ float seg_len(const BwdArgs& a, int64_t j) {
+    return (float)(min64(a.T, (j + 1) * kSeg) - j * kSeg);
+}
+
+__device__ __forceinline__ float group_len(const BwdArgs& a, int g) {
+    const GroupSpan s = group_span(a, g);
+    return s.j1 > s.j0 ? (float)(min64(a.T, s.j1 * kSeg) - s.j0 * kSeg) : 0.f;
+}
+
+__device__ __forceinline__ Rec load_rec(const BwdArgs& a, int64_t si) {
+    const int64_t SP = a.B * a.P * a.C;
+    return Rec{a.fs[si], a.fs[SP + si], a.fs[2 * SP + si], a.fs[3 * SP + si]};
+}
+
+// B: per channel, segment records combined left to right -> each segment's starting state
+// (and gw, gu zeroed for the atomics of E).
+__global__ void __launch_bounds__(kScanThreadsB) bwd_seg_carry(BwdArgs a) {
+    __shared__ Rec agg[kGroups][kScanCh];
+    const int lane = threadIdx.x % kScanCh, g = threadIdx.x / kScanCh;
+    const int64_t c = (int64_t)blockIdx.x * kScanCh + lane, b = blockIdx.y;
+    const bool live = c < a.C;
+    const float w2 = live ? a.w[c] * kLog2e : 0.f;
+    const GroupSpan sp = group_span(a, g);
     const int64_t SP = a.B * a.P * a.C;
     Rec run = rec_identity();
-    for (int64_t j0 = 0; j0 < a.P; j0 += kScanBlk) {
-        const int nb = (int)min64(kScanBlk, a.P - j0);
+    if (live) {
+        if (b == 0 && g == 0) {  // E accumulates into these
+            a.gw[c] = 0.f;
+            a.gu[c] = 0.f;
+        }
+        for (int64_t j0 = sp.j0; j0 < sp.j1; j0 += kScanBlk) {
+            const int nb = (int)min64(kScanBlk, sp.j1 - j0);
+            Rec seg[kScanBlk];
+#pragma unroll
+            for (int i = 0; i < kScanBlk; ++i)
+                if (i < nb) seg[i] = load_rec(a, seg_index(a, b, j0 + i, c));
+#pragma unroll
+            for (int i = 0; i < kScanBlk; ++i)
+                if (i < nb) run = rec_combine(run, seg[i], seg_len(a, j0 + i), w2);
+        }
+    }
+    agg[g][lane] = run;
+    __syncthreads();
+    if (!live) return;
+    Rec carry = rec_identity();  // the groups before this one, in time order
+    for (int q = 0; q < g; ++q) carry = rec_combine(carry, agg[q][lane], group_len(a, q), w2);
+    for (int64_t j0 = sp.j0; j0 < sp.j1; j0 += kScanBlk) {
+        const int nb = (int)min64(kScanBlk, sp.j1 - j0);
         Rec seg[kScanBlk];
+#pragma unroll
+        for (int i = 0; i < kScanBlk; ++i)
+            if (i < nb) seg[i] = load_rec(a, seg_index(a, b, j0 + i, c));
 #pragma unroll
         for (int i = 0; i < kScanBlk; ++i) {
             if (i < nb) {
                 const int64_t si = seg_index(a, b, j0 + i, c);
-                seg[i] = Rec{a.fs[si], a.fs[SP + si], a.fs[2 * SP + si], a.fs[3 * SP + si]};
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < kScanBlk; ++i) {
-            if (i < nb) {
-                const int64_t j = j0 + i, si = seg_index(a, b, j, c);
-                a.fs[si] = run.a;
-                a.fs[SP + si] = run.b;
-                a.fs[2 * SP + si] = run.anc;
-                a.fs[3 * SP + si] = run.n;
-                const float len = (float)(min64(a.T, (j + 1) * kSeg) - j * kSeg);
-                run = rec_combine(run, seg[i], len, w2);
+                a.fs[si] = carry.a;
+                a.fs[SP + si] = carry.b;
+                a.fs[2 * SP + si] = carry.anc;
+                a.fs[3 * SP + si] = carry.n;
+                carry = rec_combine(carry, seg[i], seg_len(a, j0 + i), w2);
             }
         }
     }
@@ -271,24 +317,59 @@ __global__ void __launch_bounds__(kThreads) bwd_seg_local(BwdArgs a) {
     a.as[4 * SP + si] = fmaf(ls.Rj, w2, ls.Rq);
 }
 
-// D: per channel, local sums composed right to left -> each segment's incoming sums
-__global__ void __launch_bounds__(kThreads) bwd_seg_adjoint_carry(BwdArgs a) {
-    const int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    const int64_t b = blockIdx.y;
-    if (c >= a.C) return;
-    const float w2 = a.w[c] * kLog2e;
+// What leaves a span of len steps to its left: its local sums plus the sums entering it from
+// the right carried across it (X decays by e^{-w len}; X' also gains len X).
+__device__ __forceinline__ Adj adj_compose(const Adj& loc, const Adj& in, float len, float w2) {
+    const float rin = in.r + len * w2;
+    const float rn = fminf(loc.r, rin);
+    const float fl = ex2(rn - loc.r), fi = ex2(rn - rin);
+    Adj out;
+    out.x = fmaf(in.x, fi, loc.x * fl);
+    out.y = fmaf(in.y, fi, loc.y * fl);
+    out.xp = fmaf(fmaf(len, in.x, in.xp), fi, loc.xp * fl);
+    out.yp = fmaf(fmaf(len, in.y, in.yp), fi, loc.yp * fl);
+    out.r = rn;
+    return out;
+}
+
+__device__ __forceinline__ Adj load_adj(const BwdArgs& a, int64_t si) {
     const int64_t SP = a.B * a.P * a.C;
-    Adj in = adj_empty();  // entering the last segment from its right: nothing
-    for (int64_t j1 = a.P; j1 > 0; j1 -= kScanBlk) {
-        const int nb = (int)min64(kScanBlk, j1);
+    return Adj{a.as[si], a.as[SP + si], a.as[2 * SP + si], a.as[3 * SP + si], a.as[4 * SP + si]};
+}
+
+// D: per channel, local sums composed right to left -> each segment's incoming sums
+__global__ void __launch_bounds__(kScanThreadsB) bwd_seg_adjoint_carry(BwdArgs a) {
+    __shared__ Adj agg[kGroups][kScanCh];
+    const int lane = threadIdx.x % kScanCh, g = threadIdx.x / kScanCh;
+    const int64_t c = (int64_t)blockIdx.x * kScanCh + lane, b = blockIdx.y;
+    const bool live = c < a.C;
+    const float w2 = live ? a.w[c] * kLog2e : 0.f;
+    const GroupSpan sp = group_span(a, g);
+    const int64_t SP = a.B * a.P * a.C;
+    Adj run = adj_empty();
+    if (live) {
+        for (int64_t j1 = sp.j1; j1 > sp.j0; j1 -= kScanBlk) {
+            const int nb = (int)min64(kScanBlk, j1 - sp.j0);
+            Adj loc[kScanBlk];
+#pragma unroll
+            for (int i = 0; i < kScanBlk; ++i)
+                if (i < nb) loc[i] = load_adj(a, seg_index(a, b, j1 - 1 - i, c));
+#pragma unroll
+            for (int i = 0; i < kScanBlk; ++i)
+                if (i < nb) run = adj_compose(loc[i], run, seg_len(a, j1 - 1 - i), w2);
+        }
+    }
+    agg[g][lane] = run;
+    __syncthreads();
+    if (!live) return;
+    Adj in = adj_empty();  // the groups after this one, composed right to left
+    for (int q = kGroups - 1; q > g; --q) in = adj_compose(agg[q][lane], in, group_len(a, q), w2);
+    for (int64_t j1 = sp.j1; j1 > sp.j0; j1 -= kScanBlk) {
+        const int nb = (int)min64(kScanBlk, j1 - sp.j0);
         Adj loc[kScanBlk];
 #pragma unroll
-        for (int i = 0; i < kScanBlk; ++i) {
-            if (i < nb) {
-                const int64_t si = seg_index(a, b, j1 - 1 - i, c);
-                loc[i] = Adj{a.as[si], a.as[SP + si], a.as[2 * SP + si], a.as[3 * SP + si], a.as[4 * SP + si]};
-            }
-        }
+        for (int i = 0; i < kScanBlk; ++i)
+            if (i < nb) loc[i] = load_adj(a, seg_index(a, b, j1 - 1 - i, c));
 #pragma unroll
         for (int i = 0; i < kScanBlk; ++i) {
             if (i < nb) {
@@ -298,19 +379,7 @@ __global__ void __launch_bounds__(kThreads) bwd_seg_adjoint_carry(BwdArgs a) {
                 a.as[2 * SP + si] = in.xp;
                 a.as[3 * SP + si] = in.yp;
                 a.as[4 * SP + si] = in.r;
-                // what leaves this segment to its left: the local sums plus the incoming ones
-                // carried across the segment's len steps
-                const float len = (float)(min64(a.T, (j + 1) * kSeg) - j * kSeg);
-                const float rin = in.r + len * w2;
-                const float rn = fminf(loc[i].r, rin);
-                const float fl = ex2(rn - loc[i].r), fi = ex2(rn - rin);
-                Adj out;
-                out.x = fmaf(in.x, fi, loc[i].x * fl);
-                out.y = fmaf(in.y, fi, loc[i].y * fl);
-                out.xp = fmaf(fmaf(len, in.x, in.xp), fi, loc[i].xp * fl);
-                out.yp = fmaf(fmaf(len, in.y, in.yp), fi, loc[i].yp * fl);
-                out.r = rn;
-                in = out;
+                in = adj_compose(loc[i], in, seg_len(a, j), w2);
             }
         }
     }
@@ -396,11 +465,12 @@ cudaError_t launch_backward(int64_t B, int64_t T, int64_t C, const float* w, con
     a.fs = static_cast<float*>(ws);
     a.as = a.fs + 4 * SP;
     const unsigned cx = (unsigned)((C + kThreads - 1) / kThreads);
-    const dim3 seg_grid(cx, (unsigned)a.P, (unsigned)B), chan_grid(cx, (unsigned)B);
+    const dim3 seg_grid(cx, (unsigned)a.P, (unsigned)B);
+    const dim3 scan_grid((unsigned)((C + kScanCh - 1) / kScanCh), (unsigned)B);
     bwd_seg_forward<<<seg_grid, kThreads, 0, s>>>(a);
-    bwd_seg_carry<<<chan_grid, kThreads, 0, s>>>(a);
+    bwd_seg_carry<<<scan_grid, kScanThreadsB, 0, s>>>(a);
     bwd_seg_local<<<seg_grid, kThreads, 0, s>>>(a);
-    bwd_seg_adjoint_carry<<<chan_grid, kThreads, 0, s>>>(a);
+    bwd_seg_adjoint_carry<<<scan_grid, kScanThreadsB, 0, s>>>(a);
     bwd_seg_grads<<<seg_grid, kThreads, kGradSmem, s>>>(a);
     return cudaGetLastError();
 }
