@@ -56,51 +56,65 @@ __device__ __forceinline__ float* chunk_state(const EagleArgs& a, int64_t b, int
     return a.ch + ((b * a.H + h) * a.P + c) * kSS;
 }
 
+// Both chunk kernels run 128 threads per (chunk, head, sequence): two per value column j, each
+// holding 32 key rows of the column's state.  Lanes 0-15 of a warp take rows 0-31 and lanes
+// 16-31 rows 32-63 of the same 16 columns; a thread's register block i (four rows) is key rows
+// 32 half + 4 ((i + half) mod 8): the two halves of a warp then read different banks of a
+// shared row in the same instruction (each half's lanes read one address, a broadcast).
+constexpr int kChunkThreads = 128;
+
+__device__ __forceinline__ int row_block(int half, int i) { return 32 * half + 4 * ((i + half) & 7); }
+
 // 1: U_c[m][j] = sum_{l < len} e^{-(len-1-l) w_m} k_l[m] v_l[j]
-__global__ void __launch_bounds__(kHead) eagle_chunk_sum(EagleArgs a, const __grid_constant__ CUtensorMap tmk,
-                                                         const __grid_constant__ CUtensorMap tmv) {
+__global__ void __launch_bounds__(kChunkThreads) eagle_chunk_sum(EagleArgs a, const __grid_constant__ CUtensorMap tmk,
+                                                                 const __grid_constant__ CUtensorMap tmv) {
     __shared__ __align__(128) float kp[kEL][kHead];
     __shared__ __align__(128) float vs[kEL][kHead];
     __shared__ uint64_t bar;
-    const int j = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, half = lane >> 4;
+    const int j = (tid >> 5) * 16 + (lane & 15);
     const int64_t c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int64_t t0 = c * kEL;
     const int len = (int)min64(kEL, a.T - t0);
-    if (j == 0) {
+    if (tid == 0) {
         mbar_init(&bar, 1);
         fence_mbar_init();
         mbar_arrive_expect_tx(&bar, 2 * kTileBytes);
         tma_load_3d(&kp[0][0], &tmk, (int)(h * kHead), (int)t0, (int)b, &bar);
         tma_load_3d(&vs[0][0], &tmv, (int)(h * kHead), (int)t0, (int)b, &bar);
     }
-    const float w2 = a.w[h * kHead + j] * kLog2e;  // here thread j scales key row m = j
-    __syncthreads();                                // the barrier is initialised
+    const int sm_m = tid & 63, sm_l0 = tid >> 6;  // the decay scaling: key row sm_m, every other token
+    const float w2 = a.w[h * kHead + sm_m] * kLog2e;
+    __syncthreads();  // the barrier is initialised
     wait_tiles(a, &bar);
-    for (int l = 0; l < len; ++l) kp[l][j] *= ex2(-(float)(len - 1 - l) * w2);
+    for (int l = sm_l0; l < len; l += 2) kp[l][sm_m] *= ex2(-(float)(len - 1 - l) * w2);
     __syncthreads();
-    float2 S[kHead / 2];
+    float2 S[16];
 #pragma unroll
-    for (int i = 0; i < kHead / 2; ++i) S[i] = make_float2(0.f, 0.f);
+    for (int i = 0; i < 16; ++i) S[i] = make_float2(0.f, 0.f);
     for (int l = 0; l < len; ++l) {
         const float vj = vs[l][j];
         const float2 vv = make_float2(vj, vj);
 #pragma unroll
-        for (int i = 0; i < kHead / 2; i += 2) {
-            const float4 kk = *reinterpret_cast<const float4*>(&kp[l][2 * i]);
-            S[i] = __ffma2_rn(make_float2(kk.x, kk.y), vv, S[i]);
-            S[i + 1] = __ffma2_rn(make_float2(kk.z, kk.w), vv, S[i + 1]);
+        for (int i = 0; i < 8; ++i) {
+            const float4 kk = *reinterpret_cast<const float4*>(&kp[l][row_block(half, i)]);
+            S[2 * i] = __ffma2_rn(make_float2(kk.x, kk.y), vv, S[2 * i]);
+            S[2 * i + 1] = __ffma2_rn(make_float2(kk.z, kk.w), vv, S[2 * i + 1]);
         }
     }
     float* out = chunk_state(a, b, h, c) + j;
 #pragma unroll
-    for (int i = 0; i < kHead / 2; ++i) {
-        out[(2 * i) * kHead] = S[i].x;
-        out[(2 * i + 1) * kHead] = S[i].y;
+    for (int i = 0; i < 8; ++i) {
+        const int m = row_block(half, i);
+        out[(m + 0) * kHead] = S[2 * i].x;
+        out[(m + 1) * kHead] = S[2 * i].y;
+        out[(m + 2) * kHead] = S[2 * i + 1].x;
+        out[(m + 3) * kHead] = S[2 * i + 1].y;
     }
 }
 
 constexpr int kScanThreads = 256;
-constexpr int kScanBlk = 8;  // chunk sums loaded before any is overwritten
+constexpr int kScanBlk = 16;  // chunk sums loaded before any is overwritten
 
 // 2: per state entry (b, h, m, j), in time order: the slot of chunk c receives S_start(c),
 // then S <- e^{-len_c w_m} S + U_c; the state after the last chunk is the final state.
@@ -137,19 +151,20 @@ __global__ void __launch_bounds__(kScanThreads) eagle_state_scan(EagleArgs a) {
 // 3: each chunk's tokens from its starting state: S <- diag(d) S + k_l v_l^T, y_l = r_l^T S
 constexpr size_t kOutSmem = 3 * (size_t)kTileBytes + 128;  // r, k, v tiles and the barrier
 
-__global__ void __launch_bounds__(kHead) eagle_chunk_out(EagleArgs a, const __grid_constant__ CUtensorMap tmr,
-                                                         const __grid_constant__ CUtensorMap tmk,
-                                                         const __grid_constant__ CUtensorMap tmv) {
+__global__ void __launch_bounds__(kChunkThreads) eagle_chunk_out(EagleArgs a, const __grid_constant__ CUtensorMap tmr,
+                                                                 const __grid_constant__ CUtensorMap tmk,
+                                                                 const __grid_constant__ CUtensorMap tmv) {
     extern __shared__ __align__(128) unsigned char smem[];
     float(*rs)[kHead] = reinterpret_cast<float(*)[kHead]>(smem);
     float(*ks)[kHead] = reinterpret_cast<float(*)[kHead]>(smem + kTileBytes);
     float(*vs)[kHead] = reinterpret_cast<float(*)[kHead]>(smem + 2 * kTileBytes);
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 3 * kTileBytes);
-    const int j = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, half = lane >> 4;
+    const int j = (tid >> 5) * 16 + (lane & 15);
     const int64_t c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int64_t t0 = c * kEL;
     const int len = (int)min64(kEL, a.T - t0);
-    if (j == 0) {
+    if (tid == 0) {
         mbar_init(bar, 1);
         fence_mbar_init();
         mbar_arrive_expect_tx(bar, 3 * kTileBytes);
@@ -157,33 +172,41 @@ __global__ void __launch_bounds__(kHead) eagle_chunk_out(EagleArgs a, const __gr
         tma_load_3d(&ks[0][0], &tmk, (int)(h * kHead), (int)t0, (int)b, bar);
         tma_load_3d(&vs[0][0], &tmv, (int)(h * kHead), (int)t0, (int)b, bar);
     }
-    // the starting state and the decays while the tiles are in flight
+    // this thread's half of the starting state and its decays while the tiles are in flight
     const float* st = chunk_state(a, b, h, c) + j;
-    float2 S[kHead / 2], d[kHead / 2];
+    const float* wh = a.w + h * kHead;
+    float2 S[16], d[16];
 #pragma unroll
-    for (int i = 0; i < kHead / 2; ++i) {
-        S[i] = make_float2(st[(2 * i) * kHead], st[(2 * i + 1) * kHead]);
-        d[i] = make_float2(ex2(-a.w[h * kHead + 2 * i] * kLog2e), ex2(-a.w[h * kHead + 2 * i + 1] * kLog2e));
+    for (int i = 0; i < 8; ++i) {
+        const int m = row_block(half, i);
+        S[2 * i] = make_float2(st[(m + 0) * kHead], st[(m + 1) * kHead]);
+        S[2 * i + 1] = make_float2(st[(m + 2) * kHead], st[(m + 3) * kHead]);
+        d[2 * i] = make_float2(ex2(-wh[m] * kLog2e), ex2(-wh[m + 1] * kLog2e));
+        d[2 * i + 1] = make_float2(ex2(-wh[m + 2] * kLog2e), ex2(-wh[m + 3] * kLog2e));
     }
     __syncthreads();  // the barrier is initialised
     wait_tiles(a, bar);
+    float* yrow = a.y + (b * a.T + t0) * a.C + h * kHead + j;
     for (int l = 0; l < len; ++l) {
         const float vj = vs[l][j];
         const float2 vv = make_float2(vj, vj);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                          make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int i = 0; i < kHead / 2; i += 2) {
-            const float4 kk = *reinterpret_cast<const float4*>(&ks[l][2 * i]);
-            const float4 rr = *reinterpret_cast<const float4*>(&rs[l][2 * i]);
-            S[i] = __ffma2_rn(d[i], S[i], __fmul2_rn(make_float2(kk.x, kk.y), vv));
-            S[i + 1] = __ffma2_rn(d[i + 1], S[i + 1], __fmul2_rn(make_float2(kk.z, kk.w), vv));
-            acc[(i / 2) & 3] = __ffma2_rn(make_float2(rr.x, rr.y), S[i], acc[(i / 2) & 3]);
-            acc[(i / 2) & 3] = __ffma2_rn(make_float2(rr.z, rr.w), S[i + 1], acc[(i / 2) & 3]);
+        for (int i = 0; i < 8; ++i) {
+            const int m = row_block(half, i);
+            const float4 kk = *reinterpret_cast<const float4*>(&ks[l][m]);
+            const float4 rr = *reinterpret_cast<const float4*>(&rs[l][m]);
+            S[2 * i] = __ffma2_rn(d[2 * i], S[2 * i], __fmul2_rn(make_float2(kk.x, kk.y), vv));
+            S[2 * i + 1] = __ffma2_rn(d[2 * i + 1], S[2 * i + 1], __fmul2_rn(make_float2(kk.z, kk.w), vv));
+            acc[i & 3] = __ffma2_rn(make_float2(rr.x, rr.y), S[2 * i], acc[i & 3]);
+            acc[i & 3] = __ffma2_rn(make_float2(rr.z, rr.w), S[2 * i + 1], acc[i & 3]);
         }
         const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
-        const float2 s = __fadd2_rn(s01, s23);
-        a.y[(b * a.T + t0 + l) * a.C + h * kHead + j] = s.x + s.y;
+        const float2 sp = __fadd2_rn(s01, s23);
+        float yv = sp.x + sp.y;
+        yv += __shfl_xor_sync(0xffffffffu, yv, 16);  // the other 32 key rows
+        if (half == 0) yrow[(int64_t)l * a.C] = yv;
     }
 }
 
@@ -262,10 +285,10 @@ cudaError_t launch_eagle_forward(int64_t B, int64_t T, int64_t C, const float* w
     a.spin_limit = kSpinLimitDefault;
     if (!a.dev_err) return cudaErrorInvalidValue;
     const dim3 grid((unsigned)a.P, (unsigned)H, (unsigned)B);
-    eagle_chunk_sum<<<grid, kHead, 0, s>>>(a, tmk, tmv);
+    eagle_chunk_sum<<<grid, kChunkThreads, 0, s>>>(a, tmk, tmv);
     const int64_t entries = B * H * kSS;
     eagle_state_scan<<<(unsigned)((entries + kScanThreads - 1) / kScanThreads), kScanThreads, 0, s>>>(a);
-    eagle_chunk_out<<<grid, kHead, kOutSmem, s>>>(a, tmr, tmk, tmv);
+    eagle_chunk_out<<<grid, kChunkThreads, kOutSmem, s>>>(a, tmr, tmk, tmv);
     return cudaGetLastError();
 }
 
