@@ -191,13 +191,26 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The largest of every rank's x (a time): one all-reduce of a scalar, on the GPU under
+    NCCL, on the host under gloo.  Every rank must call it, in the same order."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_set_seed(base_seed, rank, i):
+    """Seed of input set i on a rank: every rank draws its own batch (weak scaling)."""
+    return base_seed + 100 * rank + i
+
+
+def weak_scaling_value(world, n_elem_per_rank, ms_max):
+    """Whole-job throughput: the elements all ranks processed over the slowest rank's time."""
+    return world * n_elem_per_rank / (ms_max * 1e-3)
 
 
 # ----------------------------------------------------------------------------
@@ -539,7 +552,7 @@ def run_ours(args):
 
     spec = synth.FORWARD[WORKLOAD]
     n_elem = spec.B * spec.T * spec.C
-    sets = [ForwardSet(spec, spec.seed + 100 * rank + i, dev) for i in range(N_SETS)]
+    sets = [ForwardSet(spec, rank_set_seed(spec.seed, rank, i), dev) for i in range(N_SETS)]
     ws = wkv.Workspace(dev, wkv.workspace_size(spec.B, spec.T, spec.C))
     path = wkv.auto_path(spec.B, spec.T, spec.C)
 
@@ -587,7 +600,7 @@ def run_ours(args):
 
     ms_total = max_over_ranks(e0.elapsed_time(e1), world)
     ms_per_step = ms_total / K
-    value = world * n_elem / (ms_per_step * 1e-3)
+    value = weak_scaling_value(world, n_elem, ms_per_step)
     # The forward's own launch duration, right after the timed region: a graph of GRAPH_STEPS
     # back-to-back forwards on the rotating input sets, CUDA events around whole replays.  Event
     # nodes inside a graph add several microseconds to the launch they bracket, so the
@@ -621,7 +634,7 @@ def run_ours(args):
     if not args.no_e2e:
         ms_e2e, h2d, d2h = e2e_bench(torch, wkv, sets, ws, min(K, 240), dev)
         ms_e2e = max_over_ranks(ms_e2e, world)
-        e2e = {"value": world * n_elem / (ms_e2e * 1e-3), "unit": "elements/s", "ms_per_step": ms_e2e,
+        e2e = {"value": weak_scaling_value(world, n_elem, ms_e2e), "unit": "elements/s", "ms_per_step": ms_e2e,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     cpu = None
