@@ -415,8 +415,8 @@ def eagle_bench(torch, wkv, dev, peak, decode=True):
     out = {"eagle_forward": {"workload": spec.name, "launch_ms": f_ms, "alg_bytes_per_launch": alg,
                              "achieved_gbs": alg / (f_ms * 1e-3) / 1e9, "frac": alg / (f_ms * 1e-3) / 1e9 / peak,
                              "elements_per_s": n / (f_ms * 1e-3),
-                             "note": "three launches (chunk sums, scan over chunks, chunk outputs), fp32 on "
-                                     "CUDA cores"}}
+                             "note": "three launches: chunk sums (tcgen05 tf32 product, split operands), "
+                                     "scan over chunks, chunk outputs (CUDA cores)"}}
     del sets, ws
     if decode:
         N, L, Cd = 256, 32, 4096

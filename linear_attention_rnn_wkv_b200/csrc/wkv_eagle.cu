@@ -65,52 +65,161 @@ constexpr int kChunkThreads = 128;
 
 __device__ __forceinline__ int row_block(int half, int i) { return 32 * half + 4 * ((i + half) & 7); }
 
-// 1: U_c[m][j] = sum_{l < len} e^{-(len-1-l) w_m} k_l[m] v_l[j]
-__global__ void __launch_bounds__(kChunkThreads) eagle_chunk_sum(EagleArgs a, const __grid_constant__ CUtensorMap tmk,
-                                                                 const __grid_constant__ CUtensorMap tmv) {
-    __shared__ __align__(128) float kp[kEL][kHead];
-    __shared__ __align__(128) float vs[kEL][kHead];
-    __shared__ uint64_t bar;
-    const int tid = threadIdx.x, lane = tid & 31, half = lane >> 4;
-    const int j = (tid >> 5) * 16 + (lane & 15);
+// ---------------------------------------------------------------------------------------------
+// Tensor-core pieces (tcgen05, tf32).  An operand is 64 rows x 64 K fp32 stored K-major in
+// 8-row x 16-byte core matrices: element (row, k) at byte (row/8)*2048 + (k/4)*128 + (row%8)*16
+// + (k%4)*4, so the descriptor's leading offset (next 4 k) is 128 B and its stride offset (next
+// 8 rows) 2048 B; an MMA consumes K = 8 (two core-matrix columns), the next one starts 256 B on.
+// fp32 accuracy from split operands: x = hi + lo with hi = x cut to tf32 (its low 13 mantissa
+// bits cleared, exact) and lo = x - hi (exact, |lo| < 2^-10 |x|); a product is taken as
+// hi*hi + hi*lo + lo*hi, the dropped lo*lo below 2^-20 of it.
+// ---------------------------------------------------------------------------------------------
+constexpr uint32_t kOpBytes = 64 * 64 * sizeof(float);
+
+__device__ __forceinline__ int op_index(int row, int k) { return (row >> 3) * 512 + (k >> 2) * 32 + (row & 7) * 4 + (k & 3); }
+
+__device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
+    hi = __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
+    lo = x - hi;
+}
+
+// shared-memory matrix descriptor: start, leading offset 128 B, stride offset 2048 B, version 1,
+// no swizzle
+__device__ __forceinline__ uint64_t op_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(128u >> 4) << 16) | ((uint64_t)(2048u >> 4) << 32) |
+           ((uint64_t)1 << 46);
+}
+
+// instruction descriptor: fp32 accumulate, tf32 A and B, both K-major, M x N
+__host__ __device__ constexpr uint32_t tf32_idesc(int M, int N) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(ad), "l"(bd), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tm_alloc(uint32_t* slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tm_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tm_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tm_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 16 consecutive fp32 columns of this warp's 32 TMEM lanes
+__device__ __forceinline__ void tm_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15])::"memory");
+}
+
+// 1: U_c = (K ⊙ D')^T V as one tensor-core product per (chunk, head, sequence):
+//    U_c[m][j] = sum_{l < len} (k_l[m] e^{-(len-1-l) w_m}) v_l[j], M = 64 key rows, N = 64 value
+//    columns, K = the chunk's 64 tokens (tokens past T enter as zeros).  The threads write both
+//    operands transposed (key and value channel as the row, token as K) and split; one thread
+//    issues 8 K-steps x 3 MMAs; the accumulator (M = 64: rows 16q..16q+15 in lanes 32q..32q+15)
+//    is read back by the warp of each quadrant.
+constexpr size_t kSumSmem = 4 * (size_t)kOpBytes + 64;
+
+__global__ void __launch_bounds__(kChunkThreads) eagle_chunk_sum(EagleArgs a) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    float* Ahi = reinterpret_cast<float*>(smem);
+    float* Alo = Ahi + 4096;
+    float* Bhi = Alo + 4096;
+    float* Blo = Bhi + 4096;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 4 * kOpBytes);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + 4 * kOpBytes + 8);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int64_t t0 = c * kEL;
     const int len = (int)min64(kEL, a.T - t0);
+    const int64_t row0 = (b * a.T + t0) * a.C + h * kHead;
+    if (warp == 0) tm_alloc(tslot, 64);
     if (tid == 0) {
-        mbar_init(&bar, 1);
+        mbar_init(bar, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(&bar, 2 * kTileBytes);
-        tma_load_3d(&kp[0][0], &tmk, (int)(h * kHead), (int)t0, (int)b, &bar);
-        tma_load_3d(&vs[0][0], &tmv, (int)(h * kHead), (int)t0, (int)b, &bar);
     }
-    const int sm_m = tid & 63, sm_l0 = tid >> 6;  // the decay scaling: key row sm_m, every other token
-    const float w2 = a.w[h * kHead + sm_m] * kLog2e;
-    __syncthreads();  // the barrier is initialised
-    wait_tiles(a, &bar);
-    for (int l = sm_l0; l < len; l += 2) kp[l][sm_m] *= ex2(-(float)(len - 1 - l) * w2);
-    __syncthreads();
-    float2 S[16];
+    const int ch = tid & 63, t_first = tid >> 6;  // channel (A's / B's row); tokens t_first + 2i
+    const float w2 = a.w[h * kHead + ch] * kLog2e;
+    constexpr int kPer = kEL / 2;  // tokens per thread
+    float kx[kPer], vx[kPer];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) S[i] = make_float2(0.f, 0.f);
-    for (int l = 0; l < len; ++l) {
-        const float vj = vs[l][j];
-        const float2 vv = make_float2(vj, vj);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float4 kk = *reinterpret_cast<const float4*>(&kp[l][row_block(half, i)]);
-            S[2 * i] = __ffma2_rn(make_float2(kk.x, kk.y), vv, S[2 * i]);
-            S[2 * i + 1] = __ffma2_rn(make_float2(kk.z, kk.w), vv, S[2 * i + 1]);
+    for (int i = 0; i < kPer; ++i) {  // every load issued before any is used
+        const int t = t_first + 2 * i;
+        kx[i] = 0.f;
+        vx[i] = 0.f;
+        if (t < len) {
+            kx[i] = a.k[row0 + (int64_t)t * a.C + ch];
+            vx[i] = a.v[row0 + (int64_t)t * a.C + ch];
         }
     }
-    float* out = chunk_state(a, b, h, c) + j;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int m = row_block(half, i);
-        out[(m + 0) * kHead] = S[2 * i].x;
-        out[(m + 1) * kHead] = S[2 * i].y;
-        out[(m + 2) * kHead] = S[2 * i + 1].x;
-        out[(m + 3) * kHead] = S[2 * i + 1].y;
+    for (int i = 0; i < kPer; ++i) {
+        const int t = t_first + 2 * i;
+        const int o = op_index(ch, t);
+        // past the sequence the token is zero and so is its weight (2^{+n w} there could be inf)
+        const float f = t < len ? ex2(-(float)(len - 1 - t) * w2) : 0.f;
+        float hi, lo;
+        split_tf32(kx[i] * f, hi, lo);
+        Ahi[o] = hi;
+        Alo[o] = lo;
+        split_tf32(vx[i], hi, lo);
+        Bhi[o] = hi;
+        Blo[o] = lo;
     }
+    fence_proxy_async_smem();  // the operands, written by the threads, are read by the tensor core
+    tm_fence_before();
+    __syncthreads();
+    tm_fence_after();
+    const uint32_t tmem = *tslot;
+    if (tid == 0) {
+        constexpr uint32_t id = tf32_idesc(64, 64);
+        const uint32_t ah = smem_u32(Ahi), al = smem_u32(Alo), bh = smem_u32(Bhi), bl = smem_u32(Blo);
+#pragma unroll
+        for (uint32_t st = 0; st < kEL / 8; ++st) {
+            const uint32_t off = 256u * st;
+            mma_tf32(tmem, op_desc(ah + off), op_desc(bh + off), id, st);
+            mma_tf32(tmem, op_desc(ah + off), op_desc(bl + off), id, 1);
+            mma_tf32(tmem, op_desc(al + off), op_desc(bh + off), id, 1);
+        }
+        mma_commit(bar);
+    }
+    if (!mbar_wait(bar, 0, a.spin_limit) && lane == 0) atomicCAS(a.dev_err, kDevOk, (uint32_t)kDevTimeoutCopy);
+    tm_fence_after();
+    float* out = chunk_state(a, b, h, c) + (int64_t)(16 * warp + lane) * kHead;
+#pragma unroll
+    for (int cb = 0; cb < kHead; cb += 16) {
+        uint32_t r[16];
+        tm_ld16(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)cb, r);
+        if (lane < 16) {
+#pragma unroll
+            for (int q = 0; q < 16; q += 4)
+                *reinterpret_cast<float4*>(out + cb + q) = make_float4(__uint_as_float(r[q]), __uint_as_float(r[q + 1]),
+                                                                       __uint_as_float(r[q + 2]), __uint_as_float(r[q + 3]));
+        }
+    }
+    tm_fence_before();
+    __syncthreads();
+    if (warp == 0) tm_dealloc(tmem, 64);
 }
 
 constexpr int kScanThreads = 256;
@@ -154,7 +263,7 @@ constexpr size_t kOutSmem = 3 * (size_t)kTileBytes + 128;  // r, k, v tiles and 
 __global__ void __launch_bounds__(kChunkThreads) eagle_chunk_out(EagleArgs a, const __grid_constant__ CUtensorMap tmr,
                                                                  const __grid_constant__ CUtensorMap tmk,
                                                                  const __grid_constant__ CUtensorMap tmv) {
-    extern __shared__ __align__(128) unsigned char smem[];
+    extern __shared__ __align__(1024) unsigned char smem[];
     float(*rs)[kHead] = reinterpret_cast<float(*)[kHead]>(smem);
     float(*ks)[kHead] = reinterpret_cast<float(*)[kHead]>(smem + kTileBytes);
     float(*vs)[kHead] = reinterpret_cast<float(*)[kHead]>(smem + 2 * kTileBytes);
@@ -265,6 +374,8 @@ cudaError_t launch_eagle_forward(int64_t B, int64_t T, int64_t C, const float* w
     if (dev >= 64 || !(attr_done & (1ull << dev))) {
         e = cudaFuncSetAttribute(eagle_chunk_out, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kOutSmem);
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(eagle_chunk_sum, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSumSmem);
+        if (e != cudaSuccess) return e;
         if (dev < 64) attr_done |= 1ull << dev;
     }
     EagleArgs a;
@@ -285,7 +396,7 @@ cudaError_t launch_eagle_forward(int64_t B, int64_t T, int64_t C, const float* w
     a.spin_limit = kSpinLimitDefault;
     if (!a.dev_err) return cudaErrorInvalidValue;
     const dim3 grid((unsigned)a.P, (unsigned)H, (unsigned)B);
-    eagle_chunk_sum<<<grid, kChunkThreads, 0, s>>>(a, tmk, tmv);
+    eagle_chunk_sum<<<grid, kChunkThreads, kSumSmem, s>>>(a);
     const int64_t entries = B * H * kSS;
     eagle_state_scan<<<(unsigned)((entries + kScanThreads - 1) / kScanThreads), kScanThreads, 0, s>>>(a);
     eagle_chunk_out<<<grid, kChunkThreads, kOutSmem, s>>>(a, tmr, tmk, tmv);
