@@ -92,6 +92,15 @@ def test_binding_refuses_cpu_tensors():
         wkv.wkv_forward(torch.ones(4), torch.zeros(4), k, k)
     with pytest.raises(TypeError):
         wkv.token_shift_mix(torch.ones(4), k)
+    with pytest.raises(TypeError):
+        wkv.wkv_backward(torch.ones(4), torch.zeros(4), k, k, k)
+    with pytest.raises(TypeError):
+        wkv.token_shift_mix3(torch.ones(4), torch.ones(4), torch.ones(4), k)
+    k64 = torch.zeros(1, 4, 64)
+    with pytest.raises(TypeError):
+        wkv.eagle_forward(torch.ones(64), k64, k64, k64)
+    with pytest.raises(TypeError):
+        wkv.eagle_decode_step(torch.ones(1, 64), k64, k64, k64, torch.zeros(1, 4, 1, 64, 64))
 
 
 def test_backward_validation_without_launch():
