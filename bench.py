@@ -231,6 +231,33 @@ def time_oracle(spec, inputs, min_seconds, min_passes):
     return n * passes / el, passes, el, oracle.num_threads()
 
 
+def time_oracle_extras(spec, inputs, seconds=2.0):
+    """The oracle's two other timings: the same recurrence on one host thread (a bounded sample
+    of whole prefills of the workload), and the direct O(T^2) form on the 1x64x64 workload."""
+    import oracle
+    import synth
+    cores = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        rate1, passes1, el1, _ = time_oracle(spec, inputs, seconds, 1)
+    finally:
+        oracle.set_num_threads(cores)
+    small = synth.FORWARD["fwd_64x64"]
+    w, u, k, v = synth.forward_inputs(small)
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        oracle.wkv_direct(w, u, k, v)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= seconds / 4 and passes >= 3:
+            break
+    n_small = small.B * small.T * small.C
+    return {"single_thread": {"value": rate1, "cores": 1,
+                              "sample": f"{passes1} passes of the whole prefill ({el1:.1f} s)"},
+            "direct_64x64": {"value": n_small * passes / el, "unit": "elements/s", "cores": cores,
+                             "sample": f"{passes} passes of eq. 1 as written, O(T^2), on 1x64x64"}}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -643,6 +670,7 @@ def run_ours(args):
         cpu = {"value": rate, "unit": "elements/s", "cores": cores, "kind": "oracle",
                "sample": f"{passes} passes of the whole {spec.B}x{spec.T}x{spec.C} prefill through the fp64 "
                          f"stabilised recurrence ({el:.1f} s)"}
+        cpu.update(time_oracle_extras(spec, synth.forward_inputs(spec)))
 
     if rank == 0:
         line = {

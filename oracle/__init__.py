@@ -80,6 +80,8 @@ def load(path: str):
               L.oracle_wkv_backward_direct, L.oracle_eagle_recurrent, L.oracle_eagle_direct):
         f.restype = None
     L.oracle_num_threads.restype = ctypes.c_int
+    L.oracle_set_num_threads.argtypes = [ctypes.c_int]
+    L.oracle_set_num_threads.restype = None
     return L
 
 
@@ -95,6 +97,11 @@ def lib():
 
 def num_threads() -> int:
     return int(lib().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's parallel loops (independent channels: results are unchanged)."""
+    lib().oracle_set_num_threads(int(n))
 
 
 def _f64(a):

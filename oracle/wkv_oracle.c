@@ -70,6 +70,17 @@ int oracle_num_threads(void)
 #endif
 }
 
+/* Threads for the parallel loops that follow (timing only: every loop distributes independent
+ * channels, so the results do not depend on it). */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /*
  * Direct evaluation of the wkv_t equation ([MATH] "The WKV operator: attention
  * with a fixed decay"; [WIKI] eq. 1), O(T^2) per channel, no stabilisation.
