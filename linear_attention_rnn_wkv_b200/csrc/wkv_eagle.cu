@@ -8,18 +8,17 @@
 //
 // Prefill, time-parallel in chunks of kEL tokens (three launches):
 //   1 eagle_chunk_sum   each chunk's own contribution to the state at its end, from zero:
-//                       U_c = sum_l diag(d)^{len-1-l} k_l v_l^T (decayed keys formed once per
-//                       chunk in shared memory, then one fused multiply-add per state entry
-//                       and token);
+//                       U_c = sum_l diag(d)^{len-1-l} k_l v_l^T = (K ⊙ D')^T V, one tensor-core
+//                       product (tcgen05, tf32 operands split hi + lo for fp32-level error);
 //   2 eagle_state_scan  per state entry, the chunks in time order: S_start(c) and, after the
 //                       last chunk, the final state (S <- d^len S + U_c);
 //   3 eagle_chunk_out   each chunk's tokens again from its S_start: update, then read-out.
 // Decode (eagle_decode): one token of the recurrence per (row, head), the state read and
 // written once (section "O(N) Inference Characteristics": one matrix-vector product per token).
 //
-// Arithmetic is fp32 on the CUDA cores (packed f32x2 where a lane holds two key rows); the
-// decay powers are single exponentials 2^{-n w log2 e} of exact integer n, so no rounding
-// accumulates in them.
+// The scan, the outputs and the decode are fp32 on the CUDA cores (packed f32x2 where a lane
+// holds two key rows); the decay powers are single exponentials 2^{-n w log2 e} of exact
+// integer n, so no rounding accumulates in them.
 #include <cuda_runtime.h>
 
 #include "wkv_device.cuh"
