@@ -75,3 +75,57 @@ def test_eagle_resume_anywhere(T, N, cut, seed):
     y2, _, st2 = oracle.eagle_recurrent(w, r[:, c:], k[:, c:], v[:, c:], N=N, state_in=st1)
     assert np.all(np.abs(np.concatenate([y1, y2], axis=1) - y) <= 1e-13 * s + 1e-300)
     assert np.allclose(st2, st_all, rtol=1e-12, atol=1e-12)
+
+
+@settings(max_examples=20, deadline=None, derandomize=True)
+@given(B=st.integers(1, 2), T=st.integers(1, 6), C=st.integers(1, 3), seed=st.integers(0, 2**31 - 1))
+def test_backward_matches_finite_differences(B, T, C, seed):
+    """Every gradient of L = sum(gy * y) against central differences of the direct forward."""
+    g = np.random.default_rng(seed)
+    w = np.exp(g.uniform(-3, 1, C))
+    u = g.normal(0, 0.5, C)
+    k = g.normal(0, 1, (B, T, C))
+    v = g.normal(0, 1, (B, T, C))
+    gy = g.normal(0, 1, (B, T, C))
+    gk, gv, gw, gu, (sk, sv, sw, su) = oracle.wkv_backward(w, u, k, v, gy)
+
+    def loss(w_, u_, k_, v_):
+        return float((oracle.wkv_direct(w_, u_, k_, v_)[0] * gy).sum())
+
+    h = 1e-6
+    for arr, grad, scale, pos in ((k, gk, sk, 2), (v, gv, sv, 3), (w, gw, sw, 0), (u, gu, su, 1)):
+        for idx in np.ndindex(arr.shape):
+            plus, minus = arr.copy(), arr.copy()
+            plus[idx] += h
+            minus[idx] -= h
+            args_p = [w, u, k, v]
+            args_m = [w, u, k, v]
+            args_p[pos], args_m[pos] = plus, minus
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(fd - grad[idx]) <= 1e-6 * (scale[idx] + 1e-9)
+
+
+@SETTINGS
+@given(n=st.integers(1, 64), seed=st.integers(0, 2**31 - 1))
+def test_gate_symmetry(n, seed):
+    """sigma(r) + sigma(-r) = 1: gate(r, x) + gate(-r, x) = x."""
+    g = np.random.default_rng(seed)
+    r = g.normal(0, 4, n)
+    x = g.normal(0, 1, n)
+    assert np.allclose(oracle.gate(r, x) + oracle.gate(-r, x), x, rtol=1e-14, atol=1e-15)
+
+
+@SETTINGS
+@given(B=st.integers(1, 2), T=st.integers(1, 8), C=st.integers(1, 5), seed=st.integers(0, 2**31 - 1))
+def test_token_shift3_is_three_lerps(B, T, C, seed):
+    """The three-mu shift is the one-mu shift with each projection's mu, and a lerp: linear in
+    mu with the current token at mu = 1."""
+    g = np.random.default_rng(seed)
+    mus = [g.uniform(0, 1, C) for _ in range(3)]
+    x = g.normal(0, 1, (B, T, C))
+    xl = g.normal(0, 1, (B, C))
+    outs = oracle.token_shift3(*mus, x, xl)
+    for o, mu in zip(outs, mus):
+        assert np.array_equal(o, oracle.token_shift(mu, x, xl))
+    ones = oracle.token_shift(np.ones(C), x, xl)
+    assert np.array_equal(ones, x)
