@@ -268,8 +268,9 @@ wkv_status wkv_forward_chunked_noalloc(int64_t B, int64_t T, int64_t C, wkv_dtyp
  *   workspace      caller-owned device scratch, ws_bytes >= eagle_forward_workspace_size()
  * C must be a multiple of 64 (else WKV_ERR_UNSUPPORTED), C/64 and B at most 65535.  T = 0
  * writes state_out only (state_in, or zeros).  Time-parallel over 64-token chunks: each
- * chunk's own state contribution, a scan over the chunks per state entry, then each chunk's
- * outputs from its starting state.  Status codes as wkv_forward.
+ * chunk's own state contribution (a tensor-core product with operands split into two tf32
+ * parts, for fp32-level error), a scan over the chunks per state entry, then each chunk's
+ * outputs from its starting state (fp32).  Status codes as wkv_forward.
  */
 wkv_status eagle_forward(int64_t B, int64_t T, int64_t C, const float* w, const float* r, const float* k,
                          const float* v, const float* state_in, float* y, float* state_out, void* workspace,
