@@ -441,6 +441,39 @@ def pin_backward_closed_forms(L):
     assert np.allclose(gv.sum(axis=1), gy.sum(axis=1), rtol=1e-12, atol=1e-12)
 
 
+def pin_backward_magnitude_scales(L):
+    """The backward's magnitude scales (each gradient's terms added up with |gy| for gy and
+    |v| + |y| for v - y) where every sign is fixed: with gy >= 0 and v >= 0 (so y >= 0, a convex
+    combination) they follow from the gradients and the pinned forward alone.  y_t is linear in
+    v (y_t = sum_i beta_{t,i} v_i / D_t with D_t independent of v), so running the direct forward
+    on a value sequence zeroed outside a set of tokens picks out those tokens' weighted values:
+      sv = gv,   sk = 2 v gv - gk,
+      su = 2 sum_t gy_t y_t(v kept at token t only) - gu,
+      sw = 2 sum_t gy_t [(t - 1) y_t(v kept before t) - y_t(i v_i kept before t)] + gw."""
+    for seed, (B, T, C) in ((45, (1, 7, 3)), (46, (2, 5, 2))):
+        w, u, k, v = _rand_case(seed, B, T, C)
+        v = np.abs(v) + 0.1
+        gy = np.abs(_rng(seed + 100).normal(0, 1, k.shape)) + 0.05
+        gk, gv, gw, gu, (sk, sv, sw, su) = oracle.wkv_backward(w, u, k, v, gy, L=L)
+        assert np.allclose(sv, gv, rtol=1e-13, atol=0)
+        assert np.allclose(sk, 2 * v * gv - gk, rtol=1e-11, atol=1e-14 * np.max(sk))
+        cur = np.zeros(C)
+        past = np.zeros(C)
+        idx = np.arange(T, dtype=np.float64)[None, :, None]
+        for t in range(T):
+            only = np.zeros_like(v)
+            only[:, t] = v[:, t]
+            cur += (gy[:, t] * oracle.wkv_direct(w, u, k, only, L=L)[0][:, t]).sum(axis=0)
+            if t > 0:
+                before = v.copy()
+                before[:, t:] = 0.0
+                yb = oracle.wkv_direct(w, u, k, before, L=L)[0][:, t]
+                yi = oracle.wkv_direct(w, u, k, idx * before, L=L)[0][:, t]
+                past += (gy[:, t] * ((t - 1) * yb - yi)).sum(axis=0)
+        assert np.allclose(su, 2 * cur - gu, rtol=1e-11, atol=0)
+        assert np.allclose(sw, 2 * past + gw, rtol=1e-10, atol=1e-13 * np.max(sw))
+
+
 # ----------------------------------------------------------------------------
 # Eagle (RWKV-5) matrix-state WKV ("RWKV (Attention-RNN Hybrid)", section
 # "Versions: RWKV-4 -> Eagle -> Finch"): S_t = diag(d) S_{t-1} + k_t v_t^T,
@@ -556,6 +589,22 @@ def pin_eagle_bilinear_and_heads(L):
     assert not np.allclose(y3[:, :, N:2 * N], y1[:, :, N:2 * N])
 
 
+def pin_eagle_magnitude_scale(L):
+    """Eagle's magnitude scale s is the read-out of |r|, |k|, |v| and |S_in|: it equals the
+    (pinned) direct sum evaluated on those absolute values, and with non-negative inputs it is
+    y itself, bit for bit (the same products in the same order)."""
+    B, T, H, N = 2, 10, 2, 4
+    w, r, k, v = _eagle_case(56, B, T, H, N)
+    S0 = _rng(156).normal(0, 1, (B, H, N, N))
+    for st_in in (None, S0):
+        _, s, _ = oracle.eagle_recurrent(w, r, k, v, N=N, state_in=st_in, L=L)
+        sd = oracle.eagle_direct(w, np.abs(r), np.abs(k), np.abs(v), N=N,
+                                 state_in=None if st_in is None else np.abs(st_in), L=L)
+        assert np.allclose(s, sd, rtol=1e-12, atol=0)
+    y, s, _ = oracle.eagle_recurrent(w, np.abs(r), np.abs(k), np.abs(v), N=N, state_in=np.abs(S0), L=L)
+    assert np.array_equal(s, y)
+
+
 ALL_PINS = [
     pin_worked_example,
     pin_routes_agree,
@@ -577,10 +626,12 @@ ALL_PINS = [
     pin_token_shift3,
     pin_backward_finite_differences,
     pin_backward_closed_forms,
+    pin_backward_magnitude_scales,
     pin_eagle_hand_example,
     pin_eagle_linear_attention,
     pin_eagle_no_memory,
     pin_eagle_one_token_from_state,
     pin_eagle_routes_and_split,
     pin_eagle_bilinear_and_heads,
+    pin_eagle_magnitude_scale,
 ]

@@ -58,6 +58,18 @@ MUTANTS = {
     "eagle_direct_decay_off_by_one": ("exp(-(double)(t - i) * w[h * N + m])", "exp(-(double)(t - 1 - i) * w[h * N + m])"),
     "eagle_direct_state_in_undecayed": ("exp(-(double)(t + 1) * w[h * N + m]) * state_in",
                                         "exp(-(double)t * w[h * N + m]) * state_in"),
+    "eagle_scale_inflated": ("acc_s += fabs(rm) * Sa[m * N + j];", "acc_s += 1000.0 * fabs(rm) * Sa[m * N + j];"),
+    "eagle_scale_state_signed": ("Sa[m * N + j] = d * Sa[m * N + j] + fabs(km) * fabs(vj);",
+                                 "Sa[m * N + j] = d * Sa[m * N + j] + km * vj;"),
+    "backward_sk_inflated": ("if (sk) sk[at3(b, i, c, T, C)] += gm * beta * (fabs(vi) + fabs(yt));",
+                             "if (sk) sk[at3(b, i, c, T, C)] += 1000.0 * gm * beta * (fabs(vi) + fabs(yt));"),
+    "backward_sv_inflated": ("if (sv) sv[at3(b, t, c, T, C)] += gm * alpha;",
+                             "if (sv) sv[at3(b, t, c, T, C)] += 1000.0 * gm * alpha;"),
+    "backward_sw_inflated": ("swc += gm * (double)(t - 1 - i) * beta * (fabs(vi) + fabs(yt));",
+                             "swc += 1000.0 * gm * (double)(t - 1 - i) * beta * (fabs(vi) + fabs(yt));"),
+    "backward_su_inflated": ("suc += gm * alpha * (fabs(vt) + fabs(yt));", "suc += 1000.0 * gm * alpha * (fabs(vt) + fabs(yt));"),
+    "backward_scale_difference": ("if (sk) sk[at3(b, i, c, T, C)] += gm * beta * (fabs(vi) + fabs(yt));",
+                                  "if (sk) sk[at3(b, i, c, T, C)] += gm * beta * fabs(vi - yt);"),
 }
 
 
