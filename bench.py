@@ -3,23 +3,27 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Workload (one step = one pass of the whole hot path over one batch): prefill of
-B=8 sequences x T=1024 tokens x C=768 channels in fp32 (keys N(0,3) with 1% set to
-+40, values N(0,1), w = exp(U(-5,1)), u ~ N(0,0.5)) through wkv_forward, which also
-returns the final state, then one fused decode step (token shift + WKV update) that
-continues all 8 sequences from that state.  Metric: WKV forward B*T*C elements/s.
-The same JSON line also carries the decode throughput of 256 sessions x 32 layers x
-4096 channels (tokens/s, a token being one session's step through all 32 layers).
+Headline workload (one step = one pass of the whole hot path over one batch): the prefill
+of the largest forward configuration, B=1 sequence x T=16384 tokens x C=4096 channels in
+fp32 (keys N(0,3) with 1% set to +40, values N(0,1), w = exp(U(-5,1)), u ~ N(0,0.5))
+through wkv_forward, which also returns the final state, then one fused decode step (token
+shift + WKV update) that continues the sequence from that state.  Metric: WKV forward
+B*T*C elements/s.
 
-Timing: W untimed warm-up steps, then exactly K steps replayed from CUDA graphs,
-bracketed by a barrier and a device synchronise, timed with CUDA events; the max over
-ranks is taken.  Six input sets (453 MB, over three times the 126 MB L2) rotate
-between steps so no step finds its inputs in L2.  The timed graphs carry no event nodes.
-The forward kernel's own launch duration (for the roofline) is timed right after the timed
-region: a graph of back-to-back forwards on the same rotating inputs, events around whole
-replays.
+Timing: W untimed warm-up steps, then the K-step CUDA graph is replayed R times; each
+replay is exactly K steps, bracketed by a barrier and a device synchronise and timed with
+CUDA events on the launching stream; the median replay gives ms_per_step, and the max over
+ranks is taken.  The inputs of one step (805 MB) are over six times the 126 MB L2, so no
+step finds its inputs in L2.  The forward kernel's own launch duration (for the roofline)
+is timed right after: a graph of back-to-back forwards, events around whole replays.
 
---impl reference times the fp64 CPU oracle (plain C, OpenMP) on this workload.
+The same JSON line carries one row per benchmark configuration ("configs": the four
+forward workloads and the 256 x 32 x 4096 decode step), each timed the same way on
+rotating input sets larger than twice the L2, with its algorithmic bandwidth, its fraction
+of the measured copy peak and the fp64 oracle's rate on the host cores; and the next rows
+(gated forward, three-mu token shift, backward, Eagle prefill and decode).
+
+--impl reference times the fp64 CPU oracle (plain C, OpenMP) on the headline workload.
 """
 from __future__ import annotations
 
@@ -37,31 +41,38 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = "fwd_8x1024x768"
+WORKLOAD = "fwd_1x16384x4096"
 METRIC = "WKV forward B*T*C elements/s"
-N_SETS = 6
+L2_BYTES = 126e6
 GRAPH_STEPS = 60
+REPLAYS = 9
+REF_CHANNELS = 512                                # channels per step of the CPU reference arm
 ALG_BYTES_PER_ELEM = {"f32": 12, "bf16": 6}     # k + v read, y written, per element
 DECODE_ALG_BYTES_PER_ELEM = 48                    # x_t, x_prev, k, v, a, b, p in; a, b, p, y, xbar out
+FORWARD_CONFIGS = ("fwd_64x64", "fwd_8x1024x768", "fwd_4x4096x2048_bf16", "fwd_1x16384x4096")
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=6000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration rows")
+    ap.add_argument("--no-next", action="store_true", help="skip the next rows (gated, shift3, backward, Eagle)")
     ap.add_argument("--profile-forward", metavar="WORKLOAD", default=None,
                     help="only run 2 + 3 eager forward launches of a forward workload (e.g. fwd_1x16384x4096) "
                          "and exit: a short, self-contained command to capture under a profiler")
+    ap.add_argument("--profile-step", action="store_true",
+                    help="only run 3 + 2 eager headline steps (forward with state + fused decode) and exit")
     ap.add_argument("--profile-eagle", action="store_true",
                     help="only run 2 + 3 eager Eagle prefills on eagle_8x1024x768 and exit, for a profiler")
     ap.add_argument("--profile-backward", metavar="WORKLOAD", default=None,
-                    help="only run 2 + 3 eager backward calls (five launches each) on a forward workload's shape "
-                         "(fp32) and exit, for a profiler")
+                    help="only run 2 + 3 eager backward calls on a forward workload's shape (fp32) and exit, "
+                         "for a profiler")
     return ap.parse_args()
 
 
@@ -156,17 +167,17 @@ def kernel_source_digest():
 
 def profiled_traffic(workload):
     """DRAM bytes per launch of the forward kernel from the committed ncu summary, if it
-    was taken on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", f"tmem_kernel_{workload}.md")
+    was taken on the current kernel source (else None), and the file it came from."""
+    rel = os.path.join("profiles", f"tmem_kernel_{workload}.md")
     try:
-        txt = open(path).read()
+        txt = open(os.path.join(ROOT, rel)).read()
     except OSError:
-        return None
+        return None, None
     m_src = re.search(r"kernel_source_digest:\s*([0-9a-f]+)", txt)
     m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
     if not m_src or not m_tr or m_src.group(1) != kernel_source_digest():
-        return None
-    return float(m_tr.group(1))
+        return None, None
+    return float(m_tr.group(1)), rel
 
 
 def dist_setup(n_gpus):
@@ -213,8 +224,14 @@ def weak_scaling_value(world, n_elem_per_rank, ms_max):
     return world * n_elem_per_rank / (ms_max * 1e-3)
 
 
+def sets_for(bytes_per_set, floor=1, cap=8):
+    """Rotating input sets whose total exceeds twice the L2."""
+    n = int(-(-2 * L2_BYTES // max(bytes_per_set, 1))) + 1
+    return max(floor, min(cap, n))
+
+
 # ----------------------------------------------------------------------------
-# CPU oracle timing (cpu_baseline leg and --impl reference)
+# CPU oracle timing (cpu_baseline legs and --impl reference)
 # ----------------------------------------------------------------------------
 
 def time_oracle(spec, inputs, min_seconds, min_passes):
@@ -229,6 +246,43 @@ def time_oracle(spec, inputs, min_seconds, min_passes):
             break
     n = spec.B * spec.T * spec.C
     return n * passes / el, passes, el, oracle.num_threads()
+
+
+def oracle_row(spec, seconds=2.0):
+    """The fp64 oracle's stabilised recurrence on one forward workload, on the host cores,
+    whole prefills of the workload for about `seconds` (at least one)."""
+    import synth
+    rate, passes, el, cores = time_oracle(spec, synth.forward_inputs(spec), seconds, 1)
+    return {"value": rate, "unit": "elements/s", "cores": cores, "kind": "oracle",
+            "sample": f"{passes} passes of the whole {spec.B}x{spec.T}x{spec.C} prefill through the fp64 "
+                      f"stabilised recurrence ({el:.1f} s)"}
+
+
+def oracle_decode_row(seconds=2.0, n_sample=32):
+    """The fp64 oracle's decode step (one token through the stabilised recurrence, token shift
+    included) on the first n_sample sessions of the 256 x 32 x 4096 decode workload."""
+    import numpy as np
+    import oracle
+    import synth
+    spec = synth.DECODE["decode_256x32x4096"]
+    mu, w, u = synth.decode_params(spec)
+    x_t, k, v = (np.ascontiguousarray(a[:n_sample]) for a in synth.decode_step_inputs(spec, 0))
+    x_p = np.ascontiguousarray(synth.warmup_last_x(spec)[:n_sample])
+    st = np.ascontiguousarray(synth.filler_state(spec)[:, :n_sample], dtype=np.float64)
+    sa = np.abs(st[0])
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        oracle.decode_token_shift(mu, x_t, x_p)
+        oracle.decode_step(w, u, k, v, st, sa)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= seconds and passes >= 1:
+            break
+    rows = n_sample * spec.L * spec.C
+    return {"value": n_sample * passes / el, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "row_channels_per_s": rows * passes / el,
+            "sample": f"{passes} fp64 decode steps (token shift + stabilised update) of {n_sample} of the 256 "
+                      f"sessions x 32 layers x 4096 channels ({el:.1f} s)"}
 
 
 def time_oracle_extras(spec, inputs, seconds=2.0):
@@ -259,16 +313,23 @@ def time_oracle_extras(spec, inputs, seconds=2.0):
 
 
 def run_reference(args):
+    """The oracle as it stands on the host cores, on the headline workload's distributions:
+    each step is a bounded sample of the prefill, the first REF_CHANNELS channels over all T
+    tokens (the channels are independent, so the rate does not depend on which)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    import numpy as np
     import synth
-    spec = synth.FORWARD[WORKLOAD]
-    inputs = synth.forward_inputs(spec)
     import oracle
+    spec = synth.FORWARD[WORKLOAD]
+    w, u, k, v = synth.forward_inputs(spec)
+    c = REF_CHANNELS
+    inputs = (w[:c].copy(), u[:c].copy(), np.ascontiguousarray(k[:, :, :c]), np.ascontiguousarray(v[:, :, :c]))
+    del k, v
     for _ in range(max(args.warmup, 0)):
         oracle.wkv_recurrent(*inputs)
-    n = spec.B * spec.T * spec.C
+    n = spec.B * spec.T * c
     t0 = time.perf_counter()
     for _ in range(args.steps):
         oracle.wkv_recurrent(*inputs)
@@ -280,8 +341,8 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "B": spec.B, "T": spec.T, "C": spec.C, "io": "f32"},
         "cpu_baseline": {"value": value, "unit": "elements/s", "cores": oracle.num_threads(), "kind": "oracle",
-                         "sample": f"each step: the whole {spec.B}x{spec.T}x{spec.C} prefill through the fp64 "
-                                   f"stabilised recurrence (no decode step)"},
+                         "sample": f"each step: channels 0..{c - 1} of the {spec.B}x{spec.T}x{spec.C} prefill "
+                                   f"({n} elements) through the fp64 stabilised recurrence (no decode step)"},
         "e2e": {"value": value, "unit": "elements/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -292,86 +353,183 @@ def run_reference(args):
 # ----------------------------------------------------------------------------
 
 class ForwardSet:
-    """One rotating input set: the prefill batch plus the decode token that follows it."""
+    """One rotating input set of a forward workload plus the decode token that follows it."""
 
-    def __init__(self, spec, seed, dev):
+    def __init__(self, spec, seed, dev, with_decode=True, with_r=False):
         import numpy as np
         import torch
         import synth
         s = synth.ForwardSpec(spec.name, spec.B, spec.T, spec.C, spec.dtype, spec.k_std, spec.w_lo, spec.w_hi,
                               spec.spike_prob, spec.spike_value, seed)
         w, u, k, v = synth.forward_inputs(s)
+        td = torch.bfloat16 if spec.dtype == "bf16" else torch.float32
         self.host = (k, v)
         self.w = torch.from_numpy(w).to(dev)
         self.u = torch.from_numpy(u).to(dev)
-        self.k = torch.from_numpy(k).to(dev)
-        self.v = torch.from_numpy(v).to(dev)
+        self.k = torch.from_numpy(k).to(dev).to(td)
+        self.v = torch.from_numpy(v).to(dev).to(td)
         self.y = torch.empty_like(self.k)
         self.state = torch.empty((3, spec.B, spec.C), dtype=torch.float32, device=dev)
-        B, C = spec.B, spec.C
-        r = np.random.default_rng(seed)
-        self.mu = torch.from_numpy(r.uniform(0, 1, (1, C)).astype(np.float32)).to(dev)
-        self.w1 = self.w.reshape(1, C)
-        self.u1 = self.u.reshape(1, C)
-        self.x_t = torch.from_numpy(r.normal(0, 1, (B, 1, C)).astype(np.float32)).to(dev)
-        self.x_prev = torch.from_numpy(r.normal(0, 1, (B, 1, C)).astype(np.float32)).to(dev)
-        self.k1 = torch.from_numpy(r.normal(0, 1, (B, 1, C)).astype(np.float32)).to(dev)
-        self.v1 = torch.from_numpy(r.normal(0, 1, (B, 1, C)).astype(np.float32)).to(dev)
-        self.xbar1 = torch.empty_like(self.x_t)
-        self.y1 = torch.empty_like(self.x_t)
-        self.state4 = self.state.view(3, B, 1, C)
-        self.r = torch.from_numpy(synth.receptance(s)).to(dev)  # receptance for the gated forward
+        self.r = torch.from_numpy(synth.receptance(s)).to(dev).to(td) if with_r else None
+        if with_decode:
+            B, C = spec.B, spec.C
+            r = np.random.default_rng(seed)
+            self.mu = torch.from_numpy(r.uniform(0, 1, (1, C)).astype(np.float32)).to(dev)
+            self.w1 = self.w.reshape(1, C)
+            self.u1 = self.u.reshape(1, C)
+            self.x_t = torch.from_numpy(r.normal(0, 1, (B, 1, C)).astype(np.float32)).to(dev)
+            self.x_prev = torch.from_numpy(r.normal(0, 1, (B, 1, C)).astype(np.float32)).to(dev)
+            self.k1 = torch.from_numpy(r.normal(0, 1, (B, 1, C)).astype(np.float32)).to(dev)
+            self.v1 = torch.from_numpy(r.normal(0, 1, (B, 1, C)).astype(np.float32)).to(dev)
+            self.xbar1 = torch.empty_like(self.x_t)
+            self.y1 = torch.empty_like(self.x_t)
+            self.state4 = self.state.view(3, B, 1, C)
 
 
-def step(wkv, s, ws, ev=None):
+def step(wkv, s, ws):
     """One pass of the hot path: prefill forward (with state_out) then the fused decode step."""
-    if ev is not None:
-        ev[0].record()
     wkv.wkv_forward(s.w, s.u, s.k, s.v, workspace=ws, y=s.y, state_out=s.state)
-    if ev is not None:
-        ev[1].record()
     wkv.wkv_decode_step_fused(s.mu, s.w1, s.u1, s.x_t, s.x_prev, s.k1, s.v1, s.state4, xbar=s.xbar1, y=s.y1)
 
 
-def capture(torch, wkv, sets, ws, nsteps, with_events):
-    g = torch.cuda.CUDAGraph()
-    # external=True makes a captured record an event-record node (timed on every replay)
-    evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
-           for _ in range(nsteps)] if with_events else [None] * nsteps
-    with torch.cuda.graph(g):
-        for i in range(nsteps):
-            step(wkv, sets[i % len(sets)], ws, evs[i])
-    return g, evs
-
-
-def graph_ms(torch, fn, n_calls):
-    """Mean time of fn(i) for i in range(n_calls), captured in one CUDA graph, 10 replays."""
-    for i in range(min(n_calls, 6)):
-        fn(i)
-    torch.cuda.synchronize()
+def capture(torch, fn, n_calls):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for i in range(n_calls):
             fn(i)
+    return g
+
+
+def graph_ms(torch, fn, n_calls, replays=5):
+    """Per-call time of fn(i), i in range(n_calls), captured in one CUDA graph: the median over
+    `replays` replays, CUDA events around each whole replay on the current stream."""
+    for i in range(min(n_calls, 8)):
+        fn(i)
+    torch.cuda.synchronize()
+    g = capture(torch, fn, n_calls)
     g.replay()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(10):
+    out = []
+    for _ in range(replays):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
         g.replay()
-    e1.record()
+        e1.record()
+        torch.cuda.synchronize()
+        out.append(e0.elapsed_time(e1) / n_calls)
+    del g
+    return statistics.median(out)
+
+
+def event_node_ms(torch, fn, n_calls):
+    """Per-call time of fn(i) from event-record nodes captured around every call inside one
+    graph (each node adds a little time to the call it brackets)."""
+    evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+           for _ in range(n_calls)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n_calls):
+            evs[i][0].record()
+            fn(i)
+            evs[i][1].record()
+    for _ in range(3):
+        g.replay()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / (10 * n_calls)
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
     del g
     return ms
 
 
-def next_rows_bench(torch, wkv, sets, ws, spec, peak):
+def forward_config_row(torch, wkv, dev, name, peak, cpu_seconds):
+    """One forward benchmark configuration: the default path on rotating input sets (total
+    over twice the L2), back-to-back launches in a graph, median of 5 replays."""
+    import synth
+    spec = synth.FORWARD[name]
+    esz = 2 if spec.dtype == "bf16" else 4
+    n = spec.B * spec.T * spec.C
+    per_set = 3 * n * esz
+    n_sets = sets_for(per_set) if per_set > 4096 * 16 else 1
+    sets = [ForwardSet(spec, spec.seed + 17 * i, dev, with_decode=False) for i in range(n_sets)]
+    td = torch.bfloat16 if spec.dtype == "bf16" else torch.float32
+    ws = wkv.Workspace(dev, wkv.workspace_size(spec.B, spec.T, spec.C, td))
+
+    def fwd(i):
+        s = sets[i % n_sets]
+        wkv.wkv_forward(s.w, s.u, s.k, s.v, workspace=ws, y=s.y, state_out=s.state)
+
+    calls = GRAPH_STEPS if n < 1e6 else 4 * n_sets * max(1, 20 // (4 * n_sets))
+    ms = graph_ms(torch, fwd, calls)
+    wkv.forward_status(ws.buf)
+    alg = ALG_BYTES_PER_ELEM[spec.dtype] * n
+    row = {"workload": name, "B": spec.B, "T": spec.T, "C": spec.C, "io": spec.dtype,
+           "path": wkv.auto_path(spec.B, spec.T, spec.C, td), "launch_ms": ms, "elements_per_s": n / (ms * 1e-3),
+           "alg_bytes_per_launch": alg, "achieved_gbs": alg / (ms * 1e-3) / 1e9,
+           "frac": alg / (ms * 1e-3) / 1e9 / peak,
+           "l2": f"{n_sets} rotating input set(s) of {per_set / 1e6:.1f} MB",
+           "timing": f"graph of {calls} back-to-back forwards (with state_out), median of 5 replays"}
+    if name == "fwd_64x64":
+        # latency of one launch: events around a single eager call, median of 50
+        lat = []
+        for _ in range(50):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fwd(0)
+            e1.record()
+            torch.cuda.synchronize()
+            lat.append(e0.elapsed_time(e1))
+        row["latency_ms"] = statistics.median(lat)
+        row["latency_timing"] = "events around one eager call, median of 50"
+        row["frac_note"] = "a 50 KB problem is latency-bound: the fraction is reported, not a target"
+    if cpu_seconds:
+        row["cpu_baseline"] = oracle_row(spec, cpu_seconds)
+    del sets, ws
+    torch.cuda.empty_cache()
+    return row
+
+
+def decode_bench(torch, wkv, dev, steps, peak):
+    """256 sessions x 32 layers x 4096 channels, fused decode, 4 input sets in rotation
+    (each 403 MB of x, k, v)."""
+    N, L, C = 256, 32, 4096
+    g = torch.Generator(device=dev)
+    g.manual_seed(1005)
+    mu = torch.rand((L, C), generator=g, device=dev)
+    w = torch.exp(torch.rand((L, C), generator=g, device=dev) * 6 - 5)
+    u = torch.randn((L, C), generator=g, device=dev) * 0.5
+    st = torch.empty((3, N, L, C), device=dev)
+    st[2].normal_(1.0, 1.0, generator=g)
+    st[1].normal_(0.0, 1.0, generator=g).abs_().add_(1.0)
+    st[0].normal_(0.0, 1.0, generator=g).mul_(st[1])
+    sets = [tuple(torch.randn((N, L, C), generator=g, device=dev) for _ in range(3)) for _ in range(4)]
+    xbar = torch.empty((N, L, C), device=dev)
+    y = torch.empty((N, L, C), device=dev)
+
+    def one(i):
+        x_t, k, v = sets[i % 4]
+        x_prev = sets[(i - 1) % 4][0]
+        wkv.wkv_decode_step_fused(mu, w, u, x_t, x_prev, k, v, st, xbar=xbar, y=y)
+
+    ms = graph_ms(torch, one, 8, replays=max(3, steps // 8))
+    alg = DECODE_ALG_BYTES_PER_ELEM * N * L * C
+    del sets, st
+    torch.cuda.empty_cache()
+    return {"workload": f"decode_{N}x{L}x{C}", "metric": "decode tokens/s (session steps through all 32 layers)",
+            "value": N / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "alg_bytes_per_step": alg,
+            "achieved_gbs": alg / (ms * 1e-3) / 1e9, "frac": alg / (ms * 1e-3) / 1e9 / peak,
+            "l2": "4 rotating sets of x, k, v (403 MB each); state 403 MB updated in place",
+            "timing": "graph of 8 fused decode steps, median over replays"}
+
+
+def next_rows_bench(torch, wkv, dev, peak):
     """The fused receptance-gated forward (y = sigma(r) * wkv: k, v, r read and y written once,
     16 B/element fp32), the three-mu token shift (x read, three blends written, 16 B/element)
-    and the backward (k, v, gy read, gk, gv written: 20 B/element) on the bench workload,
-    rotating input sets, next to the plain forward timed the same way."""
+    and the backward (k, v, gy read, gk, gv written: 20 B/element) on the 8 x 1024 x 768
+    workload, rotating input sets, next to the plain forward timed the same way."""
+    import synth
+    spec = synth.FORWARD["fwd_8x1024x768"]
     n = spec.B * spec.T * spec.C
+    sets = [ForwardSet(spec, rank_set_seed(spec.seed, 0, i), dev, with_decode=False, with_r=True) for i in range(4)]
+    ws = wkv.Workspace(dev, wkv.workspace_size(spec.B, spec.T, spec.C))
 
     def plain(i):
         s = sets[i % len(sets)]
@@ -381,15 +539,15 @@ def next_rows_bench(torch, wkv, sets, ws, spec, peak):
         s = sets[i % len(sets)]
         wkv.wkv_forward(s.w, s.u, s.k, s.v, workspace=ws, y=s.y, state_out=s.state, r=s.r)
 
-    mu = [torch.rand(spec.C, device=sets[0].k.device) for _ in range(3)]
+    mu = [torch.rand(spec.C, device=dev) for _ in range(3)]
 
     def shift3(i):
         s = sets[i % len(sets)]
         wkv.token_shift_mix3(mu[0], mu[1], mu[2], s.k)
 
     gy = torch.randn_like(sets[0].k)
-    bws = torch.empty(int(wkv.lib().wkv_backward_workspace_size(spec.B, spec.T, spec.C)), dtype=torch.uint8,
-                      device=sets[0].k.device)
+    bws = torch.zeros(int(wkv.lib().wkv_backward_workspace_size(spec.B, spec.T, spec.C)), dtype=torch.uint8,
+                      device=dev)
 
     def backward(i):
         s = sets[i % len(sets)]
@@ -398,20 +556,21 @@ def next_rows_bench(torch, wkv, sets, ws, spec, peak):
     plain_ms = graph_ms(torch, plain, GRAPH_STEPS)
     gated_ms = graph_ms(torch, gated, GRAPH_STEPS)
     shift_ms = graph_ms(torch, shift3, GRAPH_STEPS)
-    bwd_ms = graph_ms(torch, backward, 6)
+    bwd_ms = graph_ms(torch, backward, 8)
     b_gbs = 20 * n / (bwd_ms * 1e-3) / 1e9
     g_gbs = 16 * n / (gated_ms * 1e-3) / 1e9
     t_gbs = 16 * n / (shift_ms * 1e-3) / 1e9
+    del sets, ws, bws
+    torch.cuda.empty_cache()
     return {
-        "gated_forward": {"launch_ms": gated_ms, "alg_bytes_per_launch": 16 * n, "achieved_gbs": g_gbs,
-                          "frac": g_gbs / peak, "plain_forward_launch_ms": plain_ms,
-                          "timing": f"graph of {GRAPH_STEPS} back-to-back launches, 10 replays, after the timed region"},
-        "token_shift3": {"launch_ms": shift_ms, "alg_bytes_per_launch": 16 * n, "achieved_gbs": t_gbs,
-                         "frac": t_gbs / peak},
-        "backward": {"launch_ms": bwd_ms, "alg_bytes_per_launch": 20 * n, "achieved_gbs": b_gbs,
-                     "frac": b_gbs / peak,
-                     "note": "k, v, gy read and gk, gv written once (20 B/element); the five kernels read k, v "
-                             "three times and gy twice (40 B/element moved)"},
+        "gated_forward": {"workload": spec.name, "launch_ms": gated_ms, "alg_bytes_per_launch": 16 * n,
+                          "achieved_gbs": g_gbs, "frac": g_gbs / peak, "plain_forward_launch_ms": plain_ms,
+                          "timing": f"graph of {GRAPH_STEPS} back-to-back launches, median of 5 replays"},
+        "token_shift3": {"workload": spec.name, "launch_ms": shift_ms, "alg_bytes_per_launch": 16 * n,
+                         "achieved_gbs": t_gbs, "frac": t_gbs / peak},
+        "backward": {"workload": spec.name, "launch_ms": bwd_ms, "alg_bytes_per_launch": 20 * n,
+                     "achieved_gbs": b_gbs, "frac": b_gbs / peak,
+                     "note": "k, v, gy read and gk, gv written once (20 B/element)"},
     }
 
 
@@ -441,9 +600,7 @@ def eagle_bench(torch, wkv, dev, peak, decode=True):
     f_ms = graph_ms(torch, fwd, 12)
     out = {"eagle_forward": {"workload": spec.name, "launch_ms": f_ms, "alg_bytes_per_launch": alg,
                              "achieved_gbs": alg / (f_ms * 1e-3) / 1e9, "frac": alg / (f_ms * 1e-3) / 1e9 / peak,
-                             "elements_per_s": n / (f_ms * 1e-3),
-                             "note": "three launches: chunk sums (tcgen05 tf32 product, split operands), "
-                                     "scan over chunks, chunk outputs (CUDA cores)"}}
+                             "elements_per_s": n / (f_ms * 1e-3)}}
     del sets, ws
     if decode:
         N, L, Cd = 256, 32, 4096
@@ -468,69 +625,7 @@ def eagle_bench(torch, wkv, dev, peak, decode=True):
     return out
 
 
-def forward_only_ms(torch, wkv, sets, ws):
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        for i in range(GRAPH_STEPS):
-            s = sets[i % len(sets)]
-            wkv.wkv_forward(s.w, s.u, s.k, s.v, workspace=ws, y=s.y, state_out=s.state)
-    g.replay()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(10):
-        g.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / (10 * GRAPH_STEPS)
-
-
-def decode_bench(torch, wkv, dev, steps):
-    """256 sessions x 32 layers x 4096 channels, fused decode, 4 input sets in rotation."""
-    import numpy as np
-    N, L, C = 256, 32, 4096
-    g = torch.Generator(device=dev)
-    g.manual_seed(1005)
-    mu = torch.rand((L, C), generator=g, device=dev)
-    w = torch.exp(torch.rand((L, C), generator=g, device=dev) * 6 - 5)
-    u = torch.randn((L, C), generator=g, device=dev) * 0.5
-    st = torch.empty((3, N, L, C), device=dev)
-    st[2].normal_(1.0, 1.0, generator=g)
-    st[1].normal_(0.0, 1.0, generator=g).abs_().add_(1.0)
-    st[0].normal_(0.0, 1.0, generator=g).mul_(st[1])
-    sets = [tuple(torch.randn((N, L, C), generator=g, device=dev) for _ in range(3)) for _ in range(4)]
-    xbar = torch.empty((N, L, C), device=dev)
-    y = torch.empty((N, L, C), device=dev)
-
-    def one(i):
-        x_t, k, v = sets[i % 4]
-        x_prev = sets[(i - 1) % 4][0]
-        wkv.wkv_decode_step_fused(mu, w, u, x_t, x_prev, k, v, st, xbar=xbar, y=y)
-
-    for i in range(4):
-        one(i)
-    nper = 8
-    gr = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gr):
-        for i in range(nper):
-            one(i)
-    gr.replay()
-    torch.cuda.synchronize()
-    reps = max(1, steps // nper)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(reps):
-        gr.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / (reps * nper)
-    del gr
-    return {"workload": f"decode_{N}x{L}x{C}", "metric": "decode tokens/s (session steps through all 32 layers)",
-            "value": N / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": reps * nper,
-            "hbm_gbs": DECODE_ALG_BYTES_PER_ELEM * N * L * C / (ms * 1e-3) / 1e9}
-
-
-def e2e_bench(torch, wkv, sets, ws, steps, dev):
+def e2e_bench(torch, wkv, sets, ws, steps):
     """Through the public API with host buffers: per step, copy k and v from pinned host
     memory, run the step, read y back to pinned host memory.  Copies ride a second
     stream so the next step's upload overlaps this step's kernels and download."""
@@ -579,26 +674,26 @@ def run_ours(args):
 
     spec = synth.FORWARD[WORKLOAD]
     n_elem = spec.B * spec.T * spec.C
-    sets = [ForwardSet(spec, rank_set_seed(spec.seed, rank, i), dev) for i in range(N_SETS)]
+    n_sets = 2  # each set's k, v, y (805 MB) is over six times the L2 by itself
+    sets = [ForwardSet(spec, rank_set_seed(spec.seed, rank, i), dev) for i in range(n_sets)]
     ws = wkv.Workspace(dev, wkv.workspace_size(spec.B, spec.T, spec.C))
     path = wkv.auto_path(spec.B, spec.T, spec.C)
 
+    def one(i):
+        step(wkv, sets[i % n_sets], ws)
+
     # eager warm-up (sets kernel attributes, first-touch), then W untimed graph steps
-    for s in sets:
-        step(wkv, s, ws)
+    for i in range(n_sets):
+        one(i)
     torch.cuda.synchronize()
     wkv.forward_status(ws.buf)
 
     K = args.steps
-    per = min(GRAPH_STEPS, K)
-    main_g, _ = capture(torch, wkv, sets, ws, per, with_events=False)
-    rem = K % per
-    rem_g = capture(torch, wkv, sets, ws, rem, with_events=False)[0] if rem else None
-    reps = K // per
-    warm_g, _ = capture(torch, wkv, sets, ws, min(max(args.warmup, 1), GRAPH_STEPS), with_events=False)
-    for _ in range(max(1, (args.warmup + GRAPH_STEPS - 1) // GRAPH_STEPS)):
-        warm_g.replay()
+    main_g = capture(torch, one, K)
+    warm_g = capture(torch, one, max(args.warmup, 3))
+    warm_g.replay()
     torch.cuda.synchronize()
+    del warm_g
 
     clocks = ClockSampler(local)
     if rank == 0:
@@ -609,63 +704,74 @@ def run_ours(args):
         main_g.replay()
         torch.cuda.synchronize()
 
-    barrier(world)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    replay_ms = []
     t_wall0 = time.time()
-    e0.record()
-    for _ in range(reps):
+    for _ in range(REPLAYS):
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
         main_g.replay()
-    if rem_g is not None:
-        rem_g.replay()
-    e1.record()
-    torch.cuda.synchronize()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        replay_ms.append(max_over_ranks(e0.elapsed_time(e1), world))
     t_wall1 = time.time()
-    barrier(world)
     clocks.stop()
     wkv.forward_status(ws.buf)
+    del main_g
 
-    ms_total = max_over_ranks(e0.elapsed_time(e1), world)
-    ms_per_step = ms_total / K
+    ms_per_step = statistics.median(replay_ms) / K
     value = weak_scaling_value(world, n_elem, ms_per_step)
-    # The forward's own launch duration, right after the timed region: a graph of GRAPH_STEPS
-    # back-to-back forwards on the rotating input sets, CUDA events around whole replays.  Event
-    # nodes inside a graph add several microseconds to the launch they bracket, so the
-    # per-launch figure they give (also reported) overstates the kernel's time.
-    fwd_ms = forward_only_ms(torch, wkv, sets, ws)
-    launch_timing = (f"graph of {GRAPH_STEPS} back-to-back forwards on the rotating input sets, CUDA events around "
-                     "10 replays, right after the timed region")
+
+    def fwd(i):
+        s = sets[i % n_sets]
+        wkv.wkv_forward(s.w, s.u, s.k, s.v, workspace=ws, y=s.y, state_out=s.state)
+
+    # The forward's own launch duration, right after the timed region: back-to-back forwards
+    # in a graph, events around whole replays (median of 5).  Event nodes inside a graph add a
+    # little to the launch they bracket; that figure is reported beside it.
+    fwd_ms = max_over_ranks(graph_ms(torch, fwd, 20), world)
     try:
-        ev_g, ev_list = capture(torch, wkv, sets, ws, per, with_events=True)
-        for _ in range(3):
-            ev_g.replay()
-        torch.cuda.synchronize()
-        fwd_ms_nodes = statistics.mean(a.elapsed_time(b) for a, b in ev_list)
-        del ev_g
+        nodes_ms = event_node_ms(torch, fwd, 10)
     except Exception:
-        fwd_ms_nodes = float("nan")
-    fwd_ms = max_over_ranks(fwd_ms, world)
-    fwd_ms_nodes = max_over_ranks(fwd_ms_nodes, world)  # every rank takes part, failed or not
-    fwd_ms_nodes = None if fwd_ms_nodes != fwd_ms_nodes else fwd_ms_nodes
+        nodes_ms = float("nan")
+    nodes_ms = max_over_ranks(nodes_ms, world)  # every rank takes part, failed or not
+    nodes_ms = None if nodes_ms != nodes_ms else nodes_ms
 
     peaks, peak_kind = measured_peaks()
+    peak = peaks["hbm_gbs"]
     alg = ALG_BYTES_PER_ELEM[spec.dtype] * n_elem
     achieved = alg / (fwd_ms * 1e-3) / 1e9
-    traffic = profiled_traffic(WORKLOAD)
+    traffic, traffic_src = profiled_traffic(WORKLOAD)
 
-    del main_g, rem_g, warm_g
-    dec = None if args.no_decode else decode_bench(torch, wkv, dev, 400)
-    nxt = next_rows_bench(torch, wkv, sets, ws, spec, peaks["hbm_gbs"])
-    nxt.update(eagle_bench(torch, wkv, dev, peaks["hbm_gbs"], decode=not args.no_decode))
     e2e = None
     if not args.no_e2e:
-        ms_e2e, h2d, d2h = e2e_bench(torch, wkv, sets, ws, min(K, 240), dev)
+        ms_e2e, h2d, d2h = e2e_bench(torch, wkv, sets[:1], ws, max(3, min(K, 20)))
         ms_e2e = max_over_ranks(ms_e2e, world)
         e2e = {"value": weak_scaling_value(world, n_elem, ms_e2e), "unit": "elements/s", "ms_per_step": ms_e2e,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del sets
+    torch.cuda.empty_cache()
+
+    cpu_s = 0.0 if (args.no_cpu or rank != 0 or world != 1) else 2.0
+    configs = None
+    if not args.no_configs:
+        configs = {}
+        for name in FORWARD_CONFIGS:
+            configs[name] = forward_config_row(torch, wkv, dev, name, peak, cpu_s)
+        if not args.no_decode:
+            d = decode_bench(torch, wkv, dev, 200, peak)
+            if cpu_s:
+                d["cpu_baseline"] = oracle_decode_row(cpu_s)
+            configs[d["workload"]] = d
+    nxt = None
+    if not args.no_next:
+        nxt = next_rows_bench(torch, wkv, dev, peak)
+        nxt.update(eagle_bench(torch, wkv, dev, peak, decode=not args.no_decode))
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu:
+    if cpu_s:
         rate, passes, el, cores = time_oracle(spec, synth.forward_inputs(spec), 5.0, 3)
         cpu = {"value": rate, "unit": "elements/s", "cores": cores, "kind": "oracle",
                "sample": f"{passes} passes of the whole {spec.B}x{spec.T}x{spec.C} prefill through the fp64 "
@@ -678,19 +784,26 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "B": spec.B, "T": spec.T, "C": spec.C, "io": spec.dtype,
+                       "state_out": True,
                        "step": "prefill forward (with final state) + one fused decode step of the same batch",
-                       "forward_path": path, "l2": f"{N_SETS} rotating input sets "
-                                                    f"({N_SETS * 3 * n_elem * 4 / 1e6:.0f} MB > 3x L2)",
-                       "graph": f"CUDA graphs of {per} steps"},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                         "kernel": f"wkv_forward ({path})", "launch_ms": fwd_ms, "launch_timing": launch_timing,
-                         "launch_ms_event_nodes": fwd_ms_nodes,
+                       "forward_path": path,
+                       "l2": f"inputs larger than L2: each step reads {2 * n_elem * 4 / 1e6:.0f} MB and writes "
+                             f"{n_elem * 4 / 1e6:.0f} MB; {n_sets} sets rotate",
+                       "graph": f"one CUDA graph of {K} steps, replayed {REPLAYS} times; median replay",
+                       "replay_ms": replay_ms},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "traffic_source": (f"{traffic_src} (ncu dram__bytes of the same kernel source; not "
+                                            "measured in this run)") if traffic_src else None,
+                         "kernel": f"wkv_forward ({path})", "launch_ms": fwd_ms,
+                         "launch_timing": "graph of 20 back-to-back forwards on the rotating input sets, CUDA "
+                                          "events around each replay, median of 5, right after the timed region",
+                         "launch_ms_event_nodes": nodes_ms,
                          "alg_bytes_per_launch": alg, "peak_kind": f"{peak_kind} hbm_gbs"},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 2 * K,
-            "decode": dec,
+            "configs": configs,
             "next_rows": nxt,
             "clocks": clocks.summary(t_wall0, t_wall1) if rank == 0 else None,
         }
@@ -723,6 +836,23 @@ def profile_forward(name):
                       "io": spec.dtype}))
 
 
+def profile_step():
+    """Three warm-up and two profiled eager headline steps (forward with state + fused decode)
+    on one input set."""
+    import torch
+    import linear_attention_rnn_wkv_b200 as wkv
+    import synth
+    spec = synth.FORWARD[WORKLOAD]
+    dev = torch.device("cuda", 0)
+    s = ForwardSet(spec, spec.seed, dev)
+    ws = wkv.Workspace(dev, wkv.workspace_size(spec.B, spec.T, spec.C))
+    for _ in range(5):
+        step(wkv, s, ws)
+    torch.cuda.synchronize()
+    wkv.forward_status(ws.buf)
+    print(json.dumps({"profile_step": WORKLOAD, "steps": 5}))
+
+
 def profile_backward(name):
     """Two warm-up and three profiled eager backward calls on one forward workload's shape, in
     fp32 (the backward's only I/O type)."""
@@ -734,7 +864,7 @@ def profile_backward(name):
     w, u, k, v = synth.forward_inputs(spec)
     gy = synth.grad_output(spec)
     t = [torch.from_numpy(a.astype("float32")).to(dev) for a in (w, u, k, v, gy)]
-    ws = torch.empty(int(wkv.lib().wkv_backward_workspace_size(spec.B, spec.T, spec.C)), dtype=torch.uint8,
+    ws = torch.zeros(int(wkv.lib().wkv_backward_workspace_size(spec.B, spec.T, spec.C)), dtype=torch.uint8,
                      device=dev)
     for _ in range(5):
         wkv.wkv_backward(*t, workspace=ws)
@@ -762,6 +892,9 @@ def main():
     args = parse()
     if args.profile_forward:
         profile_forward(args.profile_forward)
+        return
+    if args.profile_step:
+        profile_step()
         return
     if args.profile_backward:
         profile_backward(args.profile_backward)

@@ -65,7 +65,7 @@ typedef enum wkv_dtype {
 } wkv_dtype;
 
 typedef enum wkv_path {
-    WKV_PATH_AUTO = 0,     /* pick from the measured table for (B*C, T, dtype) */
+    WKV_PATH_AUTO = 0,     /* the fastest path measured at the nearest (dtype, B*C, T) grid point */
     WKV_PATH_SERIAL = 1,   /* one thread per (b, c) scanning all of T */
     WKV_PATH_CHUNKED = 2   /* time-parallel: chunk summaries, carry scan, fix-up */
 } wkv_path;
@@ -99,7 +99,8 @@ wkv_status wkv_forward(int64_t B, int64_t T, int64_t C, wkv_dtype io, const floa
  *             (resumable / piecewise prefill; state_out may alias state_in);
  *   path      WKV_PATH_AUTO, WKV_PATH_SERIAL or WKV_PATH_CHUNKED;
  *   chunk     time steps per chunk for the chunked path (0 = default; else 4, 8 or 16
- *             steps per warp).
+ *             steps per warp).  With WKV_PATH_AUTO and chunk 0 the chunk length comes
+ *             from the same measured table as the path (8 or 16).
  */
 wkv_status wkv_forward_ex(int64_t B, int64_t T, int64_t C, wkv_dtype io, const float* w, const float* u,
                           const void* k, const void* v, const float* state_in, void* y, float* state_out,
@@ -134,17 +135,24 @@ wkv_status wkv_forward_gated(int64_t B, int64_t T, int64_t C, wkv_dtype io, cons
  *   gk, gv        [B, T, C] fp32 (written; must not overlap the inputs)
  *   gw, gu        [C] fp32 (written: zeroed, then accumulated on the device)
  *   workspace     caller-owned device scratch of ws_bytes >= wkv_backward_workspace_size()
- *                 (per channel and segment: a forward state record and the adjoint sums)
- * Time-parallel over segments of 32 steps: the segments' forward states and adjoint sums are
- * each combined by one scan per channel, then every segment recomputes its outputs and writes
- * its gradients; nothing per position is kept in global memory.
+ *                 (per channel and segment: a starting state, and the published forward
+ *                 record and adjoint sums), zero-filled once before its first use
+ *                 (wkv_workspace_init); one workspace must not serve two backward calls that
+ *                 can run at the same time
+ * Time-parallel over segments of 32 steps, two launches: the segments in time order, each
+ * taking its starting state from the records of the segments before it by a bounded
+ * look-back; then the segments in reverse time order, each recomputing its outputs, taking
+ * the adjoint sums of the segments after it by a bounded look-back and writing its
+ * gradients.  k, v are read twice, gy once; nothing per position is kept in global memory.
+ * A look-back that gives up is recorded in the device-wide word that wkv_get_device_status
+ * reports (the gradients are then invalid).
  * Status codes as wkv_forward; B and ceil(T / 32) must be <= 65535.
  */
 wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
                         const float* v, const float* gy, float* gk, float* gv, float* gw, float* gu,
                         void* workspace, size_t ws_bytes, cudaStream_t stream);
 
-/* Workspace bytes wkv_backward needs (36 per batch row, channel and 32 steps). */
+/* Workspace bytes wkv_backward needs (64, plus 88 per batch row, channel and 32 steps). */
 size_t wkv_backward_workspace_size(int64_t B, int64_t T, int64_t C);
 
 /* Workspace bytes wkv_forward needs for this shape (the largest over all paths). */
@@ -233,7 +241,8 @@ wkv_status wkv_decode_step_fused(int64_t N, int64_t L, int64_t C, const float* m
  * call allocates nothing (no cudaMalloc, no allocating library routine).
  *  - Shapes whose scratch would exceed 32 MiB are rejected with WKV_ERR_INVALID_ARG
  *    before anything is enqueued (e.g. 8 x 1024 x 768 fp32 needs ~6.3 MB; 1 x 16384 x
- *    4096 fp32 needs more and is rejected).  T must be >= 1; B = 0 or C = 0 is a no-op.
+ *    4096 fp32 needs more and is rejected).  B = 0 or C = 0 is a no-op; T = 0 writes
+ *    state_out only (state_in, or the empty state), as wkv_forward_ex does.
  *  - All calls on a device share the array and it keeps the last call's contents; each
  *    call clears the counters that must start at zero.  Calls that can overlap on the
  *    GPU race on the array: order them (same stream, or events).
@@ -241,7 +250,9 @@ wkv_status wkv_decode_step_fused(int64_t N, int64_t L, int64_t C, const float* m
  *    (cudaGetSymbolAddress) with that device current and zero-fills the array once;
  *    make that first call before any stream capture.
  *  - A device-side wait that runs out (only possible when calls overlap) is recorded
- *    in the array and cleared by the next call; it is not reported to the caller.
+ *    in the array's header, which the next call clears, and in the library's
+ *    device-wide error word, which wkv_get_device_status reports.
+ *  - WKV_ERR_CUDA leaves the cause in wkv_last_cuda_error, as for the other calls.
  */
 wkv_status wkv_forward_chunked_noalloc(int64_t B, int64_t T, int64_t C, wkv_dtype io, const float* w,
                                        const float* u, const void* k, const void* v, const float* state_in,
@@ -297,7 +308,9 @@ const char* wkv_status_string(wkv_status status);
 /* The cudaError_t of the last WKV_ERR_CUDA returned on this host thread (0 if none). */
 int wkv_last_cuda_error(void);
 
-/* The path WKV_PATH_AUTO picks for this shape (WKV_PATH_SERIAL or WKV_PATH_CHUNKED). */
+/* The path WKV_PATH_AUTO picks for this shape (WKV_PATH_SERIAL or WKV_PATH_CHUNKED): the
+ * fastest one measured on a B200 at the grid point nearest to (dtype, B*C, T) on a log scale
+ * (csrc/wkv_path_table.h, written by the package's tuning script, tune.py). */
 wkv_path wkv_forward_auto_path(int64_t B, int64_t T, int64_t C, wkv_dtype io);
 
 /* Library version, major * 10000 + minor * 100 + patch. */

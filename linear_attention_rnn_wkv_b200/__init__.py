@@ -199,7 +199,8 @@ def wkv_forward(w, u, k, v, state_in=None, want_state=True, path="auto", chunk=0
 
 def wkv_backward(w, u, k, v, gy, workspace=None):
     """Gradients of sum(gy * y) for the forward from the empty state over fp32 [B, T, C]:
-    returns (gk, gv, gw, gu) with gk, gv [B, T, C] and gw, gu [C]."""
+    returns (gk, gv, gw, gu) with gk, gv [B, T, C] and gw, gu [C].  A workspace passed in must
+    have been zero-filled before its first use (e.g. torch.zeros) and be reused only in order."""
     for t, name in ((k, "k"), (v, "v"), (gy, "gy")):
         _cuda_f32(t, name)
     if k.dim() != 3 or v.shape != k.shape or gy.shape != k.shape:
@@ -212,7 +213,7 @@ def wkv_backward(w, u, k, v, gy, workspace=None):
     gu = torch.empty_like(gw)
     nbytes = int(lib().wkv_backward_workspace_size(B, T, C))
     ws = workspace if workspace is not None and workspace.numel() >= nbytes else \
-        torch.empty(max(nbytes, 16), dtype=torch.uint8, device=k.device)
+        torch.zeros(max(nbytes, 64), dtype=torch.uint8, device=k.device)
     _check(lib().wkv_backward(B, T, C, w.data_ptr(), u.data_ptr(), k.data_ptr(), v.data_ptr(), gy.data_ptr(),
                               gk.data_ptr(), gv.data_ptr(), gw.data_ptr(), gu.data_ptr(), ws.data_ptr(), ws.numel(),
                               _stream(k.device)), "wkv_backward")

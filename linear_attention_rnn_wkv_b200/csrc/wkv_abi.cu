@@ -8,6 +8,9 @@
 #include "wkv_device.cuh"
 #include "wkv_eagle_internal.h"
 #include "wkv_internal.h"
+#include "wkv_path_table.h"
+
+#include <cmath>
 
 namespace {
 
@@ -59,15 +62,37 @@ uint32_t* wkvb::device_status_word() {
     return w ? w + 2 : nullptr;
 }
 
+int wkvb::record_cuda_error(cudaError_t e) { return (int)cuda_fail(e); }
+
 namespace {
 
-// Default path table: the chunked scan exposes T-parallelism and wins unless there
-// are enough independent channels to fill every SM with serial scans.
-wkv_path auto_path(int64_t B, int64_t T, int64_t C, wkv_dtype io) {
-    (void)io;
-    const int64_t BC = B * C;
-    if (T <= 64 && BC >= 148 * 1024) return WKV_PATH_SERIAL;
-    return WKV_PATH_CHUNKED;
+// Index of the grid value nearest to x on a log scale (ties to the larger).
+template <int N>
+int nearest_log(const long long (&grid)[N], int64_t x) {
+    int best = 0;
+    double bd = 1e300;
+    const double lx = log2((double)(x > 0 ? x : 1));
+    for (int i = 0; i < N; ++i) {
+        const double d = fabs(log2((double)grid[i]) - lx);
+        if (d <= bd) {
+            bd = d;
+            best = i;
+        }
+    }
+    return best;
+}
+
+// The path (and chunk length) WKV_PATH_AUTO takes: the measured winner at the nearest grid
+// point of the tuning table (wkv_path_table.h: I/O dtype, channels B*C, tokens T); a point
+// too large to have been measured takes the nearest measured point with fewer tokens.
+wkv_path auto_path(int64_t B, int64_t T, int64_t C, wkv_dtype io, int* chunk = nullptr) {
+    const int d = io == WKV_BF16 ? 1 : 0;
+    const int ib = nearest_log(kTuneBC, B * C);
+    int it = nearest_log(kTuneT, T);
+    while (it > 0 && kTunePath[d][ib][it] == 0) --it;
+    const int code = kTunePath[d][ib][it];
+    if (chunk) *chunk = code == 8 ? 8 : 16;
+    return code == 1 ? WKV_PATH_SERIAL : WKV_PATH_CHUNKED;
 }
 
 wkv_status forward_impl(int64_t B, int64_t T, int64_t C, wkv_dtype io, const float* w, const float* u,
@@ -105,7 +130,11 @@ wkv_status forward_impl(int64_t B, int64_t T, int64_t C, wkv_dtype io, const flo
     a.state_out = state_out;
     a.spin_limit = spin_limit;
 
-    if (path == WKV_PATH_AUTO) path = auto_path(B, T, C, io);
+    if (path == WKV_PATH_AUTO) {
+        int tuned_chunk = 16;
+        path = auto_path(B, T, C, io, &tuned_chunk);
+        if (chunk == 0) chunk = tuned_chunk;
+    }
     if (path == WKV_PATH_SERIAL) {
         a.err = workspace && ws_bytes >= kWsHeaderBytes ? &static_cast<WsHeader*>(workspace)->error : status_word();
         a.dev_err = device_status_word();
@@ -199,9 +228,9 @@ wkv_status token_shift_mix3(int64_t B, int64_t T, int64_t C, const float* mu_r, 
 size_t wkv_backward_workspace_size(int64_t B, int64_t T, int64_t C) {
     int64_t n = 0;
     if (!sizes_ok(B, T, C, &n) || n > INT64_MAX / 64) return 0;
-    // per (b, segment, c): a forward state record (4 floats) and the adjoint sums with their
-    // reference (5 floats)
-    return (size_t)B * (size_t)backward_segments(T) * (size_t)C * 9 * sizeof(float);
+    // a 64-byte header; per (b, segment, c): a starting state (4 floats), the published
+    // forward record (4 tagged 64-bit words) and adjoint sums with their reference (5 words)
+    return backward_workspace_bytes(B, T, C);
 }
 
 wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,

@@ -18,19 +18,22 @@
 //   X_local = sum_{t in span} e^{-(t-t0) w} gy_t / D_t,  X'_local = the same weighted by (t - t0),
 // which can be accumulated walking left to right.
 //
-// Time-parallel in segments of kSeg steps, one thread per (b, c, segment), five launches:
-//   A  each segment's forward recurrence from the empty state -> its state record;
-//   B  per channel, the records combined in time order -> each segment's starting state
-//      (and gw, gu zeroed for the atomics of E), two-level over groups of segments;
-//   C  each segment's forward from its starting state, accumulating its local (X, Y, X', Y')
-//      left to right as each D_t and y_t appears;
-//   D  per channel, the local sums composed right to left -> each segment's incoming sums,
-//      two-level like B;
-//   E  each segment's forward again, keeping per position the output's reference exponent q_t,
-//      1 / Dn_t (D_t = Dn_t 2^{q_t}) and y_t in shared memory, then its adjoint recurrence from
-//      the incoming sums -> gk, gv, and gw, gu partials added with atomics.
-// k, v are read three times and gy twice (40 B per element with gk, gv written); nothing per
-// position is stored in global memory.
+// Time-parallel in segments of kSeg steps, one thread per (b, c, segment), two launches, each
+// handing its units out by an atomic ticket so that every wait is on a smaller ticket:
+//   A  the segments in time order: each segment's forward recurrence from the empty state
+//      gives its record, a decoupled look-back over the earlier segments of its channel folds
+//      their published records into its starting state (written for R), and the state at its
+//      end is published for the later segments; gw, gu are zeroed for R's atomics;
+//   R  the segments in reverse time order: each runs its forward from its starting state,
+//      keeping per position the output's reference exponent q_t, 1 / Dn_t (D_t = Dn_t 2^{q_t})
+//      and y_t in shared memory while it accumulates its local (X, Y, X', Y') left to right;
+//      publishes them; folds in the published sums of the later segments of its channel (a
+//      decoupled look-back towards the end of the sequence) to get its incoming sums; publishes
+//      what leaves it to the left; then runs its adjoint recurrence from the incoming sums ->
+//      gk, gv, and gw, gu partials added with atomics.
+// k, v are read once by A and once by R, gy once, and gk, gv written once (28 B per element);
+// R's adjoint pass reads its segment's k, v, gy again straight after its forward pass, from
+// the L2.  Nothing per position is stored in global memory.
 // Numerics: the forward keeps an anchored reference p = anc - n w (no drift from rounding
 // p - w); the adjoint sums are held relative to a reference r (X = x 2^{-r}) chosen so every
 // rescaling exponent is <= 0, and e^{k_i} X_i = x 2^{k_i log2 e - r} <= x because k_i never
@@ -43,9 +46,13 @@ namespace {
 
 constexpr int kSeg = 32;           // time steps per segment
 constexpr int kBlk = 16;           // steps whose loads are issued together
-constexpr int kScanBlk = 8;        // segment records loaded together by the per-channel scans
 constexpr int kThreads = 128;      // threads per block (channels of one (b, segment))
 constexpr float kRNone = 3.0e38f;  // reference of an empty adjoint sum
+// Later segments' published sums read per look-back round trip.
+#ifndef WKV_BWD_LOOKAHEAD
+#define WKV_BWD_LOOKAHEAD 4
+#endif
+constexpr int kBwdLook = WKV_BWD_LOOKAHEAD;
 // E's per-position values: [kSeg][3][kThreads] floats, each thread its own column
 constexpr size_t kGradSmem = (size_t)kSeg * 3 * kThreads * sizeof(float);
 static_assert(kGradSmem <= 48 * 1024, "fits the default dynamic shared memory limit");
@@ -145,12 +152,29 @@ __device__ __forceinline__ float ld_in(const float* p) {
 }
 __device__ __forceinline__ void hold(float& x) { asm volatile("" : "+f"(x)); }
 
+// Workspace header of the backward: the reverse pass's ticket and completion counters and the
+// launch epoch that tags its published sums (advanced by each launch's last block).
+struct BwdHeader {
+    uint32_t ticket, done, epoch;        // the reverse pass (R)
+    uint32_t error;                      // first give-up of either pass
+    uint32_t ticket_f, done_f, epoch_f;  // the forward pass (A)
+    uint32_t pad[9];
+};
+constexpr size_t kBwdHeaderBytes = sizeof(BwdHeader);
+static_assert(kBwdHeaderBytes == 64, "header size");
+
 struct BwdArgs {
     int64_t B, T, C, P;  // P segments of kSeg steps (the last may be shorter)
     const float *w, *u, *k, *v, *gy;
     float *gk, *gv, *gw, *gu;
-    float* fs;  // [4][B][P][C] segment records, then starting states
-    float* as;  // [5][B][P][C] local adjoint sums, then incoming sums
+    float* fs;           // [4][B][P][C] the segments' starting states
+    uint64_t* fslots;    // [B][P][4][C] tagged words: a segment's forward record, later the
+                         // state at its end (the inclusive record)
+    uint64_t* slots;     // [B][P][5][C] tagged words: a segment's local adjoint sums, later what
+                         // leaves it to the left (the inclusive sums)
+    BwdHeader* hdr;
+    uint32_t* dev_err;   // the library's device-wide error word
+    uint32_t spin_limit;
 };
 
 __device__ __forceinline__ int64_t seg_index(const BwdArgs& a, int64_t b, int64_t j, int64_t c) {
@@ -197,128 +221,132 @@ __device__ __forceinline__ void forward_span(const BwdArgs& a, int64_t base, int
     }
 }
 
-// A: each segment's forward from the empty state -> its record
-__global__ void __launch_bounds__(kThreads) bwd_seg_forward(BwdArgs a) {
-    const int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    const int64_t j = blockIdx.y, b = blockIdx.z;
-    if (c >= a.C) return;
-    const float w2 = a.w[c] * kLog2e, u2 = a.u[c] * kLog2e;
-    const int64_t t0 = j * kSeg, t1 = min64(a.T, t0 + kSeg);
-    FwdState s{0.f, 0.f, kPEmpty, 0.f};
-    forward_span<false, false>(a, b * a.T * a.C + c, t0, t1, s, u2, w2, [](int, const FwdOut&, float) {});
-    const int64_t si = seg_index(a, b, j, c), SP = a.B * a.P * a.C;
-    a.fs[si] = s.a;
-    a.fs[SP + si] = s.bb;
-    a.fs[2 * SP + si] = s.anc;
-    a.fs[3 * SP + si] = s.n;
+// Published forward records: four 64-bit words per (sequence, segment, channel), (a | tag),
+// (b | tag), (anc | tag), (n | tag), word-major per (sequence, segment); the same fence-free
+// protocol as the adjoint sums below (kind 1 the segment's own record, 2 the state at its end).
+__device__ __forceinline__ uint64_t* fwd_slot(const BwdArgs& a, int64_t b, int64_t j) {
+    return a.fslots + (b * a.P + j) * 4 * a.C;
 }
 
-// The two per-channel scans (B, D) split a channel's segments into kGroups consecutive groups:
-// every group folds its own segments (in parallel with the others), each group then combines
-// the aggregates of the groups before it (B) or after it (D), and walks its segments again from
-// that carry, writing each segment's carry.  The serial chain per channel is one group long.
-constexpr int kGroups = 8;
-constexpr int kScanCh = 32;  // channels per scan block: one warp per group
-constexpr int kScanThreadsB = kScanCh * kGroups;
-
-struct GroupSpan {
-    int64_t j0, j1;  // the group's segments [j0, j1) (possibly empty)
-};
-
-__device__ __forceinline__ GroupSpan group_span(const BwdArgs& a, int g) {
-    const int64_t per = (a.P + kGroups - 1) / kGroups;
-    const int64_t j0 = min64(a.P, g * per);
-    return GroupSpan{j0, min64(a.P, j0 + per)};
+__device__ __forceinline__ void rec_publish(const BwdArgs& a, int64_t b, int64_t j, int64_t c, const Rec& r,
+                                            uint32_t tag) {
+    uint64_t* p = fwd_slot(a, b, j) + c;
+    const float f[4] = {r.a, r.b, r.anc, r.n};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) st_relaxed_u64(p + i * a.C, ((uint64_t)tag << 32) | __float_as_uint(f[i]));
 }
 
-__device__ __forceinline__ float seg_len(const BwdArgs& a, int64_t j) {
-    return (float)(min64(a.T, (j + 1) * kSeg) - j * kSeg);
+// 2 the state at the segment's end, 1 its own record, 0 nothing usable yet
+__device__ __forceinline__ int rec_read(const BwdArgs& a, int64_t b, int64_t j, int64_t c, uint32_t tag_loc,
+                                        uint32_t tag_incl, Rec& out) {
+    const uint64_t* p = fwd_slot(a, b, j) + c;
+    uint64_t wd[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) wd[i] = ld_relaxed_u64(p + i * a.C);
+    const uint32_t t0 = (uint32_t)(wd[0] >> 32);
+    bool same = t0 == tag_loc || t0 == tag_incl;
+#pragma unroll
+    for (int i = 1; i < 4; ++i) same = same && (uint32_t)(wd[i] >> 32) == t0;
+    if (!same) return 0;
+    out = Rec{__uint_as_float((uint32_t)wd[0]), __uint_as_float((uint32_t)wd[1]), __uint_as_float((uint32_t)wd[2]),
+              __uint_as_float((uint32_t)wd[3])};
+    return t0 == tag_incl ? 2 : 1;
 }
 
-__device__ __forceinline__ float group_len(const BwdArgs& a, int g) {
-    const GroupSpan s = group_span(a, g);
-    return s.j1 > s.j0 ? (float)(min64(a.T, s.j1 * kSeg) - s.j0 * kSeg) : 0.f;
-}
-
-__device__ __forceinline__ Rec load_rec(const BwdArgs& a, int64_t si) {
-    const int64_t SP = a.B * a.P * a.C;
-    return Rec{a.fs[si], a.fs[SP + si], a.fs[2 * SP + si], a.fs[3 * SP + si]};
-}
-
-// B: per channel, segment records combined left to right -> each segment's starting state
-// (and gw, gu zeroed for the atomics of E).
-__global__ void __launch_bounds__(kScanThreadsB) bwd_seg_carry(BwdArgs a) {
-    __shared__ Rec agg[kGroups][kScanCh];
-    const int lane = threadIdx.x % kScanCh, g = threadIdx.x / kScanCh;
-    const int64_t c = (int64_t)blockIdx.x * kScanCh + lane, b = blockIdx.y;
-    const bool live = c < a.C;
-    const float w2 = live ? a.w[c] * kLog2e : 0.f;
-    const GroupSpan sp = group_span(a, g);
-    const int64_t SP = a.B * a.P * a.C;
-    Rec run = rec_identity();
+// A: the segments in time order (an atomic ticket hands the first segments out first), 128
+// channels of one (sequence, segment) per block: each segment's forward from the empty state
+// gives its record; a decoupled look-back over the earlier segments of its channel (each a
+// smaller ticket) folds their records into its starting state, which it writes, and the state
+// at its end is published for the later segments.  gw, gu are zeroed here for R's atomics.
+__global__ void __launch_bounds__(kThreads) bwd_seg_starts(BwdArgs a, int64_t cx) {
+    __shared__ uint32_t s_ticket, s_epoch;
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        s_ticket = atomicAdd(&a.hdr->ticket_f, 1u);
+        s_epoch = (*reinterpret_cast<volatile uint32_t*>(&a.hdr->epoch_f) + 1u) & 0x3FFFFFFFu;
+    }
+    __syncthreads();
+    const int64_t unit = s_ticket;
+    const uint32_t epoch30 = s_epoch;
+    const uint32_t tag_loc = (epoch30 << 2) | 1u, tag_incl = (epoch30 << 2) | 2u;
+    const int64_t per_seg = a.B * cx;
+    const int64_t j = unit / per_seg;
+    const int64_t b = (unit % per_seg) / cx, cb = unit % cx;
+    const int64_t c = cb * kThreads + tid;
+    const bool live = unit < a.P * per_seg && c < a.C;
     if (live) {
-        if (b == 0 && g == 0) {  // E accumulates into these
+        if (b == 0 && j == 0) {  // R accumulates into these
             a.gw[c] = 0.f;
             a.gu[c] = 0.f;
         }
-        for (int64_t j0 = sp.j0; j0 < sp.j1; j0 += kScanBlk) {
-            const int nb = (int)min64(kScanBlk, sp.j1 - j0);
-            Rec seg[kScanBlk];
+        const float w2 = a.w[c] * kLog2e, u2 = a.u[c] * kLog2e;
+        const int64_t t0 = j * kSeg, t1 = min64(a.T, t0 + kSeg);
+        FwdState s{0.f, 0.f, kPEmpty, 0.f};
+        forward_span<false, false>(a, b * a.T * a.C + c, t0, t1, s, u2, w2, [](int, const FwdOut&, float) {});
+        const Rec local{s.a, s.bb, s.anc, s.n};
+        const float len = (float)(t1 - t0);
+        Rec run = rec_identity();  // the earlier segments, folded newest first
+        if (j == 0) {
+            if (a.P > 1) rec_publish(a, b, j, c, local, tag_incl);
+        } else {
+            rec_publish(a, b, j, c, local, tag_loc);
+            float span = 0.f;
+            int64_t m = j - 1;
+            bool done = false;
+            uint32_t nap = 32;
+            for (uint32_t it = 0; it <= a.spin_limit && !done; ++it) {
+                Rec rec[kBwdLook];
+                int kind[kBwdLook];
 #pragma unroll
-            for (int i = 0; i < kScanBlk; ++i)
-                if (i < nb) seg[i] = load_rec(a, seg_index(a, b, j0 + i, c));
+                for (int d = 0; d < kBwdLook; ++d)
+                    kind[d] = m - d >= 0 ? rec_read(a, b, m - d, c, tag_loc, tag_incl, rec[d]) : 0;
+                bool progressed = false;
 #pragma unroll
-            for (int i = 0; i < kScanBlk; ++i)
-                if (i < nb) run = rec_combine(run, seg[i], seg_len(a, j0 + i), w2);
-        }
-    }
-    agg[g][lane] = run;
-    __syncthreads();
-    if (!live) return;
-    Rec carry = rec_identity();  // the groups before this one, in time order
-    for (int q = 0; q < g; ++q) carry = rec_combine(carry, agg[q][lane], group_len(a, q), w2);
-    for (int64_t j0 = sp.j0; j0 < sp.j1; j0 += kScanBlk) {
-        const int nb = (int)min64(kScanBlk, sp.j1 - j0);
-        Rec seg[kScanBlk];
-#pragma unroll
-        for (int i = 0; i < kScanBlk; ++i)
-            if (i < nb) seg[i] = load_rec(a, seg_index(a, b, j0 + i, c));
-#pragma unroll
-        for (int i = 0; i < kScanBlk; ++i) {
-            if (i < nb) {
-                const int64_t si = seg_index(a, b, j0 + i, c);
-                a.fs[si] = carry.a;
-                a.fs[SP + si] = carry.b;
-                a.fs[2 * SP + si] = carry.anc;
-                a.fs[3 * SP + si] = carry.n;
-                carry = rec_combine(carry, seg[i], seg_len(a, j0 + i), w2);
+                for (int d = 0; d < kBwdLook; ++d) {
+                    if (done || kind[d] == 0) break;
+                    progressed = true;
+                    run = rec_combine(rec[d], run, span, w2);
+                    if (kind[d] == 2) {
+                        done = true;
+                    } else {
+                        span += (float)kSeg;  // every segment before the last is whole
+                        if (--m < 0) done = true;
+                    }
+                }
+                if (progressed) {
+                    nap = 32;
+                } else {
+                    __nanosleep(nap);
+                    nap = nap < 512 ? nap * 2 : 512;
+                }
             }
+            if (!done) {  // gave up: record it, go on with what is there (the gradients are invalid)
+                atomicCAS(&a.hdr->error, kDevOk, (uint32_t)kDevTimeoutCarry);
+                atomicCAS(a.dev_err, kDevOk, (uint32_t)kDevTimeoutCarry);
+            }
+            if (j + 1 < a.P) rec_publish(a, b, j, c, rec_combine(run, local, len, w2), tag_incl);
+        }
+        const int64_t si = seg_index(a, b, j, c), SP = a.B * a.P * a.C;
+        a.fs[si] = run.a;
+        a.fs[SP + si] = run.b;
+        a.fs[2 * SP + si] = run.anc;
+        a.fs[3 * SP + si] = run.n;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const uint32_t finished = atomicAdd(&a.hdr->done_f, 1u) + 1u;
+        if (finished == gridDim.x) {
+            atomicExch(&a.hdr->ticket_f, 0u);
+            atomicExch(&a.hdr->done_f, 0u);
+            atomicExch(&a.hdr->epoch_f, epoch30);
         }
     }
-}
-
-// C: each segment's forward from its starting state -> its local adjoint sums
-__global__ void __launch_bounds__(kThreads) bwd_seg_local(BwdArgs a) {
-    const int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    const int64_t j = blockIdx.y, b = blockIdx.z;
-    if (c >= a.C) return;
-    const float w2 = a.w[c] * kLog2e, u2 = a.u[c] * kLog2e;
-    const int64_t t0 = j * kSeg, t1 = min64(a.T, t0 + kSeg);
-    const int64_t base = b * a.T * a.C + c;
-    const int64_t si = seg_index(a, b, j, c), SP = a.B * a.P * a.C;
-    FwdState s = load_state(a, si);
-    LocalSums ls{0.f, 0.f, 0.f, 0.f, kRNone, 0.f};
-    forward_span<true, true>(a, base, t0, t1, s, u2, w2,
-                             [&](int i, const FwdOut& o, float g) { ls.add((float)i, g, o, w2); });
-    a.as[si] = ls.x;
-    a.as[SP + si] = ls.y;
-    a.as[2 * SP + si] = ls.xp;
-    a.as[3 * SP + si] = ls.yp;
-    a.as[4 * SP + si] = fmaf(ls.Rj, w2, ls.Rq);
 }
 
 // What leaves a span of len steps to its left: its local sums plus the sums entering it from
-// the right carried across it (X decays by e^{-w len}; X' also gains len X).
+// the right carried across it (X decays by e^{-w len}; X' also gains len X).  Spans compose
+// associatively: (A then B) leaves adj_compose(loc_A, loc_B, len_A) given nothing from the right.
 __device__ __forceinline__ Adj adj_compose(const Adj& loc, const Adj& in, float len, float w2) {
     const float rin = in.r + len * w2;
     const float rn = fminf(loc.r, rin);
@@ -332,112 +360,178 @@ __device__ __forceinline__ Adj adj_compose(const Adj& loc, const Adj& in, float 
     return out;
 }
 
-__device__ __forceinline__ Adj load_adj(const BwdArgs& a, int64_t si) {
-    const int64_t SP = a.B * a.P * a.C;
-    return Adj{a.as[si], a.as[SP + si], a.as[2 * SP + si], a.as[3 * SP + si], a.as[4 * SP + si]};
+// Published adjoint sums: five 64-bit words per (sequence, segment, channel), each the value's
+// bits in the low half and the launch epoch with the record's kind (1 local sums, 2 inclusive)
+// in the high half.  Aligned 64-bit accesses are single-copy atomic, so a reader that finds one
+// tag in all five words holds one consistent record: no fence and no flag.  The local sums are
+// overwritten by the inclusive ones (same thread, word by word), so a reader may catch mixed
+// tags and then reads again.  Words are stored word-major per (sequence, segment), so a warp's
+// access to one word of 32 channels is contiguous.
+__device__ __forceinline__ uint64_t* adj_slot(const BwdArgs& a, int64_t b, int64_t j) {
+    return a.slots + (b * a.P + j) * 5 * a.C;
 }
 
-// D: per channel, local sums composed right to left -> each segment's incoming sums
-__global__ void __launch_bounds__(kScanThreadsB) bwd_seg_adjoint_carry(BwdArgs a) {
-    __shared__ Adj agg[kGroups][kScanCh];
-    const int lane = threadIdx.x % kScanCh, g = threadIdx.x / kScanCh;
-    const int64_t c = (int64_t)blockIdx.x * kScanCh + lane, b = blockIdx.y;
-    const bool live = c < a.C;
-    const float w2 = live ? a.w[c] * kLog2e : 0.f;
-    const GroupSpan sp = group_span(a, g);
-    const int64_t SP = a.B * a.P * a.C;
-    Adj run = adj_empty();
-    if (live) {
-        for (int64_t j1 = sp.j1; j1 > sp.j0; j1 -= kScanBlk) {
-            const int nb = (int)min64(kScanBlk, j1 - sp.j0);
-            Adj loc[kScanBlk];
+__device__ __forceinline__ void adj_publish(const BwdArgs& a, int64_t b, int64_t j, int64_t c, const Adj& s,
+                                            uint32_t tag) {
+    uint64_t* p = adj_slot(a, b, j) + c;
+    const float f[5] = {s.x, s.y, s.xp, s.yp, s.r};
 #pragma unroll
-            for (int i = 0; i < kScanBlk; ++i)
-                if (i < nb) loc[i] = load_adj(a, seg_index(a, b, j1 - 1 - i, c));
+    for (int i = 0; i < 5; ++i) st_relaxed_u64(p + i * a.C, ((uint64_t)tag << 32) | __float_as_uint(f[i]));
+}
+
+// 2 inclusive, 1 local sums, 0 nothing usable yet (stale, or caught half overwritten)
+__device__ __forceinline__ int adj_read(const BwdArgs& a, int64_t b, int64_t j, int64_t c, uint32_t tag_loc,
+                                        uint32_t tag_incl, Adj& out) {
+    const uint64_t* p = adj_slot(a, b, j) + c;
+    uint64_t wd[5];
 #pragma unroll
-            for (int i = 0; i < kScanBlk; ++i)
-                if (i < nb) run = adj_compose(loc[i], run, seg_len(a, j1 - 1 - i), w2);
-        }
+    for (int i = 0; i < 5; ++i) wd[i] = ld_relaxed_u64(p + i * a.C);
+    const uint32_t t0 = (uint32_t)(wd[0] >> 32);
+    bool same = t0 == tag_loc || t0 == tag_incl;
+#pragma unroll
+    for (int i = 1; i < 5; ++i) same = same && (uint32_t)(wd[i] >> 32) == t0;
+    if (!same) return 0;
+    out = Adj{__uint_as_float((uint32_t)wd[0]), __uint_as_float((uint32_t)wd[1]), __uint_as_float((uint32_t)wd[2]),
+              __uint_as_float((uint32_t)wd[3]), __uint_as_float((uint32_t)wd[4])};
+    return t0 == tag_incl ? 2 : 1;
+}
+
+// R: the segments in reverse time order, 128 channels of one (sequence, segment) per block
+__global__ void __launch_bounds__(kThreads) bwd_seg_reverse(BwdArgs a, int64_t cx) {
+    extern __shared__ float sm[];  // [kSeg][3][kThreads]: q, 1 / Dn, y per position
+    __shared__ uint32_t s_ticket, s_epoch;
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        s_ticket = atomicAdd(&a.hdr->ticket, 1u);
+        s_epoch = (*reinterpret_cast<volatile uint32_t*>(&a.hdr->epoch) + 1u) & 0x3FFFFFFFu;
     }
-    agg[g][lane] = run;
     __syncthreads();
-    if (!live) return;
-    Adj in = adj_empty();  // the groups after this one, composed right to left
-    for (int q = kGroups - 1; q > g; --q) in = adj_compose(agg[q][lane], in, group_len(a, q), w2);
-    for (int64_t j1 = sp.j1; j1 > sp.j0; j1 -= kScanBlk) {
-        const int nb = (int)min64(kScanBlk, j1 - sp.j0);
-        Adj loc[kScanBlk];
+    const int64_t unit = s_ticket;
+    const uint32_t epoch30 = s_epoch;
+    const uint32_t tag_loc = (epoch30 << 2) | 1u, tag_incl = (epoch30 << 2) | 2u;
+    // tickets hand out the last segments first, then (sequence, channel block) within a segment
+    const int64_t per_seg = a.B * cx;
+    const int64_t j = a.P - 1 - unit / per_seg;
+    const int64_t b = (unit % per_seg) / cx, cb = unit % cx;
+    const int64_t c = cb * kThreads + tid;
+    const bool live = unit < a.P * per_seg && c < a.C;
+    if (live) {
+        const float w2 = a.w[c] * kLog2e, u2 = a.u[c] * kLog2e;
+        const int64_t t0 = j * kSeg, t1 = min64(a.T, t0 + kSeg);
+        const int64_t base = b * a.T * a.C + c;
+        const int64_t si = seg_index(a, b, j, c);
+        // forward from the starting state: per-position values kept, local sums accumulated
+        FwdState fsd = load_state(a, si);
+        LocalSums ls{0.f, 0.f, 0.f, 0.f, kRNone, 0.f};
+        forward_span<true, true>(a, base, t0, t1, fsd, u2, w2, [&](int i, const FwdOut& o, float g) {
+            sm[(i * 3 + 0) * kThreads + tid] = o.q;
+            sm[(i * 3 + 1) * kThreads + tid] = o.rd;
+            sm[(i * 3 + 2) * kThreads + tid] = o.y;
+            ls.add((float)i, g, o, w2);
+        });
+        const Adj local{ls.x, ls.y, ls.xp, ls.yp, fmaf(ls.Rj, w2, ls.Rq)};
+        const float len = (float)(t1 - t0);
+        // the incoming sums: the later segments' sums composed, nearest first, until one that
+        // already holds everything to its right (or the sequence's end)
+        Adj incoming = adj_empty();
+        if (j + 1 < a.P) {
+            adj_publish(a, b, j, c, local, tag_loc);
+            Adj acc = adj_empty();
+            float span = 0.f;
+            int64_t m = j + 1;
+            bool done = false;
+            uint32_t nap = 32;
+            for (uint32_t it = 0; it <= a.spin_limit && !done; ++it) {
+                // kBwdLook slots per round trip: all loads issued before any is examined
+                Adj rec[kBwdLook];
+                int kind[kBwdLook];
 #pragma unroll
-        for (int i = 0; i < kScanBlk; ++i)
-            if (i < nb) loc[i] = load_adj(a, seg_index(a, b, j1 - 1 - i, c));
+                for (int d = 0; d < kBwdLook; ++d)
+                    kind[d] = m + d < a.P ? adj_read(a, b, m + d, c, tag_loc, tag_incl, rec[d]) : 0;
+                bool progressed = false;
 #pragma unroll
-        for (int i = 0; i < kScanBlk; ++i) {
-            if (i < nb) {
-                const int64_t j = j1 - 1 - i, si = seg_index(a, b, j, c);
-                a.as[si] = in.x;
-                a.as[SP + si] = in.y;
-                a.as[2 * SP + si] = in.xp;
-                a.as[3 * SP + si] = in.yp;
-                a.as[4 * SP + si] = in.r;
-                in = adj_compose(loc[i], in, seg_len(a, j), w2);
+                for (int d = 0; d < kBwdLook; ++d) {
+                    if (done || kind[d] == 0) break;
+                    progressed = true;
+                    if (kind[d] == 2) {
+                        incoming = adj_compose(acc, rec[d], span, w2);
+                        done = true;
+                    } else {
+                        acc = adj_compose(acc, rec[d], span, w2);
+                        span += (float)(min64(a.T, (m + 1) * kSeg) - m * kSeg);
+                        if (++m >= a.P) {
+                            incoming = acc;
+                            done = true;
+                        }
+                    }
+                }
+                if (progressed) {
+                    nap = 32;
+                } else {
+                    __nanosleep(nap);
+                    nap = nap < 512 ? nap * 2 : 512;
+                }
+            }
+            if (!done) {  // gave up: record it, go on with what is there (the gradients are invalid)
+                atomicCAS(&a.hdr->error, kDevOk, (uint32_t)kDevTimeoutCarry);
+                atomicCAS(a.dev_err, kDevOk, (uint32_t)kDevTimeoutCarry);
+                incoming = acc;
             }
         }
-    }
-}
-
-// E: each segment's forward again (per-position values into shared memory), then its adjoint
-// recurrence from its incoming sums -> gradients
-__global__ void __launch_bounds__(kThreads) bwd_seg_grads(BwdArgs a) {
-    extern __shared__ float sm[];  // [kSeg][3][kThreads]
-    const int tid = threadIdx.x;
-    const int64_t c = (int64_t)blockIdx.x * kThreads + tid;
-    const int64_t j = blockIdx.y, b = blockIdx.z;
-    if (c >= a.C) return;  // no block-wide synchronisation below: each thread uses its own column
-    const float w2 = a.w[c] * kLog2e, u2 = a.u[c] * kLog2e;
-    const int64_t t0 = j * kSeg, t1 = min64(a.T, t0 + kSeg);
-    const int64_t base = b * a.T * a.C + c;
-    const int64_t si = seg_index(a, b, j, c), SP = a.B * a.P * a.C;
-    FwdState fsd = load_state(a, si);
-    forward_span<true, false>(a, base, t0, t1, fsd, u2, w2, [&](int i, const FwdOut& o, float) {
-        sm[(i * 3 + 0) * kThreads + tid] = o.q;
-        sm[(i * 3 + 1) * kThreads + tid] = o.rd;
-        sm[(i * 3 + 2) * kThreads + tid] = o.y;
-    });
-    Adj s{a.as[si], a.as[SP + si], a.as[2 * SP + si], a.as[3 * SP + si], a.as[4 * SP + si]};
-    float sgw = 0.f, sgu = 0.f;
-    auto step = [&](int64_t t, float kt, float vt, float g) {
-        const int i = (int)(t - t0);
-        const FwdOut o{sm[(i * 3 + 0) * kThreads + tid], sm[(i * 3 + 1) * kThreads + tid],
-                       sm[(i * 3 + 2) * kThreads + tid]};
-        float gk, gv;
-        adj_step(s, kt * kLog2e, vt, g, o, u2, w2, gk, gv, sgw, sgu);
-        a.gk[base + t * a.C] = gk;
-        a.gv[base + t * a.C] = gv;
-    };
-    int64_t t = t1;
-    for (; t - kBlk >= t0; t -= kBlk) {
-        float kb[kBlk], vb[kBlk], gb[kBlk];
+        if (j > 0) adj_publish(a, b, j, c, adj_compose(local, incoming, len, w2), tag_incl);
+        // the adjoint recurrence right to left from the incoming sums
+        Adj st = incoming;
+        float sgw = 0.f, sgu = 0.f;
+        auto step = [&](int64_t t, float kt, float vt, float g) {
+            const int i = (int)(t - t0);
+            const FwdOut o{sm[(i * 3 + 0) * kThreads + tid], sm[(i * 3 + 1) * kThreads + tid],
+                           sm[(i * 3 + 2) * kThreads + tid]};
+            float gk, gv;
+            adj_step(st, kt * kLog2e, vt, g, o, u2, w2, gk, gv, sgw, sgu);
+            a.gk[base + t * a.C] = gk;
+            a.gv[base + t * a.C] = gv;
+        };
+        int64_t t = t1;
+        for (; t - kBlk >= t0; t -= kBlk) {
+            float kb[kBlk], vb[kBlk], gb[kBlk];
 #pragma unroll
-        for (int i = 0; i < kBlk; ++i) {
-            const int64_t at = base + (t - 1 - i) * a.C;
-            kb[i] = a.k[at];
-            vb[i] = a.v[at];
-            gb[i] = a.gy[at];
+            for (int i = 0; i < kBlk; ++i) {
+                const int64_t at = base + (t - 1 - i) * a.C;
+                kb[i] = a.k[at];
+                vb[i] = a.v[at];
+                gb[i] = a.gy[at];
+            }
+#pragma unroll
+            for (int i = 0; i < kBlk; ++i) step(t - 1 - i, kb[i], vb[i], gb[i]);
         }
-#pragma unroll
-        for (int i = 0; i < kBlk; ++i) step(t - 1 - i, kb[i], vb[i], gb[i]);
+        for (; t > t0; --t) {
+            const int64_t at = base + (t - 1) * a.C;
+            step(t - 1, a.k[at], a.v[at], a.gy[at]);
+        }
+        atomicAdd(&a.gw[c], sgw);
+        atomicAdd(&a.gu[c], sgu);
     }
-    for (; t > t0; --t) {
-        const int64_t at = base + (t - 1) * a.C;
-        step(t - 1, a.k[at], a.v[at], a.gy[at]);
+    // the launch's last block resets the counters and advances the epoch
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const uint32_t finished = atomicAdd(&a.hdr->done, 1u) + 1u;
+        if (finished == gridDim.x) {
+            atomicExch(&a.hdr->ticket, 0u);
+            atomicExch(&a.hdr->done, 0u);
+            atomicExch(&a.hdr->epoch, epoch30);
+        }
     }
-    atomicAdd(&a.gw[c], sgw);
-    atomicAdd(&a.gu[c], sgu);
 }
 
 }  // namespace
 
 int64_t backward_segments(int64_t T) { return (T + kSeg - 1) / kSeg; }
+
+size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t C) {
+    const size_t bpc = (size_t)B * (size_t)backward_segments(T) * (size_t)C;
+    return kBwdHeaderBytes + bpc * 4 * sizeof(float) + bpc * 4 * sizeof(uint64_t) + bpc * 5 * sizeof(uint64_t);
+}
 
 cudaError_t launch_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
                             const float* v, const float* gy, float* gk, float* gv, float* gw, float* gu, void* ws,
@@ -462,16 +556,28 @@ cudaError_t launch_backward(int64_t B, int64_t T, int64_t C, const float* w, con
     a.gw = gw;
     a.gu = gu;
     const int64_t SP = B * a.P * C;
-    a.fs = static_cast<float*>(ws);
-    a.as = a.fs + 4 * SP;
-    const unsigned cx = (unsigned)((C + kThreads - 1) / kThreads);
-    const dim3 seg_grid(cx, (unsigned)a.P, (unsigned)B);
-    const dim3 scan_grid((unsigned)((C + kScanCh - 1) / kScanCh), (unsigned)B);
-    bwd_seg_forward<<<seg_grid, kThreads, 0, s>>>(a);
-    bwd_seg_carry<<<scan_grid, kScanThreadsB, 0, s>>>(a);
-    bwd_seg_local<<<seg_grid, kThreads, 0, s>>>(a);
-    bwd_seg_adjoint_carry<<<scan_grid, kScanThreadsB, 0, s>>>(a);
-    bwd_seg_grads<<<seg_grid, kThreads, kGradSmem, s>>>(a);
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    a.hdr = reinterpret_cast<BwdHeader*>(base);
+    a.fs = reinterpret_cast<float*>(base + kBwdHeaderBytes);
+    a.fslots = reinterpret_cast<uint64_t*>(base + kBwdHeaderBytes + (size_t)SP * 4 * sizeof(float));
+    a.slots = a.fslots + (size_t)SP * 4;
+    a.dev_err = device_status_word();
+    if (!a.dev_err) return cudaErrorInvalidValue;
+    a.spin_limit = kSpinLimitDefault;
+    const int64_t cx = (C + kThreads - 1) / kThreads;
+    const int64_t units = a.P * B * cx;
+    if (units > INT32_MAX) return cudaErrorInvalidValue;
+    static uint64_t attr_done = 0;  // per device; set once so captured launches issue no attribute call
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64 || !(attr_done & (1ull << dev))) {
+        e = cudaFuncSetAttribute(bwd_seg_reverse, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGradSmem);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) attr_done |= 1ull << dev;
+    }
+    bwd_seg_starts<<<(unsigned)units, kThreads, 0, s>>>(a, cx);
+    bwd_seg_reverse<<<(unsigned)units, kThreads, kGradSmem, s>>>(a, cx);
     return cudaGetLastError();
 }
 

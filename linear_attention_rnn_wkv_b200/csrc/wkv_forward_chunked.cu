@@ -466,11 +466,6 @@ cudaError_t launch_lc(const ForwardArgs& a, const ChunkGeom& g, const ChunkParam
 
 }  // namespace
 
-// Bulk rows run the tensor-memory pipeline (1) or the shared-memory one (0).
-#ifndef WKV_FORWARD_TMEM
-#define WKV_FORWARD_TMEM 1
-#endif
-
 bool chunk_geometry(int64_t B, int64_t T, int64_t C, int io, int chunk, ChunkGeom* g) {
     const int esize = io == 1 ? 2 : 4;
     const bool bulk = ((C * esize) % 16) == 0;
@@ -505,11 +500,11 @@ bool chunk_geometry(int64_t B, int64_t T, int64_t C, int io, int chunk, ChunkGeo
     return true;
 }
 
-bool chunked_path_fuses_gate(const ChunkGeom& g) { return g.pipe && WKV_FORWARD_TMEM; }
+bool chunked_path_fuses_gate(const ChunkGeom& g) { return g.pipe; }
 
 cudaError_t launch_forward_chunked(const ForwardArgs& a, const ChunkGeom& g, void* ws, int64_t drop_unit,
                                    cudaStream_t s) {
-    if (g.pipe) return WKV_FORWARD_TMEM ? launch_forward_tmem(a, g, ws, drop_unit, s) : launch_forward_pipe(a, g, ws, drop_unit, s);
+    if (g.pipe) return launch_forward_tmem(a, g, ws, drop_unit, s);
     unsigned char* base = static_cast<unsigned char*>(ws);
     const size_t flags_bytes = ((size_t)g.U * 4 + 15) / 16 * 16;
     ChunkParams cp;

@@ -1,15 +1,14 @@
 // Persistent, warp-specialised chunked WKV forward that parks each tile in tensor memory
 // (the default chunked path when rows are 16-byte multiples).
 //
-// The arithmetic and the inter-CTA protocol are those of the shared-memory pipeline
-// (wkv_forward_pipe.cu): a unit is a tile of Ts = 8 * LC time steps by 64 channels; units
-// are taken by an atomic ticket in time-segment-major order; each unit's chunk summaries
-// fold into a tile aggregate, a decoupled look-back over earlier segments of the same
-// channel group yields the carry, and each chunk is re-scanned from its carry to write y
-// (the decay telescopes: RWKV transformer-math page, aicassindra.com, section "Why it
-// collapses into a recurrence").
+// A unit is a tile of Ts = 8 * LC time steps by 64 channels; units are taken by an atomic
+// ticket in time-segment-major order; each unit's chunk summaries fold into a tile
+// aggregate, a decoupled look-back over earlier segments of the same channel group yields
+// the carry, and each chunk is re-scanned from its carry to write y (the decay telescopes:
+// RWKV transformer-math page, aicassindra.com, section "Why it collapses into a
+// recurrence").
 //
-// What changes is where a tile waits for its carry.  A unit's k and v rows are needed
+// Where a tile waits for its carry matters most.  A unit's k and v rows are needed
 // twice, by the summaries and, after the look-back, by the re-scan; in between the tile
 // sits idle for several microseconds.  Here the TMA lands a tile in a shared-memory stage,
 // each summarising warp copies its chunk into its quadrant of the SM's tensor memory
@@ -145,12 +144,35 @@ __device__ __forceinline__ void gate_pair(float (&y)[2], const float (&r)[2]) {
 constexpr int kNWS = 8;   // chunks per tile (summarising warps, emitting warps)
 constexpr int kNL = 3;    // look-back warps
 constexpr int kCg = 64;   // channels per tile (a lane owns a pair)
-// Emitting warp sets: each set has a warp per chunk index and takes every kES-th unit.
-#ifndef WKV_TMEM_EMIT_SETS
-#define WKV_TMEM_EMIT_SETS 1
+// What the summarising warps park in tensor memory beside the values: each key's exponent
+// as seen from the chunk's last row, x_i = k_i log2 e - (L - 1 - i) w log2 e, exactly as the
+// summary used it (1), or the raw keys, from which the emitters recompute it (0).
+#ifndef WKV_TMEM_PARK_EXPONENT
+#define WKV_TMEM_PARK_EXPONENT 1
 #endif
-constexpr int kES = WKV_TMEM_EMIT_SETS;
-constexpr int kThreads = (1 + kNL + (1 + kES) * kNWS) * 32;
+constexpr bool kParkExponent = WKV_TMEM_PARK_EXPONENT != 0;
+constexpr int kThreads = (1 + kNL + 2 * kNWS) * 32;
+
+// What every role needs to know about a unit, worked out once by the producer (per
+// shared-memory stage) and copied with the unit into its tensor-memory slot: the tile's
+// geometry, and the channels' w and u (bulk-copied; entries past the last channel are
+// left from an earlier unit and only feed lanes whose results are discarded).
+struct UnitInfo {
+    int64_t row0;  // element offset of (b, t0, c0) in [B][T][C]
+    int64_t bc0;   // b * C + c0: the state index of the tile's first channel
+    int32_t unit;  // ticket, or -1 past the end
+    int32_t j;     // time segment
+    int32_t g;     // channel group
+    int32_t len;   // rows in the tile
+    int32_t nch;   // channels in the tile (even)
+    int32_t b, c0, t0;  // sequence, first channel, first row (tensor-map coordinates)
+};
+struct UnitBlock {
+    UnitInfo info;
+    float w[kCg];
+    float u[kCg];
+};
+static_assert(sizeof(UnitBlock) % 16 == 0, "unit blocks are copied as 16-byte words");
 
 template <typename TIO, int LC, int NS, int NT, bool GATE = false>
 struct TmLayout {
@@ -158,30 +180,40 @@ struct TmLayout {
     static constexpr int Ts = kNWS * LC;
     static constexpr size_t tile = sizeof(TIO) * Ts * Cg;  // one array (k or v)
     static constexpr size_t stage = align128(2 * tile);     // shared-memory stage: k tile, v tile
-    // unit slot: chunk records [NWS][Cg], carries [Cg], chunk maxima [NWS][Cg]
+    // unit slot: chunk records [NWS][Cg], carries [Cg], chunk maxima [NWS][Cg], the unit's block
     static constexpr size_t recs_off = 0;
     static constexpr size_t carry_off = recs_off + sizeof(Rec) * kNWS * Cg;
     static constexpr size_t mx_off = carry_off + sizeof(Rec) * Cg;
-    static constexpr size_t slot = align128(mx_off + sizeof(float) * kNWS * Cg);
+    static constexpr size_t ub_off = mx_off + sizeof(float) * kNWS * Cg;
+    static constexpr size_t slot = align128(ub_off + sizeof(UnitBlock));
     static constexpr int BR = kBoxRows < Ts ? kBoxRows : Ts;  // rows per TMA box
     static constexpr int NB = Ts / BR;
     static constexpr size_t slots_off = NS * stage;
     static constexpr size_t bars_off = slots_off + NT * slot;
-    static constexpr int NBARS = NS * (NB + 1) + NT * 3;  // per stage: NB full + 1 empty; per slot: chunks, carry, empty
-    static constexpr size_t misc_off = bars_off + NBARS * 8;  // slot unit ids [NT], end index, epoch, tensor memory base
-    static constexpr size_t stage_unit_off = misc_off + NT * 8 + 8 + 8;  // stage unit ids [NS]
+    // per stage: NB full + 1 empty + 1 unit block; per slot: chunks, carry, empty
+    static constexpr int NBARS = NS * (NB + 2) + NT * 3;
+    static constexpr size_t misc_off = bars_off + NBARS * 8;  // end index, epoch, tensor memory base
+    static constexpr size_t stage_ub_off = align128(misc_off + 16);  // the stages' unit blocks [NS]
     // gated forward: each emitting warp's chunk of r (TMA box of LC rows x Cg) and its barrier
     static constexpr size_t rbuf_bytes = align128(sizeof(TIO) * LC * Cg);
-    static constexpr size_t rbuf_off = align128(stage_unit_off + NS * 8);
+    static constexpr size_t rbuf_off = align128(stage_ub_off + NS * sizeof(UnitBlock));
     static constexpr size_t rbar_off = rbuf_off + (GATE ? kNWS * rbuf_bytes : 0);
-    static constexpr size_t total = rbar_off + (GATE ? kNWS * 8 : 0);
+    // each emitting warp's chunk of y, written row by row and stored by one TMA copy; the gated
+    // forward writes each output over its own receptance in the r buffer
+    static constexpr size_t ybuf_bytes = align128(sizeof(TIO) * LC * Cg);
+    static constexpr size_t ybuf_off = GATE ? rbuf_off : align128(rbar_off);
+    static constexpr size_t total = GATE ? rbar_off + kNWS * 8 : ybuf_off + kNWS * ybuf_bytes;
     // tensor memory: words per row per lane, columns per chunk array, per chunk, per unit and quadrant
     static constexpr int W = Pk<TIO>::W;
-    static constexpr int CPA = LC * W;
-    static constexpr int CPC = 2 * CPA;
+    // words per row of the first array: the key's exponent as an fp32 pair, or the raw keys
+    static constexpr int WK = kParkExponent ? 2 : W;
+    static constexpr int CPAK = LC * WK;  // columns of a chunk's first array (exponents or keys)
+    static constexpr int CPAV = LC * W;   // columns of a chunk's values
+    static constexpr int CPC = CPAK + CPAV;
     static constexpr int CPU = (kNWS / 4) * CPC;
-    static constexpr int SR = 8 / W;   // rows per tensor-memory slice (8 words: two slices of k and v
-    static constexpr int SW = SR * W;  // stay in registers while the next pair is read)
+    static constexpr int SR = 8 / W;     // rows per tensor-memory slice (two slices of each array
+    static constexpr int SWK = SR * WK;  // stay in registers while the next pair is read)
+    static constexpr int SW = SR * W;
     static_assert(NT * CPU <= 512, "unit slots exceed the tensor memory");
     static_assert(LC % SR == 0, "slices must tile a chunk");
 };
@@ -189,11 +221,12 @@ struct TmLayout {
 template <typename TIO, int LC, int NS, int NT, bool GATE>
 __global__ void __launch_bounds__(kThreads, 1)
     tmem_kernel(ForwardArgs args, PipeParams pp, const __grid_constant__ CUtensorMap tmk,
-                const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmr) {
+                const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmr,
+                const __grid_constant__ CUtensorMap tmy) {
     using Lay = TmLayout<TIO, LC, NS, NT, GATE>;
-    static_assert(!GATE || kES == 1, "one r buffer per chunk index");
     constexpr int V = 2;
-    constexpr int Cg = Lay::Cg, Ts = Lay::Ts, NB = Lay::NB, BR = Lay::BR, W = Lay::W, SR = Lay::SR, SW = Lay::SW;
+    constexpr int Cg = Lay::Cg, Ts = Lay::Ts, NB = Lay::NB, BR = Lay::BR, W = Lay::W, SR = Lay::SR, SW = Lay::SW,
+                  SWK = Lay::SWK;
     constexpr int W_L0 = 1, W_S0 = 1 + kNL, W_E0 = 1 + kNL + kNWS;
     // Where a unit takes its slot.  With few slots (fp32: 4) they are the scarce resource and
     // the summarisers take one only once the rows have landed; with more (bf16: 8) the
@@ -203,22 +236,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     static_assert(W_S0 % 4 == 0 && W_E0 % 4 == 0, "a chunk's summariser and emitter must share a quadrant");
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bars_off);
-    int64_t* slot_unit = reinterpret_cast<int64_t*>(smem + Lay::misc_off);
-    volatile int64_t* s_iend = reinterpret_cast<volatile int64_t*>(slot_unit + NT);
-    uint32_t* s_epoch = reinterpret_cast<uint32_t*>(slot_unit + NT + 1);
+    volatile int64_t* s_iend = reinterpret_cast<volatile int64_t*>(smem + Lay::misc_off);
+    uint32_t* s_epoch = reinterpret_cast<uint32_t*>(smem + Lay::misc_off + 8);
     uint32_t* s_tmem = s_epoch + 1;
-    int64_t* stage_unit = reinterpret_cast<int64_t*>(smem + Lay::stage_unit_off);
-    auto dfull = [&](int s, int b) { return &bars[s * (NB + 1) + b]; };
-    auto dempty = [&](int s) { return &bars[s * (NB + 1) + NB]; };
-    auto chunks_bar = [&](int t) { return &bars[NS * (NB + 1) + t * 3 + 0]; };
-    auto carry_bar = [&](int t) { return &bars[NS * (NB + 1) + t * 3 + 1]; };
-    auto uempty = [&](int t) { return &bars[NS * (NB + 1) + t * 3 + 2]; };
+    auto dfull = [&](int s, int b) { return &bars[s * (NB + 2) + b]; };
+    auto dempty = [&](int s) { return &bars[s * (NB + 2) + NB]; };
+    auto dunit = [&](int s) { return &bars[s * (NB + 2) + NB + 1]; };  // the stage's unit block is written
+    auto chunks_bar = [&](int t) { return &bars[NS * (NB + 2) + t * 3 + 0]; };
+    auto carry_bar = [&](int t) { return &bars[NS * (NB + 2) + t * 3 + 1]; };
+    auto uempty = [&](int t) { return &bars[NS * (NB + 2) + t * 3 + 2]; };
     auto ktile = [&](int s) { return reinterpret_cast<TIO*>(smem + s * Lay::stage); };
     auto vtile = [&](int s) { return reinterpret_cast<TIO*>(smem + s * Lay::stage + Lay::tile); };
     auto slotp = [&](int t) { return smem + Lay::slots_off + t * Lay::slot; };
     auto recs = [&](int t) { return reinterpret_cast<Rec*>(slotp(t) + Lay::recs_off); };
     auto carries = [&](int t) { return reinterpret_cast<Rec*>(slotp(t) + Lay::carry_off); };
     auto chunk_max = [&](int t) { return reinterpret_cast<float*>(slotp(t) + Lay::mx_off); };
+    auto slot_ub = [&](int t) { return reinterpret_cast<UnitBlock*>(slotp(t) + Lay::ub_off); };
+    auto stage_ub = [&](int s) { return reinterpret_cast<UnitBlock*>(smem + Lay::stage_ub_off) + s; };
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -236,6 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < NS; ++s) {
             for (int b = 0; b < NB; ++b) mbar_init(dfull(s, b), 1);
             mbar_init(dempty(s), kNWS);
+            mbar_init(dunit(s), 1);
         }
         if (GATE)
             for (int e = 0; e < kNWS; ++e) mbar_init(reinterpret_cast<uint64_t*>(smem + Lay::rbar_off) + e, 1);
@@ -258,54 +293,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // this warp's quadrant; the columns of chunk c's array a (0 k, 1 v) in unit slot t
     const uint32_t tq = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    auto tcol = [&](int t, int c, int a) { return (uint32_t)(t * Lay::CPU + (c >> 2) * Lay::CPC + a * Lay::CPA); };
-
-    struct Geo {
-        int64_t j, g, b, c0, t0;
-        int len, nch;
-    };
-    auto geo = [&](int64_t unit) {
-        Geo q;
-        q.j = unit / pp.G;
-        q.g = unit % pp.G;
-        q.b = q.g / pp.groups_per_b;
-        q.c0 = (q.g % pp.groups_per_b) * Cg;
-        q.t0 = q.j * Ts;
-        q.len = (int)min64(Ts, T - q.t0);
-        q.nch = (int)min64(Cg, C - q.c0);
-        return q;
-    };
+    auto tcol = [&](int t, int c, int a) { return (uint32_t)(t * Lay::CPU + (c >> 2) * Lay::CPC + a * Lay::CPAK); };
 
     if (warp == 0) {
         // ------------------------------- producer -------------------------------
+        // Lane 0 takes the tickets, works out each unit's geometry once for every other role
+        // and issues the copies: the k and v boxes (`full`) and the tile's w and u (`unit`, with
+        // the geometry).  The next ticket is requested as soon as the current unit's copies are
+        // issued, so its round trip overlaps the wait for the next free stage (safe: the
+        // block handles its units in ticket order whatever it has taken, and every
+        // cross-block wait is on a smaller ticket).
         if (lane == 0) {
+            uint32_t tk_next = atomicAdd(&pp.hdr->ticket, 1u);
             for (int64_t i = 0;; ++i) {
                 const int s = (int)(i % NS);
                 if (i >= NS && !mbar_wait(dempty(s), (uint32_t)((i / NS - 1) & 1), lim)) report(kDevTimeoutCopy);
                 const int t = (int)(i % NT);
                 if (!kLateSlot && i >= NT && !mbar_wait(uempty(t), (uint32_t)((i / NT - 1) & 1), lim))
                     report(kDevTimeoutCopy);
-                const uint32_t tk = atomicAdd(&pp.hdr->ticket, 1u);
+                const uint32_t tk = tk_next;
                 if (tk >= (uint32_t)pp.U + gridDim.x) report(kDevBadWorkspace);
+                UnitBlock* ub = stage_ub(s);
                 if (tk >= (uint32_t)pp.U) {
                     *s_iend = i;
-                    stage_unit[s] = -1;
-                    if (!kLateSlot) slot_unit[t] = -1;
+                    ub->info.unit = -1;
                     for (int b = 0; b < NB; ++b) mbar_arrive(dfull(s, b));
+                    mbar_arrive(dunit(s));
                     break;
                 }
                 const int64_t unit = tk;
+                const int64_t j = unit / pp.G, g = unit % pp.G;
+                const int64_t b = g / pp.groups_per_b;
+                const int64_t c0 = (g % pp.groups_per_b) * Cg, t0 = j * Ts;
+                const int nch = (int)min64(Cg, C - c0);
                 WKV_TRACE_EVENT(unit, 0);
-                stage_unit[s] = unit;
-                if (!kLateSlot) slot_unit[t] = unit;
-                const Geo q = geo(unit);
 #pragma unroll
-                for (int b = 0; b < NB; ++b) {
-                    uint64_t* fb = dfull(s, b);
+                for (int bx = 0; bx < NB; ++bx) {
+                    uint64_t* fb = dfull(s, bx);
                     mbar_arrive_expect_tx(fb, 2u * (uint32_t)(BR * Cg * sizeof(TIO)));
-                    tma_load_3d(ktile(s) + b * BR * Cg, &tmk, (int)q.c0, (int)(q.t0 + b * BR), (int)q.b, fb);
-                    tma_load_3d(vtile(s) + b * BR * Cg, &tmv, (int)q.c0, (int)(q.t0 + b * BR), (int)q.b, fb);
+                    tma_load_3d(ktile(s) + bx * BR * Cg, &tmk, (int)c0, (int)(t0 + bx * BR), (int)b, fb);
+                    tma_load_3d(vtile(s) + bx * BR * Cg, &tmv, (int)c0, (int)(t0 + bx * BR), (int)b, fb);
                 }
+                UnitInfo& q = ub->info;
+                q.row0 = (b * T + t0) * C + c0;
+                q.bc0 = b * C + c0;
+                q.unit = (int32_t)unit;
+                q.j = (int32_t)j;
+                q.g = (int32_t)g;
+                q.len = (int)min64(Ts, T - t0);
+                q.nch = nch;
+                q.b = (int32_t)b;
+                q.c0 = (int32_t)c0;
+                q.t0 = (int32_t)t0;
+                // w and u of the tile's channels (nch is a multiple of 4: 16-byte rows); the
+                // barrier's one arrival comes after the geometry above is written
+                const uint32_t wbytes = (uint32_t)nch * (uint32_t)sizeof(float);
+                mbar_arrive_expect_tx(dunit(s), 2u * wbytes);
+                bulk_g2s(ub->w, args.w + c0, wbytes, dunit(s));
+                bulk_g2s(ub->u, args.u + c0, wbytes, dunit(s));
+                tk_next = atomicAdd(&pp.hdr->ticket, 1u);
             }
         }
         __syncwarp();
@@ -330,18 +376,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (gone) break;
             if (!got && lane == 0) report(kDevTimeoutCarry);
-            const int64_t unit = slot_unit[t];
+            const UnitInfo q = slot_ub(t)->info;
+            const int64_t unit = q.unit;
             if (unit < 0) {
                 if (lane == 0) mbar_arrive(carry_bar(t));
                 break;
             }
             if (lane == 0) WKV_TRACE_EVENT(unit, 3);
-            const Geo q = geo(unit);
             const int cl = lane * V;
             const bool lane_active = cl < q.nch;
             float w2[V];
-#pragma unroll
-            for (int c = 0; c < V; ++c) w2[c] = lane_active ? args.w[q.c0 + cl + c] * kLog2e : 0.f;
+            {
+                const float2 wp = *reinterpret_cast<const float2*>(slot_ub(t)->w + cl);
+                w2[0] = wp.x * kLog2e;
+                w2[1] = wp.y * kLog2e;
+            }
             // the first read of the newest predecessor's slot overlaps the scan
             RawPair first;
             if (q.j > 0 && lane_active) first = load_pair<Cg>(pp.slot + ((q.j - 1) * pp.G + q.g) * 4 * Cg, cl);
@@ -370,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (q.j == 0) {
 #pragma unroll
                 for (int c = 0; c < V; ++c)
-                    run[c] = (args.state_in && lane_active) ? rec_from_state(args.state_in, q.b * C + q.c0 + cl + c, BC)
+                    run[c] = (args.state_in && lane_active) ? rec_from_state(args.state_in, q.bc0 + cl + c, BC)
                                                             : rec_identity();
             } else {
 #pragma unroll
@@ -445,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane_active && q.j == pp.S - 1 && args.state_out) {
 #pragma unroll
                 for (int c = 0; c < V; ++c) {
-                    const int64_t bc = q.b * C + q.c0 + cl + c;
+                    const int64_t bc = q.bc0 + cl + c;
                     args.state_out[bc] = inc[c].a;
                     args.state_out[BC + bc] = inc[c].b;
                     args.state_out[2 * BC + bc] = rec_p(inc[c], w2[c]) * kLn2;
@@ -460,14 +509,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s = (int)(i % NS);
             const int t = (int)(i % NT);
             const uint32_t ph = (uint32_t)((i / NS) & 1);
+            if (!mbar_wait(dunit(s), ph, lim) && lane == 0) report(kDevTimeoutCopy);
             if (!mbar_wait(dfull(s, sw * LC / BR), ph, lim) && lane == 0) report(kDevTimeoutCopy);
-            const int64_t unit = stage_unit[s];
+            const UnitBlock* sub = stage_ub(s);
+            const UnitInfo q = sub->info;
+            const int64_t unit = q.unit;
             // with late slots, the unit slot (tensor-memory columns and records) is taken only
             // now that the rows are here, so a slot is held from the summaries to the re-scan's end
-            if (kLateSlot) {
-                if (i >= NT && !mbar_wait(uempty(t), (uint32_t)((i / NT - 1) & 1), lim) && lane == 0)
-                    report(kDevTimeoutCopy);
-                if (sw == 0 && lane == 0) slot_unit[t] = unit;
+            if (kLateSlot && i >= NT && !mbar_wait(uempty(t), (uint32_t)((i / NT - 1) & 1), lim) && lane == 0)
+                report(kDevTimeoutCopy);
+            if (sw == 0) {
+                // the unit block goes with the unit into its slot (the stage is reused first)
+                const uint4* src = reinterpret_cast<const uint4*>(sub);
+                uint4* dst = reinterpret_cast<uint4*>(slot_ub(t));
+                for (int x = lane; x < (int)(sizeof(UnitBlock) / 16); x += 32) dst[x] = src[x];
             }
             if (unit < 0) {
                 __syncwarp();
@@ -476,14 +531,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             if (sw == 0 && lane == 0) WKV_TRACE_EVENT(unit, 1);
-            const Geo q = geo(unit);
             const int cl = lane * V;
             const bool lane_active = cl < q.nch;
             const int r_begin = sw * LC;
             const int r_cnt = max(0, min(LC, q.len - r_begin));
             if (r_cnt > 0) {
-                const float2 w2p = lane_active ? make_float2(args.w[q.c0 + cl] * kLog2e, args.w[q.c0 + cl + 1] * kLog2e)
-                                               : make_float2(0.f, 0.f);
+                const float2 wraw = *reinterpret_cast<const float2*>(sub->w + cl);
+                const float2 w2p = make_float2(wraw.x * kLog2e, wraw.y * kLog2e);
                 const float2 L2 = make_float2(kLog2e, kLog2e);
                 const TIO* kt = ktile(s);
                 const TIO* vt = vtile(s);
@@ -500,21 +554,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // tensor memory
 #pragma unroll
                     for (int h = 0; h < LC / SR; ++h) {
-                        uint32_t kw[SW];
+                        uint32_t kw[SWK];
 #pragma unroll
                         for (int rr = 0; rr < SR; ++rr) {
                             const int r = h * SR + rr;
-                            Pk<TIO>::load(kt + (r_begin + r) * Cg + cl, &kw[rr * W]);
+                            uint32_t raw[W];
+                            Pk<TIO>::load(kt + (r_begin + r) * Cg + cl, raw);
                             const float back = FULL ? -(float)(LC - 1 - r) : -(float)(r_cnt - 1 - r);
-                            gx[r] = __ffma2_rn(make_float2(back, back), w2p,
-                                               __fmul2_rn(Pk<TIO>::unpack(&kw[rr * W]), L2));
+                            gx[r] = __ffma2_rn(make_float2(back, back), w2p, __fmul2_rn(Pk<TIO>::unpack(raw), L2));
                             if (FULL || r < r_cnt) {
                                 M0 = fmaxf(M0, gx[r].x);
                                 M1 = fmaxf(M1, gx[r].y);
                             }
+                            if (kParkExponent) {
+                                kw[rr * 2] = __float_as_uint(gx[r].x);
+                                kw[rr * 2 + 1] = __float_as_uint(gx[r].y);
+                            } else {
+#pragma unroll
+                                for (int x = 0; x < W; ++x) kw[rr * W + x] = raw[x];
+                            }
                         }
-                        TmemIO<SW>::st(tq + tcol(t, sw, 0) + h * SW, kw);
-                        TmemIO<SW>::wait_st(kw);
+                        TmemIO<SWK>::st(tq + tcol(t, sw, 0) + h * SWK, kw);
+                        TmemIO<SWK>::wait_st(kw);
                     }
                     // pass 2: v rows -> the chunk's sums relative to its maximum; rows to tensor
                     // memory
@@ -558,13 +619,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // --------------------------------- emit ---------------------------------
-        const int ew = (warp - W_E0) % kNWS;  // chunk index (the same quadrant as its summariser)
-        const int es = (warp - W_E0) / kNWS;  // emitting set: units es, es + kES, ...
+        const int ew = warp - W_E0;  // chunk index (the same quadrant as its summariser)
         // gated forward: this warp's chunk of r arrives by TMA in its own buffer
         uint64_t* rbar = reinterpret_cast<uint64_t*>(smem + Lay::rbar_off) + ew;
         const TIO* rbuf = reinterpret_cast<const TIO*>(smem + Lay::rbuf_off + ew * Lay::rbuf_bytes);
+        // this warp's chunk of y: written row by row, then stored by one TMA tensor copy (rows past
+        // T and channels past C are clipped by the copy)
+        TIO* ybuf = reinterpret_cast<TIO*>(smem + Lay::ybuf_off + ew * Lay::ybuf_bytes);
         uint32_t rphase = 0;
-        for (int64_t i = es;; i += kES) {
+        for (int64_t i = 0;; ++i) {
             const int t = (int)(i % NT);
             const uint32_t ph = (uint32_t)((i / NT) & 1);
             bool got = false, gone = false;
@@ -585,12 +648,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!WKV_WAIT_HINT) __nanosleep(32);
                 }
                 if (gone) break;
-                const int64_t u0 = slot_unit[t];
-                if (got && u0 >= 0) {
-                    const Geo q0 = geo(u0);
+                const UnitInfo q0 = slot_ub(t)->info;
+                if (got && q0.unit >= 0) {
                     if (q0.len > ew * LC) {
                         r_pending = true;
                         if (lane == 0) {
+                            bulk_wait_read();  // the previous chunk's outputs have left the buffer
                             mbar_arrive_expect_tx(rbar, (uint32_t)(LC * Cg * sizeof(TIO)));
                             tma_load_3d(const_cast<TIO*>(rbuf), &tmr, (int)q0.c0, (int)(q0.t0 + ew * LC), (int)q0.b, rbar);
                         }
@@ -603,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     got = true;
                     break;
                 }
-                // past the end: with several emitting sets, only one meets the sentinel unit
+                // past the end (the producer has recorded the last unit)
                 if (*s_iend < i) {
                     gone = true;
                     break;
@@ -612,26 +675,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (gone) break;
             if (!got && lane == 0) report(kDevTimeoutCarry);
-            const int64_t unit = slot_unit[t];
+            const UnitInfo q = slot_ub(t)->info;
+            const int64_t unit = q.unit;
             if (unit < 0) break;
             tc_fence_after();
             if (ew == 0 && lane == 0) WKV_TRACE_EVENT(unit, 8);
-            const Geo q = geo(unit);
             const int cl = lane * V;
             const bool lane_active = cl < q.nch;
             const int r_begin = ew * LC;
             const int r_cnt = max(0, min(LC, q.len - r_begin));
             if (r_cnt > 0) {
                 // the first slice's rows are read while the carry is combined below
-                uint32_t kw[SW], vw[SW];
-                TmemIO<SW>::ld(tq + tcol(t, ew, 0), kw);
+                uint32_t kw[SWK], vw[SW];
+                TmemIO<SWK>::ld(tq + tcol(t, ew, 0), kw);
                 TmemIO<SW>::ld(tq + tcol(t, ew, 1), vw);
                 float w2[V], u2[V], a[V], bb[V], R[V], nn[V];
                 bool lazy_ok = true;
+                const float2 wv = *reinterpret_cast<const float2*>(slot_ub(t)->w + cl);
+                const float2 uv = *reinterpret_cast<const float2*>(slot_ub(t)->u + cl);
+                w2[0] = wv.x * kLog2e;
+                w2[1] = wv.y * kLog2e;
+                u2[0] = uv.x * kLog2e;
+                u2[1] = uv.y * kLog2e;
 #pragma unroll
                 for (int c = 0; c < V; ++c) {
-                    w2[c] = lane_active ? args.w[q.c0 + cl + c] * kLog2e : 0.f;
-                    u2[c] = lane_active ? args.u[q.c0 + cl + c] * kLog2e : 0.f;
                     const Rec cr = lane_active
                                        ? rec_combine(carries(t)[cl + c], recs(t)[ew * Cg + cl + c], (float)r_begin, w2[c])
                                        : rec_identity();
@@ -641,8 +708,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     nn[c] = cr.n;
                     lazy_ok = lazy_ok && fabsf(u2[c]) <= kLazyLimit && w2[c] <= kLazyLimit;
                 }
-                TIO* yg = static_cast<TIO*>(args.y) + (q.b * T + q.t0) * C + q.c0;
-                TmemIO<SW>::wait_ld(kw);
+                TIO* yg = static_cast<TIO*>(args.y) + q.row0;
+                TmemIO<SWK>::wait_ld(kw);
                 TmemIO<SW>::wait_ld(vw);
                 if (GATE && r_pending) {
                     if (!mbar_wait(rbar, rphase, lim) && lane == 0) report(kDevTimeoutCopy);
@@ -665,8 +732,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int mode = lazy_ok ? 1 : 2;
                 float2 fSa = make_float2(0.f, 0.f), fSb = fSa, fnG = fSa, fic = fSa;
                 if (WKV_PIPE_FRAME && lazy_ok) {
-                    const float2 k0 = Pk<TIO>::unpack(&kw[0]);
-                    const float k0v[2] = {k0.x, k0.y};
+                    float h0v[2];  // the first token's exponent at the chunk's last row
+                    if (kParkExponent) {
+                        h0v[0] = __uint_as_float(kw[0]);
+                        h0v[1] = __uint_as_float(kw[1]);
+                    } else {
+                        const float2 k0 = Pk<TIO>::unpack(&kw[0]);
+                        const float fc1 = 1.f - (float)r_cnt;
+                        h0v[0] = fmaf(fc1, w2[0], k0.x * kLog2e);
+                        h0v[1] = fmaf(fc1, w2[1], k0.y * kLog2e);
+                    }
                     float fa[V], fb[V], fg[V], fi[V];
                     bool ok = true;
                     const float fc = (float)r_cnt;
@@ -674,7 +749,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < V; ++c) {
                         const float M = lane_active ? chunk_max(t)[ew * Cg + cl + c] : 0.f;
                         const float hK = fmaf(-fc, w2[c], fmaf(-nn[c], w2[c], R[c]));  // history, at the last row
-                        const float h0 = fmaf(-(fc - 1.f), w2[c], k0v[c] * kLog2e);     // first token, same
+                        const float h0 = h0v[c];
                         const float bonus = u2[c] - w2[c];
                         const float dom = fminf(fmaxf(hK, h0), fmaxf(hK, h0 + bonus));
                         const float G = fmaxf(fminf(M, dom + 100.f), hK - 64.f);
@@ -699,25 +774,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // read from tensor memory while this slice is computed
                     const float2 L2 = make_float2(kLog2e, kLog2e);
                     const float2 w2p = make_float2(w2[0], w2[1]);
-                    TIO* yrow = yg + (int64_t)r_begin * C + cl;
+                    // the previous chunk's copy must have read the buffer before it is overwritten
+                    if (lane == 0) bulk_wait_read();
+                    __syncwarp();
+                    TIO* yrow = ybuf + cl;
                     auto emit = [&](auto full_c) {
                         constexpr bool FULL = decltype(full_c)::value;
 #pragma unroll
                         for (int h = 0; h < LC / SR; ++h) {
-                            uint32_t kn[SW], vn[SW];
+                            uint32_t kn[SWK], vn[SW];
                             if (h + 1 < LC / SR) {
-                                TmemIO<SW>::ld(tq + tcol(t, ew, 0) + (h + 1) * SW, kn);
+                                TmemIO<SWK>::ld(tq + tcol(t, ew, 0) + (h + 1) * SWK, kn);
                                 TmemIO<SW>::ld(tq + tcol(t, ew, 1) + (h + 1) * SW, vn);
                             }
 
 #pragma unroll
                             for (int rr = 0; rr < SR; ++rr) {
                                 const int r = h * SR + rr;
-                                const float2 kp = Pk<TIO>::unpack(&kw[rr * W]);
                                 const float2 vp = Pk<TIO>::unpack(&vw[rr * W]);
-                                // k - G first: the large cancellation happens inside one rounding
-                                const float back = FULL ? (float)(r + 1 - LC) : back0 + (float)r;
-                                const float2 x = __ffma2_rn(make_float2(back, back), w2p, __ffma2_rn(kp, L2, fnG));
+                                float2 x;
+                                if (kParkExponent) {
+                                    // the summary's own exponent, moved into the frame
+                                    x = __fadd2_rn(make_float2(__uint_as_float(kw[rr * 2]), __uint_as_float(kw[rr * 2 + 1])),
+                                                   fnG);
+                                } else {
+                                    // k - G first: the large cancellation happens inside one rounding
+                                    const float2 kp = Pk<TIO>::unpack(&kw[rr * W]);
+                                    const float back = FULL ? (float)(r + 1 - LC) : back0 + (float)r;
+                                    x = __ffma2_rn(make_float2(back, back), w2p, __ffma2_rn(kp, L2, fnG));
+                                }
                                 const float2 e = make_float2(ex2(x.x), ex2(x.y));
                                 const float2 ec = __fmul2_rn(e, fic);
                                 const float2 num = __ffma2_rn(ec, vp, fSa);
@@ -740,16 +825,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 }
                                 fSa = __ffma2_rn(e, vp, fSa);
                                 fSb = __fadd2_rn(fSb, e);
-                                if (lane_active && (FULL || r < r_cnt)) Vec<TIO, V>::store(yrow + (int64_t)r * C, yy);
+                                Vec<TIO, V>::store(yrow + r * Cg, yy);
                             }
                             if (h + 1 < LC / SR) {
-                                TmemIO<SW>::wait_ld(kn);
+                                TmemIO<SWK>::wait_ld(kn);
                                 TmemIO<SW>::wait_ld(vn);
 #pragma unroll
-                                for (int x = 0; x < SW; ++x) {
-                                    kw[x] = kn[x];
-                                    vw[x] = vn[x];
-                                }
+                                for (int x = 0; x < SWK; ++x) kw[x] = kn[x];
+#pragma unroll
+                                for (int x = 0; x < SW; ++x) vw[x] = vn[x];
                             }
                         }
                     };
@@ -757,6 +841,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         emit(std::true_type{});
                     else
                         emit(std::false_type{});
+                    fence_proxy_async_smem();  // the rows written by the lanes, read by the TMA engine
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(&tmy, ybuf, q.c0, q.t0 + r_begin, q.b);
+                        bulk_commit();
+                    }
                 } else {
                 const float2 L2 = make_float2(kLog2e, kLog2e), nL2 = make_float2(-kLog2e, -kLog2e);
                 const float2 w2p = make_float2(w2[0], w2[1]), u2p = make_float2(u2[0], u2[1]);
@@ -769,9 +859,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int h = 0; h < LC / SR; ++h) {
                     if (h > 0) {
-                        TmemIO<SW>::ld(tq + tcol(t, ew, 0) + h * SW, kw);
+                        TmemIO<SWK>::ld(tq + tcol(t, ew, 0) + h * SWK, kw);
                         TmemIO<SW>::ld(tq + tcol(t, ew, 1) + h * SW, vw);
-                        TmemIO<SW>::wait_ld(kw);
+                        TmemIO<SWK>::wait_ld(kw);
                         TmemIO<SW>::wait_ld(vw);
                     }
 #pragma unroll
@@ -779,13 +869,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int r = h * SR + rr;
                         if (!lane_active || r >= r_cnt) continue;
                         const int row = r_begin + r;
-                        const float2 kp = Pk<TIO>::unpack(&kw[rr * W]);
                         const float2 vp = Pk<TIO>::unpack(&vw[rr * W]);
+                        float2 kp;
+                        if (!kParkExponent) {
+                            kp = Pk<TIO>::unpack(&kw[rr * W]);
+                        } else if (mode != 0) {
+                            // the steps below need the keys themselves, which tensor memory does
+                            // not hold: this rare lane reads them again
+                            float kv2[V];
+                            Vec<TIO, V>::load(static_cast<const TIO*>(args.k) + q.row0 + (int64_t)row * C + cl, kv2);
+                            kp = make_float2(kv2[0], kv2[1]);
+                        }
                         float yy[V];
                         if (mode == 0) {
-                            // k - G first: the large cancellation happens inside one rounding
-                            const float back = back0 + (float)r;
-                            const float2 x = __ffma2_rn(make_float2(back, back), w2p, __ffma2_rn(kp, L2, fnG));
+                            float2 x;
+                            if (kParkExponent) {
+                                x = __fadd2_rn(make_float2(__uint_as_float(kw[rr * 2]), __uint_as_float(kw[rr * 2 + 1])), fnG);
+                            } else {
+                                // k - G first: the large cancellation happens inside one rounding
+                                const float back = back0 + (float)r;
+                                x = __ffma2_rn(make_float2(back, back), w2p, __ffma2_rn(kp, L2, fnG));
+                            }
                             const float2 e = make_float2(ex2(x.x), ex2(x.y));
                             const float2 ec = __fmul2_rn(e, fic);
                             const float2 num = __ffma2_rn(ec, vp, fSa);
@@ -840,6 +944,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ew == 0 && lane == 0) WKV_TRACE_EVENT(unit, 9);
             if (lane == 0) mbar_arrive(uempty(t));
         }
+        // the chunks' stores must be done before the block's shared memory goes away
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -866,7 +973,8 @@ struct TmConfig {
     static constexpr int NT0 = 512 / TmLayout<TIO, LC, 1, 1>::CPU;
     static constexpr int NT = NT0 > 8 ? 8 : NT0;
     static constexpr size_t fixed = TmLayout<TIO, LC, 0, NT, GATE>::total;  // everything but the stages
-    static constexpr size_t per_stage = TmLayout<TIO, LC, 1, NT>::stage + (TmLayout<TIO, LC, 1, NT>::NB + 1) * 8;
+    static constexpr size_t per_stage =
+        TmLayout<TIO, LC, 1, NT>::stage + (TmLayout<TIO, LC, 1, NT>::NB + 2) * 8 + sizeof(UnitBlock);
     static constexpr int NS0 = (int)((232448 - fixed) / per_stage);
     static constexpr int NS = NS0 > 4 ? 4 : NS0;
 };
@@ -879,17 +987,15 @@ cudaError_t launch_tmem_g(const ForwardArgs& a, const ChunkGeom& g, const PipePa
     // a look-back warp waits on unit i's slot only after finishing unit i - kNL, so the
     // slot's previous phase (unit i - NT) is complete whenever NT >= kNL
     static_assert(NT >= kNL, "fewer unit slots than look-back warps");
-    // an emitting warp waits on unit i's slot only after finishing unit i - kES; the slot's
-    // previous unit i - NT must be one it has handled, so NT is a multiple of kES
-    static_assert(NT % kES == 0, "unit slots must divide among the emitting sets");
     using Lay = TmLayout<TIO, LC, NS, NT, GATE>;
     static_assert(Lay::total <= 232448, "shared memory layout over the per-CTA limit");
     static_assert(Lay::Ts % Lay::BR == 0, "tile rows must be a multiple of the box rows");
     static_assert(LC <= Lay::BR && Lay::BR % LC == 0, "a chunk must lie inside one box");
     auto kern = tmem_kernel<TIO, LC, NS, NT, GATE>;
-    CUtensorMap tmk, tmv, tmr;
+    CUtensorMap tmk, tmv, tmr, tmy;
     if (!make_tile_map(&tmk, a.k, a.B, a.T, a.C, a.io, Lay::Cg, Lay::BR) ||
-        !make_tile_map(&tmv, a.v, a.B, a.T, a.C, a.io, Lay::Cg, Lay::BR))
+        !make_tile_map(&tmv, a.v, a.B, a.T, a.C, a.io, Lay::Cg, Lay::BR) ||
+        !make_tile_map(&tmy, a.y, a.B, a.T, a.C, a.io, Lay::Cg, LC))
         return cudaErrorInvalidValue;
     if (GATE ? !make_tile_map(&tmr, a.r, a.B, a.T, a.C, a.io, Lay::Cg, LC) : false) return cudaErrorInvalidValue;
     if (!GATE) tmr = tmk;  // unused
@@ -911,7 +1017,7 @@ cudaError_t launch_tmem_g(const ForwardArgs& a, const ChunkGeom& g, const PipePa
     }
     const int64_t nsm = dev < 64 ? sms[dev] : 148;
     const int64_t grid = g.U < nsm ? g.U : nsm;
-    kern<<<(unsigned)grid, kThreads, Lay::total, s>>>(a, pp, tmk, tmv, tmr);
+    kern<<<(unsigned)grid, kThreads, Lay::total, s>>>(a, pp, tmk, tmv, tmr, tmy);
     return cudaGetLastError();
 }
 

@@ -34,6 +34,10 @@ struct ForwardArgs {
 // wkv_get_device_status.
 uint32_t* device_status_word();
 
+// Records e as the host thread's last CUDA error (reported by wkv_last_cuda_error) and
+// returns the WKV_ERR_CUDA status code, for entry points outside the main ABI file.
+int record_cuda_error(cudaError_t e);
+
 // ----- serial path: one thread per (b, c) -----
 cudaError_t launch_forward_serial(const ForwardArgs& a, cudaStream_t s);
 
@@ -43,7 +47,7 @@ struct ChunkGeom {
     int NW;       // warps per CTA (= chunks per tile)
     int LC;       // time steps per chunk
     bool bulk;    // rows copied with cp.async.bulk
-    bool pipe;    // persistent warp-specialised kernel (wkv_forward_pipe.cu)
+    bool pipe;    // persistent warp-specialised kernel (wkv_forward_tmem.cu)
     int64_t Cg;   // channels per tile (32 * V)
     int64_t Ts;   // time steps per tile (NW * LC)
     int64_t groups_per_b;
@@ -83,15 +87,14 @@ cudaError_t launch_token_shift3(int64_t B, int64_t T, int64_t C, const float* mu
 // y <- sigma(r) * y over n elements of dtype io (0 fp32, 1 bf16), in place
 cudaError_t launch_gate(int64_t n, int io, const void* r, void* y, cudaStream_t s);
 
-// WKV backward (fp32): gk, gv [B,T,C]; gw, gu [C] (zeroed here, then accumulated); ws holds
-// 3 * B*T*C + 9 * B*P*C floats, P = backward_segments(T)
+// WKV backward (fp32): gk, gv [B,T,C]; gw, gu [C] (zeroed here, then accumulated); ws (zero-
+// filled before its first use) holds backward_workspace_bytes(B, T, C), P = backward_segments(T)
 int64_t backward_segments(int64_t T);
+size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t C);
 cudaError_t launch_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
                             const float* v, const float* gy, float* gk, float* gv, float* gw, float* gu, void* ws,
                             cudaStream_t s);
 
-cudaError_t launch_forward_pipe(const ForwardArgs& a, const ChunkGeom& g, void* ws, int64_t drop_unit,
-                                cudaStream_t s);
 cudaError_t launch_forward_tmem(const ForwardArgs& a, const ChunkGeom& g, void* ws, int64_t drop_unit,
                                 cudaStream_t s);
 

@@ -19,8 +19,9 @@
 // host-side stand-in), so the first call on each device looks up the real address
 // with cudaGetSymbolAddress while that device is current and caches it.  Make that
 // first call outside any stream capture.  A device-side wait that runs out (possible
-// only when calls overlap) is recorded in the array's header and cleared by the next
-// call; it is not reported to the caller.
+// only when calls overlap) is recorded in the array's header, which the next call
+// clears, and in the library's device-wide error word, which wkv_get_device_status
+// reports (and clears).
 #include <mutex>
 
 #include "wkv.h"
@@ -67,11 +68,19 @@ extern "C" wkv_status wkv_forward_chunked_noalloc(int64_t B, int64_t T, int64_t 
     if (B < 0 || T < 0 || C < 0) return WKV_ERR_INVALID_ARG;
     if (io != WKV_F32 && io != WKV_BF16) return WKV_ERR_UNSUPPORTED;
     if (B == 0 || C == 0) return WKV_OK;  // no channels: nothing to compute
-    if (T == 0) return WKV_ERR_INVALID_ARG;  // the chunked kernel needs at least one token
-    if (B > INT64_MAX / T || B * T > INT64_MAX / C) return WKV_ERR_INVALID_ARG;
-    if (!w || !u || !k || !v || !y) return WKV_ERR_INVALID_ARG;
+    if (B > INT64_MAX / C || B * C > INT64_MAX / 3) return WKV_ERR_INVALID_ARG;
+    if (T > 0 && B * C > INT64_MAX / T) return WKV_ERR_INVALID_ARG;
     auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-    if (!al(w) || !al(u) || !al(k) || !al(v) || !al(y) || !al(state_in) || !al(state_out)) return WKV_ERR_MISALIGNED;
+    if (!w || !u) return WKV_ERR_INVALID_ARG;
+    if (!al(w) || !al(u) || !al(state_in) || !al(state_out)) return WKV_ERR_MISALIGNED;
+    if (T == 0) {
+        // no tokens: the state passes through (state_in, or the empty state), as in wkv_forward_ex
+        if (!state_out) return WKV_OK;
+        const cudaError_t e = launch_state_passthrough(B * C, state_in, state_out, stream);
+        return e == cudaSuccess ? WKV_OK : (wkv_status)record_cuda_error(e);
+    }
+    if (!k || !v || !y) return WKV_ERR_INVALID_ARG;
+    if (!al(k) || !al(v) || !al(y)) return WKV_ERR_MISALIGNED;
 
     // the default tile if its scratch fits, else the longer tile (fewer records)
     ChunkGeom g;
@@ -81,10 +90,10 @@ extern "C" wkv_status wkv_forward_chunked_noalloc(int64_t B, int64_t T, int64_t 
 
     void* scratch = nullptr;
     cudaError_t e = scratch_for_current_device(&scratch, stream);
-    if (e != cudaSuccess) return WKV_ERR_CUDA;
+    if (e != cudaSuccess) return (wkv_status)record_cuda_error(e);
     // error word, failing unit, ticket and completion counters must start at zero; keep the epoch
     e = cudaMemsetAsync(scratch, 0, 4 * sizeof(uint32_t), stream);
-    if (e != cudaSuccess) return WKV_ERR_CUDA;
+    if (e != cudaSuccess) return (wkv_status)record_cuda_error(e);
 
     ForwardArgs a;
     a.B = B;
@@ -100,8 +109,8 @@ extern "C" wkv_status wkv_forward_chunked_noalloc(int64_t B, int64_t T, int64_t 
     a.state_out = state_out;
     a.err = static_cast<uint32_t*>(scratch);
     a.dev_err = device_status_word();
-    if (!a.dev_err) return WKV_ERR_CUDA;
+    if (!a.dev_err) return (wkv_status)record_cuda_error(cudaGetLastError());
     a.spin_limit = kSpinLimitDefault;
     e = launch_forward_chunked(a, g, scratch, -1, stream);
-    return e == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+    return e == cudaSuccess ? WKV_OK : (wkv_status)record_cuda_error(e);
 }

@@ -72,6 +72,20 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* tm, in
         : "memory");
 }
 
+// Shared -> global tensor copy of one box (the TMA engine clips rows and channels that fall
+// outside the tensor), tracked by this thread's bulk async-group.  Coordinates are
+// non-negative and x is a multiple of 16 bytes' worth of elements.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* tm, const void* src, int x, int y, int z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(tm),
+                 "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// waits until this thread's committed bulk stores have read their shared-memory source
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// waits until this thread's committed bulk stores are complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 struct PipeParams {
     int64_t groups_per_b, G, S, U;
     uint64_t* slot;     // [U][Cg][4] tagged words: a tile's aggregate, later its inclusive prefix

@@ -104,13 +104,23 @@ def test_eagle_forward_resumes_from_state():
     _check(np.concatenate([y1, y2], axis=1), st2, w, r, k, v)
 
 
-def test_eagle_full_size_sampled():
-    """eagle_8x1024x768 at full size (the bench's launch), sampled heads against the oracle."""
+def test_eagle_full_size_all_heads():
+    """eagle_8x1024x768 at full size (the bench's launch): every sequence-head against the oracle."""
     spec = synth.EAGLE["eagle_8x1024x768"]
     w, r, k, v = synth.eagle_inputs(spec)
     y, st = _gpu_forward(w, r, k, v)
-    rng = np.random.default_rng(7)
-    for b, h in zip(rng.integers(0, spec.B, 6), rng.integers(0, spec.C // 64, 6)):
+    _check(y, st, w, r, k, v)
+
+
+def test_eagle_long_workload_sampled_heads():
+    """eagle_4x4096x2048 at full size (32 heads, 4096 tokens): 24 sampled sequence-heads, the
+    last one included, against the oracle."""
+    spec = synth.EAGLE["eagle_4x4096x2048"]
+    w, r, k, v = synth.eagle_inputs(spec)
+    y, st = _gpu_forward(w, r, k, v)
+    rng = np.random.default_rng(8)
+    pairs = list(zip(rng.integers(0, spec.B, 23), rng.integers(0, spec.C // 64, 23))) + [(spec.B - 1, spec.C // 64 - 1)]
+    for b, h in pairs:
         sl = slice(h * 64, (h + 1) * 64)
         _check(y[b:b + 1, :, sl], st[b:b + 1, h:h + 1], w[sl], r[b:b + 1, :, sl], k[b:b + 1, :, sl],
                v[b:b + 1, :, sl])

@@ -79,24 +79,18 @@ def test_gate_limits_are_exact(path, chunk):
     assert torch.count_nonzero(y_shut).item() == 0
 
 
-def test_gated_full_size_sampled():
-    """fwd_8x1024x768 at full size through the default path, sampled channels against the
-    oracle (the whole workload's oracle would take minutes)."""
-    import torch
+def test_gated_full_size_all_elements():
+    """fwd_8x1024x768 at full size through the default path: every element of the gated output
+    against the oracle's sigma(r) * wkv."""
     import linear_attention_rnn_wkv_b200 as wkv
     spec = synth.FORWARD["fwd_8x1024x768"]
     w, u, k, v = synth.forward_inputs(spec)
     r = synth.receptance(spec)
     o, _ = wkv.wkv_forward(to_gpu(w), to_gpu(u), to_gpu(k), to_gpu(v), r=to_gpu(r))
     o = o.cpu().numpy()
-    rng = np.random.default_rng(5)
-    bs = rng.integers(0, spec.B, 64)
-    cs = rng.integers(0, spec.C, 64)
-    for b, c in zip(bs, cs):
-        y_ref, s_ref, _, _ = oracle.wkv_recurrent(w[c:c + 1], u[c:c + 1], k[b:b + 1, :, c:c + 1],
-                                                  v[b:b + 1, :, c:c + 1])
-        o_ref = oracle.gate(r[b:b + 1, :, c:c + 1], y_ref)
-        assert scaled_output_error(o[b:b + 1, :, c:c + 1], o_ref, s_ref) <= TOL_Y["f32"]
+    y_ref, s_ref, _, _ = oracle.wkv_recurrent(w, u, k, v)
+    o_ref = oracle.gate(r, y_ref)
+    assert scaled_output_error(o, o_ref, s_ref) <= TOL_Y["f32"]
 
 
 def test_token_shift_three_mu():
