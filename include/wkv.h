@@ -216,7 +216,10 @@ wkv_status token_shift_mix3(int64_t B, int64_t T, int64_t C, const float* mu_r, 
                             float* xv, cudaStream_t stream);
 
 /*
- * Fused decode step: the token-shift lerp and the WKV decode step in one kernel.
+ * Fused decode step: the token-shift lerp ("RWKV" transformer-math page, section "Token shift:
+ * a two-tap causal convolution": xbar = mu x_t + (1 - mu) x_{t-1}) and the WKV decode step
+ * (aiwiki "RWKV": the one-token decode step; the same arithmetic as wkv_decode_step) in one
+ * kernel, each input and state element read once.
  *   mu, w, u      [L][C] fp32
  *   x_t, x_prev   [N][L][C] fp32: this token's input and the previous token's
  *   xbar          [N][L][C] fp32: mu * x_t + (1 - mu) * x_prev (written)

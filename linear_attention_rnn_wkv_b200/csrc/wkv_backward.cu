@@ -50,7 +50,7 @@ constexpr int kThreads = 128;      // threads per block (channels of one (b, seg
 constexpr float kRNone = 3.0e38f;  // reference of an empty adjoint sum
 // Later segments' published sums read per look-back round trip.
 #ifndef WKV_BWD_LOOKAHEAD
-#define WKV_BWD_LOOKAHEAD 4
+#define WKV_BWD_LOOKAHEAD 1
 #endif
 constexpr int kBwdLook = WKV_BWD_LOOKAHEAD;
 // E's per-position values: [kSeg][3][kThreads] floats, each thread its own column

@@ -260,11 +260,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t T = args.T, C = args.C, BC = args.B * args.C;
     const uint32_t lim = args.spin_limit;
 
+    if (tid == 0) WKV_TRACE_BLOCK(pp.U, 0);
     if (warp == 0) {
         tmem_alloc(s_tmem, 512);
         tmem_relinquish();
     }
+    // the producer's first ticket and the launch's epoch: both round trips start before the
+    // barrier set-up and overlap each other (the producer is thread 0)
+    uint32_t first_ticket = 0;
     if (tid == 0) {
+        first_ticket = atomicAdd(&pp.hdr->ticket, 1u);
         *s_epoch = (*reinterpret_cast<volatile uint32_t*>(&pp.hdr->epoch) + 1u) & 0x3FFFFFFFu;
         *s_iend = INT64_MAX;
         for (int s = 0; s < NS; ++s) {
@@ -304,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // block handles its units in ticket order whatever it has taken, and every
         // cross-block wait is on a smaller ticket).
         if (lane == 0) {
-            uint32_t tk_next = atomicAdd(&pp.hdr->ticket, 1u);
+            uint32_t tk_next = first_ticket;
             for (int64_t i = 0;; ++i) {
                 const int s = (int)(i % NS);
                 if (i >= NS && !mbar_wait(dempty(s), (uint32_t)((i / NS - 1) & 1), lim)) report(kDevTimeoutCopy);
@@ -956,6 +961,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_dealloc(tmem, 512);
     }
     if (tid == 0) {
+        WKV_TRACE_BLOCK(pp.U, 1);
         __threadfence();
         const uint32_t finished = atomicAdd(&pp.hdr->done, 1u) + 1u;
         if (finished == gridDim.x) {

@@ -28,8 +28,17 @@ __device__ __forceinline__ void wkv_trace(int64_t unit, int ev) {
     }
 }
 #define WKV_TRACE_EVENT(unit, ev) wkv_trace(unit, ev)
+// per block, after the units' events: [2] = block start, block end
+__device__ __forceinline__ void wkv_trace_block(int64_t units, int ev) {
+    if (!g_wkv_trace) return;
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    g_wkv_trace[units * 11 + blockIdx.x * 2 + ev] = t;
+}
+#define WKV_TRACE_BLOCK(units, ev) wkv_trace_block(units, ev)
 #else
 #define WKV_TRACE_EVENT(unit, ev) ((void)0)
+#define WKV_TRACE_BLOCK(units, ev) ((void)0)
 #endif
 // events: 0 ticket, 1 tile loaded, 2 chunks summarised, 3 look-back start, 4 summaries
 // scanned, 5 carry known, 6 carry handed over, 7 records published, 8 emit start, 9 emit end
