@@ -48,14 +48,12 @@ constexpr int kSeg = 32;           // time steps per segment
 constexpr int kBlk = 16;           // steps whose loads are issued together
 constexpr int kThreads = 128;      // threads per block (channels of one (b, segment))
 constexpr float kRNone = 3.0e38f;  // reference of an empty adjoint sum
-// Later segments' published sums read per look-back round trip.
-#ifndef WKV_BWD_LOOKAHEAD
-#define WKV_BWD_LOOKAHEAD 1
-#endif
-constexpr int kBwdLook = WKV_BWD_LOOKAHEAD;
-// E's per-position values: [kSeg][3][kThreads] floats, each thread its own column
-constexpr size_t kGradSmem = (size_t)kSeg * 3 * kThreads * sizeof(float);
-static_assert(kGradSmem <= 48 * 1024, "fits the default dynamic shared memory limit");
+// Segments per block: their records and adjoint sums are combined in shared memory, and the
+// look-backs walk over groups of this many segments.
+constexpr int kGroupSegs = 4;
+constexpr int kGroupThreads = kGroupSegs * kThreads;
+// R's per-position values: [kGroupSegs][kSeg][3][kThreads] floats, each thread its own column
+constexpr size_t kGradSmem = (size_t)kGroupSegs * kSeg * 3 * kThreads * sizeof(float);
 
 struct Adj {
     float x, y, xp, yp, r;  // X, Y, X', Y' relative to 2^{-r}
@@ -221,46 +219,62 @@ __device__ __forceinline__ void forward_span(const BwdArgs& a, int64_t base, int
     }
 }
 
-// Published forward records: four 64-bit words per (sequence, segment, channel), (a | tag),
-// (b | tag), (anc | tag), (n | tag), word-major per (sequence, segment); the same fence-free
-// protocol as the adjoint sums below (kind 1 the segment's own record, 2 the state at its end).
-__device__ __forceinline__ uint64_t* fwd_slot(const BwdArgs& a, int64_t b, int64_t j) {
-    return a.fslots + (b * a.P + j) * 4 * a.C;
+// Published records, one per (sequence, group of kGroupSegs segments, channel): the forward
+// pass's record has four 64-bit words, (a | tag), (b | tag), (anc | tag), (n | tag), the
+// reverse pass's adjoint sums five, (x, y, x', y', r); each word holds the value's bits in its
+// low half and the launch epoch with the record's kind (1 the group's own record, 2 inclusive:
+// everything before it, or after it, folded in) in its high half.  Aligned 64-bit accesses are
+// single-copy atomic, so a reader that finds one tag in all the words holds one consistent
+// record: no fence and no flag.  The group's own record is overwritten by the inclusive one
+// (same thread, word by word), so a reader may catch mixed tags and then reads again.  Words
+// are stored word-major per (sequence, group), so a warp's access to one word of 32 channels
+// is contiguous.
+template <int NW>
+__device__ __forceinline__ void slot_publish(uint64_t* p, int64_t C, const float (&f)[NW], uint32_t tag) {
+#pragma unroll
+    for (int i = 0; i < NW; ++i) st_relaxed_u64(p + i * C, ((uint64_t)tag << 32) | __float_as_uint(f[i]));
 }
 
-__device__ __forceinline__ void rec_publish(const BwdArgs& a, int64_t b, int64_t j, int64_t c, const Rec& r,
-                                            uint32_t tag) {
-    uint64_t* p = fwd_slot(a, b, j) + c;
-    const float f[4] = {r.a, r.b, r.anc, r.n};
+// 2 inclusive, 1 the group's own record, 0 nothing usable yet
+template <int NW>
+__device__ __forceinline__ int slot_read(const uint64_t* p, int64_t C, uint32_t tag_loc, uint32_t tag_incl,
+                                         float (&f)[NW]) {
+    uint64_t wd[NW];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) st_relaxed_u64(p + i * a.C, ((uint64_t)tag << 32) | __float_as_uint(f[i]));
-}
-
-// 2 the state at the segment's end, 1 its own record, 0 nothing usable yet
-__device__ __forceinline__ int rec_read(const BwdArgs& a, int64_t b, int64_t j, int64_t c, uint32_t tag_loc,
-                                        uint32_t tag_incl, Rec& out) {
-    const uint64_t* p = fwd_slot(a, b, j) + c;
-    uint64_t wd[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) wd[i] = ld_relaxed_u64(p + i * a.C);
+    for (int i = 0; i < NW; ++i) wd[i] = ld_relaxed_u64(p + i * C);
     const uint32_t t0 = (uint32_t)(wd[0] >> 32);
     bool same = t0 == tag_loc || t0 == tag_incl;
 #pragma unroll
-    for (int i = 1; i < 4; ++i) same = same && (uint32_t)(wd[i] >> 32) == t0;
+    for (int i = 1; i < NW; ++i) same = same && (uint32_t)(wd[i] >> 32) == t0;
     if (!same) return 0;
-    out = Rec{__uint_as_float((uint32_t)wd[0]), __uint_as_float((uint32_t)wd[1]), __uint_as_float((uint32_t)wd[2]),
-              __uint_as_float((uint32_t)wd[3])};
+#pragma unroll
+    for (int i = 0; i < NW; ++i) f[i] = __uint_as_float((uint32_t)wd[i]);
     return t0 == tag_incl ? 2 : 1;
 }
 
-// A: the segments in time order (an atomic ticket hands the first segments out first), 128
-// channels of one (sequence, segment) per block: each segment's forward from the empty state
-// gives its record; a decoupled look-back over the earlier segments of its channel (each a
-// smaller ticket) folds their records into its starting state, which it writes, and the state
-// at its end is published for the later segments.  gw, gu are zeroed here for R's atomics.
-__global__ void __launch_bounds__(kThreads) bwd_seg_starts(BwdArgs a, int64_t cx) {
+__device__ __forceinline__ int64_t num_groups(const BwdArgs& a) { return (a.P + kGroupSegs - 1) / kGroupSegs; }
+
+__device__ __forceinline__ float span_len(const BwdArgs& a, int64_t j0, int64_t j1) {  // steps of segments [j0, j1)
+    return j1 > j0 ? (float)(min64(a.T, j1 * kSeg) - j0 * kSeg) : 0.f;
+}
+
+__device__ __forceinline__ void give_up(const BwdArgs& a) {
+    atomicCAS(&a.hdr->error, kDevOk, (uint32_t)kDevTimeoutCarry);
+    atomicCAS(a.dev_err, kDevOk, (uint32_t)kDevTimeoutCarry);
+}
+
+// A: groups of kGroupSegs segments in time order (an atomic ticket hands the first groups out
+// first), one block of kGroupSegs x 128 threads per (group, sequence, channel block): each
+// segment's forward from the empty state gives its record; the block folds its segments'
+// records in shared memory; a decoupled look-back over the earlier groups of the channel (each
+// a smaller ticket) gives the group's starting state, from which every segment's starting
+// state follows and is written; the state at the group's end is published for later groups.
+// gw, gu are zeroed here for R's atomics.
+__global__ void __launch_bounds__(kGroupThreads) bwd_seg_starts(BwdArgs a, int64_t cx) {
+    __shared__ Rec s_rec[kGroupSegs][kThreads];  // each segment's record, then its in-group prefix
+    __shared__ Rec s_carry[kThreads];            // the state entering the group
     __shared__ uint32_t s_ticket, s_epoch;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, tc = tid % kThreads, gs = tid / kThreads;
     if (tid == 0) {
         s_ticket = atomicAdd(&a.hdr->ticket_f, 1u);
         s_epoch = (*reinterpret_cast<volatile uint32_t*>(&a.hdr->epoch_f) + 1u) & 0x3FFFFFFFu;
@@ -269,68 +283,82 @@ __global__ void __launch_bounds__(kThreads) bwd_seg_starts(BwdArgs a, int64_t cx
     const int64_t unit = s_ticket;
     const uint32_t epoch30 = s_epoch;
     const uint32_t tag_loc = (epoch30 << 2) | 1u, tag_incl = (epoch30 << 2) | 2u;
-    const int64_t per_seg = a.B * cx;
-    const int64_t j = unit / per_seg;
-    const int64_t b = (unit % per_seg) / cx, cb = unit % cx;
-    const int64_t c = cb * kThreads + tid;
-    const bool live = unit < a.P * per_seg && c < a.C;
+    const int64_t per_grp = a.B * cx, NG = num_groups(a);
+    const int64_t J = unit / per_grp;
+    const int64_t b = (unit % per_grp) / cx, cb = unit % cx;
+    const int64_t c = cb * kThreads + tc;
+    const int64_t j = J * kGroupSegs + gs;
+    const bool chan = unit < NG * per_grp && c < a.C;
+    const bool live = chan && j < a.P;
+    const float w2 = chan ? a.w[c] * kLog2e : 0.f;
     if (live) {
         if (b == 0 && j == 0) {  // R accumulates into these
             a.gw[c] = 0.f;
             a.gu[c] = 0.f;
         }
-        const float w2 = a.w[c] * kLog2e, u2 = a.u[c] * kLog2e;
-        const int64_t t0 = j * kSeg, t1 = min64(a.T, t0 + kSeg);
-        FwdState s{0.f, 0.f, kPEmpty, 0.f};
-        forward_span<false, false>(a, b * a.T * a.C + c, t0, t1, s, u2, w2, [](int, const FwdOut&, float) {});
-        const Rec local{s.a, s.bb, s.anc, s.n};
-        const float len = (float)(t1 - t0);
-        Rec run = rec_identity();  // the earlier segments, folded newest first
-        if (j == 0) {
-            if (a.P > 1) rec_publish(a, b, j, c, local, tag_incl);
+        const float u2 = a.u[c] * kLog2e;
+        FwdState st{0.f, 0.f, kPEmpty, 0.f};
+        forward_span<false, false>(a, b * a.T * a.C + c, j * kSeg, min64(a.T, (j + 1) * kSeg), st, u2, w2,
+                                   [](int, const FwdOut&, float) {});
+        s_rec[gs][tc] = Rec{st.a, st.bb, st.anc, st.n};
+    } else {
+        s_rec[gs][tc] = rec_identity();
+    }
+    __syncthreads();
+    if (gs == 0 && chan) {
+        // the group's segments folded in time order; each slot keeps its in-group prefix
+        Rec agg = rec_identity();
+#pragma unroll
+        for (int g = 0; g < kGroupSegs; ++g) {
+            const Rec r = s_rec[g][tc];
+            s_rec[g][tc] = agg;
+            const int64_t jg = J * kGroupSegs + g;
+            if (jg < a.P) agg = rec_combine(agg, r, span_len(a, jg, jg + 1), w2);
+        }
+        uint64_t* my = a.fslots + (b * NG + J) * 4 * a.C + c;
+        Rec run = rec_identity();  // the earlier groups, folded newest first
+        if (J == 0) {
+            if (NG > 1) slot_publish<4>(my, a.C, {agg.a, agg.b, agg.anc, agg.n}, tag_incl);
         } else {
-            rec_publish(a, b, j, c, local, tag_loc);
+            slot_publish<4>(my, a.C, {agg.a, agg.b, agg.anc, agg.n}, tag_loc);
             float span = 0.f;
-            int64_t m = j - 1;
+            int64_t m = J - 1;
             bool done = false;
             uint32_t nap = 32;
             for (uint32_t it = 0; it <= a.spin_limit && !done; ++it) {
-                Rec rec[kBwdLook];
-                int kind[kBwdLook];
-#pragma unroll
-                for (int d = 0; d < kBwdLook; ++d)
-                    kind[d] = m - d >= 0 ? rec_read(a, b, m - d, c, tag_loc, tag_incl, rec[d]) : 0;
-                bool progressed = false;
-#pragma unroll
-                for (int d = 0; d < kBwdLook; ++d) {
-                    if (done || kind[d] == 0) break;
-                    progressed = true;
-                    run = rec_combine(rec[d], run, span, w2);
-                    if (kind[d] == 2) {
-                        done = true;
-                    } else {
-                        span += (float)kSeg;  // every segment before the last is whole
-                        if (--m < 0) done = true;
-                    }
-                }
-                if (progressed) {
-                    nap = 32;
-                } else {
+                float f[4];
+                const int kind = slot_read<4>(a.fslots + (b * NG + m) * 4 * a.C + c, a.C, tag_loc, tag_incl, f);
+                if (kind == 0) {
                     __nanosleep(nap);
                     nap = nap < 512 ? nap * 2 : 512;
+                    continue;
+                }
+                nap = 32;
+                run = rec_combine(Rec{f[0], f[1], f[2], f[3]}, run, span, w2);
+                if (kind == 2) {
+                    done = true;
+                } else {
+                    span += (float)(kGroupSegs * kSeg);  // every group before the last is whole
+                    if (--m < 0) done = true;
                 }
             }
-            if (!done) {  // gave up: record it, go on with what is there (the gradients are invalid)
-                atomicCAS(&a.hdr->error, kDevOk, (uint32_t)kDevTimeoutCarry);
-                atomicCAS(a.dev_err, kDevOk, (uint32_t)kDevTimeoutCarry);
+            if (!done) give_up(a);  // go on with what is there (the gradients are then invalid)
+            if (J + 1 < NG) {
+                const Rec inc = rec_combine(run, agg, span_len(a, J * kGroupSegs, (J + 1) * kGroupSegs), w2);
+                slot_publish<4>(my, a.C, {inc.a, inc.b, inc.anc, inc.n}, tag_incl);
             }
-            if (j + 1 < a.P) rec_publish(a, b, j, c, rec_combine(run, local, len, w2), tag_incl);
         }
+        s_carry[tc] = run;
+    }
+    __syncthreads();
+    if (live) {
+        // this segment's starting state: the group's, then the group's segments before it
+        const Rec st = rec_combine(s_carry[tc], s_rec[gs][tc], span_len(a, J * kGroupSegs, j), w2);
         const int64_t si = seg_index(a, b, j, c), SP = a.B * a.P * a.C;
-        a.fs[si] = run.a;
-        a.fs[SP + si] = run.b;
-        a.fs[2 * SP + si] = run.anc;
-        a.fs[3 * SP + si] = run.n;
+        a.fs[si] = st.a;
+        a.fs[SP + si] = st.b;
+        a.fs[2 * SP + si] = st.anc;
+        a.fs[3 * SP + si] = st.n;
     }
     __syncthreads();
     if (tid == 0) {
@@ -360,47 +388,19 @@ __device__ __forceinline__ Adj adj_compose(const Adj& loc, const Adj& in, float 
     return out;
 }
 
-// Published adjoint sums: five 64-bit words per (sequence, segment, channel), each the value's
-// bits in the low half and the launch epoch with the record's kind (1 local sums, 2 inclusive)
-// in the high half.  Aligned 64-bit accesses are single-copy atomic, so a reader that finds one
-// tag in all five words holds one consistent record: no fence and no flag.  The local sums are
-// overwritten by the inclusive ones (same thread, word by word), so a reader may catch mixed
-// tags and then reads again.  Words are stored word-major per (sequence, segment), so a warp's
-// access to one word of 32 channels is contiguous.
-__device__ __forceinline__ uint64_t* adj_slot(const BwdArgs& a, int64_t b, int64_t j) {
-    return a.slots + (b * a.P + j) * 5 * a.C;
-}
-
-__device__ __forceinline__ void adj_publish(const BwdArgs& a, int64_t b, int64_t j, int64_t c, const Adj& s,
-                                            uint32_t tag) {
-    uint64_t* p = adj_slot(a, b, j) + c;
-    const float f[5] = {s.x, s.y, s.xp, s.yp, s.r};
-#pragma unroll
-    for (int i = 0; i < 5; ++i) st_relaxed_u64(p + i * a.C, ((uint64_t)tag << 32) | __float_as_uint(f[i]));
-}
-
-// 2 inclusive, 1 local sums, 0 nothing usable yet (stale, or caught half overwritten)
-__device__ __forceinline__ int adj_read(const BwdArgs& a, int64_t b, int64_t j, int64_t c, uint32_t tag_loc,
-                                        uint32_t tag_incl, Adj& out) {
-    const uint64_t* p = adj_slot(a, b, j) + c;
-    uint64_t wd[5];
-#pragma unroll
-    for (int i = 0; i < 5; ++i) wd[i] = ld_relaxed_u64(p + i * a.C);
-    const uint32_t t0 = (uint32_t)(wd[0] >> 32);
-    bool same = t0 == tag_loc || t0 == tag_incl;
-#pragma unroll
-    for (int i = 1; i < 5; ++i) same = same && (uint32_t)(wd[i] >> 32) == t0;
-    if (!same) return 0;
-    out = Adj{__uint_as_float((uint32_t)wd[0]), __uint_as_float((uint32_t)wd[1]), __uint_as_float((uint32_t)wd[2]),
-              __uint_as_float((uint32_t)wd[3]), __uint_as_float((uint32_t)wd[4])};
-    return t0 == tag_incl ? 2 : 1;
-}
-
-// R: the segments in reverse time order, 128 channels of one (sequence, segment) per block
-__global__ void __launch_bounds__(kThreads) bwd_seg_reverse(BwdArgs a, int64_t cx) {
-    extern __shared__ float sm[];  // [kSeg][3][kThreads]: q, 1 / Dn, y per position
+// R: groups in reverse time order, one block of kGroupSegs x 128 threads per (group, sequence,
+// channel block): each segment's forward from its starting state keeps its per-position
+// values in shared memory while it accumulates its local adjoint sums; the block composes its
+// segments' sums right to left; a decoupled look-back over the later groups of the channel
+// (each a smaller ticket) gives the sums entering the group; what leaves it is published for
+// earlier groups; each segment's incoming sums follow, and its adjoint pass writes gk, gv and
+// adds its gw, gu partials.
+__global__ void __launch_bounds__(kGroupThreads) bwd_seg_reverse(BwdArgs a, int64_t cx) {
+    extern __shared__ float sm[];               // [kGroupSegs][kSeg][3][kThreads]: q, 1 / Dn, y
+    __shared__ Adj s_in[kGroupSegs][kThreads];  // each segment's local sums, then its in-group incoming
+    __shared__ Adj s_gin[kThreads];             // the sums entering the group from its right
     __shared__ uint32_t s_ticket, s_epoch;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, tc = tid % kThreads, gs = tid / kThreads;
     if (tid == 0) {
         s_ticket = atomicAdd(&a.hdr->ticket, 1u);
         s_epoch = (*reinterpret_cast<volatile uint32_t*>(&a.hdr->epoch) + 1u) & 0x3FFFFFFFu;
@@ -409,83 +409,98 @@ __global__ void __launch_bounds__(kThreads) bwd_seg_reverse(BwdArgs a, int64_t c
     const int64_t unit = s_ticket;
     const uint32_t epoch30 = s_epoch;
     const uint32_t tag_loc = (epoch30 << 2) | 1u, tag_incl = (epoch30 << 2) | 2u;
-    // tickets hand out the last segments first, then (sequence, channel block) within a segment
-    const int64_t per_seg = a.B * cx;
-    const int64_t j = a.P - 1 - unit / per_seg;
-    const int64_t b = (unit % per_seg) / cx, cb = unit % cx;
-    const int64_t c = cb * kThreads + tid;
-    const bool live = unit < a.P * per_seg && c < a.C;
+    // tickets hand out the last groups first, then (sequence, channel block) within a group
+    const int64_t per_grp = a.B * cx, NG = num_groups(a);
+    const int64_t J = NG - 1 - unit / per_grp;
+    const int64_t b = (unit % per_grp) / cx, cb = unit % cx;
+    const int64_t c = cb * kThreads + tc;
+    const int64_t j = J * kGroupSegs + gs;
+    const bool chan = unit < NG * per_grp && c < a.C;
+    const bool live = chan && j < a.P;
+    const float w2 = chan ? a.w[c] * kLog2e : 0.f, u2 = chan ? a.u[c] * kLog2e : 0.f;
+    const int64_t t0 = j * kSeg, t1 = min64(a.T, t0 + kSeg);
+    const int64_t base = b * a.T * a.C + c;
+    float* my_sm = sm + (size_t)gs * kSeg * 3 * kThreads;
     if (live) {
-        const float w2 = a.w[c] * kLog2e, u2 = a.u[c] * kLog2e;
-        const int64_t t0 = j * kSeg, t1 = min64(a.T, t0 + kSeg);
-        const int64_t base = b * a.T * a.C + c;
-        const int64_t si = seg_index(a, b, j, c);
         // forward from the starting state: per-position values kept, local sums accumulated
-        FwdState fsd = load_state(a, si);
+        FwdState fsd = load_state(a, seg_index(a, b, j, c));
         LocalSums ls{0.f, 0.f, 0.f, 0.f, kRNone, 0.f};
         forward_span<true, true>(a, base, t0, t1, fsd, u2, w2, [&](int i, const FwdOut& o, float g) {
-            sm[(i * 3 + 0) * kThreads + tid] = o.q;
-            sm[(i * 3 + 1) * kThreads + tid] = o.rd;
-            sm[(i * 3 + 2) * kThreads + tid] = o.y;
+            my_sm[(i * 3 + 0) * kThreads + tc] = o.q;
+            my_sm[(i * 3 + 1) * kThreads + tc] = o.rd;
+            my_sm[(i * 3 + 2) * kThreads + tc] = o.y;
             ls.add((float)i, g, o, w2);
         });
-        const Adj local{ls.x, ls.y, ls.xp, ls.yp, fmaf(ls.Rj, w2, ls.Rq)};
-        const float len = (float)(t1 - t0);
-        // the incoming sums: the later segments' sums composed, nearest first, until one that
+        s_in[gs][tc] = Adj{ls.x, ls.y, ls.xp, ls.yp, fmaf(ls.Rj, w2, ls.Rq)};
+    } else {
+        s_in[gs][tc] = adj_empty();
+    }
+    __syncthreads();
+    if (gs == 0 && chan) {
+        // the group's segments composed right to left; each slot keeps what enters its segment
+        // from the group's later segments
+        Adj run = adj_empty();
+#pragma unroll
+        for (int g = kGroupSegs - 1; g >= 0; --g) {
+            const Adj loc = s_in[g][tc];
+            s_in[g][tc] = run;
+            const int64_t jg = J * kGroupSegs + g;
+            if (jg < a.P) run = adj_compose(loc, run, span_len(a, jg, jg + 1), w2);
+        }
+        uint64_t* my = a.slots + (b * NG + J) * 5 * a.C + c;
+        // the sums entering the group: the later groups' composed, nearest first, until one that
         // already holds everything to its right (or the sequence's end)
-        Adj incoming = adj_empty();
-        if (j + 1 < a.P) {
-            adj_publish(a, b, j, c, local, tag_loc);
+        Adj gin = adj_empty();
+        if (J + 1 < NG) {
+            slot_publish<5>(my, a.C, {run.x, run.y, run.xp, run.yp, run.r}, tag_loc);
             Adj acc = adj_empty();
             float span = 0.f;
-            int64_t m = j + 1;
+            int64_t m = J + 1;
             bool done = false;
             uint32_t nap = 32;
             for (uint32_t it = 0; it <= a.spin_limit && !done; ++it) {
-                // kBwdLook slots per round trip: all loads issued before any is examined
-                Adj rec[kBwdLook];
-                int kind[kBwdLook];
-#pragma unroll
-                for (int d = 0; d < kBwdLook; ++d)
-                    kind[d] = m + d < a.P ? adj_read(a, b, m + d, c, tag_loc, tag_incl, rec[d]) : 0;
-                bool progressed = false;
-#pragma unroll
-                for (int d = 0; d < kBwdLook; ++d) {
-                    if (done || kind[d] == 0) break;
-                    progressed = true;
-                    if (kind[d] == 2) {
-                        incoming = adj_compose(acc, rec[d], span, w2);
-                        done = true;
-                    } else {
-                        acc = adj_compose(acc, rec[d], span, w2);
-                        span += (float)(min64(a.T, (m + 1) * kSeg) - m * kSeg);
-                        if (++m >= a.P) {
-                            incoming = acc;
-                            done = true;
-                        }
-                    }
-                }
-                if (progressed) {
-                    nap = 32;
-                } else {
+                float f[5];
+                const int kind = slot_read<5>(a.slots + (b * NG + m) * 5 * a.C + c, a.C, tag_loc, tag_incl, f);
+                if (kind == 0) {
                     __nanosleep(nap);
                     nap = nap < 512 ? nap * 2 : 512;
+                    continue;
+                }
+                nap = 32;
+                const Adj rec{f[0], f[1], f[2], f[3], f[4]};
+                if (kind == 2) {
+                    gin = adj_compose(acc, rec, span, w2);
+                    done = true;
+                } else {
+                    acc = adj_compose(acc, rec, span, w2);
+                    span += span_len(a, m * kGroupSegs, (m + 1) * kGroupSegs);
+                    if (++m >= NG) {
+                        gin = acc;
+                        done = true;
+                    }
                 }
             }
-            if (!done) {  // gave up: record it, go on with what is there (the gradients are invalid)
-                atomicCAS(&a.hdr->error, kDevOk, (uint32_t)kDevTimeoutCarry);
-                atomicCAS(a.dev_err, kDevOk, (uint32_t)kDevTimeoutCarry);
-                incoming = acc;
+            if (!done) {  // gave up: go on with what is there (the gradients are then invalid)
+                give_up(a);
+                gin = acc;
             }
         }
-        if (j > 0) adj_publish(a, b, j, c, adj_compose(local, incoming, len, w2), tag_incl);
-        // the adjoint recurrence right to left from the incoming sums
-        Adj st = incoming;
+        if (J > 0) {
+            const Adj out = adj_compose(run, gin, span_len(a, J * kGroupSegs, (J + 1) * kGroupSegs), w2);
+            slot_publish<5>(my, a.C, {out.x, out.y, out.xp, out.yp, out.r}, tag_incl);
+        }
+        s_gin[tc] = gin;
+    }
+    __syncthreads();
+    if (live) {
+        // the sums entering this segment: its group's later segments', with the group's own
+        // incoming sums carried across them
+        Adj st = adj_compose(s_in[gs][tc], s_gin[tc], span_len(a, j + 1, (J + 1) * kGroupSegs), w2);
         float sgw = 0.f, sgu = 0.f;
         auto step = [&](int64_t t, float kt, float vt, float g) {
             const int i = (int)(t - t0);
-            const FwdOut o{sm[(i * 3 + 0) * kThreads + tid], sm[(i * 3 + 1) * kThreads + tid],
-                           sm[(i * 3 + 2) * kThreads + tid]};
+            const FwdOut o{my_sm[(i * 3 + 0) * kThreads + tc], my_sm[(i * 3 + 1) * kThreads + tc],
+                           my_sm[(i * 3 + 2) * kThreads + tc]};
             float gk, gv;
             adj_step(st, kt * kLog2e, vt, g, o, u2, w2, gk, gv, sgw, sgu);
             a.gk[base + t * a.C] = gk;
@@ -529,8 +544,10 @@ __global__ void __launch_bounds__(kThreads) bwd_seg_reverse(BwdArgs a, int64_t c
 int64_t backward_segments(int64_t T) { return (T + kSeg - 1) / kSeg; }
 
 size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t C) {
-    const size_t bpc = (size_t)B * (size_t)backward_segments(T) * (size_t)C;
-    return kBwdHeaderBytes + bpc * 4 * sizeof(float) + bpc * 4 * sizeof(uint64_t) + bpc * 5 * sizeof(uint64_t);
+    const int64_t P = backward_segments(T);
+    const size_t bpc = (size_t)B * (size_t)P * (size_t)C;
+    const size_t bgc = (size_t)B * (size_t)((P + kGroupSegs - 1) / kGroupSegs) * (size_t)C;
+    return kBwdHeaderBytes + bpc * 4 * sizeof(float) + bgc * 9 * sizeof(uint64_t);
 }
 
 cudaError_t launch_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
@@ -559,13 +576,14 @@ cudaError_t launch_backward(int64_t B, int64_t T, int64_t C, const float* w, con
     unsigned char* base = static_cast<unsigned char*>(ws);
     a.hdr = reinterpret_cast<BwdHeader*>(base);
     a.fs = reinterpret_cast<float*>(base + kBwdHeaderBytes);
+    const int64_t NG = (a.P + kGroupSegs - 1) / kGroupSegs;
     a.fslots = reinterpret_cast<uint64_t*>(base + kBwdHeaderBytes + (size_t)SP * 4 * sizeof(float));
-    a.slots = a.fslots + (size_t)SP * 4;
+    a.slots = a.fslots + (size_t)(B * NG * C) * 4;
     a.dev_err = device_status_word();
     if (!a.dev_err) return cudaErrorInvalidValue;
     a.spin_limit = kSpinLimitDefault;
     const int64_t cx = (C + kThreads - 1) / kThreads;
-    const int64_t units = a.P * B * cx;
+    const int64_t units = NG * B * cx;
     if (units > INT32_MAX) return cudaErrorInvalidValue;
     static uint64_t attr_done = 0;  // per device; set once so captured launches issue no attribute call
     int dev = 0;
@@ -576,8 +594,8 @@ cudaError_t launch_backward(int64_t B, int64_t T, int64_t C, const float* w, con
         if (e != cudaSuccess) return e;
         if (dev < 64) attr_done |= 1ull << dev;
     }
-    bwd_seg_starts<<<(unsigned)units, kThreads, 0, s>>>(a, cx);
-    bwd_seg_reverse<<<(unsigned)units, kThreads, kGradSmem, s>>>(a, cx);
+    bwd_seg_starts<<<(unsigned)units, kGroupThreads, 0, s>>>(a, cx);
+    bwd_seg_reverse<<<(unsigned)units, kGroupThreads, kGradSmem, s>>>(a, cx);
     return cudaGetLastError();
 }
 

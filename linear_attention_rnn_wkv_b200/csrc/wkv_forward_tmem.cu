@@ -151,6 +151,13 @@ constexpr int kCg = 64;   // channels per tile (a lane owns a pair)
 #define WKV_TMEM_PARK_EXPONENT 1
 #endif
 constexpr bool kParkExponent = WKV_TMEM_PARK_EXPONENT != 0;
+// Where the summarising warps take their weights 2^(x_i - M): the MUFU pipe (0), a polynomial on
+// the FMA pipe for every row (1) or for every other row (2), to unload the MUFU pipe that the
+// emitting warps' exponentials and reciprocals need.
+#ifndef WKV_TMEM_SOFT_EXP2
+#define WKV_TMEM_SOFT_EXP2 0
+#endif
+constexpr int kSoftExp2 = WKV_TMEM_SOFT_EXP2;
 constexpr int kThreads = (1 + kNL + 2 * kNWS) * 32;
 
 // What every role needs to know about a unit, worked out once by the producer (per
@@ -594,7 +601,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             Pk<TIO>::load(vt + (r_begin + r) * Cg + cl, &vw[rr * W]);
                             if (FULL || r < r_cnt) {
                                 const float2 x = __fadd2_rn(gx[r], nM);
-                                const float2 e = make_float2(ex2(x.x), ex2(x.y));
+                                const float2 e = (kSoftExp2 == 1 || (kSoftExp2 == 2 && (r & 1)))
+                                                     ? exp2_fma2(x)
+                                                     : make_float2(ex2(x.x), ex2(x.y));
                                 sa = __ffma2_rn(e, Pk<TIO>::unpack(&vw[rr * W]), sa);
                                 sb = __fadd2_rn(sb, e);
                             }
@@ -949,8 +958,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ew == 0 && lane == 0) WKV_TRACE_EVENT(unit, 9);
             if (lane == 0) mbar_arrive(uempty(t));
         }
-        // the chunks' stores must be done before the block's shared memory goes away
-        if (lane == 0) bulk_wait_all();
+        // the chunks' stores must have read their rows before the block's shared memory goes
+        // away (their writes complete on their own; the kernel's end orders them for later work)
+        if (lane == 0) bulk_wait_read();
         __syncwarp();
     }
 

@@ -59,7 +59,7 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 
 // Suspend-time hint of the mbarrier waits, in nanoseconds (0: poll with a short sleep).
 #ifndef WKV_WAIT_HINT
-#define WKV_WAIT_HINT 1000
+#define WKV_WAIT_HINT 250
 #endif
 
 // Bounded wait on an mbarrier phase; returns false if it ran out.  With a hint, a waiting
@@ -92,8 +92,6 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* tm, const void* 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // waits until this thread's committed bulk stores have read their shared-memory source
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// waits until this thread's committed bulk stores are complete
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 struct PipeParams {
     int64_t groups_per_b, G, S, U;

@@ -118,10 +118,10 @@ def test_backward_validation_without_launch():
     assert bwd(1, 4, 4, nbytes=16) == 1          # workspace too small
     assert bwd(70000, 1, 4) == 3                 # batch above the grid's z limit
     assert bwd(1, 32 * 65535 + 1, 4) == 3        # more 32-step segments than the grid's y limit
-    # a 64-byte header, then 88 B per (b, 32-step segment, c)
-    assert L.wkv_backward_workspace_size(2, 3, 5) == 64 + 2 * 1 * 5 * 88
-    assert L.wkv_backward_workspace_size(1, 130, 2) == 64 + 1 * 5 * 2 * 88
-    assert L.wkv_backward_workspace_size(1, 128, 2) == 64 + 1 * 4 * 2 * 88
+    # a 64-byte header, 16 B per (b, 32-step segment, c), 72 B per (b, group of 4 segments, c)
+    assert L.wkv_backward_workspace_size(2, 3, 5) == 64 + 2 * 1 * 5 * 16 + 2 * 1 * 5 * 72
+    assert L.wkv_backward_workspace_size(1, 130, 2) == 64 + 1 * 5 * 2 * 16 + 1 * 2 * 2 * 72
+    assert L.wkv_backward_workspace_size(1, 128, 2) == 64 + 1 * 4 * 2 * 16 + 1 * 1 * 2 * 72
 
 
 def test_gated_and_shift3_validation_without_launch():
