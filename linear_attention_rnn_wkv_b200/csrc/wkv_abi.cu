@@ -167,32 +167,9 @@ bool f32_args_ok(std::initializer_list<const void*> ps) {
     return true;
 }
 
-// Evaluates the library's polynomial 2^x (exp2_fma2) elementwise, for its accuracy test.
-__global__ void exp2_fma_kernel(int64_t n, const float* x, float* y) {
-    const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 2;
-    if (i + 1 < n) {
-        const float2 r = exp2_fma2(make_float2(x[i], x[i + 1]));
-        y[i] = r.x;
-        y[i + 1] = r.y;
-    } else if (i < n) {
-        y[i] = exp2_fma2(make_float2(x[i], 0.f)).x;
-    }
-}
-
 }  // namespace
 
 extern "C" {
-
-/* Test hook: y = the library's FMA-pipe 2^x over n floats (device pointers). */
-wkv_status wkv_testhook_exp2_fma(int64_t n, const float* x, float* y, cudaStream_t stream) {
-    if (n < 0 || (n > 0 && (!x || !y))) return WKV_ERR_INVALID_ARG;
-    if (n == 0) return WKV_OK;
-    const int64_t blocks = ((n + 1) / 2 + 255) / 256;
-    if (blocks > INT32_MAX) return WKV_ERR_INVALID_ARG;
-    exp2_fma_kernel<<<(unsigned)blocks, 256, 0, stream>>>(n, x, y);
-    const cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? WKV_OK : cuda_fail(e);
-}
 
 size_t wkv_forward_workspace_size(int64_t B, int64_t T, int64_t C, wkv_dtype io) {
     int64_t n = 0;

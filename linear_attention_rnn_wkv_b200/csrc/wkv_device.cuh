@@ -55,31 +55,6 @@ __device__ __forceinline__ float rcp(float x) {
     return y;
 }
 
-// 2^x for a pair of x <= 0 (weights against a maximum) on the FMA and integer pipes, leaving
-// the MUFU pipe to the other exponentials.  Cody-Waite style split x = n + f, n the nearest
-// integer (found by adding and subtracting 1.5 * 2^23, which rounds to nearest) and f in
-// [-1/2, 1/2]; 2^f from a degree-5 polynomial whose coefficients were fitted for this library
-// to 2^f on [-1/2, 1/2] (Lawson's iteratively reweighted least squares towards the minimax
-// relative error: 7.5e-8 in exact arithmetic, 2.4e-7 with fp32 Horner steps); n is then added
-// to the exponent field (the low bits of x + 1.5 * 2^23 hold n, so shifting them left by 23
-// gives n << 23).  x is clamped below at -120 first, so a weight under 2^-120 (negligible
-// next to the maximum's 1) comes out as 2^-120 and every exponent stays in the normal range.
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-    x.x = fmaxf(x.x, -120.f);
-    x.y = fmaxf(x.y, -120.f);
-    const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
-    const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-    float2 p = make_float2(1.327647129e-03f, 1.327647129e-03f);
-    p = __ffma2_rn(p, f, make_float2(9.675540961e-03f, 9.675540961e-03f));
-    p = __ffma2_rn(p, f, make_float2(5.550713092e-02f, 5.550713092e-02f));
-    p = __ffma2_rn(p, f, make_float2(2.402212024e-01f, 2.402212024e-01f));
-    p = __ffma2_rn(p, f, make_float2(6.931469440e-01f, 6.931469440e-01f));
-    p = __ffma2_rn(p, f, make_float2(1.000000119e+00f, 1.000000119e+00f));
-    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
 // exp in the chosen domain
 template <bool NAT>
 __device__ __forceinline__ float expd(float x) {
@@ -295,6 +270,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     asm volatile(
         "{\n\t.reg .pred P;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking test: true once the phase with the given parity has completed (the thread is
+// never suspended, so a caller that must also watch another condition sees it promptly).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, P;\n\t}"
         : "=r"(ok)
         : "r"(smem_u32(bar)), "r"(parity)

@@ -151,13 +151,6 @@ constexpr int kCg = 64;   // channels per tile (a lane owns a pair)
 #define WKV_TMEM_PARK_EXPONENT 1
 #endif
 constexpr bool kParkExponent = WKV_TMEM_PARK_EXPONENT != 0;
-// Where the summarising warps take their weights 2^(x_i - M): the MUFU pipe (0), a polynomial on
-// the FMA pipe for every row (1) or for every other row (2), to unload the MUFU pipe that the
-// emitting warps' exponentials and reciprocals need.
-#ifndef WKV_TMEM_SOFT_EXP2
-#define WKV_TMEM_SOFT_EXP2 0
-#endif
-constexpr int kSoftExp2 = WKV_TMEM_SOFT_EXP2;
 constexpr int kThreads = (1 + kNL + 2 * kNWS) * 32;
 
 // What every role needs to know about a unit, worked out once by the producer (per
@@ -374,9 +367,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int t = (int)(i % NT);
             const uint32_t ph = (uint32_t)((i / NT) & 1);
             bool got = false, gone = false;
+            // polled without suspending, so a warp whose unit lies past the end sees the
+            // producer's end index at once (a suspended wait here held blocks ~3 us at the end)
             for (uint32_t it = 0; it <= lim; ++it) {
-                if (WKV_WAIT_HINT ? mbar_try_wait_hint(chunks_bar(t), ph, WKV_WAIT_HINT)
-                                  : mbar_try_wait(chunks_bar(t), ph)) {
+                if (mbar_test_wait(chunks_bar(t), ph)) {
                     got = true;
                     break;
                 }
@@ -384,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     gone = true;
                     break;
                 }
-                if (!WKV_WAIT_HINT) __nanosleep(32);
+                __nanosleep(it < 256 ? 64 : 512);  // the bound stays ~0.1 s of waiting
             }
             if (gone) break;
             if (!got && lane == 0) report(kDevTimeoutCarry);
@@ -601,9 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             Pk<TIO>::load(vt + (r_begin + r) * Cg + cl, &vw[rr * W]);
                             if (FULL || r < r_cnt) {
                                 const float2 x = __fadd2_rn(gx[r], nM);
-                                const float2 e = (kSoftExp2 == 1 || (kSoftExp2 == 2 && (r & 1)))
-                                                     ? exp2_fma2(x)
-                                                     : make_float2(ex2(x.x), ex2(x.y));
+                                const float2 e = make_float2(ex2(x.x), ex2(x.y));
                                 sa = __ffma2_rn(e, Pk<TIO>::unpack(&vw[rr * W]), sa);
                                 sb = __fadd2_rn(sb, e);
                             }
@@ -963,6 +955,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) bulk_wait_read();
         __syncwarp();
     }
+    if (lane == 0) WKV_TRACE_WARP(pp.U, warp);
 
     tc_fence_before();
     __syncthreads();

@@ -36,7 +36,23 @@ __device__ __forceinline__ void wkv_trace_block(int64_t units, int ev) {
     g_wkv_trace[units * 11 + blockIdx.x * 2 + ev] = t;
 }
 #define WKV_TRACE_BLOCK(units, ev) wkv_trace_block(units, ev)
+// per block and warp, after the blocks' events: [24] = each warp's role end (warps 0-19), then
+// the block's SM id
+__device__ __forceinline__ void wkv_trace_warp(int64_t units, int warp) {
+    if (!g_wkv_trace) return;
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    unsigned long long* base = g_wkv_trace + units * 11 + 2 * 148 + blockIdx.x * 24;
+    base[warp] = t;
+    if (warp == 0) {
+        unsigned sm;
+        asm volatile("mov.u32 %0, %smid;" : "=r"(sm));
+        base[20] = sm;
+    }
+}
+#define WKV_TRACE_WARP(units, warp) wkv_trace_warp(units, warp)
 #else
+#define WKV_TRACE_WARP(units, warp) ((void)0)
 #define WKV_TRACE_EVENT(unit, ev) ((void)0)
 #define WKV_TRACE_BLOCK(units, ev) ((void)0)
 #endif
