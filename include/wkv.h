@@ -281,18 +281,33 @@ wkv_status wkv_forward_chunked_noalloc(int64_t B, int64_t T, int64_t C, wkv_dtyp
  *   y              [B, T, C] fp32 (written; must not alias the inputs)
  *   state_out      [B][C/64][64][64] fp32, the state after the last token, or NULL
  *   workspace      caller-owned device scratch, ws_bytes >= eagle_forward_workspace_size()
+ *                  (none when eagle_forward_workspace_size() is 0: workspace may then be NULL)
  * C must be a multiple of 64 (else WKV_ERR_UNSUPPORTED), C/64 and B at most 65535.  T = 0
- * writes state_out only (state_in, or zeros).  Time-parallel over 64-token chunks: each
- * chunk's own state contribution (a tensor-core product with operands split into two tf32
- * parts, for fp32-level error), a scan over the chunks per state entry, then each chunk's
- * outputs from its starting state (fp32).  Status codes as wkv_forward.
+ * writes state_out only (state_in, or zeros).  Two forms, chosen from the shape
+ * (eagle_forward_launches):
+ *   one launch: a block per (sequence, head) walks its 64-token chunks in order; per 16-token
+ *     block the outputs are the state's read-out plus the block's own causal attention, and the
+ *     state advances by the block's key-value sum, every product on the tensor cores (tcgen05,
+ *     operands split into two tf32 parts for fp32-level error) and the state kept in fp32
+ *     registers.  A head with a channel of |w| > 5.5 (decay below 0.004 per token) runs the
+ *     same launch token by token on the CUDA cores instead.  Used when B * C/64 >= 24 or the
+ *     sequence has at most 8 chunks.
+ *   three launches, time-parallel over all chunk-heads: each chunk's own state contribution (a
+ *     tensor-core product as above), a scan over the chunks per state entry, then each chunk's
+ *     outputs from its starting state (fp32 CUDA cores).  For few heads with long sequences.
+ * Status codes as wkv_forward.
  */
 wkv_status eagle_forward(int64_t B, int64_t T, int64_t C, const float* w, const float* r, const float* k,
                          const float* v, const float* state_in, float* y, float* state_out, void* workspace,
                          size_t ws_bytes, cudaStream_t stream);
 
-/* Workspace bytes eagle_forward needs: 16 KiB per sequence, head and 64-token chunk. */
+/* Workspace bytes eagle_forward needs: 0 for the one-launch form, else 16 KiB per sequence,
+ * head and 64-token chunk. */
 size_t eagle_forward_workspace_size(int64_t B, int64_t T, int64_t C);
+
+/* Kernel launches eagle_forward makes for this shape: 1 (the one-launch form) or 3; 0 for an
+ * invalid shape.  No device call. */
+int eagle_forward_launches(int64_t B, int64_t T, int64_t C);
 
 /*
  * Eagle decode: one token for N sessions x L layers (section "O(N) Inference

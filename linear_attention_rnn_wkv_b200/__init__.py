@@ -75,6 +75,8 @@ def lib():
                 L.eagle_forward.argtypes = [i64, i64, i64] + [vp] * 8 + [sz, vp]
                 L.eagle_forward_workspace_size.argtypes = [i64, i64, i64]
                 L.eagle_forward_workspace_size.restype = sz
+                L.eagle_forward_launches.argtypes = [i64, i64, i64]
+                L.eagle_forward_launches.restype = i32
                 L.eagle_decode_step.argtypes = [i64, i64, i64] + [vp] * 7
                 L.wkv_decode_step_fused.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
                 L.token_shift_mix.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp]

@@ -252,7 +252,9 @@ wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float* w, const f
 size_t eagle_forward_workspace_size(int64_t B, int64_t T, int64_t C) {
     int64_t n = 0;
     if (!sizes_ok(B, T, C, &n) || C % 64 != 0) return 0;
-    // per (b, head, chunk): one 64 x 64 fp32 state (the chunk's sum, then its starting state)
+    // the one-launch form needs no scratch; the three-launch form one 64 x 64 fp32 state per
+    // (b, head, chunk) (the chunk's sum, then its starting state)
+    if (eagle_uses_sequence_kernel(B, T, C)) return 0;
     const int64_t heads = B * (C / 64), chunks = eagle_chunks(T);
     if (chunks != 0 && heads > INT64_MAX / 16384 / chunks) return 0;
     return (size_t)heads * (size_t)chunks * 64 * 64 * sizeof(float);
@@ -272,9 +274,16 @@ wkv_status eagle_forward(int64_t B, int64_t T, int64_t C, const float* w, const 
     // TMA coordinates are 32-bit
     if (B > 65535 || C / 64 > 65535 || T > INT32_MAX || C > INT32_MAX || B * (C / 64) > INT32_MAX / 16)
         return WKV_ERR_UNSUPPORTED;
-    if (n > 0 && (!workspace || ws_bytes < eagle_forward_workspace_size(B, T, C))) return WKV_ERR_INVALID_ARG;
+    const size_t need = eagle_forward_workspace_size(B, T, C);
+    if (n > 0 && need > 0 && (!workspace || ws_bytes < need)) return WKV_ERR_INVALID_ARG;
     cudaError_t e = launch_eagle_forward(B, T, C, w, r, k, v, state_in, y, state_out, workspace, stream);
     return e == cudaSuccess ? WKV_OK : cuda_fail(e);
+}
+
+int eagle_forward_launches(int64_t B, int64_t T, int64_t C) {
+    int64_t n = 0;
+    if (!sizes_ok(B, T, C, &n) || C % 64 != 0) return 0;
+    return eagle_uses_sequence_kernel(B, T, C) ? 1 : 3;
 }
 
 wkv_status eagle_decode_step(int64_t N, int64_t L, int64_t C, const float* w, const float* r, const float* k,

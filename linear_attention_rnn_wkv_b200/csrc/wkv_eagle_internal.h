@@ -10,6 +10,10 @@ namespace wkvb {
 // Chunks of the prefill's time-parallel form (tokens per chunk: 64).
 int64_t eagle_chunks(int64_t T);
 
+// True when the prefill of this shape runs as one launch of one block per (sequence, head)
+// (eagle_seq_tc); otherwise three launches over all chunk-heads (chunk sums, state scan, outputs).
+bool eagle_uses_sequence_kernel(int64_t B, int64_t T, int64_t C);
+
 // Prefill over [B, T, C] (C a multiple of 64); ws holds B * H * eagle_chunks(T) * 64 * 64 floats.
 cudaError_t launch_eagle_forward(int64_t B, int64_t T, int64_t C, const float* w, const float* r, const float* k,
                                  const float* v, const float* state_in, float* y, float* state_out, void* ws,

@@ -199,7 +199,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-bool make_tile_map(CUtensorMap* tm, const void* base, int64_t B, int64_t T, int64_t C, int io, int Cg, int Ts) {
+bool make_tile_map(CUtensorMap* tm, const void* base, int64_t B, int64_t T, int64_t C, int io, int Cg, int Ts,
+                   bool swizzle128 = false) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t es = io == 1 ? 2 : 4;
@@ -209,7 +210,8 @@ bool make_tile_map(CUtensorMap* tm, const void* base, int64_t B, int64_t T, int6
     cuuint32_t estr[3] = {1, 1, 1};
     const CUresult r = fn(tm, io == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
                           const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }

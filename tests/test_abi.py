@@ -147,13 +147,19 @@ def test_eagle_validation_without_launch():
     assert fwd(1, 4, 64, r=None) == 1            # null input
     assert fwd(1, 4, 64, y=FAKE + 4) == 2        # misaligned output
     assert fwd(1, 4, 64, state_in=FAKE + 8) == 2  # misaligned optional state
-    assert fwd(1, 4, 64, nbytes=16) == 1         # workspace too small
+    assert fwd(1, 1000, 64, nbytes=16) == 1      # workspace too small (the three-launch form)
     assert fwd(70000, 1, 64) == 3                # batch above the grid's z limit
     assert fwd(0, 4, 64) == 0 and fwd(1, 4, 0) == 0  # empty calls
-    # one 64 x 64 fp32 state per (sequence, head, 64-token chunk)
-    assert L.eagle_forward_workspace_size(2, 65, 128) == 2 * 2 * 2 * 64 * 64 * 4
-    assert L.eagle_forward_workspace_size(1, 64, 64) == 64 * 64 * 4
-    assert L.eagle_forward_workspace_size(1, 4, 96) == 0
+    # the one-launch form (24 or more sequence-heads, or at most 8 chunks) needs no scratch; the
+    # three-launch form one 64 x 64 fp32 state per (sequence, head, 64-token chunk)
+    assert L.eagle_forward_launches(2, 65, 128) == 1 and L.eagle_forward_workspace_size(2, 65, 128) == 0
+    assert L.eagle_forward_launches(8, 1024, 768) == 1 and L.eagle_forward_workspace_size(8, 1024, 768) == 0
+    assert L.eagle_forward_launches(1, 512, 64) == 1 and L.eagle_forward_workspace_size(1, 512, 64) == 0
+    assert L.eagle_forward_launches(1, 513, 64) == 3
+    assert L.eagle_forward_workspace_size(1, 1000, 64) == 16 * 64 * 64 * 4
+    assert L.eagle_forward_workspace_size(2, 1000, 640) == 2 * 10 * 16 * 64 * 64 * 4
+    assert L.eagle_forward_launches(3, 5000, 448) == 3 and L.eagle_forward_launches(4, 5000, 384) == 1
+    assert L.eagle_forward_workspace_size(1, 4, 96) == 0 and L.eagle_forward_launches(1, 4, 96) == 0
 
     def dec(N, L_, C, state=FAKE, y=FAKE):
         return L.eagle_decode_step(N, L_, C, FAKE, FAKE, FAKE, FAKE, state, y, None)

@@ -65,6 +65,39 @@ def test_eagle_forward_matches_oracle(shape, with_state):
     _check(y, st, w, r, k, v, state_in)
 
 
+@pytest.mark.parametrize("shape", [(2, 700, 768), (4, 333, 512), (3, 1000, 512), (2, 1000, 256)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_eagle_forward_both_forms(shape):
+    """Shapes on either side of the choice between the one-launch form (a block per sequence-head
+    walking its chunks: 24 or more sequence-heads) and the three-launch form (few heads, more than
+    8 chunks), ragged last chunks, with and without a given state, every element checked."""
+    import linear_attention_rnn_wkv_b200 as wkv
+    B, T, C = shape
+    launches = wkv.lib().eagle_forward_launches(B, T, C)
+    assert launches == (1 if B * (C // 64) >= 24 else 3)
+    spec, (w, r, k, v) = _case(B, T, C, seed=2300 + B + T + C)
+    y, st = _gpu_forward(w, r, k, v)
+    _check(y, st, w, r, k, v)
+    S0 = synth.eagle_state(spec)
+    y, st = _gpu_forward(w, r, k, v, S0)
+    _check(y, st, w, r, k, v, S0)
+
+
+def test_eagle_forward_fast_decay_head():
+    """A head holding one channel with w = 7 (decay e^-7 per token, beyond the range the
+    one-launch form's scaled operands admit) runs token by token in the same launch while the
+    other heads use the tensor cores; every element against the oracle, for both forms."""
+    import linear_attention_rnn_wkv_b200 as wkv
+    for B, T, C in ((3, 150, 512), (1, 600, 192)):
+        spec, (w, r, k, v) = _case(B, T, C, seed=2310 + T)
+        w = w.copy()
+        w[64 + 5] = 7.0
+        assert wkv.lib().eagle_forward_launches(B, T, C) == (1 if B * (C // 64) >= 24 or T <= 512 else 3)
+        S0 = synth.eagle_state(spec)
+        y, st = _gpu_forward(w, r, k, v, S0)
+        _check(y, st, w, r, k, v, S0)
+
+
 def test_eagle_forward_decay_extremes():
     """No decay (w = 0: causal linear attention) and total decay (w = 1e4: only the current
     token, y_t = (r_t . k_t) v_t) on the GPU."""
