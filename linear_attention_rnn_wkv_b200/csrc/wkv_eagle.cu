@@ -425,12 +425,13 @@ __global__ void __launch_bounds__(kHead) eagle_decode(int64_t L, int64_t C, int6
 //    A_I, run the state from block to block (thread t of warp w holds key rows
 //    32 (w / 4) + 16 (t / 16) .. + 15 of value column 16 (w % 4) + t % 16) and read y out.  Lane 0 of warp 8 issues A and the U_I, lane 0 of warp 9 the Y_I (two
 //    issuing warps keep the tensor core fed).  Hand-overs are mbarriers with bounded waits:
-//    ops (operands of a chunk written, to both issuers), diag (A_I written), sready[4] (Ŝ^T of a
-//    block written, one per buffer: block g uses buffer g % 4), raw (a chunk's rows landed), and
-//    tensor-core commits U, A (warp 8, in that order), Y[4] (per Ŝ^T buffer) and done[2] (every
-//    product of warp 9 in a chunk, per chunk parity).  Rc and the Y accumulator have a buffer
-//    per chunk parity, so the math warps build chunk c + 1's operands while chunk c's last Y
-//    products run and read chunk c's y out after chunk c + 1's state chain.
+//    kv (Kt and V^T of a chunk written), ops (all its operands written), diag (A_I written),
+//    s123 and s0 (once per chunk each: Ŝ^T of its blocks 1-3, and of the next chunk's block 0,
+//    written; block I uses buffer I), raw (a chunk's rows landed), and tensor-core commits U, A (warp
+//    8, in that order), Y0 (block 0's Y product), diagdone (the diagonal products) and done[2]
+//    (every product of warp 9 in a chunk, per chunk parity).  Rc and the Y accumulator have a
+//    buffer per chunk parity, so the math warps build chunk c + 1's operands while chunk c's Y
+//    products run and read chunk c's y out before chunk c + 1's state chain.
 // ---------------------------------------------------------------------------------------------
 // Per-chunk event trace of block 0 (profiling builds only): compiled with -DWKV_TRACE, the
 // sequence kernel stamps %globaltimer at its hand-overs into the buffer registered with
@@ -466,7 +467,7 @@ constexpr uint32_t kSqAd = 18 * kBOp;                  // A_I hi (4 x 512 B), th
 constexpr uint32_t kSqPw = kSqAd + 4096;               // d^e table
 constexpr uint32_t kSqW2 = kSqPw + kPwRows * kPwStride * 4;  // w log2e of the head's 64 channels
 constexpr uint32_t kSqBar = kSqW2 + 64 * 4;            // mbarriers, the TMEM address, the form flag
-constexpr uint32_t kSqY = (kSqBar + 128 + 1023) / 1024 * 1024;  // y tile [64 tokens][64 columns], TMA store source
+constexpr uint32_t kSqY = (kSqBar + 256 + 1023) / 1024 * 1024;  // y tile [64 tokens][64 columns], TMA store source
 constexpr uint32_t kSqRaw = kSqY + kTileBytes;         // the chunk's r, k, v rows: 6 boxes [64 tokens][32 channels]
 constexpr uint32_t kRawBox = kEL * 32 * 4;             // 8 KB, 128-byte rows with the 128-byte swizzle
 constexpr size_t kSqSmem = kSqRaw + 6 * kRawBox;
@@ -478,7 +479,8 @@ static_assert(2 * kTileBytes + 4 * kTileBytes <= kSqPw, "token-by-token staging 
 
 constexpr uint32_t kColA = 0, kColU = 64, kColY = 320, kSeqCols = 512;  // TMEM columns (Y: two buffers of 64)
 
-enum { kBarOps = 0, kBarDiag, kBarS0, kBarA = kBarS0 + 4, kBarU, kBarY0, kBarDone = kBarY0 + 4, kBarRaw = kBarDone + 2, kNumSeqBars };
+enum { kBarOps = 0, kBarKV, kBarDiag, kBarS0, kBarS123, kBarA, kBarU, kBarY0, kBarDiagDone, kBarDone, kBarRaw = kBarDone + 2, kNumSeqBars };
+static_assert(kNumSeqBars * 8 + 8 <= 256, "barriers, TMEM address and form flag fit their area");
 
 // bf16 K-major operand index (in elements) of (row, k) for a K-wide operand
 template <int K>
@@ -643,7 +645,7 @@ __global__ void __launch_bounds__(kSeqThreads, 1) eagle_seq_tc(EagleArgs a, cons
     }
     if (tid == 0) {
         for (int i = 0; i < kNumSeqBars; ++i)
-            mbar_init(&bars[i], (i == kBarOps || i == kBarDiag || (i >= kBarS0 && i < kBarS0 + 4)) ? kSeqMath : 1);
+            mbar_init(&bars[i], (i == kBarOps || i == kBarKV || i == kBarDiag || i == kBarS0 || i == kBarS123) ? kSeqMath : 1);
         fence_mbar_init();
     }
     __syncthreads();
@@ -689,12 +691,11 @@ __global__ void __launch_bounds__(kSeqThreads, 1) eagle_seq_tc(EagleArgs a, cons
                 asm volatile("" : "+l"(q1k), "+l"(q256));
                 auto D = [&](uint32_t off) { return q1k + (off >> 4); };
                 if (warp == 8) {
-                    seq_wait(a, &bars[kBarOps], par);
+                    seq_wait(a, &bars[kBarKV], par);
                     tm_fence_after();
                     EAGLE_TRACE(c, 0);
-                    if (c + 1 < P) load_raw(c + 1);  // the raw stage is consumed
-                    // U_I^T = V_I^T Kt_I (M = 64 columns, N = 64 key rows, K = the block's 16 tokens):
-                    // first, the state chain waits for it
+                    // U_I^T = V_I^T Kt_I (M = 64 columns, N = 64 key rows, K = the block's 16 tokens),
+                    // as soon as Kt and V^T are written: the state chain waits for it
 #pragma unroll
                     for (uint32_t I = 0; I < 4; ++I)
                         mma_product<1>(tmem + kColU + 64 * I, D(kSqVt + 256 * I), D(kSqVt + kBOp + 256 * I),
@@ -702,17 +703,20 @@ __global__ void __launch_bounds__(kSeqThreads, 1) eagle_seq_tc(EagleArgs a, cons
                     mma_commit(&bars[kBarU]);
                     EAGLE_TRACE(c, 9);
                     // A = Rc Kc^T (M = N = 64 tokens, K = 64 key rows)
+                    seq_wait(a, &bars[kBarOps], par);
+                    tm_fence_after();
                     const uint32_t rc = kSqRc + 2 * kBOp * (uint32_t)(c & 1);
                     mma_product<4>(tmem + kColA, D(rc), D(rc + kBOp), D(kSqKc), D(kSqKc + kBOp), id64, 0);
                     mma_commit(&bars[kBarA]);
                     EAGLE_TRACE(c, 1);
+                    if (c + 1 < P) load_raw(c + 1);  // the raw stage is consumed
                 } else {
                     // Y_0^T: the state part of block 0
                     const int64_t g0 = 4 * c;
                     const uint32_t ty = tmem + kColY + 64 * (uint32_t)(c & 1);  // Y buffer of the chunk
                     const uint32_t rc = kSqRc + 2 * kBOp * (uint32_t)(c & 1);
                     seq_wait(a, &bars[kBarOps], par);
-                    seq_wait(a, &bars[kBarS0], (uint32_t)((g0 >> 2) & 1));
+                    seq_wait(a, &bars[kBarS0], par);  // Ŝ^T of block 0 (written at the end of the last chunk's chain)
                     tm_fence_after();
                     mma_product<4>(ty, D(kSqS), D(kSqS + kBOp), D(rc), D(rc + kBOp), id16, 0);
                     mma_commit(&bars[kBarY0]);
@@ -727,17 +731,16 @@ __global__ void __launch_bounds__(kSeqThreads, 1) eagle_seq_tc(EagleArgs a, cons
                         mma_product<1>(ty + 16 * I, D(kSqVt + 256 * I), D(kSqVt + kBOp + 256 * I), ob,
                                        ob + (2048 >> 4), id16, I == 0 ? 1u : 0u);
                     }
-                    // blocks 1-3: the state part, once the state before the block is written
+                    mma_commit(&bars[kBarDiagDone]);
+                    // blocks 1-3: the state part, once the chain has written the states before them
+                    seq_wait(a, &bars[kBarS123], par);
+                    tm_fence_after();
+                    EAGLE_TRACE(c, 5);
 #pragma unroll 1
                     for (uint32_t I = 1; I < 4; ++I) {
-                        const int64_t g = g0 + I;
-                        seq_wait(a, &bars[kBarS0 + I], (uint32_t)((g >> 2) & 1));
-                        tm_fence_after();
-                        EAGLE_TRACE(c, 4 + I);
                         const uint32_t sb = kSqS + 2 * kBOp * I;
                         const uint64_t orow = (2048u * I) >> 4;  // the block's 16 rows of Rc
                         mma_product<4>(ty + 16 * I, D(sb), D(sb + kBOp), D(rc) + orow, D(rc + kBOp) + orow, id16, 1);
-                        mma_commit(&bars[kBarY0 + I]);
                     }
                     mma_commit(&bars[kBarDone + (c & 1)]);
                     EAGLE_TRACE(c, 8);
@@ -788,10 +791,10 @@ __global__ void __launch_bounds__(kSeqThreads, 1) eagle_seq_tc(EagleArgs a, cons
                 const int o = 2 * bop_index<64>(j, m0 + 8 * g8);
                 store_split8(hi + o, hi + kBOp + o, x);
             }
-            fence_proxy_async_smem();
-            mbar_arrive(&bars[kBarS0 + xb]);
         };
         write_shat(0);
+        fence_proxy_async_smem();
+        mbar_arrive(&bars[kBarS0]);
 
         // y of a chunk: read back, written to the shared tile, stored by one TMA copy (rows past T
         // clipped); the copy has read the tile before the tile is written again (thread 0 waits
@@ -813,15 +816,37 @@ __global__ void __launch_bounds__(kSeqThreads, 1) eagle_seq_tc(EagleArgs a, cons
         for (int64_t c = 0; c < P; ++c) {
             const uint32_t par = (uint32_t)(c & 1);
             const int len = (int)min64(kEL, a.T - c * kEL);
-            // operands of this chunk from the raw stage: Rc and Kc (rows), then Kt and V^T (columns).
+            // operands of this chunk from the raw stage: Kt and V^T (columns), then Rc and Kc (rows).
             // Rc goes to the buffer of the chunk's parity (its last reader, the previous chunk but one,
             // is done: its y was read out); Kc, Kt, V^T and the A_I were last read by the previous
-            // chunk's A, U and diagonal products, done once its block-1 Y product (issued after them)
-            // is.
-            if (c > 0) seq_wait(a, &bars[kBarY0 + 1], par ^ 1u);
+            // chunk's A, U and diagonal products.
+            if (c > 0) seq_wait(a, &bars[kBarDiagDone], par ^ 1u);
             seq_wait(a, &bars[kBarRaw], par);
             if (tid == 0) EAGLE_TRACE(c, 10);
             const uint32_t rc = kSqRc + 2 * kBOp * (uint32_t)(c & 1);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                int m, t8;
+                col_task(i, m, t8);
+                const int I = t8 >> 4, bl = max(0, min(16, len - 16 * I));
+                float xk[8], xv[8];
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    const int li = (t8 & 15) + s;
+                    const bool in = li < bl;
+                    const float p = pw[(in ? bl - 1 - li + 8 : 8) * kPwStride + m];  // d^{bl-1-li}
+                    const float kx = *reinterpret_cast<const float*>(smem + kSqRaw + raw_off(1, t8 + s, m));
+                    xk[s] = in ? kx * p : 0.f;
+                    xv[s] = *reinterpret_cast<const float*>(smem + kSqRaw + raw_off(2, t8 + s, m));
+                }
+                const int o = 2 * bop_index<64>(m, t8);
+                store_split8(smem + kSqKt + o, smem + kSqKt + kBOp + o, xk);
+                store_split8(smem + kSqVt + o, smem + kSqVt + kBOp + o, xv);
+            }
+            fence_proxy_async_smem();
+            tm_fence_before();
+            mbar_arrive(&bars[kBarKV]);  // Kt and V^T written: U may start
+            if (tid == 0) EAGLE_TRACE(c, 24);
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
                 int l, mc8;
@@ -841,26 +866,6 @@ __global__ void __launch_bounds__(kSeqThreads, 1) eagle_seq_tc(EagleArgs a, cons
                 const int o = 2 * bop_index<64>(l, mc8);
                 store_split8(smem + rc + o, smem + rc + kBOp + o, xr);
                 store_split8(smem + kSqKc + o, smem + kSqKc + kBOp + o, xk);
-            }
-            if (tid == 0) EAGLE_TRACE(c, 24);
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                int m, t8;
-                col_task(i, m, t8);
-                const int I = t8 >> 4, bl = max(0, min(16, len - 16 * I));
-                float xk[8], xv[8];
-#pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    const int li = (t8 & 15) + s;
-                    const bool in = li < bl;
-                    const float p = pw[(in ? bl - 1 - li + 8 : 8) * kPwStride + m];  // d^{bl-1-li}
-                    const float kx = *reinterpret_cast<const float*>(smem + kSqRaw + raw_off(1, t8 + s, m));
-                    xk[s] = in ? kx * p : 0.f;
-                    xv[s] = *reinterpret_cast<const float*>(smem + kSqRaw + raw_off(2, t8 + s, m));
-                }
-                const int o = 2 * bop_index<64>(m, t8);
-                store_split8(smem + kSqKt + o, smem + kSqKt + kBOp + o, xk);
-                store_split8(smem + kSqVt + o, smem + kSqVt + kBOp + o, xv);
             }
             if (tid == 0) EAGLE_TRACE(c, 25);
             fence_proxy_async_smem();
@@ -891,9 +896,18 @@ __global__ void __launch_bounds__(kSeqThreads, 1) eagle_seq_tc(EagleArgs a, cons
                 if (tid == 0) EAGLE_TRACE(c, 14);
             };
 
-            // the state from block to block; Ŝ^T of each next block for the issuing warp (the
-            // diagonal blocks are handed over after the first block's state, which is the chain's
-            // first need)
+            // the previous chunk's y: its products ran behind this chunk's operands; once they are
+            // done, the Ŝ^T buffers of blocks 1-3 are free as well
+            if (c > 0) {
+                seq_wait(a, &bars[kBarDone + ((c - 1) & 1)], (uint32_t)(((c - 1) >> 1) & 1));
+                tm_fence_after();
+                if (tid == 0) EAGLE_TRACE(c, 11);
+                read_y(c - 1);
+            }
+
+            // the state from block to block: Ŝ^T of blocks 1-3 and of the next chunk's block 0 into
+            // their buffers, handed over together at the end (the diagonal blocks in between, after
+            // the first block's state)
             seq_wait(a, &bars[kBarU], par);
             tm_fence_after();
             if (tid == 0) EAGLE_TRACE(c, 15);
@@ -904,7 +918,6 @@ __global__ void __launch_bounds__(kSeqThreads, 1) eagle_seq_tc(EagleArgs a, cons
 #pragma unroll
                 for (int k2 = 0; k2 < 2; ++k2) {
                     const int I = I2 + k2;
-                    const int64_t g = 4 * c + I;
                     const int bl = max(0, min(16, len - 16 * I));
                     if (bl == 16) {
 #pragma unroll
@@ -915,25 +928,21 @@ __global__ void __launch_bounds__(kSeqThreads, 1) eagle_seq_tc(EagleArgs a, cons
                         for (int i = 0; i < 16; ++i) S[i] = fmaf(dbl[i], S[i], __uint_as_float(u[k2][i]));
                     }
                     if (k2 == 1) tm_fence_before();
-                    if (c + 1 < P || I < 3) {
-                        // Ŝ^T of block g + 1 into buffer (g + 1) % 4, once the Y product of block g - 3
-                        // (the buffer's last reader) is done
-                        const int64_t gn = g + 1;
-                        const int xb = (int)(gn & 3);
-                        if (gn >= 4) seq_wait(a, &bars[kBarY0 + xb], (uint32_t)(((gn - 4) >> 2) & 1));
-                        if (tid == 0) EAGLE_TRACE(c, 16 + I);
-                        write_shat(xb);
-                        if (tid == 0) EAGLE_TRACE(c, 20 + I);
+                    if (I < 3) {
+                        write_shat(I + 1);
+                        if (I == 2) {  // the states before blocks 1-3
+                            fence_proxy_async_smem();
+                            mbar_arrive(&bars[kBarS123]);
+                        }
+                    } else if (c + 1 < P) {
+                        seq_wait(a, &bars[kBarY0], par);  // block 0's Y product has read buffer 0
+                        write_shat(0);
+                        fence_proxy_async_smem();
+                        mbar_arrive(&bars[kBarS0]);  // the state before the next chunk's block 0
                     }
+                    if (tid == 0) EAGLE_TRACE(c, 16 + I);
                     if (I == 0) diag_blocks();
                 }
-            }
-            // the previous chunk's y (its products ran behind this chunk's operands and chain)
-            if (c > 0) {
-                seq_wait(a, &bars[kBarDone + ((c - 1) & 1)], (uint32_t)(((c - 1) >> 1) & 1));
-                tm_fence_after();
-                if (tid == 0) EAGLE_TRACE(c, 11);
-                read_y(c - 1);
             }
         }
         if (a.state_out)
