@@ -421,17 +421,20 @@ __global__ void __launch_bounds__(kHead) eagle_decode(int64_t L, int64_t C, int6
 //    16-byte core matrices (8 bf16 along K): element (row, k) of a K-wide operand at byte
 //    (row/8)(2K) + (k/8)128 + (row%8)16 + (k%8)2.
 //
-//    Warps 0-7 build the operands (from the chunk's rows, brought by TMA), mask and split the
-//    A_I, run the state from block to block (thread t of warp w holds key rows
-//    32 (w / 4) + 16 (t / 16) .. + 15 of value column 16 (w % 4) + t % 16) and read y out.  Lane 0 of warp 8 issues A and the U_I, lane 0 of warp 9 the Y_I (two
-//    issuing warps keep the tensor core fed).  Hand-overs are mbarriers with bounded waits:
-//    kv (Kt and V^T of a chunk written), ops (all its operands written), diag (A_I written),
-//    s123 and s0 (once per chunk each: Ŝ^T of its blocks 1-3, and of the next chunk's block 0,
-//    written; block I uses buffer I), raw (a chunk's rows landed), and tensor-core commits U, A (warp
-//    8, in that order), Y0 (block 0's Y product), diagdone (the diagonal products) and done[2]
-//    (every product of warp 9 in a chunk, per chunk parity).  Rc and the Y accumulator have a
-//    buffer per chunk parity, so the math warps build chunk c + 1's operands while chunk c's Y
-//    products run and read chunk c's y out before chunk c + 1's state chain.
+//    Roles.  Warps 0-7 build the operands from the chunk's r, k, v rows (brought by TMA with the
+//    128-byte swizzle), mask and split the A_I, run the state from block to block (thread t of
+//    warp w holds key rows 32 (w / 4) + 16 (t / 16) .. + 15 of value column 16 (w % 4) + t % 16)
+//    and read y out into a shared tile.  Lane 0 of warp 8 issues the U_I and A and the next
+//    chunk's row loads, lane 0 of warp 9 the Y_I (two issuing warps keep the tensor core fed),
+//    lane 0 of warp 10 stores each y tile by TMA.  Rc and the Y accumulator have a buffer per
+//    chunk parity, so the math warps build chunk c + 1's operands while chunk c's Y products
+//    run, and read chunk c's y out before chunk c + 1's state chain.
+//    Hand-overs are mbarriers with bounded waits: raw (a chunk's rows landed), kv (Kt and V^T
+//    of a chunk written), ops (all its operands written), diag (A_I written), s123 and s0 (once
+//    per chunk each: Ŝ^T of its blocks 1-3, and of the next chunk's block 0, written; block I
+//    uses buffer I), yt / yf (a y tile written / stored), and tensor-core commits U, A (warp 8,
+//    in that order), Y0 (block 0's Y product), diagdone (the diagonal products) and done[2]
+//    (every product of warp 9 in a chunk, per chunk parity).
 // ---------------------------------------------------------------------------------------------
 // Per-chunk event trace of block 0 (profiling builds only): compiled with -DWKV_TRACE, the
 // sequence kernel stamps %globaltimer at its hand-overs into the buffer registered with
@@ -450,7 +453,8 @@ __device__ __forceinline__ void eagle_trace(int64_t c, int ev) {
 #endif
 
 constexpr int kSeqMath = 256;                 // warps 0-7
-constexpr int kSeqThreads = kSeqMath + 64;    // and the two issuing warps
+constexpr int kSeqWarpY = 10;                 // the y-store warp
+constexpr int kSeqThreads = kSeqMath + 96;    // and the two issuing warps and the y-store warp
 constexpr int kPwRows = 25;                   // d^e, e = -8 .. 16
 constexpr int kPwStride = 68;                 // floats per row: consecutive rows 16 B apart in the banks
 constexpr float kSeqMaxW2 = 8.f;              // |w| log2e admitted by the scaled form
@@ -479,7 +483,8 @@ static_assert(2 * kTileBytes + 4 * kTileBytes <= kSqPw, "token-by-token staging 
 
 constexpr uint32_t kColA = 0, kColU = 64, kColY = 320, kSeqCols = 512;  // TMEM columns (Y: two buffers of 64)
 
-enum { kBarOps = 0, kBarKV, kBarDiag, kBarS0, kBarS123, kBarA, kBarU, kBarY0, kBarDiagDone, kBarDone, kBarRaw = kBarDone + 2, kNumSeqBars };
+enum { kBarOps = 0, kBarKV, kBarDiag, kBarS0, kBarS123, kBarA, kBarU, kBarY0, kBarDiagDone, kBarDone, kBarRaw = kBarDone + 2,
+       kBarYT, kBarYF, kNumSeqBars };
 static_assert(kNumSeqBars * 8 + 8 <= 256, "barriers, TMEM address and form flag fit their area");
 
 // bf16 K-major operand index (in elements) of (row, k) for a K-wide operand
@@ -546,19 +551,6 @@ __device__ __forceinline__ void store_split8(unsigned char* hi, unsigned char* l
     split_bf16x2(x[6], x[7], h.w, l.w);
     *reinterpret_cast<uint4*>(hi) = h;
     *reinterpret_cast<uint4*>(lo) = l;
-}
-
-// Loads issued where they stand (volatile asm keeps them in program order), so a chunk's rows
-// are in flight while the previous chunk's products run.
-__device__ __forceinline__ float4 ld_early4(const float* p) {
-    float4 x;
-    asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(x.x), "=f"(x.y), "=f"(x.z), "=f"(x.w) : "l"(p));
-    return x;
-}
-__device__ __forceinline__ float ld_early(const float* p) {
-    float x;
-    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(x) : "l"(p));
-    return x;
 }
 
 __device__ __forceinline__ void seq_wait(const EagleArgs& a, uint64_t* bar, uint32_t parity) {
@@ -645,7 +637,8 @@ __global__ void __launch_bounds__(kSeqThreads, 1) eagle_seq_tc(EagleArgs a, cons
     }
     if (tid == 0) {
         for (int i = 0; i < kNumSeqBars; ++i)
-            mbar_init(&bars[i], (i == kBarOps || i == kBarKV || i == kBarDiag || i == kBarS0 || i == kBarS123) ? kSeqMath : 1);
+            mbar_init(&bars[i], (i == kBarOps || i == kBarKV || i == kBarDiag || i == kBarS0 || i == kBarS123 || i == kBarYT)
+                                    ? kSeqMath : 1);
         fence_mbar_init();
     }
     __syncthreads();
@@ -667,7 +660,21 @@ __global__ void __launch_bounds__(kSeqThreads, 1) eagle_seq_tc(EagleArgs a, cons
     const uint32_t sm = smem_u32(smem);
     const int64_t P = a.P;
 
-    if (warp >= 8) {
+    if (warp == kSeqWarpY) {
+        // ---- lane 0 of warp 10: each chunk's y tile to global memory by one TMA store (rows past
+        // T clipped), the tile handed back once the store has read it ----
+        if (lane == 0) {
+            for (int64_t c = 0; c < P; ++c) {
+                seq_wait(a, &bars[kBarYT], (uint32_t)(c & 1));
+                tma_store_3d(&tmy, ytile, (int)(h * kHead), (int)(c * kEL), (int)b);
+                bulk_commit();
+                bulk_wait_read();
+                mbar_arrive(&bars[kBarYF]);
+            }
+            bulk_wait_all();  // the last stores are complete before the block exits
+        }
+        __syncwarp();
+    } else if (warp >= 8) {
         // ---- lane 0 of warp 8: A and the U_I; lane 0 of warp 9: the Y_I ----
         if (lane == 0) {
             constexpr uint32_t id64 = bf16_idesc(64, 64), id16 = bf16_idesc(64, 16);
@@ -712,7 +719,6 @@ __global__ void __launch_bounds__(kSeqThreads, 1) eagle_seq_tc(EagleArgs a, cons
                     if (c + 1 < P) load_raw(c + 1);  // the raw stage is consumed
                 } else {
                     // Y_0^T: the state part of block 0
-                    const int64_t g0 = 4 * c;
                     const uint32_t ty = tmem + kColY + 64 * (uint32_t)(c & 1);  // Y buffer of the chunk
                     const uint32_t rc = kSqRc + 2 * kBOp * (uint32_t)(c & 1);
                     seq_wait(a, &bars[kBarOps], par);
@@ -796,21 +802,16 @@ __global__ void __launch_bounds__(kSeqThreads, 1) eagle_seq_tc(EagleArgs a, cons
         fence_proxy_async_smem();
         mbar_arrive(&bars[kBarS0]);
 
-        // y of a chunk: read back, written to the shared tile, stored by one TMA copy (rows past T
-        // clipped); the copy has read the tile before the tile is written again (thread 0 waits
-        // for it before it hands the next chunk's operands over)
+        // y of a chunk: read back and written to the shared tile (once the y-store warp has read
+        // the previous chunk's out of it), handed to the y-store warp
         auto read_y = [&](int64_t c) {
+            if (c > 0) seq_wait(a, &bars[kBarYF], (uint32_t)((c - 1) & 1));
             uint32_t r[16];
             tm_ld16x2(tq + kColY + 64 * (uint32_t)(c & 1) + 32 * hf, r);  // tokens 32 hf + 16 up ..
 #pragma unroll
             for (int i = 0; i < 16; ++i) ytile[(32 * hf + 16 * up + i) * kHead + j] = __uint_as_float(r[i]);
             fence_proxy_async_smem();
-            asm volatile("bar.sync 1, %0;" ::"n"(kSeqMath) : "memory");
-            if (tid == 0) {
-                tma_store_3d(&tmy, ytile, (int)(h * kHead), (int)(c * kEL), (int)b);
-                bulk_commit();
-                bulk_wait_read();
-            }
+            mbar_arrive(&bars[kBarYT]);
         };
 
         for (int64_t c = 0; c < P; ++c) {

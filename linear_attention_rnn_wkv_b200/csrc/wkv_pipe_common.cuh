@@ -108,6 +108,8 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* tm, const void* 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // waits until this thread's committed bulk stores have read their shared-memory source
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// waits until this thread's committed bulk stores are complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 struct PipeParams {
     int64_t groups_per_b, G, S, U;
