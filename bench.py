@@ -575,33 +575,38 @@ def next_rows_bench(torch, wkv, dev, peak):
 
 
 def eagle_bench(torch, wkv, dev, peak, decode=True):
-    """Eagle (RWKV-5) matrix-state WKV: the prefill on eagle_8x1024x768 (r, k, v read and y
-    written once: 16 B/element, plus the final state, 16 KiB per sequence-head) over three
-    rotating input sets (> 2x L2), and the decode step for 256 sessions x 32 layers x 4096
-    channels (each 64 x 64 state read and written once, r, k, v read and y written)."""
+    """Eagle (RWKV-5) matrix-state WKV: the prefill on eagle_8x1024x768 (three rotating input
+    sets, > 2x L2) and eagle_4x4096x2048 (two sets of 1.6 GB), r, k, v read and y written once:
+    16 B/element, plus the final state, 16 KiB per sequence-head; and the decode step for 256
+    sessions x 32 layers x 4096 channels (each 64 x 64 state read and written once, r, k, v read
+    and y written)."""
     import synth
-    spec = synth.EAGLE["eagle_8x1024x768"]
-    B, T, C = spec.B, spec.T, spec.C
-    H = C // 64
+    out = {}
     g = torch.Generator(device=dev)
-    g.manual_seed(spec.seed)
-    w = torch.exp(torch.rand(C, generator=g, device=dev) * (spec.w_hi - spec.w_lo) + spec.w_lo)
-    sets = [[torch.randn((B, T, C), generator=g, device=dev) for _ in range(3)] for _ in range(3)]
-    y = torch.empty((B, T, C), device=dev)
-    st = torch.empty((B, H, 64, 64), device=dev)
-    ws = torch.empty(int(wkv.lib().eagle_forward_workspace_size(B, T, C)), dtype=torch.uint8, device=dev)
+    for key, name, n_sets in (("eagle_forward", "eagle_8x1024x768", 3), ("eagle_forward_long", "eagle_4x4096x2048", 2)):
+        spec = synth.EAGLE[name]
+        B, T, C = spec.B, spec.T, spec.C
+        H = C // 64
+        g.manual_seed(spec.seed)
+        w = torch.exp(torch.rand(C, generator=g, device=dev) * (spec.w_hi - spec.w_lo) + spec.w_lo)
+        sets = [[torch.randn((B, T, C), generator=g, device=dev) for _ in range(3)] for _ in range(n_sets)]
+        y = torch.empty((B, T, C), device=dev)
+        st = torch.empty((B, H, 64, 64), device=dev)
+        ws = torch.empty(int(wkv.lib().eagle_forward_workspace_size(B, T, C)), dtype=torch.uint8, device=dev)
 
-    def fwd(i):
-        r, k, v = sets[i % 3]
-        wkv.eagle_forward(w, r, k, v, y=y, state_out=st, workspace=ws)
+        def fwd(i, sets=sets, w=w, y=y, st=st, ws=ws):
+            r, k, v = sets[i % len(sets)]
+            wkv.eagle_forward(w, r, k, v, y=y, state_out=st, workspace=ws)
 
-    n = B * T * C
-    alg = 16 * n + B * H * 64 * 64 * 4
-    f_ms = graph_ms(torch, fwd, 12)
-    out = {"eagle_forward": {"workload": spec.name, "launch_ms": f_ms, "alg_bytes_per_launch": alg,
-                             "achieved_gbs": alg / (f_ms * 1e-3) / 1e9, "frac": alg / (f_ms * 1e-3) / 1e9 / peak,
-                             "elements_per_s": n / (f_ms * 1e-3)}}
-    del sets, ws
+        n = B * T * C
+        alg = 16 * n + B * H * 64 * 64 * 4
+        f_ms = graph_ms(torch, fwd, 12)
+        out[key] = {"workload": spec.name, "launch_ms": f_ms, "alg_bytes_per_launch": alg,
+                    "achieved_gbs": alg / (f_ms * 1e-3) / 1e9, "frac": alg / (f_ms * 1e-3) / 1e9 / peak,
+                    "elements_per_s": n / (f_ms * 1e-3), "launches": int(wkv.lib().eagle_forward_launches(B, T, C)),
+                    "l2": f"{n_sets} rotating input sets of {3 * n * 4 / 1e6:.0f} MB"}
+        del sets, ws, y, st, w
+        torch.cuda.empty_cache()
     if decode:
         N, L, Cd = 256, 32, 4096
         Hd = Cd // 64
