@@ -161,6 +161,29 @@ struct BwdHeader {
 constexpr size_t kBwdHeaderBytes = sizeof(BwdHeader);
 static_assert(kBwdHeaderBytes == 64, "header size");
 
+// Per-block event trace (profiling builds only): compiled with -DWKV_TRACE, each block stamps
+// %globaltimer at its phase boundaries into the buffer registered with wkv_bwd_trace_set_buffer
+// ([2][units][8] u64: the forward pass's blocks, then the reverse pass's, indexed by ticket;
+// slot 7 the SM id); normal builds define the hook away.
+#ifdef WKV_TRACE
+static __device__ unsigned long long* g_bwd_trace = nullptr;
+__device__ __forceinline__ void bwd_trace(int pass, int64_t units, int64_t unit, int ev) {
+    if (!g_bwd_trace || threadIdx.x != 0) return;
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    unsigned long long* p = g_bwd_trace + ((int64_t)pass * units + unit) * 8;
+    p[ev] = t;
+    if (ev == 0) {
+        unsigned sm;
+        asm volatile("mov.u32 %0, %smid;" : "=r"(sm));
+        p[7] = sm;
+    }
+}
+#define BWD_TRACE(pass, unit, ev) bwd_trace(pass, (int64_t)gridDim.x, unit, ev)
+#else
+#define BWD_TRACE(pass, unit, ev) ((void)0)
+#endif
+
 struct BwdArgs {
     int64_t B, T, C, P;  // P segments of kSeg steps (the last may be shorter)
     const float *w, *u, *k, *v, *gy;
@@ -280,6 +303,7 @@ __global__ void __launch_bounds__(kGroupThreads) bwd_seg_starts(BwdArgs a, int64
         s_epoch = (*reinterpret_cast<volatile uint32_t*>(&a.hdr->epoch_f) + 1u) & 0x3FFFFFFFu;
     }
     __syncthreads();
+    BWD_TRACE(0, s_ticket, 0);
     const int64_t unit = s_ticket;
     const uint32_t epoch30 = s_epoch;
     const uint32_t tag_loc = (epoch30 << 2) | 1u, tag_incl = (epoch30 << 2) | 2u;
@@ -301,10 +325,12 @@ __global__ void __launch_bounds__(kGroupThreads) bwd_seg_starts(BwdArgs a, int64
         forward_span<false, false>(a, b * a.T * a.C + c, j * kSeg, min64(a.T, (j + 1) * kSeg), st, u2, w2,
                                    [](int, const FwdOut&, float) {});
         s_rec[gs][tc] = Rec{st.a, st.bb, st.anc, st.n};
+        BWD_TRACE(0, s_ticket, 1);
     } else {
         s_rec[gs][tc] = rec_identity();
     }
     __syncthreads();
+    BWD_TRACE(0, s_ticket, 2);
     if (gs == 0 && chan) {
         // the group's segments folded in time order; each slot keeps its in-group prefix
         Rec agg = rec_identity();
@@ -343,6 +369,7 @@ __global__ void __launch_bounds__(kGroupThreads) bwd_seg_starts(BwdArgs a, int64
                 }
             }
             if (!done) give_up(a);  // go on with what is there (the gradients are then invalid)
+            BWD_TRACE(0, s_ticket, 3);
             if (J + 1 < NG) {
                 const Rec inc = rec_combine(run, agg, span_len(a, J * kGroupSegs, (J + 1) * kGroupSegs), w2);
                 slot_publish<4>(my, a.C, {inc.a, inc.b, inc.anc, inc.n}, tag_incl);
@@ -351,6 +378,7 @@ __global__ void __launch_bounds__(kGroupThreads) bwd_seg_starts(BwdArgs a, int64
         s_carry[tc] = run;
     }
     __syncthreads();
+    BWD_TRACE(0, s_ticket, 4);
     if (live) {
         // this segment's starting state: the group's, then the group's segments before it
         const Rec st = rec_combine(s_carry[tc], s_rec[gs][tc], span_len(a, J * kGroupSegs, j), w2);
@@ -360,6 +388,7 @@ __global__ void __launch_bounds__(kGroupThreads) bwd_seg_starts(BwdArgs a, int64
         a.fs[2 * SP + si] = st.anc;
         a.fs[3 * SP + si] = st.n;
     }
+    BWD_TRACE(0, s_ticket, 5);
     __syncthreads();
     if (tid == 0) {
         __threadfence();
@@ -406,6 +435,7 @@ __global__ void __launch_bounds__(kGroupThreads) bwd_seg_reverse(BwdArgs a, int6
         s_epoch = (*reinterpret_cast<volatile uint32_t*>(&a.hdr->epoch) + 1u) & 0x3FFFFFFFu;
     }
     __syncthreads();
+    BWD_TRACE(1, s_ticket, 0);
     const int64_t unit = s_ticket;
     const uint32_t epoch30 = s_epoch;
     const uint32_t tag_loc = (epoch30 << 2) | 1u, tag_incl = (epoch30 << 2) | 2u;
@@ -432,10 +462,12 @@ __global__ void __launch_bounds__(kGroupThreads) bwd_seg_reverse(BwdArgs a, int6
             ls.add((float)i, g, o, w2);
         });
         s_in[gs][tc] = Adj{ls.x, ls.y, ls.xp, ls.yp, fmaf(ls.Rj, w2, ls.Rq)};
+        BWD_TRACE(1, s_ticket, 1);
     } else {
         s_in[gs][tc] = adj_empty();
     }
     __syncthreads();
+    BWD_TRACE(1, s_ticket, 2);
     if (gs == 0 && chan) {
         // the group's segments composed right to left; each slot keeps what enters its segment
         // from the group's later segments
@@ -484,6 +516,7 @@ __global__ void __launch_bounds__(kGroupThreads) bwd_seg_reverse(BwdArgs a, int6
                 give_up(a);
                 gin = acc;
             }
+            BWD_TRACE(1, s_ticket, 3);
         }
         if (J > 0) {
             const Adj out = adj_compose(run, gin, span_len(a, J * kGroupSegs, (J + 1) * kGroupSegs), w2);
@@ -492,6 +525,7 @@ __global__ void __launch_bounds__(kGroupThreads) bwd_seg_reverse(BwdArgs a, int6
         s_gin[tc] = gin;
     }
     __syncthreads();
+    BWD_TRACE(1, s_ticket, 4);
     if (live) {
         // the sums entering this segment: its group's later segments', with the group's own
         // incoming sums carried across them
@@ -523,10 +557,12 @@ __global__ void __launch_bounds__(kGroupThreads) bwd_seg_reverse(BwdArgs a, int6
             const int64_t at = base + (t - 1) * a.C;
             step(t - 1, a.k[at], a.v[at], a.gy[at]);
         }
+        BWD_TRACE(1, s_ticket, 5);
         atomicAdd(&a.gw[c], sgw);
         atomicAdd(&a.gu[c], sgu);
     }
     // the launch's last block resets the counters and advances the epoch
+    BWD_TRACE(1, s_ticket, 6);
     __syncthreads();
     if (tid == 0) {
         __threadfence();
@@ -540,6 +576,13 @@ __global__ void __launch_bounds__(kGroupThreads) bwd_seg_reverse(BwdArgs a, int6
 }
 
 }  // namespace
+
+#ifdef WKV_TRACE
+extern "C" void wkv_bwd_trace_set_buffer(void* buf) {
+    unsigned long long* p = static_cast<unsigned long long*>(buf);
+    cudaMemcpyToSymbol(g_bwd_trace, &p, sizeof(p));
+}
+#endif
 
 int64_t backward_segments(int64_t T) { return (T + kSeg - 1) / kSeg; }
 
