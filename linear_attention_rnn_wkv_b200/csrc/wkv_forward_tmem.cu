@@ -144,13 +144,9 @@ __device__ __forceinline__ void gate_pair(float (&y)[2], const float (&r)[2]) {
 constexpr int kNWS = 8;   // chunks per tile (summarising warps, emitting warps)
 constexpr int kNL = 3;    // look-back warps
 constexpr int kCg = 64;   // channels per tile (a lane owns a pair)
-// What the summarising warps park in tensor memory beside the values: each key's exponent
-// as seen from the chunk's last row, x_i = k_i log2 e - (L - 1 - i) w log2 e, exactly as the
-// summary used it (1), or the raw keys, from which the emitters recompute it (0).
-#ifndef WKV_TMEM_PARK_EXPONENT
-#define WKV_TMEM_PARK_EXPONENT 1
-#endif
-constexpr bool kParkExponent = WKV_TMEM_PARK_EXPONENT != 0;
+// Beside the values, the summarising warps park in tensor memory each key's exponent as
+// seen from the chunk's last row, x_i = k_i log2 e - (L - 1 - i) w log2 e, exactly as the
+// summary used it, so the emitters need not recompute it.
 constexpr int kThreads = (1 + kNL + 2 * kNWS) * 32;
 
 // What every role needs to know about a unit, worked out once by the producer (per
@@ -205,9 +201,9 @@ struct TmLayout {
     static constexpr size_t total = GATE ? rbar_off + kNWS * 8 : ybuf_off + kNWS * ybuf_bytes;
     // tensor memory: words per row per lane, columns per chunk array, per chunk, per unit and quadrant
     static constexpr int W = Pk<TIO>::W;
-    // words per row of the first array: the key's exponent as an fp32 pair, or the raw keys
-    static constexpr int WK = kParkExponent ? 2 : W;
-    static constexpr int CPAK = LC * WK;  // columns of a chunk's first array (exponents or keys)
+    // words per row of the first array: the key's exponent as an fp32 pair
+    static constexpr int WK = 2;
+    static constexpr int CPAK = LC * WK;  // columns of a chunk's first array (exponents)
     static constexpr int CPAV = LC * W;   // columns of a chunk's values
     static constexpr int CPC = CPAK + CPAV;
     static constexpr int CPU = (kNWS / 4) * CPC;
@@ -572,13 +568,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 M0 = fmaxf(M0, gx[r].x);
                                 M1 = fmaxf(M1, gx[r].y);
                             }
-                            if (kParkExponent) {
-                                kw[rr * 2] = __float_as_uint(gx[r].x);
-                                kw[rr * 2 + 1] = __float_as_uint(gx[r].y);
-                            } else {
-#pragma unroll
-                                for (int x = 0; x < W; ++x) kw[rr * W + x] = raw[x];
-                            }
+                            kw[rr * 2] = __float_as_uint(gx[r].x);
+                            kw[rr * 2 + 1] = __float_as_uint(gx[r].y);
                         }
                         TmemIO<SWK>::st(tq + tcol(t, sw, 0) + h * SWK, kw);
                         TmemIO<SWK>::wait_st(kw);
@@ -643,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // this chunk's r rows now (one TMA box), so they are waiting when the rows are
                 // emitted.  The buffer is free: the previous unit's rows were read before.
                 for (uint32_t it = 0; it <= lim; ++it) {
-                    if (WKV_WAIT_HINT ? mbar_try_wait_hint(chunks_bar(t), ph, WKV_WAIT_HINT) : mbar_try_wait(chunks_bar(t), ph)) {
+                    if (mbar_try_wait_hint(chunks_bar(t), ph, kWaitHintNs)) {
                         got = true;
                         break;
                     }
@@ -651,7 +642,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         gone = true;
                         break;
                     }
-                    if (!WKV_WAIT_HINT) __nanosleep(32);
                 }
                 if (gone) break;
                 const UnitInfo q0 = slot_ub(t)->info;
@@ -668,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 got = false;
             }
             for (uint32_t it = 0; it <= lim; ++it) {
-                if (WKV_WAIT_HINT ? mbar_try_wait_hint(carry_bar(t), ph, WKV_WAIT_HINT) : mbar_try_wait(carry_bar(t), ph)) {
+                if (mbar_try_wait_hint(carry_bar(t), ph, kWaitHintNs)) {
                     got = true;
                     break;
                 }
@@ -677,7 +667,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     gone = true;
                     break;
                 }
-                if (!WKV_WAIT_HINT) __nanosleep(32);
             }
             if (gone) break;
             if (!got && lane == 0) report(kDevTimeoutCarry);
@@ -737,17 +726,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // parameters outside that step's range take the page's two-exp step.
                 int mode = lazy_ok ? 1 : 2;
                 float2 fSa = make_float2(0.f, 0.f), fSb = fSa, fnG = fSa, fic = fSa;
-                if (WKV_PIPE_FRAME && lazy_ok) {
-                    float h0v[2];  // the first token's exponent at the chunk's last row
-                    if (kParkExponent) {
-                        h0v[0] = __uint_as_float(kw[0]);
-                        h0v[1] = __uint_as_float(kw[1]);
-                    } else {
-                        const float2 k0 = Pk<TIO>::unpack(&kw[0]);
-                        const float fc1 = 1.f - (float)r_cnt;
-                        h0v[0] = fmaf(fc1, w2[0], k0.x * kLog2e);
-                        h0v[1] = fmaf(fc1, w2[1], k0.y * kLog2e);
-                    }
+                if (lazy_ok) {
+                    // the first token's exponent at the chunk's last row
+                    const float h0v[2] = {__uint_as_float(kw[0]), __uint_as_float(kw[1])};
                     float fa[V], fb[V], fg[V], fi[V];
                     bool ok = true;
                     const float fc = (float)r_cnt;
@@ -774,12 +755,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         fic = make_float2(fi[0], fi[1]);
                     }
                 }
-                const float back0 = 1.f - (float)r_cnt;  // -(steps from row 0 to the last row)
                 if (__all_sync(0xffffffffu, mode == 0 || !lane_active)) {
                     // every lane in the fixed frame: one branch-free loop, the next slice's rows
                     // read from tensor memory while this slice is computed
-                    const float2 L2 = make_float2(kLog2e, kLog2e);
-                    const float2 w2p = make_float2(w2[0], w2[1]);
                     // the previous chunk's copy must have read the buffer before it is overwritten
                     if (lane == 0) bulk_wait_read();
                     __syncwarp();
@@ -798,17 +776,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int rr = 0; rr < SR; ++rr) {
                                 const int r = h * SR + rr;
                                 const float2 vp = Pk<TIO>::unpack(&vw[rr * W]);
-                                float2 x;
-                                if (kParkExponent) {
-                                    // the summary's own exponent, moved into the frame
-                                    x = __fadd2_rn(make_float2(__uint_as_float(kw[rr * 2]), __uint_as_float(kw[rr * 2 + 1])),
-                                                   fnG);
-                                } else {
-                                    // k - G first: the large cancellation happens inside one rounding
-                                    const float2 kp = Pk<TIO>::unpack(&kw[rr * W]);
-                                    const float back = FULL ? (float)(r + 1 - LC) : back0 + (float)r;
-                                    x = __ffma2_rn(make_float2(back, back), w2p, __ffma2_rn(kp, L2, fnG));
-                                }
+                                // the summary's own exponent, moved into the frame
+                                const float2 x = __fadd2_rn(
+                                    make_float2(__uint_as_float(kw[rr * 2]), __uint_as_float(kw[rr * 2 + 1])), fnG);
                                 const float2 e = make_float2(ex2(x.x), ex2(x.y));
                                 const float2 ec = __fmul2_rn(e, fic);
                                 const float2 num = __ffma2_rn(ec, vp, fSa);
@@ -877,9 +847,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int row = r_begin + r;
                         const float2 vp = Pk<TIO>::unpack(&vw[rr * W]);
                         float2 kp;
-                        if (!kParkExponent) {
-                            kp = Pk<TIO>::unpack(&kw[rr * W]);
-                        } else if (mode != 0) {
+                        if (mode != 0) {
                             // the steps below need the keys themselves, which tensor memory does
                             // not hold: this rare lane reads them again
                             float kv2[V];
@@ -888,14 +856,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         float yy[V];
                         if (mode == 0) {
-                            float2 x;
-                            if (kParkExponent) {
-                                x = __fadd2_rn(make_float2(__uint_as_float(kw[rr * 2]), __uint_as_float(kw[rr * 2 + 1])), fnG);
-                            } else {
-                                // k - G first: the large cancellation happens inside one rounding
-                                const float back = back0 + (float)r;
-                                x = __ffma2_rn(make_float2(back, back), w2p, __ffma2_rn(kp, L2, fnG));
-                            }
+                            const float2 x =
+                                __fadd2_rn(make_float2(__uint_as_float(kw[rr * 2]), __uint_as_float(kw[rr * 2 + 1])), fnG);
                             const float2 e = make_float2(ex2(x.x), ex2(x.y));
                             const float2 ec = __fmul2_rn(e, fic);
                             const float2 num = __ffma2_rn(ec, vp, fSa);

@@ -59,33 +59,26 @@ __device__ __forceinline__ void wkv_trace_warp(int64_t units, int warp) {
 // events: 0 ticket, 1 tile loaded, 2 chunks summarised, 3 look-back start, 4 summaries
 // scanned, 5 carry known, 6 carry handed over, 7 records published, 8 emit start, 9 emit end
 
-// Rows per TMA box (a tile of Ts rows is fetched as Ts / kBoxRows boxes per array).
-#ifndef WKV_PIPE_BOXR
-#define WKV_PIPE_BOXR 32
-#endif
-
 namespace wkvb {
 namespace {
 
-constexpr int kBoxRows = WKV_PIPE_BOXR;
+// Rows per TMA box (a tile of Ts rows is fetched as Ts / kBoxRows boxes per array).
+constexpr int kBoxRows = 32;
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Suspend-time hint of the mbarrier waits, in nanoseconds (0: poll with a short sleep).
-#ifndef WKV_WAIT_HINT
-#define WKV_WAIT_HINT 250
-#endif
+// Suspend-time hint of the mbarrier waits, in nanoseconds.
+constexpr uint32_t kWaitHintNs = 250;
 
 // Bounded wait on an mbarrier phase; returns false if it ran out.  With a hint, a waiting
 // warp is parked by the hardware instead of spinning, so it takes no issue slots from the
 // warps that do the work.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
     for (uint32_t it = 0;; ++it) {
-        if (WKV_WAIT_HINT ? mbar_try_wait_hint(bar, parity, WKV_WAIT_HINT) : mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_hint(bar, parity, kWaitHintNs)) return true;
         if (it >= limit) return false;
-        if (!WKV_WAIT_HINT) __nanosleep(32);
     }
 }
 
@@ -168,22 +161,8 @@ __device__ __forceinline__ int pair_kind(const RawPair& r, uint32_t tag_agg, uin
     return t0 == tag_incl ? 2 : 1;
 }
 
-// Emitters re-scan a chunk in the fixed frame of its largest exponent (1), or carry a
-// moving reference token by token (0; always used where the frame's range check fails).
-#ifndef WKV_PIPE_FRAME
-#define WKV_PIPE_FRAME 1
-#endif
-
-// Summaries and the emitters' per-token step on f32x2 pairs (1) or per channel (0).
-#ifndef WKV_PIPE_PACKED
-#define WKV_PIPE_PACKED 1
-#endif
-
 // Predecessor slots read per look-back round trip.
-#ifndef WKV_PIPE_LOOKAHEAD
-#define WKV_PIPE_LOOKAHEAD 1
-#endif
-constexpr int kLook = WKV_PIPE_LOOKAHEAD;
+constexpr int kLook = 1;
 
 constexpr size_t align128(size_t x) { return (x + 127) / 128 * 128; }
 
