@@ -133,27 +133,31 @@ wkv_status wkv_forward_gated(int64_t B, int64_t T, int64_t C, wkv_dtype io, cons
  *   w, u          [C] fp32
  *   k, v, gy      [B, T, C] fp32
  *   gk, gv        [B, T, C] fp32 (written; must not overlap the inputs)
- *   gw, gu        [C] fp32 (written: zeroed, then accumulated on the device)
+ *   gw, gu        [C] fp32 (written: zeroed, then each block's partial sums added with atomics)
  *   workspace     caller-owned device scratch of ws_bytes >= wkv_backward_workspace_size()
- *                 (per channel and segment a starting state; per channel and group of four
- *                 segments the published forward record and adjoint sums), zero-filled once
- *                 before its first use
- *                 (wkv_workspace_init); one workspace must not serve two backward calls that
- *                 can run at the same time
- * Time-parallel over segments of 32 steps, four to a block, two launches: the groups in time
- * order, each taking its starting state from the records of the groups before it by a bounded
- * look-back; then the groups in reverse time order, each recomputing its outputs, taking the
- * adjoint sums of the groups after it by a bounded look-back and writing its gradients.  k, v are read twice, gy once; nothing per position is kept in global memory.
+ *                 (per channel and group of 128 steps the published forward record and adjoint
+ *                 sums), zero-filled once before its first use (wkv_workspace_init); one
+ *                 workspace must not serve two backward calls that can run at the same time
+ * Time-parallel over segments of 16 steps, eight to a block, in one launch whose blocks take
+ * their work in ticket order: first the groups in time order, each publishing its forward
+ * record and, by a bounded look-back over the records of the groups before it, the state at
+ * its end; then the groups in reverse time order, each recomputing its outputs from the state
+ * entering it (the same look-back), taking the adjoint sums of the groups after it by a bounded
+ * look-back and writing its gradients.  Inside a segment the forward and adjoint sums run in a
+ * fixed exponent frame where the segment's exponents fit one (the per-step stabilised
+ * recurrence elsewhere).  k, v are read twice, gy once; nothing per position is kept in global
+ * memory.
  * A look-back that gives up is recorded in the device-wide word that wkv_get_device_status
  * reports (the gradients are then invalid).
- * Status codes as wkv_forward; B and ceil(T / 32) must be <= 65535.
+ * Status codes as wkv_forward; WKV_ERR_UNSUPPORTED when (2 ceil(T / 128) - 1) B ceil(C / 32)
+ * exceeds 2^31 - 1 (one launch's blocks).
  */
 wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
                         const float* v, const float* gy, float* gk, float* gv, float* gw, float* gu,
                         void* workspace, size_t ws_bytes, cudaStream_t stream);
 
-/* Workspace bytes wkv_backward needs: 64, plus 16 per batch row, channel and 32 steps, plus 72
- * per batch row, channel and 128 steps (rounded up). */
+/* Workspace bytes wkv_backward needs: 64, plus 72 per batch row, channel and 128 steps (rounded
+ * up). */
 size_t wkv_backward_workspace_size(int64_t B, int64_t T, int64_t C);
 
 /* Workspace bytes wkv_forward needs for this shape (the largest over all paths). */

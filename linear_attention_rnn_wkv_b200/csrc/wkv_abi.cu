@@ -228,9 +228,8 @@ wkv_status token_shift_mix3(int64_t B, int64_t T, int64_t C, const float* mu_r, 
 size_t wkv_backward_workspace_size(int64_t B, int64_t T, int64_t C) {
     int64_t n = 0;
     if (!sizes_ok(B, T, C, &n) || n > INT64_MAX / 64) return 0;
-    // a 64-byte header; per (b, segment, c) a starting state (4 floats); per (b, group of four
-    // segments, c) the published forward record (4 tagged 64-bit words) and adjoint sums with
-    // their reference (5 words)
+    // a 64-byte header; per (b, group of 128 steps, c) the published forward record (4 tagged
+    // 64-bit words) and adjoint sums with their reference (5 words)
     return backward_workspace_bytes(B, T, C);
 }
 
@@ -243,8 +242,8 @@ wkv_status wkv_backward(int64_t B, int64_t T, int64_t C, const float* w, const f
     if (!w || !u || !gw || !gu) return WKV_ERR_INVALID_ARG;
     if (n > 0 && (!k || !v || !gy || !gk || !gv)) return WKV_ERR_INVALID_ARG;
     if (!f32_args_ok({w, u, k, v, gy, gk, gv, gw, gu, workspace})) return WKV_ERR_MISALIGNED;
+    if (!backward_fits(B, T, C)) return WKV_ERR_UNSUPPORTED;
     if (n > 0 && (!workspace || ws_bytes < wkv_backward_workspace_size(B, T, C))) return WKV_ERR_INVALID_ARG;
-    if (B > 65535 || backward_segments(T) > 65535) return WKV_ERR_UNSUPPORTED;
     cudaError_t e = launch_backward(B, T, C, w, u, k, v, gy, gk, gv, gw, gu, workspace, stream);
     return e == cudaSuccess ? WKV_OK : cuda_fail(e);
 }

@@ -762,8 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (lane == 0) bulk_wait_read();
                     __syncwarp();
                     TIO* yrow = ybuf + cl;
-                    auto emit = [&](auto full_c) {
-                        constexpr bool FULL = decltype(full_c)::value;
+                    {
 #pragma unroll
                         for (int h = 0; h < LC / SR; ++h) {
                             uint32_t kn[SWK], vn[SW];
@@ -812,11 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 for (int x = 0; x < SW; ++x) vw[x] = vn[x];
                             }
                         }
-                    };
-                    if (r_cnt == LC)
-                        emit(std::true_type{});
-                    else
-                        emit(std::false_type{});
+                    }
                     fence_proxy_async_smem();  // the rows written by the lanes, read by the TMA engine
                     __syncwarp();
                     if (lane == 0) {

@@ -87,9 +87,10 @@ cudaError_t launch_token_shift3(int64_t B, int64_t T, int64_t C, const float* mu
 // y <- sigma(r) * y over n elements of dtype io (0 fp32, 1 bf16), in place
 cudaError_t launch_gate(int64_t n, int io, const void* r, void* y, cudaStream_t s);
 
-// WKV backward (fp32): gk, gv [B,T,C]; gw, gu [C] (zeroed here, then accumulated); ws (zero-
-// filled before its first use) holds backward_workspace_bytes(B, T, C), P = backward_segments(T)
+// WKV backward (fp32): gk, gv [B,T,C]; gw, gu [C] (zeroed, then accumulated); ws (zero-filled) holds
+// backward_workspace_bytes(B, T, C); backward_fits says whether one launch's grid holds the shape
 int64_t backward_segments(int64_t T);
+bool backward_fits(int64_t B, int64_t T, int64_t C);
 size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t C);
 cudaError_t launch_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
                             const float* v, const float* gy, float* gk, float* gv, float* gw, float* gu, void* ws,

@@ -116,12 +116,13 @@ def test_backward_validation_without_launch():
     assert bwd(1, 4, 4, k=None) == 1             # null input
     assert bwd(1, 4, 4, gk=FAKE + 4) == 2        # misaligned output
     assert bwd(1, 4, 4, nbytes=16) == 1          # workspace too small
-    assert bwd(70000, 1, 4) == 3                 # batch above the grid's z limit
-    assert bwd(1, 32 * 65535 + 1, 4) == 3        # more 32-step segments than the grid's y limit
-    # a 64-byte header, 16 B per (b, 32-step segment, c), 72 B per (b, group of 4 segments, c)
-    assert L.wkv_backward_workspace_size(2, 3, 5) == 64 + 2 * 1 * 5 * 16 + 2 * 1 * 5 * 72
-    assert L.wkv_backward_workspace_size(1, 130, 2) == 64 + 1 * 5 * 2 * 16 + 1 * 2 * 2 * 72
-    assert L.wkv_backward_workspace_size(1, 128, 2) == 64 + 1 * 4 * 2 * 16 + 1 * 1 * 2 * 72
+    assert bwd(1 << 16, 1 << 20, 96) == 3        # more blocks than one launch's grid
+    assert bwd(1 << 16, 1 << 20, 96, nbytes=16) == 3
+    # a 64-byte header and 72 B per (b, group of 128 steps, c): the two published records
+    assert L.wkv_backward_workspace_size(2, 3, 5) == 64 + 2 * 1 * 5 * 72
+    assert L.wkv_backward_workspace_size(1, 130, 2) == 64 + 1 * 2 * 2 * 72
+    assert L.wkv_backward_workspace_size(1, 128, 2) == 64 + 1 * 1 * 2 * 72
+    assert L.wkv_backward_workspace_size(1, 129, 160) == 64 + 1 * 2 * 160 * 72
 
 
 def test_gated_and_shift3_validation_without_launch():

@@ -16,7 +16,8 @@ from parity_util import to_gpu
 pytestmark = pytest.mark.gpu
 
 TOL_GRAD = 2e-4
-# T = 3000 and 2049: 94 and 65 segments of 32 steps, several per group of the two-level scans
+# T = 3000 and 2049: 24 and 17 groups of 128 steps (eight 16-step segments each), so the
+# look-backs take several hops and the last group is ragged; C = 129: a channel block of one lane
 SHAPES = [(1, 1, 4), (2, 5, 3), (1, 64, 64), (3, 200, 96), (1, 1000, 32), (2, 130, 129), (1, 3000, 8),
           (2, 2049, 4)]
 
@@ -54,6 +55,34 @@ def test_backward_matches_oracle(shape, base):
 def test_backward_key_shift():
     """Keys shifted by +100 (exponents near 144 in base 2): the gradients do not change."""
     _check(*_case(2, 300, 64, "fwd_8x1024x768", seed=9601, k_shift=100.0))
+
+
+def test_backward_mixed_frames():
+    """Channels whose 16-step segments cannot share one exponent frame (w = 20, 9 and 12: 15 w
+    log2 e is far beyond the frame's range; u = -40, +30 and -25: the bonus outside it) beside
+    channels that can, in the same warps: the per-step lanes and the frame lanes agree with the
+    oracle."""
+    spec = synth.forward_spec_like("fwd_8x1024x768", 2, 500, 40, seed=9602)
+    w, u, k, v = synth.forward_inputs(spec)
+    w[[0, 3, 33]] = np.float32([20.0, 9.0, 12.0])
+    u[[5, 6, 38]] = np.float32([-40.0, 30.0, -25.0])
+    _check(w, u, k, v, synth.grad_output(spec))
+
+
+def test_backward_workspace_reuse():
+    """Three calls on one workspace (its counters and tags reset by each launch): each matches
+    the oracle (bits may differ between calls: a look-back folds whichever records have been
+    published by then)."""
+    import torch
+    import linear_attention_rnn_wkv_b200 as wkv
+    w, u, k, v, gy = _case(3, 700, 96, "fwd_8x1024x768", seed=9603)
+    args = [to_gpu(a) for a in (w, u, k, v, gy)]
+    ws = torch.zeros(int(wkv.lib().wkv_backward_workspace_size(3, 700, 96)), dtype=torch.uint8, device="cuda")
+    rk, rv, rw, ru, (sk, sv, sw, su) = oracle.wkv_backward(w, u, k, v, gy)
+    for _ in range(3):
+        got = [t.cpu().numpy() for t in wkv.wkv_backward(*args, workspace=ws)]
+        for g, r, sc in zip(got, (rk, rv, rw, ru), (sk, sv, sw, su)):
+            assert np.max(np.abs(g - r) / np.maximum(sc, 1e-30)) <= TOL_GRAD
 
 
 def _check_sampled(spec, n_channels, seed):
