@@ -185,6 +185,11 @@ struct LocalSums {
 __device__ __forceinline__ void cp_async4(float* dst, const float* src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
+__device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t* p) {
+    uint64_t v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
@@ -203,24 +208,30 @@ static_assert(kBwdHeaderBytes == 64, "header size");
 
 // Per-block event trace (profiling builds only): compiled with -DWKV_TRACE, each block stamps
 // %globaltimer at its phase boundaries into the buffer registered with wkv_bwd_trace_set_buffer
-// ([tickets][8] u64, slot 7 the SM id); normal builds define the hook away.
+// ([tickets][16] u64: phase times, slot 8 the reverse look-back's polls, slot 15 the SM id);
+// normal builds define the hook away.
 #ifdef WKV_TRACE
 static __device__ unsigned long long* g_bwd_trace = nullptr;
 __device__ __forceinline__ void bwd_trace(int64_t unit, int ev) {
     if (!g_bwd_trace || threadIdx.x != 0) return;
     unsigned long long t;
     asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    unsigned long long* p = g_bwd_trace + unit * 8;
+    unsigned long long* p = g_bwd_trace + unit * 16;
     p[ev] = t;
     if (ev == 0) {
         unsigned sm;
         asm volatile("mov.u32 %0, %smid;" : "=r"(sm));
-        p[7] = sm;
+        p[15] = sm;
     }
 }
+__device__ __forceinline__ void bwd_trace_value(int64_t unit, int slot, unsigned long long v) {
+    if (g_bwd_trace) g_bwd_trace[unit * 16 + slot] = v;
+}
 #define BWD_TRACE(unit, ev) bwd_trace(unit, ev)
+#define BWD_TRACE_VALUE(unit, slot, v) bwd_trace_value(unit, slot, v)
 #else
 #define BWD_TRACE(unit, ev) ((void)0)
+#define BWD_TRACE_VALUE(unit, slot, v) ((void)(v))
 #endif
 
 struct BwdArgs {
@@ -254,13 +265,16 @@ __device__ __forceinline__ void slot_publish(uint64_t* p, int64_t C, const float
     for (int i = 0; i < NW; ++i) st_relaxed_u64(p + i * C, ((uint64_t)tag << 32) | __float_as_uint(f[i]));
 }
 
-// 2 inclusive, 1 the group's own record, 0 nothing usable yet
 template <int NW>
-__device__ __forceinline__ int slot_read(const uint64_t* p, int64_t C, uint32_t tag_loc, uint32_t tag_incl,
-                                         float (&f)[NW]) {
-    uint64_t wd[NW];
+__device__ __forceinline__ void slot_load(const uint64_t* p, int64_t C, uint64_t (&wd)[NW]) {
 #pragma unroll
     for (int i = 0; i < NW; ++i) wd[i] = ld_relaxed_u64(p + i * C);
+}
+
+// 2 inclusive, 1 the group's own record, 0 nothing usable yet
+template <int NW>
+__device__ __forceinline__ int slot_decode(const uint64_t (&wd)[NW], uint32_t tag_loc, uint32_t tag_incl,
+                                           float (&f)[NW]) {
     const uint32_t t0 = (uint32_t)(wd[0] >> 32);
     bool same = t0 == tag_loc || t0 == tag_incl;
 #pragma unroll
@@ -269,6 +283,14 @@ __device__ __forceinline__ int slot_read(const uint64_t* p, int64_t C, uint32_t 
 #pragma unroll
     for (int i = 0; i < NW; ++i) f[i] = __uint_as_float((uint32_t)wd[i]);
     return t0 == tag_incl ? 2 : 1;
+}
+
+template <int NW>
+__device__ __forceinline__ int slot_read(const uint64_t* p, int64_t C, uint32_t tag_loc, uint32_t tag_incl,
+                                         float (&f)[NW]) {
+    uint64_t wd[NW];
+    slot_load<NW>(p, C, wd);
+    return slot_decode<NW>(wd, tag_loc, tag_incl, f);
 }
 
 __device__ __forceinline__ void give_up(const BwdArgs& a) {
@@ -442,9 +464,50 @@ __device__ __forceinline__ void adj_steps(const BwdArgs& a, int64_t base, const 
     }
 }
 
+// The sums entering group J from its right: the later groups' published sums composed,
+// nearest first, until one that already holds everything to its right (or the sequence's end).
+// wd holds the nearest later group's words, read before the group's own were composed.
+__device__ __forceinline__ Adj adj_lookback(const BwdArgs& a, int b, int J, int c, float w2, uint32_t tag_loc,
+                                            uint32_t tag_incl, uint64_t (&wd)[5], uint32_t& polls) {
+    Adj acc = adj_empty(), gin = adj_empty();
+    float span = 0.f;
+    int64_t mg = J + 1;
+    bool done = false;
+    uint32_t nap = 32;
+    for (uint32_t it = 0; it <= a.spin_limit && !done; ++it) {
+        float f[5];
+        if (it > 0) slot_load<5>(a.slots + ((int64_t)b * a.NG + mg) * 5 * a.C + c, a.C, wd);
+        const int kind = slot_decode<5>(wd, tag_loc, tag_incl, f);
+        ++polls;
+        if (kind == 0) {
+            __nanosleep(nap);
+            nap = nap < 512 ? nap * 2 : 512;
+            continue;
+        }
+        nap = 32;
+        const Adj rg{f[0], f[1], f[2], f[3], f[4]};
+        if (kind == 2) {
+            gin = adj_compose(acc, rg, span, w2);
+            done = true;
+        } else {
+            acc = adj_normalize(adj_compose(acc, rg, span, w2));
+            span += (float)min64(a.T - mg * kGroupSteps, kGroupSteps);
+            if (++mg >= a.NG) {
+                gin = acc;
+                done = true;
+            }
+        }
+    }
+    if (!done) {  // gave up: go on with what is there (the gradients are then invalid)
+        give_up(a);
+        gin = acc;
+    }
+    return adj_normalize(gin);
+}
+
 // Shared memory of a block: the three staged tiles, then the records (each segment's, then its
-// starting state) overlaid by the adjoint sums (each segment's local sums, then its in-group
-// incoming sums: written only after every thread has read its starting state).
+// starting state) overlaid by the adjoint sums (each segment's local sums, then its incoming
+// sums: written only after every thread has read its starting state).
 constexpr size_t kTileFloats = (size_t)kGroupSteps * kCh;
 static_assert(kTileFloats == (size_t)kSeg * kThreads, "a tile holds one element per thread and step");
 constexpr size_t kRecBytes = sizeof(Rec) * kGroupSegs * kCh, kAdjBytes = sizeof(Adj) * kGroupSegs * kCh;
@@ -458,7 +521,8 @@ __global__ void __launch_bounds__(kThreads, 4)
     float* sm = reinterpret_cast<float*>(sm4);
     Rec(*s_rec)[kCh] = reinterpret_cast<Rec(*)[kCh]>(sm + 3 * kTileFloats);
     Adj(*s_adj)[kCh] = reinterpret_cast<Adj(*)[kCh]>(sm + 3 * kTileFloats);
-    __shared__ Adj s_gin[kCh];  // the sums entering the group from its right
+    __shared__ Adj s_gin[kCh];          // the sums entering the group from its right
+    __shared__ float s_ys[kSeg * kCh];  // warp 0's outputs during the reverse look-back
     __shared__ uint32_t s_ticket, s_epoch;
     __shared__ __align__(8) uint64_t s_bar;  // the TMA copies' completion
     const int tid = threadIdx.x, lane = tid % kCh, seg = tid / kCh;
@@ -477,14 +541,15 @@ __global__ void __launch_bounds__(kThreads, 4)
         s_epoch = ep & 0x3FFFFFFFu;
     }
     __syncthreads();
-    const int64_t ticket = s_ticket;
+    const uint32_t ticket = s_ticket;
     BWD_TRACE(ticket, 0);
     const uint32_t tag_loc = (s_epoch << 2) | 1u, tag_incl = (s_epoch << 2) | 2u;
-    const bool isA = ticket < a.UA;
-    const int64_t per = a.B * a.cx, r = isA ? ticket : ticket - a.UA;
-    const int64_t J = isA ? r / per : a.NG - 1 - r / per;
-    const int64_t b = (r % per) / a.cx, cb = r % a.cx;
-    const int64_t c = cb * kCh + lane;
+    // the work item (all indices below 2^31: the grid's blocks are)
+    const bool isA = ticket < (uint32_t)a.UA;
+    const uint32_t per = (uint32_t)(a.B * a.cx), cx = (uint32_t)a.cx, r = isA ? ticket : ticket - (uint32_t)a.UA;
+    const int J = (int)(isA ? r / per : (uint32_t)a.NG - 1u - r / per);
+    const int b = (int)((r % per) / cx), cb = (int)(r % cx);
+    const int c = cb * kCh + lane;
     const bool chan = c < a.C;
     const int64_t t0 = J * kGroupSteps + (int64_t)seg * kSeg;
     const int len = chan ? seg_len(a, t0) : 0;
@@ -508,27 +573,26 @@ __global__ void __launch_bounds__(kThreads, 4)
         }
     }
     // while the copies fly: R's warp 0 takes the state entering the group (the look-back over
-    // A's records) and waits until gw, gu have been zeroed (by A's first block of this channel
-    // block, which publishes its record after the zeros); A's first blocks zero them
+    // A's records); R's warp 1 waits until gw, gu have been zeroed: A's first block of the
+    // channel block zeroes them, then (after a fence) publishes its record, which warp 1 reads
+    // with acquire semantics; the block barriers then order warp 0's atomics after that read
     Rec gstart = rec_identity();
-    if (seg == 0 && chan) {
-        if (isA) {
-            if (J == 0 && b == 0) {
-                a.gw[c] = 0.f;
-                a.gu[c] = 0.f;
+    if (isA) {
+        if (seg == 0 && chan && J == 0 && b == 0) {  // published (after a fence) by this lane
+            a.gw[c] = 0.f;
+            a.gu[c] = 0.f;
+        }
+    } else {
+        if (seg == 0) {
+            if (chan) gstart = fwd_lookback(a, b, J, c, w2, tag_loc, tag_incl);
+            if (lane == 0) BWD_TRACE(ticket, 9);
+        } else if (seg == 1 && chan && a.NG > 1) {
+            bool zeroed = false;
+            for (uint32_t it = 0; it <= a.spin_limit && !zeroed; ++it) {
+                zeroed = (uint32_t)(ld_acquire_u64(a.fslots + c) >> 32) == tag_incl;  // (b = 0, group 0) word 0
+                if (!zeroed) __nanosleep(64);
             }
-        } else {
-            gstart = fwd_lookback(a, b, J, c, w2, tag_loc, tag_incl);
-            if (a.NG > 1) {
-                const uint64_t* z = a.fslots + c;  // (b = 0, group 0) word 0
-                bool seen = false;
-                for (uint32_t it = 0; it <= a.spin_limit && !seen; ++it) {
-                    seen = (uint32_t)(ld_relaxed_u64(z) >> 32) == tag_incl;
-                    if (!seen) __nanosleep(64);
-                }
-                if (!seen) give_up(a);
-                fence_acquire_gpu();
-            }
+            if (!zeroed) give_up(a);
         }
     }
     if (TMA) {
@@ -536,6 +600,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     } else {
         cp_async_wait_all();
     }
+    BWD_TRACE(ticket, 10);
     float M = 0.f, m = 0.f;
     Rec rec = rec_identity();
     if (len == kSeg)
@@ -543,6 +608,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     else if (len > 0)
         rec = seg_record<false>(sk, sv, len, w2, M, m);
     s_rec[seg][lane] = rec;
+    BWD_TRACE(ticket, 11);
     __syncthreads();
     BWD_TRACE(ticket, 1);
 
@@ -555,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 4)
                 const int ls = seg_len(a, J * kGroupSteps + (int64_t)s * kSeg);
                 if (ls > 0) agg = rec_combine(agg, s_rec[s][lane], (float)ls, w2);
             }
-            uint64_t* my = a.fslots + (b * a.NG + J) * 4 * a.C + c;
+            uint64_t* my = a.fslots + ((int64_t)b * a.NG + J) * 4 * a.C + c;
             if (J == 0) {
                 if (b == 0) __threadfence();  // the zeros of gw, gu before the record
                 slot_publish<4>(my, a.C, {agg.a, agg.b, agg.anc, agg.n}, tag_incl);
@@ -569,7 +635,6 @@ __global__ void __launch_bounds__(kThreads, 4)
         BWD_TRACE(ticket, 2);
         return;
     }
-
     // R: each segment's starting state from the group's
     if (seg == 0 && chan) {
         Rec run = gstart;
@@ -611,6 +676,13 @@ __global__ void __launch_bounds__(kThreads, 4)
     __syncthreads();
     BWD_TRACE(ticket, 3);
     if (seg == 0 && chan) {
+        // (this warp's outputs wait in shared memory meanwhile: fewer registers at the peak)
+#pragma unroll
+        for (int i = 0; i < kSeg; ++i) s_ys[i * kCh + lane] = ys[i];
+        // the nearest later group's record is read first; it travels while the group composes
+        const bool later = J + 1 < a.NG;
+        uint64_t wd[5];
+        if (later) slot_load<5>(a.slots + ((int64_t)b * a.NG + J + 1) * 5 * a.C + c, a.C, wd);
         // the group's segments composed right to left; each slot keeps what enters its segment
         // from the group's later segments
         Adj run = adj_empty();
@@ -621,51 +693,25 @@ __global__ void __launch_bounds__(kThreads, 4)
             const int l = seg_len(a, J * kGroupSteps + (int64_t)s * kSeg);
             if (l > 0) run = adj_normalize(adj_compose(ls, run, (float)l, w2));
         }
-        uint64_t* my = a.slots + (b * a.NG + J) * 5 * a.C + c;
-        // the sums entering the group: the later groups' composed, nearest first, until one
-        // that already holds everything to its right (or the sequence's end)
+        uint64_t* my = a.slots + ((int64_t)b * a.NG + J) * 5 * a.C + c;
         Adj gin = adj_empty();
-        if (J + 1 < a.NG) {
+        if (later) {
             if (J > 0) slot_publish<5>(my, a.C, {run.x, run.y, run.xp, run.yp, run.r}, tag_loc);
-            Adj acc = adj_empty();
-            float span = 0.f;
-            int64_t mg = J + 1;
-            bool done = false;
-            uint32_t nap = 32;
-            for (uint32_t it = 0; it <= a.spin_limit && !done; ++it) {
-                float f[5];
-                const int kind = slot_read<5>(a.slots + (b * a.NG + mg) * 5 * a.C + c, a.C, tag_loc, tag_incl, f);
-                if (kind == 0) {
-                    __nanosleep(nap);
-                    nap = nap < 512 ? nap * 2 : 512;
-                    continue;
-                }
-                nap = 32;
-                const Adj rg{f[0], f[1], f[2], f[3], f[4]};
-                if (kind == 2) {
-                    gin = adj_compose(acc, rg, span, w2);
-                    done = true;
-                } else {
-                    acc = adj_normalize(adj_compose(acc, rg, span, w2));
-                    span += (float)min64(a.T - mg * kGroupSteps, kGroupSteps);
-                    if (++mg >= a.NG) {
-                        gin = acc;
-                        done = true;
-                    }
-                }
+            uint32_t polls = 0;
+            gin = adj_lookback(a, b, J, c, w2, tag_loc, tag_incl, wd, polls);
+            if (lane == 0) {
+                BWD_TRACE(ticket, 7);
+                BWD_TRACE_VALUE(ticket, 8, polls);
             }
-            if (!done) {  // gave up: go on with what is there (the gradients are then invalid)
-                give_up(a);
-                gin = acc;
-            }
-            gin = adj_normalize(gin);
         }
         if (J > 0) {
             const Adj out =
-                adj_normalize(adj_compose(run, gin, (float)min64(a.T - J * kGroupSteps, kGroupSteps), w2));
+                adj_normalize(adj_compose(run, gin, (float)min64(a.T - (int64_t)J * kGroupSteps, kGroupSteps), w2));
             slot_publish<5>(my, a.C, {out.x, out.y, out.xp, out.yp, out.r}, tag_incl);
         }
         s_gin[lane] = gin;
+#pragma unroll
+        for (int i = 0; i < kSeg; ++i) ys[i] = s_ys[i * kCh + lane];
     }
     __syncthreads();
     BWD_TRACE(ticket, 4);
@@ -673,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     if (len > 0) {
         // the sums entering this segment: its group's later segments', with the group's own
         // incoming sums carried across them
-        const float after = (float)(min64(a.T, (J + 1) * kGroupSteps) - (t0 + len));
+        const float after = (float)(min64(a.T, (int64_t)(J + 1) * kGroupSteps) - (t0 + len));
         const Adj in = adj_compose(s_adj[seg][lane], s_gin[lane], after, w2);
         if (frame) {
             // into the frame: F e^{-(len-1) w} times the sums at the segment's last position
