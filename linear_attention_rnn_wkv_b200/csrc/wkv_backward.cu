@@ -529,11 +529,13 @@ __global__ void __launch_bounds__(kThreads, 4)
     float* sk = sm + seg * kSeg * kCh + lane;  // this thread's elements of k (then 2^{x - G}),
     float* sv = sk + kTileFloats;              // of v
     float* sg = sk + 2 * kTileFloats;          // of gy (then gy / D^)
+    grid_dep_launch_dependents();
+    if (TMA && tid == 0) {
+        mbar_init(&s_bar, 1);
+        fence_mbar_init();
+    }
+    grid_dep_wait();  // global memory only from here
     if (tid == 0) {
-        if (TMA) {
-            mbar_init(&s_bar, 1);
-            fence_mbar_init();
-        }
         const unsigned long long t = atomicAdd(&a.hdr->tk, 1ull);
         const uint32_t tk = (uint32_t)t, ep = (uint32_t)(t >> 32);
         if (tk == a.units - 1u) atomicExch(&a.hdr->tk, (unsigned long long)((ep + 1u) & 0x3FFFFFFFu) << 32);
@@ -832,10 +834,9 @@ cudaError_t launch_backward(int64_t B, int64_t T, int64_t C, const float* w, con
                      make_tile_map(&tmv, v, B, T, C, 0, kCh, kGroupSteps) &&
                      make_tile_map(&tmg, gy, B, T, C, 0, kCh, kGroupSteps);
     if (tma)
-        bwd_kernel<true><<<(unsigned)units, kThreads, kSmemBytes, s>>>(a, tmk, tmv, tmg);
+        return launch_pdl(bwd_kernel<true>, dim3((unsigned)units), dim3(kThreads), kSmemBytes, s, a, tmk, tmv, tmg);
     else
-        bwd_kernel<false><<<(unsigned)units, kThreads, kSmemBytes, s>>>(a, tmk, tmv, tmg);
-    return cudaGetLastError();
+        return launch_pdl(bwd_kernel<false>, dim3((unsigned)units), dim3(kThreads), kSmemBytes, s, a, tmk, tmv, tmg);
 }
 
 }  // namespace wkvb

@@ -45,6 +45,8 @@ __global__ void __launch_bounds__(256) decode_kernel(int64_t rows, int64_t L, in
                                                      float* __restrict__ xbar, const float* __restrict__ k,
                                                      const float* __restrict__ v, float* __restrict__ st,
                                                      float* __restrict__ y) {
+    grid_dep_launch_dependents();
+    grid_dep_wait();  // before any global memory access
     const int64_t RC = rows * C;
     const int64_t c = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * V;
     if (c >= C) return;
@@ -86,6 +88,8 @@ __global__ void __launch_bounds__(256) token_shift_kernel(int64_t B, int64_t T, 
                                                           const float* __restrict__ x,
                                                           const float* __restrict__ x_last,
                                                           float* __restrict__ xbar) {
+    grid_dep_launch_dependents();
+    grid_dep_wait();  // before any global memory access
     const int64_t c = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * V;
     if (c >= C) return;
     float m[V];
@@ -117,6 +121,8 @@ __global__ void __launch_bounds__(256) token_shift3_kernel(int64_t B, int64_t T,
                                                            const float* __restrict__ x, const float* __restrict__ x_last,
                                                            float* __restrict__ xr, float* __restrict__ xk,
                                                            float* __restrict__ xv) {
+    grid_dep_launch_dependents();
+    grid_dep_wait();  // before any global memory access
     const int64_t c = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * V;
     if (c >= C) return;
     float mr[V], mk[V], mv[V];
@@ -153,6 +159,8 @@ __global__ void __launch_bounds__(256) token_shift3_kernel(int64_t B, int64_t T,
 // sigma(r) = 1 / (1 + 2^(-r log2 e)); for r -> -inf the exponential is +inf and the gate 0.
 template <typename TIO, int V>
 __global__ void __launch_bounds__(256) gate_kernel(int64_t n, const TIO* __restrict__ r, TIO* __restrict__ y) {
+    grid_dep_launch_dependents();
+    grid_dep_wait();  // before any global memory access
     const int64_t stride = (int64_t)gridDim.x * blockDim.x * V;
     for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * V; i < n; i += stride) {
         float rv[V], yv[V];
@@ -165,6 +173,8 @@ __global__ void __launch_bounds__(256) gate_kernel(int64_t n, const TIO* __restr
 }
 
 __global__ void passthrough_kernel(int64_t BC, const float* in, float* out) {
+    grid_dep_launch_dependents();
+    grid_dep_wait();  // before any global memory access
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < 3 * BC; i += (int64_t)gridDim.x * blockDim.x)
         out[i] = in ? in[i] : (i < 2 * BC ? 0.f : kPEmpty);
 }
@@ -185,16 +195,19 @@ cudaError_t launch_decode_step(int64_t N, int64_t L, int64_t C, const float* mu,
     const dim3 grid = grid2d(C, vec ? 4 : 1, rows);
     if (fused) {
         if (vec)
-            decode_kernel<true, 4><<<grid, 256, 0, s>>>(rows, L, C, mu, w, u, x_t, x_prev, xbar, k, v, state, y);
+            return launch_pdl(decode_kernel<true, 4>, dim3(grid), dim3(256), 0, s,
+                              rows, L, C, mu, w, u, x_t, x_prev, xbar, k, v, state, y);
         else
-            decode_kernel<true, 1><<<grid, 256, 0, s>>>(rows, L, C, mu, w, u, x_t, x_prev, xbar, k, v, state, y);
+            return launch_pdl(decode_kernel<true, 1>, dim3(grid), dim3(256), 0, s,
+                              rows, L, C, mu, w, u, x_t, x_prev, xbar, k, v, state, y);
     } else {
         if (vec)
-            decode_kernel<false, 4><<<grid, 256, 0, s>>>(rows, L, C, mu, w, u, x_t, x_prev, xbar, k, v, state, y);
+            return launch_pdl(decode_kernel<false, 4>, dim3(grid), dim3(256), 0, s,
+                              rows, L, C, mu, w, u, x_t, x_prev, xbar, k, v, state, y);
         else
-            decode_kernel<false, 1><<<grid, 256, 0, s>>>(rows, L, C, mu, w, u, x_t, x_prev, xbar, k, v, state, y);
+            return launch_pdl(decode_kernel<false, 1>, dim3(grid), dim3(256), 0, s,
+                              rows, L, C, mu, w, u, x_t, x_prev, xbar, k, v, state, y);
     }
-    return cudaGetLastError();
 }
 
 cudaError_t launch_token_shift(int64_t B, int64_t T, int64_t C, const float* mu, const float* x, const float* x_last,
@@ -202,17 +215,15 @@ cudaError_t launch_token_shift(int64_t B, int64_t T, int64_t C, const float* mu,
     const bool vec = (C % 4) == 0;
     const dim3 grid = grid2d(C, vec ? 4 : 1, B * T);
     if (vec)
-        token_shift_kernel<4><<<grid, 256, 0, s>>>(B, T, C, mu, x, x_last, xbar);
+        return launch_pdl(token_shift_kernel<4>, dim3(grid), dim3(256), 0, s, B, T, C, mu, x, x_last, xbar);
     else
-        token_shift_kernel<1><<<grid, 256, 0, s>>>(B, T, C, mu, x, x_last, xbar);
-    return cudaGetLastError();
+        return launch_pdl(token_shift_kernel<1>, dim3(grid), dim3(256), 0, s, B, T, C, mu, x, x_last, xbar);
 }
 
 cudaError_t launch_state_passthrough(int64_t BC, const float* state_in, float* state_out, cudaStream_t s) {
     const int64_t n = 3 * BC;
     const int64_t blocks = (n + 255) / 256 < 148 * 16 ? (n + 255) / 256 : 148 * 16;
-    passthrough_kernel<<<(unsigned)blocks, 256, 0, s>>>(BC, state_in, state_out);
-    return cudaGetLastError();
+    return launch_pdl(passthrough_kernel, dim3((unsigned)blocks), dim3(256), 0, s, BC, state_in, state_out);
 }
 
 cudaError_t launch_token_shift3(int64_t B, int64_t T, int64_t C, const float* mu_r, const float* mu_k,
@@ -221,10 +232,11 @@ cudaError_t launch_token_shift3(int64_t B, int64_t T, int64_t C, const float* mu
     const bool vec = (C % 4) == 0;
     const dim3 grid = grid2d(C, vec ? 4 : 1, B * T);
     if (vec)
-        token_shift3_kernel<4><<<grid, 256, 0, s>>>(B, T, C, mu_r, mu_k, mu_v, x, x_last, xr, xk, xv);
+        return launch_pdl(token_shift3_kernel<4>, dim3(grid), dim3(256), 0, s,
+                          B, T, C, mu_r, mu_k, mu_v, x, x_last, xr, xk, xv);
     else
-        token_shift3_kernel<1><<<grid, 256, 0, s>>>(B, T, C, mu_r, mu_k, mu_v, x, x_last, xr, xk, xv);
-    return cudaGetLastError();
+        return launch_pdl(token_shift3_kernel<1>, dim3(grid), dim3(256), 0, s,
+                          B, T, C, mu_r, mu_k, mu_v, x, x_last, xr, xk, xv);
 }
 
 cudaError_t launch_gate(int64_t n, int io, const void* r, void* y, cudaStream_t s) {
@@ -239,18 +251,17 @@ cudaError_t launch_gate(int64_t n, int io, const void* r, void* y, cudaStream_t 
         const __nv_bfloat16* rr = static_cast<const __nv_bfloat16*>(r);
         __nv_bfloat16* yy = static_cast<__nv_bfloat16*>(y);
         if (n % 8 == 0)
-            gate_kernel<__nv_bfloat16, 8><<<blocks(n / 8), 256, 0, s>>>(n, rr, yy);
+            return launch_pdl(gate_kernel<__nv_bfloat16, 8>, dim3(blocks(n / 8)), dim3(256), 0, s, n, rr, yy);
         else
-            gate_kernel<__nv_bfloat16, 1><<<blocks(n), 256, 0, s>>>(n, rr, yy);
+            return launch_pdl(gate_kernel<__nv_bfloat16, 1>, dim3(blocks(n)), dim3(256), 0, s, n, rr, yy);
     } else {
         const float* rr = static_cast<const float*>(r);
         float* yy = static_cast<float*>(y);
         if (n % 4 == 0)
-            gate_kernel<float, 4><<<blocks(n / 4), 256, 0, s>>>(n, rr, yy);
+            return launch_pdl(gate_kernel<float, 4>, dim3(blocks(n / 4)), dim3(256), 0, s, n, rr, yy);
         else
-            gate_kernel<float, 1><<<blocks(n), 256, 0, s>>>(n, rr, yy);
+            return launch_pdl(gate_kernel<float, 1>, dim3(blocks(n)), dim3(256), 0, s, n, rr, yy);
     }
-    return cudaGetLastError();
 }
 
 }  // namespace wkvb

@@ -339,6 +339,16 @@ __device__ __forceinline__ void st_relaxed_v2u64(uint64_t* p, uint64_t x, uint64
 // Makes earlier relaxed loads acquire: later accesses see what their writers released.
 __device__ __forceinline__ void fence_acquire_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialisation may
+// be scheduled while the stream's previous kernel is still running; it runs its prologue
+// (shared and tensor memory, barriers) and then waits here, before its first access to global
+// memory, until that kernel has completed and its writes are visible.  Without the attribute
+// the wait returns at once.  launch_dependents lets the next such kernel be scheduled early.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }

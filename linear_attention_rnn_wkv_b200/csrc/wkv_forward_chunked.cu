@@ -69,6 +69,8 @@ struct ChunkParams {
 
 template <typename TIO, int V, int NW, int LC, bool BULK>
 __global__ void __launch_bounds__(NW * 32) chunked_kernel(ForwardArgs args, ChunkParams cp) {
+    grid_dep_launch_dependents();
+    grid_dep_wait();  // before any global memory access
     constexpr int NT = NW * 32;
     constexpr int Cg = 32 * V;
     constexpr int Ts = NW * LC;
@@ -450,8 +452,7 @@ cudaError_t launch_t(const ForwardArgs& a, const ChunkGeom& g, const ChunkParams
         if (e != cudaSuccess) return e;
         if (dev < 64) attr_done |= 1ull << dev;
     }
-    kern<<<(unsigned)g.U, NW * 32, smem, s>>>(a, cp);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3((unsigned)g.U), dim3(NW * 32), smem, s, a, cp);
 }
 
 template <typename TIO, int V, int NW, bool BULK>

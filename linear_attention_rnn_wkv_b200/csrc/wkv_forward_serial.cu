@@ -50,6 +50,8 @@ struct SerialChannel {
 // Bulk-copy path.  Shared memory: NS stages of [TS][NT] k then [TS][NT] v, then NS mbarriers.
 template <typename TIO, int NT, int TS, int NS>
 __global__ void __launch_bounds__(NT) serial_bulk_kernel(ForwardArgs args) {
+    grid_dep_launch_dependents();
+    grid_dep_wait();  // before any global memory access
     extern __shared__ __align__(128) unsigned char smem[];
     constexpr int kStageElems = TS * NT;
     TIO* stage_base = reinterpret_cast<TIO*>(smem);
@@ -154,6 +156,8 @@ __global__ void __launch_bounds__(NT) serial_bulk_kernel(ForwardArgs args) {
 // Per-element path for C not a multiple of 16 bytes: coalesced scalar loads.
 template <typename TIO, int NT>
 __global__ void __launch_bounds__(NT) serial_plain_kernel(ForwardArgs args) {
+    grid_dep_launch_dependents();
+    grid_dep_wait();  // before any global memory access
     const int64_t B = args.B, T = args.T, C = args.C;
     const int64_t groups_per_b = (C + NT - 1) / NT;
     const int64_t b = blockIdx.x / groups_per_b;
@@ -194,11 +198,10 @@ cudaError_t launch_serial_t(const ForwardArgs& a, cudaStream_t s) {
             if (e != cudaSuccess) return e;
             if (dev < 64) attr_done |= 1ull << dev;
         }
-        kern<<<(unsigned)grid, NT, smem, s>>>(a);
+        return launch_pdl(kern, dim3((unsigned)grid), dim3(NT), smem, s, a);
     } else {
-        serial_plain_kernel<TIO, NT><<<(unsigned)grid, NT, 0, s>>>(a);
+        return launch_pdl(serial_plain_kernel<TIO, NT>, dim3((unsigned)grid), dim3(NT), 0, s, a);
     }
-    return cudaGetLastError();
 }
 
 }  // namespace

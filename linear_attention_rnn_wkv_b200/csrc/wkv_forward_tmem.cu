@@ -256,17 +256,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t T = args.T, C = args.C, BC = args.B * args.C;
     const uint32_t lim = args.spin_limit;
 
-    if (tid == 0) WKV_TRACE_BLOCK(pp.U, 0);
+    grid_dep_launch_dependents();
     if (warp == 0) {
         tmem_alloc(s_tmem, 512);
         tmem_relinquish();
     }
-    // the producer's first ticket and the launch's epoch: both round trips start before the
-    // barrier set-up and overlap each other (the producer is thread 0)
     uint32_t first_ticket = 0;
     if (tid == 0) {
-        first_ticket = atomicAdd(&pp.hdr->ticket, 1u);
-        *s_epoch = (*reinterpret_cast<volatile uint32_t*>(&pp.hdr->epoch) + 1u) & 0x3FFFFFFFu;
         *s_iend = INT64_MAX;
         for (int s = 0; s < NS; ++s) {
             for (int b = 0; b < NB; ++b) mbar_init(dfull(s, b), 1);
@@ -281,6 +277,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(uempty(t), kNWS);
         }
         fence_mbar_init();
+    }
+    // global memory only from here: the stream's previous kernel may still be running
+    grid_dep_wait();
+    if (tid == 0) {
+        WKV_TRACE_BLOCK(pp.U, 0);
+        // the producer's first ticket and the launch's epoch (two round trips in flight at once)
+        first_ticket = atomicAdd(&pp.hdr->ticket, 1u);
+        *s_epoch = (*reinterpret_cast<volatile uint32_t*>(&pp.hdr->epoch) + 1u) & 0x3FFFFFFFu;
     }
     tc_fence_before();
     __syncthreads();
@@ -983,8 +987,17 @@ cudaError_t launch_tmem_g(const ForwardArgs& a, const ChunkGeom& g, const PipePa
     }
     const int64_t nsm = dev < 64 ? sms[dev] : 148;
     const int64_t grid = g.U < nsm ? g.U : nsm;
-    kern<<<(unsigned)grid, kThreads, Lay::total, s>>>(a, pp, tmk, tmv, tmr, tmy);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = Lay::total;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = kProgrammaticLaunch ? 1 : 0;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a, pp, tmk, tmv, tmr, tmy);
 }
 
 template <typename TIO, int LC>

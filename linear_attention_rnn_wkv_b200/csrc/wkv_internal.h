@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace wkvb {
 
 // Device error codes written to the error word (first word of a status block).
@@ -12,6 +14,27 @@ enum : uint32_t { kDevOk = 0, kDevTimeoutCarry = 1, kDevTimeoutCopy = 2, kDevBad
 
 // Bounded-wait limits (iterations of a poll loop that sleeps ~64 ns per miss).
 constexpr uint32_t kSpinLimitDefault = 1u << 18;  // a few hundred ms of polling
+// Kernels that wait for their stream predecessor in-kernel (grid_dep_wait) are launched with
+// programmatic stream serialisation, so their launch and prologue overlap its tail.
+constexpr bool kProgrammaticLaunch = true;
+
+// Launches kern with programmatic stream serialisation; every kernel launched this way calls
+// grid_dep_wait before its first access to global memory.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = kProgrammaticLaunch ? 1 : 0;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 struct ForwardArgs {
     int64_t B, T, C;
