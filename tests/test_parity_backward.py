@@ -103,12 +103,12 @@ def _check_sampled(spec, n_channels, seed):
 
 
 def test_backward_full_width_sampled():
-    """fwd_8x1024x768's shape (B=8, T=1024, C=768) through the GPU, 48 sampled channels against
+    """fwd_8x1024x768's shape (B=8, T=1024, C=768) through the GPU, 96 sampled channels against
     the oracle (channels are independent; gw and gu of a channel sum over the whole batch)."""
-    _check_sampled(synth.FORWARD["fwd_8x1024x768"], 48, 11)
+    _check_sampled(synth.FORWARD["fwd_8x1024x768"], 96, 11)
 
 
 def test_backward_long_context_sampled():
-    """The long-context shape (B=1, T=16384, C=4096) through the GPU, 6 sampled channels against
+    """The long-context shape (B=1, T=16384, C=4096) through the GPU, 12 sampled channels against
     the oracle's O(T^2) gradient (the last channel included)."""
-    _check_sampled(synth.FORWARD["fwd_1x16384x4096"], 6, 12)
+    _check_sampled(synth.FORWARD["fwd_1x16384x4096"], 12, 12)
