@@ -326,10 +326,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive(dunit(s));
                     break;
                 }
-                const int64_t unit = tk;
-                const int64_t j = unit / pp.G, g = unit % pp.G;
-                const int64_t b = g / pp.groups_per_b;
-                const int64_t c0 = (g % pp.groups_per_b) * Cg, t0 = j * Ts;
+                // the unit's geometry: 32-bit divisions (tickets, G and groups per row are all
+                // below 2^31: the host checks U)
+                const uint32_t G32 = (uint32_t)pp.G, gpb32 = (uint32_t)pp.groups_per_b;
+                const uint32_t j32 = tk / G32, g32 = tk - j32 * G32;
+                const uint32_t b32 = g32 / gpb32, cg32 = g32 - b32 * gpb32;
+                const int64_t unit = tk, j = j32, g = g32, b = b32;
+                const int64_t c0 = (int64_t)cg32 * Cg, t0 = j * Ts;
                 const int nch = (int)min64(Cg, C - c0);
                 WKV_TRACE_EVENT(unit, 0);
 #pragma unroll
