@@ -15,19 +15,19 @@ constexpr long long kTuneT[kTuneNumT] = {1, 4, 16, 64, 256, 1024, 4096, 16384};
 // [dtype: 0 fp32, 1 bf16][B*C][T]
 constexpr signed char kTunePath[2][kTuneNumBC][kTuneNumT] = {
     {
-        {1, 1, 1, 1, 16, 16, 16, 16},  // B*C = 64
-        {1, 1, 1, 1, 16, 16, 16, 16},  // B*C = 512
-        {1, 1, 1, 1, 16, 16, 16, 16},  // B*C = 4096
-        {1, 1, 1, 16, 16, 16, 16, 0},  // B*C = 32768
-        {1, 1, 1, 8, 16, 16, 0, 0},  // B*C = 262144
+        {1, 1, 1, 8, 8, 16, 16, 16},  // B*C = 64
+        {1, 1, 1, 8, 8, 8, 16, 16},  // B*C = 512
+        {1, 1, 1, 16, 16, 16, 16, 16},  // B*C = 4096
+        {1, 1, 1, 8, 16, 16, 16, 0},  // B*C = 32768
+        {1, 1, 8, 8, 16, 16, 0, 0},  // B*C = 262144
         {1, 1, 8, 8, 16, 0, 0, 0},  // B*C = 1048576
     },
     {
-        {1, 1, 1, 1, 16, 16, 16, 16},  // B*C = 64
-        {1, 1, 1, 1, 16, 16, 16, 16},  // B*C = 512
-        {1, 1, 1, 1, 16, 16, 16, 16},  // B*C = 4096
-        {1, 1, 1, 1, 16, 16, 16, 0},  // B*C = 32768
-        {1, 1, 1, 1, 16, 16, 0, 0},  // B*C = 262144
+        {1, 1, 1, 8, 16, 16, 16, 16},  // B*C = 64
+        {1, 1, 1, 8, 16, 16, 16, 16},  // B*C = 512
+        {1, 1, 1, 8, 16, 16, 16, 16},  // B*C = 4096
+        {1, 1, 1, 8, 16, 16, 16, 0},  // B*C = 32768
+        {1, 1, 1, 8, 16, 16, 0, 0},  // B*C = 262144
         {1, 1, 1, 8, 16, 0, 0, 0},  // B*C = 1048576
     },
 };
