@@ -148,6 +148,10 @@ constexpr int kCg = 64;   // channels per tile (a lane owns a pair)
 // seen from the chunk's last row, x_i = k_i log2 e - (L - 1 - i) w log2 e, exactly as the
 // summary used it, so the emitters need not recompute it.
 constexpr int kThreads = (1 + kNL + 2 * kNWS) * 32;
+// The producer hands each unit's ticket to the look-back warps through a ring of this many
+// entries as soon as it has it, so a unit's look-back over its predecessors runs while its rows
+// are still loading and being summarised.
+constexpr int kRing = 16;
 
 // What every role needs to know about a unit, worked out once by the producer (per
 // shared-memory stage) and copied with the unit into its tensor-memory slot: the tile's
@@ -189,7 +193,9 @@ struct TmLayout {
     // per stage: NB full + 1 empty + 1 unit block; per slot: chunks, carry, empty
     static constexpr int NBARS = NS * (NB + 2) + NT * 3;
     static constexpr size_t misc_off = bars_off + NBARS * 8;  // end index, epoch, tensor memory base
-    static constexpr size_t stage_ub_off = align128(misc_off + 16);  // the stages' unit blocks [NS]
+    // the ticket ring: kRing tickets, then a full and an empty barrier per entry
+    static constexpr size_t ring_off = align128(misc_off + 16);
+    static constexpr size_t stage_ub_off = align128(ring_off + kRing * (4 + 16));  // the stages' unit blocks [NS]
     // gated forward: each emitting warp's chunk of r (TMA box of LC rows x Cg) and its barrier
     static constexpr size_t rbuf_bytes = align128(sizeof(TIO) * LC * Cg);
     static constexpr size_t rbuf_off = align128(stage_ub_off + NS * sizeof(UnitBlock));
@@ -249,6 +255,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto chunk_max = [&](int t) { return reinterpret_cast<float*>(slotp(t) + Lay::mx_off); };
     auto slot_ub = [&](int t) { return reinterpret_cast<UnitBlock*>(slotp(t) + Lay::ub_off); };
     auto stage_ub = [&](int s) { return reinterpret_cast<UnitBlock*>(smem + Lay::stage_ub_off) + s; };
+    volatile uint32_t* ring_tk = reinterpret_cast<volatile uint32_t*>(smem + Lay::ring_off);
+    auto ring_full = [&](int e) { return reinterpret_cast<uint64_t*>(smem + Lay::ring_off + kRing * 4) + 2 * e; };
+    auto ring_empty = [&](int e) { return reinterpret_cast<uint64_t*>(smem + Lay::ring_off + kRing * 4) + 2 * e + 1; };
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -275,6 +284,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(chunks_bar(t), kNWS);
             mbar_init(carry_bar(t), 1);
             mbar_init(uempty(t), kNWS);
+        }
+        for (int e = 0; e < kRing; ++e) {
+            mbar_init(ring_full(e), 1);
+            mbar_init(ring_empty(e), 1);
         }
         fence_mbar_init();
     }
@@ -318,6 +331,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     report(kDevTimeoutCopy);
                 const uint32_t tk = tk_next;
                 if (tk >= (uint32_t)pp.U + gridDim.x) report(kDevBadWorkspace);
+                {
+                    // the ticket to the unit's look-back warp, which starts on it at once (the
+                    // sentinel past the end too)
+                    const int e = (int)(i % kRing);
+                    if (i >= kRing && !mbar_wait(ring_empty(e), (uint32_t)((i / kRing - 1) & 1), lim))
+                        report(kDevTimeoutCopy);
+                    ring_tk[e] = tk;
+                    mbar_arrive(ring_full(e));
+                }
                 UnitBlock* ub = stage_ub(s);
                 if (tk >= (uint32_t)pp.U) {
                     *s_iend = i;
@@ -365,15 +387,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp < W_S0) {
         // ------------------------------- look-back ------------------------------
+        // Warp l takes units l, l + kNL, ...  It learns a unit's ticket from the producer's
+        // ring as soon as the producer has it and folds the records of the unit's predecessors
+        // (a decoupled look-back) while the unit's rows are still loading and being
+        // summarised.  Once the summaries are in it scans them (exclusive prefixes for the
+        // emitters); if by then the carry is not yet known, it first publishes the tile's
+        // aggregate for later segments.  Then the inclusive prefix is published and the carry
+        // handed to the emitters.
         const int l = warp - W_L0;
+        const uint32_t G32 = (uint32_t)pp.G, gpb32 = (uint32_t)pp.groups_per_b;
         for (int64_t i = l;; i += kNL) {
             const int t = (int)(i % NT);
             const uint32_t ph = (uint32_t)((i / NT) & 1);
+            const int e = (int)(i % kRing);
+            // the unit's ticket; polled without suspending, so a warp whose unit lies past the
+            // end sees the producer's end index at once
             bool got = false, gone = false;
-            // polled without suspending, so a warp whose unit lies past the end sees the
-            // producer's end index at once (a suspended wait here held blocks ~3 us at the end)
             for (uint32_t it = 0; it <= lim; ++it) {
-                if (mbar_test_wait(chunks_bar(t), ph)) {
+                if (mbar_test_wait(ring_full(e), (uint32_t)((i / kRing) & 1))) {
                     got = true;
                     break;
                 }
@@ -384,95 +415,105 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __nanosleep(it < 256 ? 64 : 512);  // the bound stays ~0.1 s of waiting
             }
             if (gone) break;
-            if (!got && lane == 0) report(kDevTimeoutCarry);
-            const UnitInfo q = slot_ub(t)->info;
-            const int64_t unit = q.unit;
-            if (unit < 0) {
+            if (!got) {  // gave up: release the unit's emitters and stop
+                if (lane == 0) {
+                    report(kDevTimeoutCarry);
+                    mbar_arrive(carry_bar(t));
+                }
+                break;
+            }
+            const uint32_t tk = ring_tk[e];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ring_empty(e));
+            if (tk >= (uint32_t)pp.U) {
+                // the sentinel: its emitters learn of the end from a hand-over, once the
+                // summarisers have passed it into the slot
+                if (!mbar_wait(chunks_bar(t), ph, lim) && lane == 0) report(kDevTimeoutCarry);
+                __syncwarp();
                 if (lane == 0) mbar_arrive(carry_bar(t));
                 break;
             }
+            // the unit's geometry (as the producer works it out)
+            const uint32_t j32 = tk / G32, g32 = tk - j32 * G32;
+            const uint32_t b32 = g32 / gpb32, cg32 = g32 - b32 * gpb32;
+            const int64_t unit = tk, j = j32, g = g32;
+            const int64_t c0 = (int64_t)cg32 * Cg, t0 = j * Ts;
+            const int nch = (int)min64(Cg, C - c0);
+            const int len = (int)min64(Ts, T - t0);
+            const int64_t bc0 = (int64_t)b32 * C + c0;
             if (lane == 0) WKV_TRACE_EVENT(unit, 3);
             const int cl = lane * V;
-            const bool lane_active = cl < q.nch;
-            float w2[V];
-            {
-                const float2 wp = *reinterpret_cast<const float2*>(slot_ub(t)->w + cl);
+            const bool lane_active = cl < nch;  // (nch is even: a lane's two channels are both in or both out)
+            float w2[V] = {0.f, 0.f};
+            if (lane_active) {
+                const float2 wp = *reinterpret_cast<const float2*>(args.w + c0 + cl);
                 w2[0] = wp.x * kLog2e;
                 w2[1] = wp.y * kLog2e;
             }
-            // the first read of the newest predecessor's slot overlaps the scan
-            RawPair first;
-            if (q.j > 0 && lane_active) first = load_pair<Cg>(pp.slot + ((q.j - 1) * pp.G + q.g) * 4 * Cg, cl);
-            // scan the chunk summaries (exclusive prefixes for the emitters) and publish the
-            // tile aggregate for later segments
-            Rec agg[V];
-            if (lane_active) {
-                Rec* rc = recs(t);
+            // the chunk summaries scanned: exclusive prefixes for the emitters, the tile aggregate
+            Rec agg[V] = {rec_identity(), rec_identity()};
+            bool scanned = false;
+            auto scan = [&]() {
+                if (lane_active) {
+                    Rec* rc = recs(t);
 #pragma unroll
-                for (int c = 0; c < V; ++c) agg[c] = rec_identity();
+                    for (int w = 0; w < kNWS; ++w) {
+                        const int lw = max(0, min(LC, len - w * LC));
 #pragma unroll
-                for (int w = 0; w < kNWS; ++w) {
-                    const int lw = max(0, min(LC, q.len - w * LC));
-#pragma unroll
-                    for (int c = 0; c < V; ++c) {
-                        const Rec r = rc[w * Cg + cl + c];
-                        rc[w * Cg + cl + c] = agg[c];  // exclusive prefix of chunk w
-                        if (lw > 0) agg[c] = rec_combine(agg[c], r, (float)lw, w2[c]);
+                        for (int c = 0; c < V; ++c) {
+                            const Rec r = rc[w * Cg + cl + c];
+                            rc[w * Cg + cl + c] = agg[c];  // exclusive prefix of chunk w
+                            if (lw > 0) agg[c] = rec_combine(agg[c], r, (float)lw, w2[c]);
+                        }
                     }
                 }
-                // (nch is even, so a lane's two channels are both in range or both out)
-                if (q.j > 0 && unit != pp.drop_unit) publish_pair<Cg>(pp.slot + unit * 4 * Cg, cl, agg[0], agg[1], tag_agg);
-            }
-            if (lane == 0) WKV_TRACE_EVENT(unit, 4);
+                scanned = true;
+                if (lane == 0) WKV_TRACE_EVENT(unit, 4);
+            };
             Rec run[V];
-            if (q.j == 0) {
+            if (j == 0) {
 #pragma unroll
                 for (int c = 0; c < V; ++c)
-                    run[c] = (args.state_in && lane_active) ? rec_from_state(args.state_in, q.bc0 + cl + c, BC)
+                    run[c] = (args.state_in && lane_active) ? rec_from_state(args.state_in, bc0 + cl + c, BC)
                                                             : rec_identity();
             } else {
 #pragma unroll
                 for (int c = 0; c < V; ++c) run[c] = rec_identity();
-                // Each lane looks back for its channel pair, kLook predecessor slots per round
-                // trip: it folds aggregates from the newest backwards and stops at the first
-                // inclusive prefix (the carry is then known) or at the first slot that is not
-                // yet published.
+                // Each lane looks back for its channel pair: it folds aggregates from the newest
+                // predecessor backwards and stops at the first inclusive prefix (the carry is then
+                // known); a slot not yet published is read again after a short sleep.
                 float span = 0.f;
-                int64_t hi = q.j - 1;
+                int64_t hi = j - 1;
                 bool done = !lane_active;
                 uint32_t nap = 64;
                 bool all_done = false;
                 for (uint32_t it = 0; it <= lim && !all_done; ++it) {
+                    RawPair raw;
+                    if (!done) raw = load_pair<Cg>(pp.slot + (hi * pp.G + g) * 4 * Cg, cl);
+                    // while the read travels: the summaries are in before the carry, so the
+                    // aggregate goes out now and later segments need not wait for this carry
+                    if (!scanned && __any_sync(0xffffffffu, mbar_test_wait(chunks_bar(t), ph))) {
+                        if (!mbar_wait(chunks_bar(t), ph, lim) && lane == 0) report(kDevTimeoutCarry);
+                        scan();
+                        if (lane_active && unit != pp.drop_unit)
+                            publish_pair<Cg>(pp.slot + unit * 4 * Cg, cl, agg[0], agg[1], tag_agg);
+                    }
                     if (!done) {
-                        RawPair raw[kLook];
-#pragma unroll
-                        for (int d = 0; d < kLook; ++d)
-                            if (hi - d >= 0)
-                                raw[d] = (it == 0 && d == 0)
-                                             ? first
-                                             : load_pair<Cg>(pp.slot + ((hi - d) * pp.G + q.g) * 4 * Cg, cl);
-                        bool progressed = false;
-#pragma unroll
-                        for (int d = 0; d < kLook; ++d) {
-                            if (done) break;
-                            Rec r0, r1;
-                            const int kind = pair_kind(raw[d], tag_agg, tag_incl, r0, r1);
-                            if (kind == 0) break;
+                        Rec r0, r1;
+                        const int kind = pair_kind(raw, tag_agg, tag_incl, r0, r1);
+                        if (kind != 0) {
                             run[0] = rec_combine(r0, run[0], span, w2[0]);
                             run[1] = rec_combine(r1, run[1], span, w2[1]);
-                            progressed = true;
                             if (kind == 2) {
                                 done = true;
                             } else {
                                 span += (float)Ts;
                                 if (--hi < 0) done = true;
                             }
-                        }
-                        if (!done && !progressed) {
-                            __nanosleep(nap);
-                            nap = nap < 1024 ? nap * 2 : 1024;
-                        } else if (progressed) {
                             nap = 64;
+                        } else {
+                            __nanosleep(nap);
+                            nap = nap < 256 ? nap * 2 : 256;
                         }
                     }
                     all_done = __all_sync(0xffffffffu, done);
@@ -483,12 +524,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (lane == 0) WKV_TRACE_EVENT(unit, 5);
-            // publish the inclusive prefix (it overwrites the aggregate), then hand the carry
-            // to the emitters
+            if (!scanned) {
+                if (!mbar_wait(chunks_bar(t), ph, lim) && lane == 0) report(kDevTimeoutCarry);
+                scan();
+            }
+            // publish the inclusive prefix (over the aggregate, if that went out), then hand the
+            // carry to the emitters
             Rec inc[V];
             if (lane_active) {
 #pragma unroll
-                for (int c = 0; c < V; ++c) inc[c] = rec_combine(run[c], agg[c], (float)q.len, w2[c]);
+                for (int c = 0; c < V; ++c) inc[c] = rec_combine(run[c], agg[c], (float)len, w2[c]);
                 if (unit != pp.drop_unit) publish_pair<Cg>(pp.slot + unit * 4 * Cg, cl, inc[0], inc[1], tag_incl);
                 Rec* cs = carries(t);
 #pragma unroll
@@ -500,10 +545,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 WKV_TRACE_EVENT(unit, 6);
                 mbar_arrive(carry_bar(t));
             }
-            if (lane_active && q.j == pp.S - 1 && args.state_out) {
+            if (lane_active && j == pp.S - 1 && args.state_out) {
 #pragma unroll
                 for (int c = 0; c < V; ++c) {
-                    const int64_t bc = q.bc0 + cl + c;
+                    const int64_t bc = bc0 + cl + c;
                     args.state_out[bc] = inc[c].a;
                     args.state_out[BC + bc] = inc[c].b;
                     args.state_out[2 * BC + bc] = rec_p(inc[c], w2[c]) * kLn2;

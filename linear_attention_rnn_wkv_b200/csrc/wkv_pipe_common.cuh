@@ -161,9 +161,6 @@ __device__ __forceinline__ int pair_kind(const RawPair& r, uint32_t tag_agg, uin
     return t0 == tag_incl ? 2 : 1;
 }
 
-// Predecessor slots read per look-back round trip.
-constexpr int kLook = 1;
-
 constexpr size_t align128(size_t x) { return (x + 127) / 128 * 128; }
 
 // Tensor maps for k and v viewed as [B][T][C] (3-D, channels innermost), box = one tile.
