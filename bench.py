@@ -156,12 +156,16 @@ def measured_peaks():
 
 
 def kernel_source_digest():
+    """A digest of the forward kernel's code (its sources with comments and whitespace
+    removed), recorded in each committed ncu summary: a summary counts only while it matches."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_attention_rnn_wkv_b200", "csrc")
     for name in ("wkv_device.cuh", "wkv_vec.cuh", "wkv_internal.h", "wkv_pipe_common.cuh", "wkv_forward_chunked.cu",
                  "wkv_forward_tmem.cu"):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            code = re.sub(r"/\*.*?\*/", " ", f.read(), flags=re.S)
+        code = re.sub(r"//[^\n]*", " ", code)
+        h.update(re.sub(r"\s+", " ", code).encode())
     return h.hexdigest()[:16]
 
 

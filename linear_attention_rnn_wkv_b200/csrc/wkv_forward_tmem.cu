@@ -15,16 +15,18 @@
 // (tcgen05.st, 512 columns x 128 lanes x 32 bits) while it reads it, and the stage is
 // free again as soon as the summaries are done.  The emitting warp of the same quadrant
 // reads the chunk back (tcgen05.ld) once the carry is known.  Tensor memory holds 4
-// (fp32) or 8 (bf16) units, so that many units per SM wait for carries at once while
-// only 2-4 shared-memory stages are needed for the loads.
+// (fp32, 16-step chunks) or 5 (bf16) units, so that many units per SM wait for carries at
+// once while only 2-4 shared-memory stages are needed for the loads.
 //
 // Roles (20 warps):
-//   warp 0          producer: a ticket once a stage and a unit slot are free, the unit's
-//                   TMA box copies (`full`, one barrier per box of rows); also allocates
-//                   and frees the tensor memory;
-//   warps 1-3       look-back, round robin over units: scan the chunk summaries, publish
-//                   the aggregate, fold predecessors' records into the carry, publish
-//                   the inclusive prefix, hand the carry over (`carry`);
+//   warp 0          producer: a ticket once a stage and a unit slot are free, handed at once
+//                   to the look-back warps (a ring of tickets), the unit's TMA box copies
+//                   (`full`, one barrier per box of rows); also allocates and frees the
+//                   tensor memory;
+//   warps 1-3       look-back, round robin over units: from the ticket on, fold the
+//                   predecessors' records into the carry while the unit's rows load; scan the
+//                   chunk summaries once they are in (publishing the aggregate if the carry
+//                   is still open), publish the inclusive prefix, hand the carry over (`carry`);
 //   warps 4-11      summarise chunk c = warp - 4: summary record, rows into tensor memory
 //                   (`chunks`; the stage is released, `dempty`);
 //   warps 12-19     emit chunk c = warp - 12 (same quadrant as its summariser): rows back
@@ -32,7 +34,8 @@
 // All waits are bounded (error word on expiry, then the pipeline keeps moving), and the
 // tensor memory is freed on every path before the CTA exits.  Deadlock freedom: a ticket
 // is taken only when its stage and slot are free, roles handle a CTA's units in ticket
-// order, and every cross-CTA wait is on a smaller ticket.
+// order, every cross-CTA wait is on a smaller ticket, and the ticket ring's producer waits
+// only for look-back warps that are working on older units.
 #include <type_traits>
 
 #include "wkv_device.cuh"
