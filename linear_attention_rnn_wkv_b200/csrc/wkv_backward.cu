@@ -693,8 +693,11 @@ __global__ void __launch_bounds__(kThreads, 4)
             const Adj ls = s_adj[s][lane];
             s_adj[s][lane] = run;
             const int l = seg_len(a, J * kGroupSteps + (int64_t)s * kSeg);
-            if (l > 0) run = adj_normalize(adj_compose(ls, run, (float)l, w2));
+            if (l > 0) run = adj_compose(ls, run, (float)l, w2);
         }
+        // (normalised once: within a group every factor is at most 1 and the sums of the
+        // normalised segment sums stay below 2^11, so the chain needs no rescaling per step)
+        run = adj_normalize(run);
         uint64_t* my = a.slots + ((int64_t)b * a.NG + J) * 5 * a.C + c;
         Adj gin = adj_empty();
         if (later) {
