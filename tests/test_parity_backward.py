@@ -17,9 +17,11 @@ pytestmark = pytest.mark.gpu
 
 TOL_GRAD = 2e-4
 # T = 3000 and 2049: 24 and 17 groups of 128 steps (eight 16-step segments each), so the
-# look-backs take several hops and the last group is ragged; C = 129: a channel block of one lane
-SHAPES = [(1, 1, 4), (2, 5, 3), (1, 64, 64), (3, 200, 96), (1, 1000, 32), (2, 130, 129), (1, 3000, 8),
-          (2, 2049, 4)]
+# look-backs take several hops and the last group is ragged; C = 129: a channel block of one lane;
+# T = 128 and 256: one and two whole groups (no ragged group), the latter with rows of 37
+# channels (not whole 16-byte units: the cp.async staging)
+SHAPES = [(1, 1, 4), (2, 5, 3), (1, 64, 64), (1, 128, 32), (2, 256, 37), (3, 200, 96), (1, 1000, 32),
+          (2, 130, 129), (1, 3000, 8), (2, 2049, 4)]
 
 
 def _case(B, T, C, base, seed, k_shift=0.0):

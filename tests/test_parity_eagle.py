@@ -22,8 +22,8 @@ pytestmark = pytest.mark.gpu
 
 TOL_EAGLE = 1e-4
 
-SHAPES = [(1, 1, 64), (2, 3, 64), (1, 63, 128), (2, 64, 64), (2, 65, 128), (1, 130, 192), (3, 200, 64),
-          (1, 1000, 64)]
+SHAPES = [(1, 1, 64), (2, 3, 64), (1, 63, 128), (2, 64, 64), (2, 65, 128), (2, 128, 128), (1, 130, 192),
+          (3, 200, 64), (1, 1000, 64)]
 
 
 def _case(B, T, C, seed):

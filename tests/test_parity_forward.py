@@ -10,7 +10,7 @@ pytestmark = pytest.mark.gpu
 
 PATHS = [("serial", 0), ("chunked", 4), ("chunked", 8), ("chunked", 16)]
 SHAPES = [(1, 1, 1), (1, 2, 3), (2, 3, 5), (1, 63, 4), (3, 64, 32), (1, 65, 129), (2, 257, 36), (1, 64, 64),
-          (2, 100, 768), (1, 33, 8), (1, 130, 136)]
+          (2, 100, 768), (1, 33, 8), (1, 130, 136), (2, 128, 64), (1, 256, 72)]
 
 
 def _inputs(B, T, C, base, dtype, seed):
